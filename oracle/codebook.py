@@ -1,0 +1,76 @@
+"""NF-k codebook straight from the construction on the page (oracle side).
+
+TEST INFRASTRUCTURE (see the package docstring).
+
+"QLoRA: Efficient Finetuning of Quantized LLMs", section "Method", paragraph
+"4-bit NormalFloat Quantization":
+  (1) estimate quantiles of a theoretical N(0, 1) distribution,
+  (2) normalize the values into [-1, 1],
+  asymmetric construction: 2^(k-1) quantiles for the negative part and
+  2^(k-1) + 1 for the positive part; unify both sets and remove one of the two
+  zeros that occur in both.  (The page's superscripts were lost in
+  extraction; "2k - 1" there is 2^(k-1).)
+
+The equation that fixes the probabilities is missing from the page.  Reading
+used here: each side takes equally spaced probabilities from 1 - delta down to
+1/2, where delta is the tail probability of the outermost value; the default
+delta = (1/(2*16) + 1/(2*15)) / 2 puts the outermost value at the centre of
+the outermost equal-mass bin, averaged over the 16- and 15-level halves.
+
+Phi^-1 is computed here by bisection on Phi(x) = erfc(-x / sqrt 2) / 2 with
+libm's erfc: a method deliberately different from the one in the CUDA
+library's host code.
+"""
+
+import math
+
+import numpy as np
+
+DEFAULT_DELTA = 0.5 * (1.0 / 32.0 + 1.0 / 30.0)
+
+
+def norm_cdf(x: float) -> float:
+    """Phi(x) of N(0, 1)."""
+    return 0.5 * math.erfc(-x / math.sqrt(2.0))
+
+
+def norm_ppf(p: float) -> float:
+    """Phi^-1(p) by bisection to adjacent doubles; Phi^-1(1/2) = 0 exactly
+    (symmetry of N(0, 1))."""
+    if not 0.0 < p < 1.0:
+        raise ValueError("p must lie in (0, 1)")
+    if p == 0.5:
+        return 0.0
+    lo, hi = -40.0, 40.0
+    for _ in range(4000):
+        mid = 0.5 * (lo + hi)
+        if mid == lo or mid == hi:
+            break
+        if norm_cdf(mid) < p:
+            lo = mid
+        else:
+            hi = mid
+    # the crossing lies in [lo, hi], two adjacent doubles: take the closer one
+    return lo if abs(norm_cdf(lo) - p) <= abs(norm_cdf(hi) - p) else hi
+
+
+def _probabilities(a: float, b: float, n: int):
+    """n equally spaced probabilities from a to b, both ends included."""
+    return [a + (b - a) * i / (n - 1) if i < n - 1 else b for i in range(n)]
+
+
+def nfk_codebook_f64(k: int = 4, delta: float = DEFAULT_DELTA) -> np.ndarray:
+    """The 2^k NF-k values in float64, ascending, in [-1, 1]."""
+    top = norm_ppf(1.0 - delta)
+    pos = [norm_ppf(p) for p in _probabilities(1.0 - delta, 0.5, 2 ** (k - 1) + 1)]
+    neg = [-norm_ppf(p) for p in _probabilities(1.0 - delta, 0.5, 2 ** (k - 1))]
+    # both sets end in 0: unify and drop one of the two zeros
+    values = pos + neg[:-1]
+    assert neg[-1] == 0.0 and pos[-1] == 0.0
+    values = sorted(v / top for v in values)
+    return np.array(values, dtype=np.float64)
+
+
+def nf4_codebook(delta: float = DEFAULT_DELTA) -> np.ndarray:
+    """NF4 as the 16 binary32 values the codec stores (rounded once)."""
+    return nfk_codebook_f64(4, delta).astype(np.float32)

@@ -1,0 +1,66 @@
+"""QLoRA linear layer, forward and backward, in float64 (oracle side).
+
+TEST INFRASTRUCTURE (see the package docstring).
+
+The layer (mbrenndoerfer.com QLoRA essay, section "Low-Rank Adaptation
+(LoRA)": x_out = (W_q + BA) x_in, with A of shape r x d and B of shape d x r;
+"QLoRA: Efficient Finetuning of Quantized LLMs", section "Method": the 4-bit
+weight is dequantized to BFloat16 and used in a 16-bit matrix multiplication;
+gradients are backpropagated through the frozen quantized weight into the
+adapters only, so there is no gradient for W).
+
+Row-vector convention, as in nn.Linear:
+  X  [M, K]  tokens x in_features          W' [N, K] dequantized weight (bf16)
+  A  [r, K]  B [N, r]  s = lora_alpha / r (the usual LoRA scale; the pages
+  print alpha and r but no formula)
+  Y  = X W'^T + s (X A^T) B^T
+and with dY = dL/dY:
+  dX = dY W' + s (dY B) A
+  dA = s (dY B)^T X
+  dB = s dY^T (X A^T)
+Every operand is exactly the bf16 (or float32) value handed to the GPU,
+widened to float64; numpy's float64 matmul is the only library step.
+"""
+
+import numpy as np
+
+
+def _f64(a) -> np.ndarray:
+    return np.asarray(a, dtype=np.float64)
+
+
+def forward(X, Wd, A, B, s: float) -> np.ndarray:
+    X, Wd, A, B = map(_f64, (X, Wd, A, B))
+    return X @ Wd.T + s * ((X @ A.T) @ B.T)
+
+
+def backward(X, Wd, A, B, s: float, dY):
+    """(dX, dA, dB)."""
+    X, Wd, A, B, dY = map(_f64, (X, Wd, A, B, dY))
+    G = dY @ B                     # [M, r]
+    dX = dY @ Wd + s * (G @ A)
+    dA = s * (G.T @ X)
+    dB = s * (dY.T @ (X @ A.T))
+    return dX, dA, dB
+
+
+def forward_rows(X, Wd, A, B, s: float, rows) -> np.ndarray:
+    """Forward restricted to the token rows `rows` (for spot checks at sizes
+    where the whole product would be slow on the CPU)."""
+    return forward(_f64(X)[rows], Wd, A, B, s)
+
+
+def backward_dx_rows(Wd, A, B, s: float, dY, rows) -> np.ndarray:
+    dYr = _f64(dY)[rows]
+    Wd, A, B = map(_f64, (Wd, A, B))
+    return dYr @ Wd + s * ((dYr @ B) @ A)
+
+
+def rel_frobenius(got, ref) -> float:
+    got, ref = _f64(got), _f64(ref)
+    den = np.linalg.norm(ref)
+    return float(np.linalg.norm(got - ref) / (den if den > 0 else 1.0))
+
+
+def max_abs(got, ref) -> float:
+    return float(np.max(np.abs(_f64(got) - _f64(ref)))) if np.size(ref) else 0.0

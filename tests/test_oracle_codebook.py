@@ -1,0 +1,68 @@
+"""Pins of the oracle's NF-k codebook against what the pages and mathematics fix.
+
+"QLoRA: Efficient Finetuning of Quantized LLMs", section "Method", paragraph
+"4-bit NormalFloat Quantization".
+"""
+
+import numpy as np
+import pytest
+from scipy import special
+
+from oracle import codebook
+from tests.conftest import read_golden
+
+FIG = {k: float(v) for k, v in read_golden("paper_figures.txt")}
+
+
+@pytest.mark.parametrize("p,x", [(float(a), float(b)) for a, b in read_golden("normal_quantiles.txt")])
+def test_norm_ppf_textbook_values(p, x):
+    assert codebook.norm_ppf(p) == pytest.approx(x, abs=2e-15, rel=2e-15)
+
+
+def test_norm_ppf_against_library_routine():
+    for p in np.linspace(0.001, 0.999, 137):
+        assert codebook.norm_ppf(float(p)) == pytest.approx(float(special.ndtri(p)), rel=1e-13, abs=1e-13)
+
+
+def test_nf4_structure_matches_the_page():
+    q = codebook.nf4_codebook()
+    assert q.dtype == np.float32
+    assert q.size == FIG["codebook_size"] == 2 ** FIG["k_bits"]
+    assert np.all(np.diff(q) > 0), "strictly increasing"
+    assert q[0] == FIG["range_lo"] and q[-1] == FIG["range_hi"], "normalized into [-1, 1]"
+    assert np.count_nonzero(q == 0.0) == 1, "exactly one exact zero"
+    # 2^(k-1) negative-part quantiles and 2^(k-1)+1 positive-part quantiles, the
+    # shared zero counted once: 7 negative, 1 zero, 8 positive
+    assert np.count_nonzero(q < 0) == FIG["negative_part_quantiles"] - 1
+    assert np.count_nonzero(q > 0) == FIG["positive_part_quantiles"] - 1
+    assert int(np.flatnonzero(q == 0.0)[0]) == 7
+
+
+def test_nf4_values_are_equally_spaced_quantiles():
+    """Undo the normalization with an independent Phi (scipy): the positive
+    values must sit at 8 equal probability steps from 1/2 to 1 - delta, the
+    negative ones at 7 equal steps (step (1) of the construction)."""
+    delta = codebook.DEFAULT_DELTA
+    q = codebook.nfk_codebook_f64(4, delta)
+    top = special.ndtri(1.0 - delta)
+    p = special.ndtr(q * top)
+    pos, neg = p[q > 0], p[q < 0]
+    np.testing.assert_allclose(np.diff(np.concatenate([[0.5], pos])), (0.5 - delta) / 8, rtol=1e-9)
+    np.testing.assert_allclose(np.diff(np.concatenate([neg, [0.5]])), (0.5 - delta) / 7, rtol=1e-9)
+    assert p[-1] == pytest.approx(1.0 - delta, rel=1e-12)
+    assert p[0] == pytest.approx(delta, rel=1e-9)
+
+
+def test_nf4_binary32_values_are_the_rounded_float64_construction():
+    q64 = codebook.nfk_codebook_f64(4)
+    assert np.array_equal(codebook.nf4_codebook(), q64.astype(np.float32))
+
+
+@pytest.mark.parametrize("k", [2, 3, 5])
+def test_nfk_general_k(k):
+    q = codebook.nfk_codebook_f64(k)
+    assert q.size == 2 ** k
+    assert q[0] == -1.0 and q[-1] == 1.0
+    assert np.count_nonzero(q == 0.0) == 1
+    assert np.count_nonzero(q < 0) == 2 ** (k - 1) - 1
+    assert np.all(np.diff(q) > 0)

@@ -1,0 +1,86 @@
+"""Pins of the oracle's QLoRA linear: brute-force loops, finite differences of
+the forward, and the special cases that reduce to a plain product.
+
+mbrenndoerfer.com QLoRA essay, section "Low-Rank Adaptation (LoRA)"
+(x_out = (W_q + BA) x_in); "QLoRA: Efficient Finetuning of Quantized LLMs",
+section "Method" (16-bit matmul with the dequantized weight) and abstract
+(gradients flow through the frozen 4-bit weight into the adapters only).
+"""
+
+import numpy as np
+
+from oracle import linear
+
+
+def _rand(rng, *shape):
+    return rng.standard_normal(shape)
+
+
+def test_forward_against_triple_loops():
+    rng = np.random.default_rng(12)
+    M, K, N, r, s = 3, 8, 5, 2, 0.75
+    X, W, A, B = _rand(rng, M, K), _rand(rng, N, K), _rand(rng, r, K), _rand(rng, N, r)
+    Y = linear.forward(X, W, A, B, s)
+    for m in range(M):
+        for n in range(N):
+            ref = 0.0
+            for k in range(K):
+                dw = sum(B[n, j] * A[j, k] for j in range(r))          # (B A)[n, k]
+                ref += (W[n, k] + s * dw) * X[m, k]
+            assert abs(Y[m, n] - ref) < 1e-12
+
+
+def test_backward_against_finite_differences():
+    rng = np.random.default_rng(13)
+    M, K, N, r, s = 4, 6, 5, 3, 0.5
+    X, W, A, B, dY = (_rand(rng, M, K), _rand(rng, N, K), _rand(rng, r, K),
+                      _rand(rng, N, r), _rand(rng, M, N))
+    dX, dA, dB = linear.backward(X, W, A, B, s, dY)
+
+    def loss(X_, A_, B_):
+        return float(np.sum(dY * linear.forward(X_, W, A_, B_, s)))
+
+    h = 1e-6
+    for name, P, G in (("X", X, dX), ("A", A, dA), ("B", B, dB)):
+        for idx in np.ndindex(P.shape):
+            Pp, Pm = P.copy(), P.copy()
+            Pp[idx] += h
+            Pm[idx] -= h
+            args_p = {"X": (Pp, A, B), "A": (X, Pp, B), "B": (X, A, Pp)}[name]
+            args_m = {"X": (Pm, A, B), "A": (X, Pm, B), "B": (X, A, Pm)}[name]
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * h)
+            assert abs(fd - G[idx]) < 1e-6 * max(1.0, abs(fd)), (name, idx)
+
+
+def test_zero_adapter_and_zero_scale_reduce_to_plain_product():
+    rng = np.random.default_rng(14)
+    M, K, N, r = 5, 16, 7, 4
+    X, W, A, dY = _rand(rng, M, K), _rand(rng, N, K), _rand(rng, r, K), _rand(rng, M, N)
+    B0 = np.zeros((N, r))
+    np.testing.assert_allclose(linear.forward(X, W, A, B0, 2.0), X @ W.T, rtol=0, atol=1e-12)
+    dX, dA, dB = linear.backward(X, W, A, B0, 2.0, dY)
+    np.testing.assert_allclose(dX, dY @ W, atol=1e-12)
+    assert np.all(dA == 0)
+    B = _rand(rng, N, r)
+    np.testing.assert_allclose(linear.forward(X, W, A, B, 0.0), X @ W.T, atol=1e-12)
+    dX, dA, dB = linear.backward(X, W, A, B, 0.0, dY)
+    assert np.all(dA == 0) and np.all(dB == 0)
+
+
+def test_row_helpers_match_full_products():
+    rng = np.random.default_rng(15)
+    M, K, N, r, s = 9, 64, 12, 4, 0.25
+    X, W, A, B, dY = (_rand(rng, M, K), _rand(rng, N, K), _rand(rng, r, K),
+                      _rand(rng, N, r), _rand(rng, M, N))
+    rows = [0, 3, 8]
+    np.testing.assert_allclose(linear.forward_rows(X, W, A, B, s, rows),
+                               linear.forward(X, W, A, B, s)[rows], atol=1e-12)
+    np.testing.assert_allclose(linear.backward_dx_rows(W, A, B, s, dY, rows),
+                               linear.backward(X, W, A, B, s, dY)[0][rows], atol=1e-12)
+
+
+def test_error_metrics():
+    ref = np.array([[3.0, 4.0]])
+    assert linear.rel_frobenius(ref, ref) == 0.0
+    assert linear.rel_frobenius(ref + np.array([[0.0, 0.5]]), ref) == 0.1
+    assert linear.max_abs(ref + 0.25, ref) == 0.25
