@@ -1,0 +1,176 @@
+"""Python binding of libqlora_b200.so (the C ABI declared in include/qlora.h).
+
+Argument marshalling only: every function forwards to the C entry point of
+the same name, passing torch device pointers and the current CUDA stream.
+PyTorch provides device memory and streams; all arithmetic of the path runs
+in the library's sm_100a kernels.  If the shared library is missing the
+import fails loudly -- there is no fallback implementation.
+"""
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqlora_b200.so")
+
+QLORA_BLOCK = 64
+QLORA_GROUP = 256
+QLORA_BF16 = 0
+QLORA_FP32 = 1
+
+STATUS = {
+    0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_SHAPE", 3: "QLORA_ERR_ALIGNMENT",
+    4: "QLORA_ERR_WORKSPACE", 5: "QLORA_ERR_CUDA", 6: "QLORA_ERR_UNSUPPORTED", 7: "QLORA_ERR_TIMEOUT",
+}
+
+# every symbol the header declares
+EXPORTS = (
+    "qlora_build_nf4_codebook", "qlora_quantize_workspace_bytes", "qlora_quantize_nf4_dq",
+    "qlora_dequantize_nf4_dq", "qlora_linear_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd",
+    "qlora_status_string", "qlora_check_device_error",
+)
+
+
+class QLoraError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+        self.status = status
+
+
+class qlora_nf4_weight(ctypes.Structure):
+    _fields_ = [
+        ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+        ("packed", ctypes.c_void_p), ("code2", ctypes.c_void_p),
+        ("c2", ctypes.c_void_p), ("mean", ctypes.c_void_p),
+        ("codebook", ctypes.c_float * 16),
+    ]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python bit_nf4_quantized_16_b200/build.py`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I64, I32, F, S = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    W = ctypes.POINTER(qlora_nf4_weight)
+    sig = {
+        "qlora_build_nf4_codebook": (ctypes.c_int, [ctypes.c_double, P]),
+        "qlora_quantize_workspace_bytes": (S, [I64, I64]),
+        "qlora_quantize_nf4_dq": (ctypes.c_int, [P, ctypes.c_int, W, P, S, P]),
+        "qlora_dequantize_nf4_dq": (ctypes.c_int, [W, P, P]),
+        "qlora_linear_workspace_bytes": (S, [I64, I64, I64, I32]),
+        "qlora_linear_fwd": (ctypes.c_int, [W, P, I64, P, P, I32, F, P, ctypes.c_int, P, P, S, P]),
+        "qlora_linear_bwd": (ctypes.c_int, [W, P, P, I64, P, P, I32, F, P, P, ctypes.c_int, P, P, P, S, P]),
+        "qlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "qlora_check_device_error": (ctypes.c_int, [P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise QLoraError(status, where)
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return QLORA_BF16
+    if t.dtype == torch.float32:
+        return QLORA_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+# ---- quantized weight container (device buffers owned by torch) ----------------
+
+class NF4Weight:
+    """Device buffers of one quantized weight plus its C descriptor."""
+
+    def __init__(self, rows: int, cols: int, codebook=None, device="cuda"):
+        if cols % QLORA_BLOCK:
+            raise ValueError("cols must be a multiple of 64")
+        nblocks = rows * cols // QLORA_BLOCK
+        ngroups = -(-nblocks // QLORA_GROUP)
+        self.rows, self.cols = rows, cols
+        self.packed = torch.empty(rows * cols // 2, dtype=torch.uint8, device=device)
+        self.code2 = torch.empty(nblocks, dtype=torch.uint8, device=device)
+        self.c2 = torch.empty(ngroups, dtype=torch.float32, device=device)
+        self.mean = torch.empty(4, dtype=torch.float32, device=device)   # 16-byte slot
+        self.codebook = list(codebook) if codebook is not None else qlora_build_nf4_codebook()
+        self.desc = qlora_nf4_weight(rows, cols, self.packed.data_ptr(), self.code2.data_ptr(),
+                                     self.c2.data_ptr(), self.mean.data_ptr(),
+                                     (ctypes.c_float * 16)(*self.codebook))
+
+    @property
+    def nbytes(self) -> int:
+        return self.packed.numel() + self.code2.numel() + 4 * self.c2.numel() + 4
+
+
+# ---- entry points (same names as the C ABI) -------------------------------------------
+
+def qlora_build_nf4_codebook(delta: float = 0.0):
+    out = (ctypes.c_float * 16)()
+    _check(lib.qlora_build_nf4_codebook(delta, ctypes.cast(out, ctypes.c_void_p)), "qlora_build_nf4_codebook")
+    return [float(v) for v in out]
+
+
+def qlora_quantize_workspace_bytes(rows: int, cols: int) -> int:
+    return lib.qlora_quantize_workspace_bytes(rows, cols)
+
+
+def qlora_quantize_nf4_dq(W: torch.Tensor, out: NF4Weight, workspace: torch.Tensor, stream=None):
+    _check(lib.qlora_quantize_nf4_dq(_ptr(W), _dtype_code(W), ctypes.byref(out.desc), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _stream(stream)),
+           "qlora_quantize_nf4_dq")
+
+
+def qlora_dequantize_nf4_dq(w: NF4Weight, out_bf16: torch.Tensor, stream=None):
+    _check(lib.qlora_dequantize_nf4_dq(ctypes.byref(w.desc), _ptr(out_bf16), _stream(stream)),
+           "qlora_dequantize_nf4_dq")
+
+
+def qlora_linear_workspace_bytes(M: int, N: int, K: int, r: int) -> int:
+    return lib.qlora_linear_workspace_bytes(M, N, K, r)
+
+
+def qlora_linear_fwd(w: NF4Weight, X, M: int, A, B, r: int, scale: float, Y, H_save=None,
+                     workspace=None, stream=None):
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.qlora_linear_fwd(ctypes.byref(w.desc), _ptr(X), M, _ptr(A), _ptr(B), r, scale, _ptr(Y),
+                                _dtype_code(Y), _ptr(H_save), _ptr(workspace), ws_bytes, _stream(stream)),
+           "qlora_linear_fwd")
+
+
+def qlora_linear_bwd(w: NF4Weight, X, dY, M: int, A, B, r: int, scale: float, H_saved, dX, dA, dB,
+                     workspace=None, stream=None):
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    dx_code = QLORA_BF16 if dX is None else _dtype_code(dX)
+    _check(lib.qlora_linear_bwd(ctypes.byref(w.desc), _ptr(X), _ptr(dY), M, _ptr(A), _ptr(B), r, scale,
+                                _ptr(H_saved), _ptr(dX), dx_code, _ptr(dA), _ptr(dB), _ptr(workspace),
+                                ws_bytes, _stream(stream)),
+           "qlora_linear_bwd")
+
+
+def qlora_status_string(status: int) -> str:
+    return lib.qlora_status_string(status).decode()
+
+
+def qlora_check_device_error(stream=None):
+    _check(lib.qlora_check_device_error(_stream(stream)), "qlora_check_device_error")

@@ -1,0 +1,186 @@
+// Host-side entry points that launch nothing: the NF4 codebook, status
+// strings, device queries and the device error word.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <mutex>
+#include <string.h>
+
+#include "common.cuh"
+
+namespace qlora {
+
+// One error word per device; kernels receive its address as a parameter.
+static __device__ int g_device_error = 0;
+
+namespace {
+constexpr int kMaxDevices = 64;
+int *g_error_ptr[kMaxDevices] = {};
+DeviceInfo g_info[kMaxDevices];
+bool g_info_ok[kMaxDevices] = {};
+std::mutex g_mutex;
+}  // namespace
+
+qlora_status device_info(DeviceInfo *out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QLORA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!g_info_ok[dev]) {
+        DeviceInfo d;
+        d.device = dev;
+        int v = 0;
+        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return QLORA_ERR_CUDA;
+        if (cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return QLORA_ERR_CUDA;
+        if (cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return QLORA_ERR_CUDA;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return QLORA_ERR_CUDA;
+        d.smem_optin = (size_t)v;
+        g_info[dev] = d;
+        g_info_ok[dev] = true;
+    }
+    *out = g_info[dev];
+    // the kernels are built for sm_100a only
+    if (out->major != 10) return QLORA_ERR_UNSUPPORTED;
+    return QLORA_OK;
+}
+
+int *device_error_word()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!g_error_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+        g_error_ptr[dev] = static_cast<int *>(p);
+    }
+    return g_error_ptr[dev];
+}
+
+qlora_status check_weight(const qlora_nf4_weight *w)
+{
+    if (!w) return QLORA_ERR_INVALID_ARG;
+    if (w->rows <= 0 || w->cols <= 0 || w->cols % QLORA_BLOCK != 0) return QLORA_ERR_SHAPE;
+    if (!w->packed || !w->code2 || !w->c2 || !w->mean) return QLORA_ERR_INVALID_ARG;
+    if (!aligned16(w->packed) || !aligned16(w->code2) || !aligned16(w->c2) || !aligned16(w->mean))
+        return QLORA_ERR_ALIGNMENT;
+    int zeros = 0;
+    for (int j = 0; j < 16; j++) {
+        if (!isfinite(w->codebook[j])) return QLORA_ERR_INVALID_ARG;
+        if (j && !(w->codebook[j - 1] < w->codebook[j])) return QLORA_ERR_INVALID_ARG;
+        zeros += w->codebook[j] == 0.0f;
+    }
+    if (zeros != 1) return QLORA_ERR_INVALID_ARG;
+    return QLORA_OK;
+}
+
+// ---- normal quantile function -----------------------------------------------------
+//
+// Algorithm AS 241 (M. J. Wichura, "The percentage points of the normal
+// distribution", Applied Statistics 37 (1988) 477-484), routine PPND16:
+// rational approximations in q = p - 1/2 for the central region |q| <= 0.425
+// and in t = sqrt(-ln min(p, 1-p)) for the tails, accurate to about 1e-16.
+static double ppnd16(double p)
+{
+    static const double a[8] = {3.3871328727963666080e0, 1.3314166789178437745e+2, 1.9715909503065514427e+3,
+                                1.3731693765509461125e+4, 4.5921953931549871457e+4, 6.7265770927008700853e+4,
+                                3.3430575583588128105e+4, 2.5090809287301226727e+3};
+    static const double b[8] = {1.0, 4.2313330701600911252e+1, 6.8718700749205790830e+2, 5.3941960214247511077e+3,
+                                2.1213794301586595867e+4, 3.9307895800092710610e+4, 2.8729085735721942674e+4,
+                                5.2264952788528545610e+3};
+    static const double c[8] = {1.42343711074968357734e0, 4.63033784615654529590e0, 5.76949722146069140550e0,
+                                3.64784832476320460504e0, 1.27045825245236838258e0, 2.41780725177450611770e-1,
+                                2.27238449892691845833e-2, 7.74545014278341407640e-4};
+    static const double d[8] = {1.0, 2.05319162663775882187e0, 1.67638483018380384940e0, 6.89767334985100004550e-1,
+                                1.48103976427480074590e-1, 1.51986665636164571966e-2, 5.47593808499534494600e-4,
+                                1.05075007164441684324e-9};
+    static const double e[8] = {6.65790464350110377720e0, 5.46378491116411436990e0, 1.78482653991729133580e0,
+                                2.96560571828504891230e-1, 2.65321895265761230930e-2, 1.24266094738807843860e-3,
+                                2.71155556874348757815e-5, 2.01033439929228813265e-7};
+    static const double f[8] = {1.0, 5.99832206555887937690e-1, 1.36929880922735805310e-1, 1.48753612908506148525e-2,
+                                7.86869131145613259100e-4, 1.84631831751005468180e-5, 1.42151175831644588870e-7,
+                                2.04426310338993978564e-15};
+    auto poly = [](const double *k, double x) {
+        double s = k[7];
+        for (int i = 6; i >= 0; i--) s = s * x + k[i];
+        return s;
+    };
+    double q = p - 0.5;
+    if (fabs(q) <= 0.425) {
+        double r = 0.180625 - q * q;
+        return q * poly(a, r) / poly(b, r);
+    }
+    double r = q < 0 ? p : 1.0 - p;
+    r = sqrt(-log(r));
+    double x;
+    if (r <= 5.0) {
+        r -= 1.6;
+        x = poly(c, r) / poly(d, r);
+    } else {
+        r -= 5.0;
+        x = poly(e, r) / poly(f, r);
+    }
+    return q < 0 ? -x : x;
+}
+
+}  // namespace qlora
+
+using namespace qlora;
+
+// NF4 construction ("QLoRA: Efficient Finetuning of Quantized LLMs", section
+// "Method", paragraph "4-bit NormalFloat Quantization"): 2^(k-1)+1 = 9
+// quantiles for the positive part and 2^(k-1) = 8 for the negative part,
+// probabilities equally spaced from 1 - delta to 1/2, union without the
+// duplicate zero, normalized by the largest magnitude into [-1, 1].
+extern "C" qlora_status qlora_build_nf4_codebook(double delta, float codebook_out[16])
+{
+    if (!codebook_out) return QLORA_ERR_INVALID_ARG;
+    if (delta <= 0.0) delta = 0.5 * (1.0 / 32.0 + 1.0 / 30.0);
+    if (!(delta < 0.5)) return QLORA_ERR_INVALID_ARG;
+    const double hi = 1.0 - delta;
+    const double top = ppnd16(hi);
+    double v[16];
+    int n = 0;
+    for (int i = 0; i < 9; i++) {        // positive part, zero included
+        double p = i < 8 ? hi + (0.5 - hi) * i / 8.0 : 0.5;
+        v[n++] = (i < 8 ? ppnd16(p) : 0.0) / top;
+    }
+    for (int i = 0; i < 7; i++) {        // negative part; its zero is the dropped duplicate
+        double p = hi + (0.5 - hi) * i / 7.0;
+        v[n++] = -ppnd16(p) / top;
+    }
+    // ascending order
+    for (int i = 1; i < 16; i++)
+        for (int j = i; j > 0 && v[j - 1] > v[j]; j--) {
+            double t = v[j];
+            v[j] = v[j - 1];
+            v[j - 1] = t;
+        }
+    for (int i = 0; i < 16; i++) codebook_out[i] = (float)v[i];
+    return QLORA_OK;
+}
+
+extern "C" const char *qlora_status_string(qlora_status status)
+{
+    switch (status) {
+    case QLORA_OK: return "QLORA_OK";
+    case QLORA_ERR_INVALID_ARG: return "QLORA_ERR_INVALID_ARG";
+    case QLORA_ERR_SHAPE: return "QLORA_ERR_SHAPE";
+    case QLORA_ERR_ALIGNMENT: return "QLORA_ERR_ALIGNMENT";
+    case QLORA_ERR_WORKSPACE: return "QLORA_ERR_WORKSPACE";
+    case QLORA_ERR_CUDA: return "QLORA_ERR_CUDA";
+    case QLORA_ERR_UNSUPPORTED: return "QLORA_ERR_UNSUPPORTED";
+    case QLORA_ERR_TIMEOUT: return "QLORA_ERR_TIMEOUT";
+    }
+    return "QLORA_ERR_UNKNOWN";
+}
+
+extern "C" qlora_status qlora_check_device_error(void *stream)
+{
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return QLORA_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (v == kDevOk) return QLORA_OK;
+    int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return QLORA_ERR_CUDA;
+    return v == kDevTimeout ? QLORA_ERR_TIMEOUT : QLORA_ERR_CUDA;
+}

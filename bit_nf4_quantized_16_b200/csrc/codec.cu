@@ -1,0 +1,425 @@
+// NF4 + double-quantization codec kernels for sm_100a.
+//
+// "QLoRA: Efficient Finetuning of Quantized LLMs", section "Method":
+//   - "4-bit NormalFloat Quantization", step (3): each block of 64 weights is
+//     rescaled by its absolute maximum into [-1, 1] and rounded to the nearest
+//     value of the 16-entry NF4 table;
+//   - "Double Quantization": the per-block 32-bit constants are quantized
+//     again (8-bit floats, groups of 256, mean subtracted);
+//   - storage vs. compute type: the weight is dequantized to BFloat16 when
+//     used.
+//
+// Three kernels, all HBM-bound streaming passes with 16-byte accesses:
+//   quantize_blocks_kernel  W -> packed codes, c1 (workspace), exact mean
+//   dq_encode_kernel        c1, mean -> code2 (E4M3), c2
+//   dequantize_kernel       packed, code2, c2, mean -> bf16 W'
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_fp16.h>
+#include <math.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "exact_mean.cuh"
+
+namespace qlora {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kUnroll = 4;
+
+// ---- small device helpers ----------------------------------------------------
+
+// Order-preserving map from binary32 to uint32: a < b (as floats, -0 < +0)
+// iff key(a) < key(b).
+__device__ __forceinline__ uint32_t sortable_key(float f)
+{
+    uint32_t b = __float_as_uint(f);
+    uint32_t s = (uint32_t)((int32_t)b >> 31);
+    return b ^ (s | 0x80000000u);
+}
+
+__device__ __forceinline__ uint4 ld_stream_v4(const void *p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t ld_stream_u32(const void *p)
+{
+    uint32_t v;
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
+// Two binary32 values rounded to nearest-even bf16, lo in bits 0-15.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    uint32_t d;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
+__device__ __forceinline__ float e4m3_to_float(uint8_t code)
+{
+    __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)code, __NV_E4M3);
+    return __half2float(__half(h));
+}
+
+// ---- pass 1: absmax, codes, exact-mean buckets -----------------------------------
+
+struct QuantParams {
+    const void *W;             // bf16 or fp32, numel elements
+    uint8_t *packed;           // numel / 2 bytes
+    float *c1;                 // nblocks floats (workspace)
+    unsigned long long *acc;   // 256 buckets (workspace, zero on entry)
+    unsigned int *ticket;      // CTA arrival counter (workspace, zero on entry)
+    float *mean_out;           // 1 float
+    int64_t nwords;            // numel / 8: one word = 8 codes = 32 bits
+    int64_t nblocks;
+    uint32_t mkey[15];         // keys of the round-down midpoints, ascending
+};
+
+// Code lookup on the top 12 bits of the key of n = x * (1/c1).  The 15
+// midpoints between neighbouring codebook values are rounded down to binary32,
+// so "n > midpoint_j" holds exactly when n is nearer to value j+1 than to
+// value j (a tie stays with the lower index), and the code is the number of
+// midpoints below n.  Each 2^20-key interval holds at most one midpoint (the
+// host checks this), so one table entry plus one carry decides the code:
+//   entry = (midpoints below the interval) << 20, plus 2^20-1 - low20(key_m)
+//   if midpoint m lies inside the interval;  code = (entry + low20(key)) >> 20.
+__device__ __forceinline__ void build_code_lut(uint32_t *lut, const uint32_t (&mkey)[15])
+{
+    for (int idx = threadIdx.x; idx < 4096; idx += blockDim.x) {
+        uint32_t lo = (uint32_t)idx << 20;
+        uint32_t below = 0, inc = 0;
+#pragma unroll
+        for (int j = 0; j < 15; j++) {
+            uint32_t k = mkey[j];
+            if (k < lo)
+                below++;
+            else if ((k >> 20) == (uint32_t)idx)
+                inc = 0xFFFFFu - (k & 0xFFFFFu);
+        }
+        lut[idx] = (below << 20) + inc;
+    }
+}
+
+__device__ __forceinline__ uint32_t code_of(const uint32_t *lut, float x, float r)
+{
+    uint32_t k = sortable_key(__fmul_rn(x, r));
+    return (lut[k >> 20] + (k & 0xFFFFFu)) >> 20;
+}
+
+template <bool kF32In>
+__global__ void __launch_bounds__(kThreads) quantize_blocks_kernel(QuantParams p)
+{
+    __shared__ uint32_t lut[4096];
+    __shared__ unsigned long long s_acc[256];
+    __shared__ bool s_last;
+    build_code_lut(lut, p.mkey);
+    s_acc[threadIdx.x] = 0;
+    __syncthreads();
+
+    const int lane = threadIdx.x & 31;
+    const int64_t stride = (int64_t)gridDim.x * kThreads;
+    for (int64_t base = (int64_t)blockIdx.x * kThreads + (threadIdx.x & ~31); base < p.nwords;
+         base += stride * kUnroll) {
+        float x[kUnroll][8];
+        bool act[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; u++) {
+            int64_t w = base + lane + u * stride;
+            act[u] = w < p.nwords;
+            if (kF32In) {
+                uint4 a = make_uint4(0, 0, 0, 0), b = a;
+                if (act[u]) {
+                    const float *src = static_cast<const float *>(p.W) + 8 * w;
+                    a = ld_stream_v4(src);
+                    b = ld_stream_v4(src + 4);
+                }
+                x[u][0] = __uint_as_float(a.x); x[u][1] = __uint_as_float(a.y);
+                x[u][2] = __uint_as_float(a.z); x[u][3] = __uint_as_float(a.w);
+                x[u][4] = __uint_as_float(b.x); x[u][5] = __uint_as_float(b.y);
+                x[u][6] = __uint_as_float(b.z); x[u][7] = __uint_as_float(b.w);
+            } else {
+                uint4 a = make_uint4(0, 0, 0, 0);
+                if (act[u]) a = ld_stream_v4(static_cast<const __nv_bfloat16 *>(p.W) + 8 * w);
+                const uint32_t v[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    x[u][2 * i] = __uint_as_float(v[i] << 16);
+                    x[u][2 * i + 1] = __uint_as_float(v[i] & 0xFFFF0000u);
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; u++) {
+            float m = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; i++) m = fmaxf(m, fabsf(x[u][i]));
+            // the 8 lanes of one block reduce together
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+            // zero block (absmax below the smallest normal): r = 0 sends every
+            // element to n = +-0, whose code is the codebook's zero
+            const float r = m < 1.17549435e-38f ? 0.0f : __frcp_rn(m);
+            uint32_t word = 0;
+#pragma unroll
+            for (int i = 0; i < 8; i++) word |= code_of(lut, x[u][i], r) << (4 * i);
+            if (act[u]) {
+                int64_t w = base + lane + u * stride;
+                reinterpret_cast<uint32_t *>(p.packed)[w] = word;
+                if ((lane & 7) == 0) {
+                    p.c1[w >> 3] = m;
+                    uint32_t bucket, sig;
+                    exact_mean_split(__float_as_uint(m), &bucket, &sig);
+                    atomicAdd(&s_acc[bucket], (unsigned long long)sig);
+                }
+            }
+        }
+    }
+    __syncthreads();
+    unsigned long long v = s_acc[threadIdx.x];
+    if (v) atomicAdd(&p.acc[threadIdx.x], v);
+    // the last CTA to finish turns the buckets into the mean
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(p.ticket, 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (s_last) {
+        __threadfence();
+        s_acc[threadIdx.x] = atomicAdd(&p.acc[threadIdx.x], 0ull);
+        __syncthreads();
+        if (threadIdx.x == 0)
+            *p.mean_out = __uint_as_float(exact_mean_bits(s_acc, (uint64_t)p.nblocks));
+    }
+}
+
+// ---- pass 2: double quantization of the block constants ----------------------------
+
+struct DqParams {
+    const float *c1;
+    const float *mean;
+    uint8_t *code2;
+    float *c2;
+    int64_t nblocks;
+    int64_t ngroups;
+};
+
+// One warp per group of 256 constants, 8 per lane.
+__global__ void __launch_bounds__(kThreads) dq_encode_kernel(DqParams p)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const float mu = *p.mean;
+    for (int64_t g = (int64_t)blockIdx.x * (kThreads / 32) + warp; g < p.ngroups;
+         g += (int64_t)gridDim.x * (kThreads / 32)) {
+        const int64_t b0 = g * QLORA_GROUP + lane * 8;
+        float d[8];
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            bool ok = b0 + i < p.nblocks;
+            d[i] = ok ? __fsub_rn(p.c1[b0 + i], mu) : 0.0f;
+            amax = fmaxf(amax, fabsf(d[i]));
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const float s = __fdiv_rn(amax, 448.0f);
+        if (lane == 0) p.c2[g] = s;
+        uint8_t e[8];
+#pragma unroll
+        for (int i = 0; i < 8; i++)
+            e[i] = s == 0.0f ? (uint8_t)0
+                             : (uint8_t)__nv_cvt_float_to_fp8(__fdiv_rn(d[i], s), __NV_SATFINITE, __NV_E4M3);
+        if (b0 + 8 <= p.nblocks) {
+            uint2 v;
+            v.x = e[0] | (e[1] << 8) | (e[2] << 16) | ((uint32_t)e[3] << 24);
+            v.y = e[4] | (e[5] << 8) | (e[6] << 16) | ((uint32_t)e[7] << 24);
+            *reinterpret_cast<uint2 *>(p.code2 + b0) = v;
+        } else {
+            for (int i = 0; i < 8; i++)
+                if (b0 + i < p.nblocks) p.code2[b0 + i] = e[i];
+        }
+    }
+}
+
+// ---- dequantize -------------------------------------------------------------------
+
+struct DeqParams {
+    const uint8_t *packed;
+    const uint8_t *code2;
+    const float *c2;
+    const float *mean;
+    __nv_bfloat16 *out;
+    int64_t nwords;
+    float q[16];
+};
+
+__global__ void __launch_bounds__(kThreads) dequantize_kernel(DeqParams p)
+{
+    __shared__ float lut[16];
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int i = 0; i < 16; i++) lut[i] = p.q[i];   // static indices keep p in the parameter bank
+    }
+    __syncthreads();
+    const float mu = *p.mean;
+    const int64_t stride = (int64_t)gridDim.x * kThreads;
+    for (int64_t w0 = (int64_t)blockIdx.x * kThreads + threadIdx.x; w0 < p.nwords; w0 += stride * kUnroll) {
+        uint32_t word[kUnroll];
+        float c1p[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; u++) {
+            int64_t w = w0 + u * stride;
+            word[u] = 0;
+            c1p[u] = 0.0f;
+            if (w < p.nwords) {
+                word[u] = ld_stream_u32(p.packed + 4 * w);
+                int64_t b = w >> 3;
+                c1p[u] = __fmaf_rn(e4m3_to_float(p.code2[b]), p.c2[b / QLORA_GROUP], mu);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; u++) {
+            int64_t w = w0 + u * stride;
+            if (w >= p.nwords) continue;
+            uint32_t o[4];
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                float lo = __fmul_rn(lut[(word[u] >> (8 * i)) & 15u], c1p[u]);
+                float hi = __fmul_rn(lut[(word[u] >> (8 * i + 4)) & 15u], c1p[u]);
+                o[i] = pack_bf16x2(lo, hi);
+            }
+            *reinterpret_cast<uint4 *>(p.out + 8 * w) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+    }
+}
+
+// ---- host helpers ----------------------------------------------------------------
+
+// Binary32 nearest below-or-equal to a double.
+float round_down_f32(double d)
+{
+    float f = (float)d;
+    if ((double)f > d) f = nextafterf(f, -INFINITY);
+    return f;
+}
+
+uint32_t host_sortable_key(float f)
+{
+    uint32_t b;
+    memcpy(&b, &f, 4);
+    uint32_t s = (uint32_t)((int32_t)b >> 31);
+    return b ^ (s | 0x80000000u);
+}
+
+// Midpoint keys for the code lookup; rejects tables the lookup cannot serve.
+qlora_status midpoint_keys(const float q[16], uint32_t out[15])
+{
+    for (int j = 0; j < 15; j++) {
+        if (!(q[j] < q[j + 1])) return QLORA_ERR_INVALID_ARG;
+        double sum = (double)q[j] + (double)q[j + 1];
+        if (sum - (double)q[j + 1] != (double)q[j]) return QLORA_ERR_UNSUPPORTED;  // inexact sum
+        float m = round_down_f32(sum / 2.0);
+        if (m == 0.0f) m = 0.0f;  // +0, never -0
+        out[j] = host_sortable_key(m);
+        if (j > 0 && (out[j] >> 20) == (out[j - 1] >> 20)) return QLORA_ERR_UNSUPPORTED;
+    }
+    return QLORA_OK;
+}
+
+int grid_for(int64_t work_items, int items_per_cta, int max_ctas)
+{
+    int64_t g = (work_items + items_per_cta - 1) / items_per_cta;
+    if (g > max_ctas) g = max_ctas;
+    return g < 1 ? 1 : (int)g;
+}
+
+}  // namespace
+
+// Workspace layout for the quantizer: [acc 256 u64][ticket u32 + pad to 16][c1 floats]
+static constexpr size_t kAccBytes = 256 * sizeof(unsigned long long) + 16;
+
+}  // namespace qlora
+
+using namespace qlora;
+
+extern "C" size_t qlora_quantize_workspace_bytes(int64_t rows, int64_t cols)
+{
+    if (rows <= 0 || cols <= 0) return kAccBytes;
+    int64_t nblocks = rows * cols / QLORA_BLOCK;
+    return kAccBytes + (size_t)((nblocks * 4 + 15) / 16 * 16);
+}
+
+extern "C" qlora_status qlora_quantize_nf4_dq(const void *W, qlora_dtype w_dtype, const qlora_nf4_weight *out,
+                                              void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!W || !out || !workspace) return QLORA_ERR_INVALID_ARG;
+    if (w_dtype != QLORA_BF16 && w_dtype != QLORA_FP32) return QLORA_ERR_INVALID_ARG;
+    QLORA_TRY(check_weight(out));
+    if (!aligned16(W) || !aligned16(workspace)) return QLORA_ERR_ALIGNMENT;
+    if (workspace_bytes < qlora_quantize_workspace_bytes(out->rows, out->cols)) return QLORA_ERR_WORKSPACE;
+    uint32_t mkey[15];
+    QLORA_TRY(midpoint_keys(out->codebook, mkey));
+    DeviceInfo dev;
+    QLORA_TRY(device_info(&dev));
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t numel = out->rows * out->cols;
+    const int64_t nblocks = numel / QLORA_BLOCK;
+    char *ws = static_cast<char *>(workspace);
+    QLORA_CUDA_TRY(cudaMemsetAsync(ws, 0, kAccBytes, s));
+
+    QuantParams qp;
+    qp.W = W;
+    qp.packed = out->packed;
+    qp.acc = reinterpret_cast<unsigned long long *>(ws);
+    qp.ticket = reinterpret_cast<unsigned int *>(ws + 256 * sizeof(unsigned long long));
+    qp.c1 = reinterpret_cast<float *>(ws + kAccBytes);
+    qp.mean_out = out->mean;
+    qp.nwords = numel / 8;
+    qp.nblocks = nblocks;
+    memcpy(qp.mkey, mkey, sizeof(mkey));
+    int grid = grid_for(qp.nwords, kThreads * kUnroll, dev.sms * 4);
+    if (w_dtype == QLORA_FP32)
+        quantize_blocks_kernel<true><<<grid, kThreads, 0, s>>>(qp);
+    else
+        quantize_blocks_kernel<false><<<grid, kThreads, 0, s>>>(qp);
+    QLORA_TRY(launch_status());
+
+    DqParams dp;
+    dp.c1 = qp.c1;
+    dp.mean = out->mean;
+    dp.code2 = out->code2;
+    dp.c2 = out->c2;
+    dp.nblocks = nblocks;
+    dp.ngroups = (nblocks + QLORA_GROUP - 1) / QLORA_GROUP;
+    dq_encode_kernel<<<grid_for(dp.ngroups, kThreads / 32, dev.sms * 8), kThreads, 0, s>>>(dp);
+    return launch_status();
+}
+
+extern "C" qlora_status qlora_dequantize_nf4_dq(const qlora_nf4_weight *w, void *out_bf16, void *stream)
+{
+    if (!w || !out_bf16) return QLORA_ERR_INVALID_ARG;
+    QLORA_TRY(check_weight(w));
+    if (!aligned16(out_bf16)) return QLORA_ERR_ALIGNMENT;
+    DeviceInfo dev;
+    QLORA_TRY(device_info(&dev));
+    DeqParams p;
+    p.packed = w->packed;
+    p.code2 = w->code2;
+    p.c2 = w->c2;
+    p.mean = w->mean;
+    p.out = static_cast<__nv_bfloat16 *>(out_bf16);
+    p.nwords = w->rows * w->cols / 8;
+    memcpy(p.q, w->codebook, sizeof(p.q));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    dequantize_kernel<<<grid_for(p.nwords, kThreads * kUnroll, dev.sms * 8), kThreads, 0, s>>>(p);
+    return launch_status();
+}

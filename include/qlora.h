@@ -1,0 +1,221 @@
+/*
+ * qlora.h -- C ABI of the B200 (sm_100a) QLoRA hot path.
+ *
+ * What is computed (all citations are to "QLoRA: Efficient Finetuning of
+ * Quantized LLMs", inquiringlines.com/papers/2305.14314, unless noted):
+ *   - a frozen weight W [N, K] is stored as 4-bit NormalFloat codes with one
+ *     absmax constant per block of 64 ("Method", paragraphs "4-bit NormalFloat
+ *     Quantization" and "Double Quantization"), and the block constants are
+ *     quantized a second time (double quantization) to 8-bit floats in groups
+ *     of 256 blocks after subtracting their mean;
+ *   - whenever the weight is used it is dequantized to BFloat16 and multiplied
+ *     in 16-bit arithmetic ("Method", storage vs. computation data type);
+ *   - the QLoRA linear layer x_out = (W_q + B A) x_in (mbrenndoerfer.com QLoRA
+ *     essay, "Low-Rank Adaptation (LoRA)"), in row-vector form
+ *         Y = X W'^T + s (X A^T) B^T,      W' = dequant(W_q),
+ *     with its backward pass dX, dA, dB; the quantized weight is frozen, so
+ *     there is no dW (abstract: gradients are backpropagated "through a
+ *     frozen, 4-bit quantized pretrained language model into Low Rank
+ *     Adapters").
+ *
+ * Conventions common to every entry point
+ *   - Pointers named "device" must point to memory of the current CUDA device;
+ *     the caller allocates and frees every buffer.  The library never
+ *     allocates device memory and never frees what it is given.
+ *   - Every device pointer must be 16-byte aligned (tensor-memory-access
+ *     copies require it); QLORA_ERR_ALIGNMENT otherwise.
+ *   - All work is enqueued on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and is asynchronous.  Argument validation is synchronous
+ *     and happens before anything is enqueued: a non-OK status means nothing
+ *     was launched.  No entry point synchronizes the stream.
+ *   - Inputs must be finite numbers; results for NaN or infinite inputs are
+ *     unspecified.
+ *   - Outputs must not alias inputs or each other.
+ *   - Matrices are row-major and dense (leading dimension = column count).
+ *   - Kernel-side failures (a bounded wait that timed out) are recorded in a
+ *     device error word, read back by qlora_check_device_error().
+ *   - The library requires a compute capability 10.0 device (B200);
+ *     QLORA_ERR_UNSUPPORTED otherwise.  There is no CPU fallback.
+ */
+#ifndef QLORA_H
+#define QLORA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QLORA_API __attribute__((visibility("default")))
+#else
+#define QLORA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Blocksize of the first quantization level: 64 consecutive elements of one
+ * row ("Method", "Double Quantization": "a blocksize of 64 for W"). */
+#define QLORA_BLOCK 64
+/* Number of first-level constants per second-level (double-quantization)
+ * group: 256 consecutive blocks in row-major block order. */
+#define QLORA_GROUP 256
+
+typedef enum {
+    QLORA_OK = 0,
+    QLORA_ERR_INVALID_ARG = 1, /* null pointer, unknown enum, negative size   */
+    QLORA_ERR_SHAPE = 2,       /* a size violates the documented constraints  */
+    QLORA_ERR_ALIGNMENT = 3,   /* a device pointer is not 16-byte aligned     */
+    QLORA_ERR_WORKSPACE = 4,   /* workspace missing or smaller than required  */
+    QLORA_ERR_CUDA = 5,        /* a CUDA runtime/driver call failed           */
+    QLORA_ERR_UNSUPPORTED = 6, /* not a compute capability 10.x device        */
+    QLORA_ERR_TIMEOUT = 7      /* a kernel's bounded wait gave up (device)    */
+} qlora_status;
+
+typedef enum { QLORA_BF16 = 0, QLORA_FP32 = 1 } qlora_dtype;
+
+/*
+ * A quantized weight W [rows, cols] (rows = N = out_features, cols = K =
+ * in_features).  Plain data: the struct holds caller-owned device pointers
+ * and a host copy of the 16-entry codebook.
+ *   packed  device, rows*cols/2 bytes.  Element (n, k) has flat index
+ *           i = n*cols + k; its 4-bit code sits in byte i/2, in bits 0-3 when
+ *           i is even and bits 4-7 when i is odd.
+ *   code2   device, nblocks = rows*cols/64 bytes: E4M3 (OCP "e4m3fn") code of
+ *           block b's constant after subtracting the mean and dividing by
+ *           the group scale.  Block b covers flat indices [64b, 64b+64).
+ *   c2      device, ngroups = ceil(nblocks/256) floats: group scale of blocks
+ *           [256g, 256g+256).
+ *   mean    device, 1 float: mean of all first-level constants of W.
+ *   codebook  host values q[0..15], strictly ascending, containing exactly
+ *           one 0; the NF4 table from qlora_build_nf4_codebook() or any other
+ *           4-bit table with the same properties.
+ */
+typedef struct {
+    int64_t rows;
+    int64_t cols;
+    uint8_t *packed;
+    uint8_t *code2;
+    float *c2;
+    float *mean;
+    float codebook[16];
+} qlora_nf4_weight;
+
+/*
+ * qlora_build_nf4_codebook -- the NF4 data type ("Method", "4-bit NormalFloat
+ * Quantization", steps (1)-(2) and the asymmetric construction: 2^(k-1)
+ * quantiles of N(0,1) for the negative part and 2^(k-1)+1 for the positive
+ * part, unified with one of the two zeros removed, normalized into [-1, 1]).
+ * The page omits the probabilities; each side uses equally spaced
+ * probabilities from 1 - delta down to 1/2, delta being the tail probability
+ * of the outermost value.  Host-only, no CUDA call.
+ *   delta          tail probability in (0, 0.5); delta <= 0 selects the
+ *                  default (1/32 + 1/30)/2.
+ *   codebook_out   host, 16 floats, written ascending: -1 first, +1 last,
+ *                  exactly one 0 at index 7.
+ * Errors: QLORA_ERR_INVALID_ARG for a null pointer or delta >= 0.5.
+ */
+QLORA_API qlora_status qlora_build_nf4_codebook(double delta, float codebook_out[16]);
+
+/*
+ * Workspace in bytes that qlora_quantize_nf4_dq needs for a rows x cols
+ * weight (first-level constants plus a few reduction slots).
+ */
+QLORA_API size_t qlora_quantize_workspace_bytes(int64_t rows, int64_t cols);
+
+/*
+ * qlora_quantize_nf4_dq -- NF4 quantization with double quantization.
+ * ("Method": "4-bit NormalFloat Quantization" step (3) and "Double
+ * Quantization".)  Per block of 64: c1 = max|x|; if c1 < 2^-126 every code is
+ * the codebook's zero, else n = RN32(x * RN32(1/c1)) and the code is the
+ * index of the codebook value nearest to n (ties: lower index).  Then
+ * mean = binary32 nearest to the exact mean of all c1 (ties to even); per
+ * group: d = RN32(c1 - mean), c2 = RN32(max|d| / 448), code2 = E4M3 with
+ * round-to-nearest-even and saturation of RN32(d / c2) (all zero if c2 = 0).
+ *   W          device, rows*cols elements of w_dtype (QLORA_BF16 or
+ *              QLORA_FP32), row-major.
+ *   out        host struct: rows, cols, the four device buffers (written) and
+ *              the codebook (read).  rows >= 1, cols % 64 == 0.
+ *   workspace  device, at least qlora_quantize_workspace_bytes(rows, cols)
+ *              bytes; contents on entry do not matter; clobbered.
+ * Errors: INVALID_ARG, SHAPE, ALIGNMENT, WORKSPACE, CUDA, UNSUPPORTED.
+ * Deterministic: the same input gives the same bytes on every call.
+ */
+QLORA_API qlora_status qlora_quantize_nf4_dq(const void *W, qlora_dtype w_dtype, const qlora_nf4_weight *out,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * qlora_dequantize_nf4_dq -- expand a quantized weight to BFloat16 ("Method":
+ * the tensor is dequantized to BFloat16 whenever it is used).  Per block:
+ * c1' = fmaf(E4M3value(code2), c2, mean) (one rounding); per element
+ * w = bf16_RNE(RN32(q[code] * c1')).
+ *   w        host struct describing the quantized weight (read only).
+ *   out_bf16 device, rows*cols bf16, row-major.
+ * Errors: INVALID_ARG, SHAPE, ALIGNMENT, CUDA, UNSUPPORTED.
+ */
+QLORA_API qlora_status qlora_dequantize_nf4_dq(const qlora_nf4_weight *w, void *out_bf16, void *stream);
+
+/*
+ * Workspace in bytes for qlora_linear_fwd / qlora_linear_bwd at these sizes
+ * (M tokens, weight N x K, rank r).  One workspace sized by this function
+ * serves both directions.
+ */
+QLORA_API size_t qlora_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t r);
+
+/*
+ * qlora_linear_fwd -- Y = X W'^T + H_b B^T with H = s X A^T (float32 sums),
+ * H_b = bf16(H); W' is the dequantized weight of `w`, expanded tile by tile
+ * on chip and never written to memory.
+ *   w       quantized weight, N = w->rows, K = w->cols; N % 8 == 0.
+ *   X       device bf16 [M, K].  M >= 0 (M == 0: nothing is done).
+ *   A       device bf16 [r, K];  B  device bf16 [N, r].
+ *   r       adapter rank, 8 <= r <= 128, r % 8 == 0.
+ *   scale   s (usually lora_alpha / r), any finite value.
+ *   Y       device [M, N] of y_dtype (QLORA_BF16 or QLORA_FP32).
+ *   H_save  device float [M, r] or NULL: receives H = s X A^T for the
+ *           backward pass.
+ *   workspace  device, >= qlora_linear_workspace_bytes(M, N, K, r) bytes.
+ * Errors: INVALID_ARG, SHAPE, ALIGNMENT, WORKSPACE, CUDA, UNSUPPORTED.
+ */
+QLORA_API qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const void *X, int64_t M, const void *A,
+                              const void *B, int32_t r, float scale, void *Y, qlora_dtype y_dtype,
+                              float *H_save, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * qlora_linear_bwd -- gradients of the layer above for dY = dL/dY:
+ *     G  = s dY B                      (float32 sums)
+ *     dX = dY W' + bf16(G) A           (W' expanded on chip, transposed use)
+ *     dA = G^T X                       (= s (dY B)^T X)
+ *     dB = dY^T H                      (= s dY^T (X A^T))
+ * dA and dB are computed from G and H carried at about 16 significant bits
+ * (each split into two bf16 terms), so their error stays at the level of
+ * float32 accumulation.  No gradient is formed for the frozen weight.
+ *   w, X, A, B, r, scale, M   as for qlora_linear_fwd.
+ *   dY       device bf16 [M, N].
+ *   H_saved  device float [M, r] from qlora_linear_fwd, or NULL to recompute.
+ *   dX       device [M, K] of dx_dtype, or NULL to skip the input gradient.
+ *   dA       device float [r, K], overwritten.
+ *   dB       device float [N, r], overwritten.
+ *   workspace  device, >= qlora_linear_workspace_bytes(M, N, K, r) bytes.
+ * Errors: INVALID_ARG, SHAPE, ALIGNMENT, WORKSPACE, CUDA, UNSUPPORTED.
+ */
+QLORA_API qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *X, const void *dY, int64_t M,
+                              const void *A, const void *B, int32_t r, float scale,
+                              const float *H_saved, void *dX, qlora_dtype dx_dtype, float *dA,
+                              float *dB, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+QLORA_API const char *qlora_status_string(qlora_status status);
+
+/*
+ * Synchronizes `stream`, then reads and clears the device error word of the
+ * current device.  Returns QLORA_OK if no kernel recorded a failure since
+ * the last call, QLORA_ERR_TIMEOUT if a bounded wait gave up, QLORA_ERR_CUDA
+ * if the synchronization itself failed.
+ */
+QLORA_API qlora_status qlora_check_device_error(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_H */

@@ -1,0 +1,100 @@
+"""The C-ABI library loads without a GPU, exports every symbol the header
+declares, and its host-only logic (codebook, status strings, workspace sizes,
+argument validation before any CUDA call) behaves as documented."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import codebook as ocb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+LIB = os.path.join(ROOT, "bit_nf4_quantized_16_b200", "libqlora_b200.so")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(LIB):
+        import importlib.util
+        spec = importlib.util.spec_from_file_location("qbuild", os.path.join(ROOT, "bit_nf4_quantized_16_b200", "build.py"))
+        mod = importlib.util.module_from_spec(spec)
+        spec.loader.exec_module(mod)
+        mod.build()
+    return ctypes.CDLL(LIB)
+
+
+def declared_symbols():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"QLORA_API\s+[\w\s\*]+?\b(qlora_\w+)\s*\(", txt)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_symbols()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_binding_lists_the_same_symbols():
+    src = open(os.path.join(ROOT, "bit_nf4_quantized_16_b200", "__init__.py")).read()
+    exports = re.search(r"EXPORTS = \((.*?)\)", src, re.S).group(1)
+    assert sorted(re.findall(r'"(qlora_\w+)"', exports)) == declared_symbols()
+
+
+def test_nf4_codebook_matches_oracle_bit_for_bit(lib):
+    out = (ctypes.c_float * 16)()
+    lib.qlora_build_nf4_codebook.argtypes = [ctypes.c_double, ctypes.c_void_p]
+    assert lib.qlora_build_nf4_codebook(0.0, ctypes.cast(out, ctypes.c_void_p)) == 0
+    got = np.array(list(out), np.float32)
+    assert np.array_equal(got.view(np.uint32), ocb.nf4_codebook().view(np.uint32))
+    for delta in (0.01, 0.05, 0.1):
+        assert lib.qlora_build_nf4_codebook(delta, ctypes.cast(out, ctypes.c_void_p)) == 0
+        ref = ocb.nfk_codebook_f64(4, delta).astype(np.float32)
+        assert np.array_equal(np.array(list(out), np.float32).view(np.uint32), ref.view(np.uint32))
+    assert lib.qlora_build_nf4_codebook(0.5, ctypes.cast(out, ctypes.c_void_p)) == 1
+    assert lib.qlora_build_nf4_codebook(0.0, None) == 1
+
+
+def test_status_strings(lib):
+    lib.qlora_status_string.restype = ctypes.c_char_p
+    assert lib.qlora_status_string(0) == b"QLORA_OK"
+    assert lib.qlora_status_string(7) == b"QLORA_ERR_TIMEOUT"
+    assert lib.qlora_status_string(99) == b"QLORA_ERR_UNKNOWN"
+
+
+def test_quantize_workspace_size(lib):
+    lib.qlora_quantize_workspace_bytes.restype = ctypes.c_size_t
+    lib.qlora_quantize_workspace_bytes.argtypes = [ctypes.c_int64, ctypes.c_int64]
+    n = lib.qlora_quantize_workspace_bytes(4096, 4096)
+    assert n >= 4 * 4096 * 4096 // 64 and n % 16 == 0
+
+
+class Weight(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("packed", ctypes.c_void_p),
+                ("code2", ctypes.c_void_p), ("c2", ctypes.c_void_p), ("mean", ctypes.c_void_p),
+                ("codebook", ctypes.c_float * 16)]
+
+
+def test_validation_happens_before_any_cuda_call(lib):
+    """Bad arguments are rejected on the host; these calls never reach CUDA."""
+    q = ocb.nf4_codebook()
+    fake = 0x10000   # aligned, never dereferenced
+    w = Weight(64, 128, fake, fake, fake, fake, (ctypes.c_float * 16)(*q))
+    f = lib.qlora_quantize_nf4_dq
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(Weight), ctypes.c_void_p, ctypes.c_size_t,
+                  ctypes.c_void_p]
+    assert f(None, 0, ctypes.byref(w), fake, 1 << 20, None) == 1            # null W
+    assert f(fake, 7, ctypes.byref(w), fake, 1 << 20, None) == 1            # bad dtype
+    bad = Weight(64, 100, fake, fake, fake, fake, (ctypes.c_float * 16)(*q))
+    assert f(fake, 0, ctypes.byref(bad), fake, 1 << 20, None) == 2          # cols % 64
+    assert f(fake + 4, 0, ctypes.byref(w), fake, 1 << 20, None) == 3        # misaligned W
+    assert f(fake, 0, ctypes.byref(w), fake, 16, None) == 4                 # workspace too small
+    unsorted = Weight(64, 128, fake, fake, fake, fake, (ctypes.c_float * 16)(*q[::-1]))
+    assert f(fake, 0, ctypes.byref(unsorted), fake, 1 << 20, None) == 1     # codebook not ascending

@@ -1,0 +1,138 @@
+"""GPU parity of the NF4 + double-quantization codec against the oracle.
+
+"QLoRA: Efficient Finetuning of Quantized LLMs", section "Method": NF4
+quantization with blocksize 64 (step (3) of "4-bit NormalFloat
+Quantization"), double quantization of the block constants, dequantization to
+BFloat16.  Packed codes, E4M3 codes, scales, mean and the dequantized bf16
+weight must match the oracle bit for bit.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import synthetic
+from oracle import codebook as ocb
+from oracle import codec as occ
+
+pytestmark = pytest.mark.gpu
+
+Q = ocb.nf4_codebook()
+
+
+@pytest.fixture(scope="module")
+def q():
+    import bit_nf4_quantized_16_b200 as q
+    assert torch.cuda.is_available()
+    return q
+
+
+def gpu_quantize(q, W: torch.Tensor):
+    rows, cols = W.shape
+    w = q.NF4Weight(rows, cols, device="cuda")
+    ws = torch.empty(q.qlora_quantize_workspace_bytes(rows, cols), dtype=torch.uint8, device="cuda")
+    q.qlora_quantize_nf4_dq(W.cuda().contiguous(), w, ws)
+    torch.cuda.synchronize()
+    return w
+
+
+def gpu_dequantize(q, w):
+    out = torch.empty(w.rows, w.cols, dtype=torch.bfloat16, device="cuda")
+    q.qlora_dequantize_nf4_dq(w, out)
+    torch.cuda.synchronize()
+    return out.view(torch.int16).cpu().numpy().view(np.uint16).ravel()
+
+
+def check_parity(q, W: torch.Tensor):
+    w = gpu_quantize(q, W)
+    ref = occ.quantize(W.float().numpy(), Q)
+    assert np.array_equal(w.packed.cpu().numpy(), ref["packed"]), "packed codes"
+    assert np.array_equal(w.code2.cpu().numpy(), ref["e"]), "E4M3 codes"
+    assert np.array_equal(w.c2.cpu().numpy().view(np.uint32), ref["c2"].view(np.uint32)), "group scales"
+    assert w.mean[0].item() == float(ref["mean"]), "mean"
+    got = gpu_dequantize(q, w)
+    want = occ.dequantize(ref["packed"], ref["e"], ref["c2"], ref["mean"], Q)
+    assert np.array_equal(got, want), "dequantized bf16"
+    return w, ref
+
+
+def test_codebook_in_weight_descriptor_is_the_oracle_table(q):
+    assert np.array_equal(np.array(q.qlora_build_nf4_codebook(), np.float32).view(np.uint32), Q.view(np.uint32))
+
+
+def test_tiny_config_fp32(q):
+    case = synthetic.tiny_linear(seed=0)
+    check_parity(q, case["W"])
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 64), (3, 192), (100, 192), (257, 320), (512, 1024)])
+def test_ragged_shapes_bf16(q, rows, cols):
+    check_parity(q, synthetic.normal((rows, cols), 0.02, seed=rows + cols, dtype=torch.bfloat16))
+
+
+def test_llama_7b_shapes_bf16(q):
+    for i, (rows, cols) in enumerate([(4096, 4096), (11008, 4096), (4096, 11008)]):
+        check_parity(q, synthetic.normal((rows, cols), 0.02, seed=40 + i, dtype=torch.bfloat16))
+
+
+def test_edge_blocks(q):
+    """Zero blocks, a subnormal block, values exactly on the round-down
+    midpoints (ties go to the lower code), and +-absmax."""
+    W = synthetic.normal((6, 256), 0.02, seed=7)
+    W[0, :64] = 0.0
+    W[1, :64] = -0.0
+    W[1, 64:128] = 0.0
+    W[1, 70] = 1e-40
+    mids = []
+    for j in range(15):
+        m = np.float32((float(Q[j]) + float(Q[j + 1])) / 2)
+        mids += [m, np.nextafter(m, np.float32(-2)), np.nextafter(m, np.float32(2))]
+    row = np.zeros(64, np.float32)
+    row[0] = 1.0
+    row[1:1 + 45] = mids
+    W[2, :64] = torch.from_numpy(row)
+    W[3, :64] = -torch.from_numpy(row)
+    check_parity(q, W)
+
+
+def test_constant_tensor_has_zero_second_level(q):
+    W = torch.full((8, 128), 0.03125, dtype=torch.bfloat16)
+    w, ref = check_parity(q, W)
+    assert np.all(ref["c2"] == 0) and np.all(ref["e"] == 0)
+
+
+def test_exact_round_trip(q):
+    rng = np.random.default_rng(9)
+    a = np.float32(0.046875)
+    codes = rng.integers(0, 16, (64, 256)).astype(np.uint8)
+    codes[:, ::64] = rng.choice([0, 15], (64, 4))
+    W = occ.bf16_bits_to_f32(occ.bf16_rne((Q[codes] * a).astype(np.float32)))
+    w = gpu_quantize(q, torch.from_numpy(W).to(torch.bfloat16))
+    got = gpu_dequantize(q, w)
+    assert np.array_equal(got, torch.from_numpy(W).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16).ravel())
+
+
+def test_deterministic_bytes(q):
+    W = synthetic.normal((1024, 4096), 0.02, seed=3, dtype=torch.bfloat16)
+    a, b = gpu_quantize(q, W), gpu_quantize(q, W)
+    for name in ("packed", "code2", "c2", "mean"):
+        assert torch.equal(getattr(a, name), getattr(b, name)), name
+
+
+def test_dequantize_of_oracle_encoded_weight(q):
+    """The dequantizer alone, fed the oracle's quantized buffers."""
+    W = synthetic.normal((300, 256), 0.02, seed=11).numpy()
+    ref = occ.quantize(W, Q)
+    w = q.NF4Weight(300, 256, device="cuda")
+    w.packed.copy_(torch.from_numpy(ref["packed"]))
+    w.code2.copy_(torch.from_numpy(ref["e"]))
+    w.c2.copy_(torch.from_numpy(ref["c2"]))
+    w.mean[0] = float(ref["mean"])
+    got = gpu_dequantize(q, w)
+    assert np.array_equal(got, occ.dequantize(ref["packed"], ref["e"], ref["c2"], ref["mean"], Q))
+
+
+def test_bits_per_parameter_from_buffer_sizes(q):
+    w = q.NF4Weight(4096, 4096, device="cuda")
+    bits = 8 * w.nbytes / (4096 * 4096)
+    assert bits == pytest.approx(occ.storage_bits_per_param(4096 * 4096), rel=1e-12)
