@@ -112,7 +112,7 @@ class NF4Weight:
         self.packed = torch.empty(rows * cols // 2, dtype=torch.uint8, device=device)
         self.code2 = torch.empty(nblocks, dtype=torch.uint8, device=device)
         self.c2 = torch.empty(ngroups, dtype=torch.float32, device=device)
-        self.mean = torch.empty(4, dtype=torch.float32, device=device)   # 16-byte slot
+        self.mean = torch.zeros(4, dtype=torch.float32, device=device)   # 16-byte slot, [0] used
         self.codebook = list(codebook) if codebook is not None else qlora_build_nf4_codebook()
         self.desc = qlora_nf4_weight(rows, cols, self.packed.data_ptr(), self.code2.data_ptr(),
                                      self.c2.data_ptr(), self.mean.data_ptr(),

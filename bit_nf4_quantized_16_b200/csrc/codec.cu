@@ -157,6 +157,7 @@ __global__ void __launch_bounds__(kThreads) quantize_blocks_kernel(QuantParams p
                 }
             }
         }
+        float c1v[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; u++) {
             float m = 0.0f;
@@ -166,22 +167,43 @@ __global__ void __launch_bounds__(kThreads) quantize_blocks_kernel(QuantParams p
             m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
             m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
             m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+            c1v[u] = m;
             // zero block (absmax below the smallest normal): r = 0 sends every
             // element to n = +-0, whose code is the codebook's zero
             const float r = m < 1.17549435e-38f ? 0.0f : __frcp_rn(m);
             uint32_t word = 0;
 #pragma unroll
             for (int i = 0; i < 8; i++) word |= code_of(lut, x[u][i], r) << (4 * i);
-            if (act[u]) {
-                int64_t w = base + lane + u * stride;
-                reinterpret_cast<uint32_t *>(p.packed)[w] = word;
-                if ((lane & 7) == 0) {
-                    p.c1[w >> 3] = m;
-                    uint32_t bucket, sig;
-                    exact_mean_split(__float_as_uint(m), &bucket, &sig);
-                    atomicAdd(&s_acc[bucket], (unsigned long long)sig);
-                }
+            if (act[u]) reinterpret_cast<uint32_t *>(p.packed)[base + lane + u * stride] = word;
+        }
+        // Gather the warp's 4*kUnroll block constants into lanes 0..4*kUnroll-1
+        // (lane 4u+g takes block g of unrolled step u), store them, and add
+        // them to the exponent buckets with one shared atomic per distinct
+        // exponent instead of one per block.
+        float cv = 0.0f;
+        bool ca = false;
+#pragma unroll
+        for (int u = 0; u < kUnroll; u++) {
+            float t = __shfl_sync(0xffffffffu, c1v[u], (lane & 3) * 8);
+            bool a = __shfl_sync(0xffffffffu, (int)act[u], (lane & 3) * 8) != 0;
+            if ((lane >> 2) == u) {
+                cv = t;
+                ca = a;
             }
+        }
+        if (lane < 4 * kUnroll && ca) p.c1[(base + 8 * (lane & 3) + (lane >> 2) * stride) >> 3] = cv;
+        uint32_t bucket, sig;
+        exact_mean_split(__float_as_uint(cv), &bucket, &sig);
+        bool pending = lane < 4 * kUnroll && ca;
+        for (;;) {
+            unsigned pend = __ballot_sync(0xffffffffu, pending);
+            if (!pend) break;
+            int leader = __ffs(pend) - 1;
+            uint32_t lb = __shfl_sync(0xffffffffu, bucket, leader);
+            bool mine = pending && bucket == lb;
+            uint32_t sum = __reduce_add_sync(0xffffffffu, mine ? sig : 0u);   // < 16 * 2^24
+            if (lane == leader) atomicAdd(&s_acc[lb], (unsigned long long)sum);
+            pending = pending && !mine;
         }
     }
     __syncthreads();

@@ -1,0 +1,221 @@
+"""GPU parity of the QLoRA linear layer (forward and backward) against the
+float64 oracle.
+
+Layer: x_out = (W_q + B A) x_in (mbrenndoerfer.com QLoRA essay, section
+"Low-Rank Adaptation (LoRA)"), with the 4-bit weight dequantized to BFloat16
+and used in a 16-bit matmul ("QLoRA: Efficient Finetuning of Quantized LLMs",
+section "Method"); gradients reach only the adapters (abstract).
+
+Tolerance: relative Frobenius error <= 5e-3 and max abs error <= 2e-2 for
+float32 outputs (fp32 accumulation).  For bf16 outputs the max-abs bound is
+widened by half a bf16 unit in the last place of the reference value, the
+rounding of the output itself.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import synthetic
+from oracle import codebook as ocb
+from oracle import codec as occ
+from oracle import linear as olin
+
+pytestmark = pytest.mark.gpu
+
+Q = ocb.nf4_codebook()
+REL_FRO = 5e-3
+MAX_ABS = 2e-2
+
+
+@pytest.fixture(scope="module")
+def q():
+    import bit_nf4_quantized_16_b200 as q
+    assert torch.cuda.is_available()
+    return q
+
+
+def half_ulp_bf16(ref):
+    a = np.abs(np.asarray(ref, np.float64))
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -126)))
+    return 2.0 ** (e - 8)
+
+
+def assert_close(got, ref, bf16_out=False, what=""):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert got.shape == ref.shape, what
+    assert np.all(np.isfinite(got)), what
+    rel = olin.rel_frobenius(got, ref)
+    assert rel <= REL_FRO, f"{what}: rel Frobenius {rel:.3e}"
+    bound = MAX_ABS + (half_ulp_bf16(ref) if bf16_out else 0.0)
+    err = np.abs(got - ref)
+    worst = np.unravel_index(np.argmax(err - bound), err.shape) if err.size else None
+    assert np.all(err <= bound), f"{what}: max abs {err.max():.3e} at {worst}"
+
+
+def oracle_weight(W):
+    ref = occ.quantize(W.float().numpy(), Q)
+    Wd = occ.dequantize(ref["packed"], ref["e"], ref["c2"], ref["mean"], Q)
+    return occ.bf16_bits_to_f32(Wd).reshape(W.shape).astype(np.float64)
+
+
+class Runner:
+    """Quantizes W on the GPU and runs the layer through the C ABI."""
+
+    def __init__(self, q, case):
+        self.q, self.c = q, case
+        N, K = case["W"].shape
+        self.w = q.NF4Weight(N, K)
+        ws = torch.empty(q.qlora_quantize_workspace_bytes(N, K), dtype=torch.uint8, device="cuda")
+        q.qlora_quantize_nf4_dq(case["W"].cuda(), self.w, ws)
+        self.X = case["X"].cuda()
+        self.A = case["A"].cuda()
+        self.B = case["B"].cuda()
+        self.dY = case["dY"].cuda()
+        self.M = case["X"].shape[0]
+        self.ws = torch.empty(q.qlora_linear_workspace_bytes(self.M, N, K, case["r"]), dtype=torch.uint8,
+                              device="cuda")
+
+    def fwd(self, ydt=torch.float32, save_h=False):
+        N = self.w.rows
+        Y = torch.empty(self.M, N, dtype=ydt, device="cuda")
+        H = torch.empty(self.M, self.c["r"], dtype=torch.float32, device="cuda") if save_h else None
+        self.q.qlora_linear_fwd(self.w, self.X, self.M, self.A, self.B, self.c["r"], self.c["scale"], Y, H, self.ws)
+        self.q.qlora_check_device_error()
+        return Y, H
+
+    def bwd(self, dxdt=torch.float32, H=None, want_dx=True):
+        N, K, r = self.w.rows, self.w.cols, self.c["r"]
+        dX = torch.empty(self.M, K, dtype=dxdt, device="cuda") if want_dx else None
+        dA = torch.empty(r, K, dtype=torch.float32, device="cuda")
+        dB = torch.empty(N, r, dtype=torch.float32, device="cuda")
+        self.q.qlora_linear_bwd(self.w, self.X, self.dY, self.M, self.A, self.B, r, self.c["scale"], H, dX, dA, dB,
+                                self.ws)
+        self.q.qlora_check_device_error()
+        return dX, dA, dB
+
+
+def np64(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def full_check(q, case, ydt=torch.float32):
+    run = Runner(q, case)
+    Wd = oracle_weight(case["W"])
+    X, A, B, dY = (np64(case[k]) for k in ("X", "A", "B", "dY"))
+    s = case["scale"]
+    Y, _ = run.fwd(ydt)
+    assert_close(np64(Y), olin.forward(X, Wd, A, B, s), bf16_out=ydt == torch.bfloat16, what="Y")
+    dX, dA, dB = run.bwd(ydt)
+    rdX, rdA, rdB = olin.backward(X, Wd, A, B, s, dY)
+    assert_close(np64(dX), rdX, bf16_out=ydt == torch.bfloat16, what="dX")
+    assert_close(np64(dA), rdA, what="dA")
+    assert_close(np64(dB), rdB, what="dB")
+    return run
+
+
+def test_tiny_config(q):
+    full_check(q, synthetic.tiny_linear(seed=0))
+
+
+def test_tiny_config_bf16_outputs(q):
+    full_check(q, synthetic.tiny_linear(seed=0), ydt=torch.bfloat16)
+
+
+@pytest.mark.parametrize("M,N,K,r", [
+    (300, 320, 448, 16),     # ragged tails in every dimension, several tiles
+    (129, 512, 256, 64),     # one token past a tile
+    (64, 264, 576, 8),       # N not a multiple of 64
+    (256, 256, 1024, 128),   # largest rank
+    (1, 512, 512, 64),       # a single token
+])
+def test_ragged_shapes(q, M, N, K, r):
+    full_check(q, synthetic.linear_case(M, N, K, r, alpha=16.0, seed=M + N + K + r))
+
+
+def test_saved_h_equals_recomputed_h(q):
+    case = synthetic.linear_case(200, 384, 512, 64, alpha=16.0, seed=5)
+    run = Runner(q, case)
+    _, H = run.fwd(save_h=True)
+    X, A = np64(case["X"]), np64(case["A"])
+    np.testing.assert_allclose(np64(H), case["scale"] * X @ A.T, rtol=1e-5, atol=1e-5)
+    a = run.bwd(H=None)
+    b = run.bwd(H=H)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_backward_without_input_gradient(q):
+    case = synthetic.linear_case(128, 256, 256, 16, alpha=32.0, seed=6)
+    run = Runner(q, case)
+    dX0, dA0, dB0 = run.bwd()
+    dX, dA, dB = run.bwd(want_dx=False)
+    assert dX is None and torch.equal(dA, dA0) and torch.equal(dB, dB0)
+
+
+def test_zero_adapter_and_zero_scale(q):
+    case = synthetic.linear_case(130, 256, 320, 16, alpha=16.0, seed=8)
+    case["B"] = torch.zeros_like(case["B"])
+    run = Runner(q, case)
+    Wd = oracle_weight(case["W"])
+    Y, _ = run.fwd()
+    assert_close(np64(Y), np64(case["X"]) @ Wd.T, what="Y with B = 0")
+    dX, dA, dB = run.bwd()
+    assert torch.count_nonzero(dA).item() == 0, "G = 0 gives dA = 0 exactly"
+    case = synthetic.linear_case(130, 256, 320, 16, alpha=0.0, seed=9)
+    run = Runner(q, case)
+    dX, dA, dB = run.bwd()
+    assert torch.count_nonzero(dA).item() == 0 and torch.count_nonzero(dB).item() == 0
+
+
+def test_zero_tokens(q):
+    case = synthetic.linear_case(4, 128, 128, 8, alpha=16.0, seed=10)
+    run = Runner(q, case)
+    run.M = 0
+    dX, dA, dB = run.bwd(want_dx=False)
+    assert torch.count_nonzero(dA).item() == 0 and torch.count_nonzero(dB).item() == 0
+
+
+def test_deterministic(q):
+    case = synthetic.linear_case(512, 512, 1024, 64, alpha=16.0, seed=12)
+    run = Runner(q, case)
+    y1, _ = run.fwd()
+    y2, _ = run.fwd()
+    assert torch.equal(y1, y2)
+    g1, g2 = run.bwd(), run.bwd()
+    for a, b in zip(g1, g2):
+        assert torch.equal(a, b)
+
+
+def test_llama7b_shapes_sampled(q):
+    """7B-shaped linears at 4096 tokens: Y and dX on sampled rows, dA and dB in
+    full (they contract over every token)."""
+    rng = np.random.default_rng(0)
+    for i, (name, N, K) in enumerate([("q", 4096, 4096), ("gate", 11008, 4096), ("down", 4096, 11008)]):
+        case = synthetic.linear_case(4096, N, K, 64, alpha=16.0, seed=100 + i, device="cpu")
+        run = Runner(q, case)
+        Wd = oracle_weight(case["W"])
+        X, A, B, dY = (np64(case[k]) for k in ("X", "A", "B", "dY"))
+        s = case["scale"]
+        rows = np.sort(rng.choice(4096, 48, replace=False))
+        Y, _ = run.fwd()
+        assert_close(np64(Y)[rows], olin.forward_rows(X, Wd, A, B, s, rows), what=f"{name} Y")
+        dX, dA, dB = run.bwd()
+        assert_close(np64(dX)[rows], olin.backward_dx_rows(Wd, A, B, s, dY, rows), what=f"{name} dX")
+        G = dY @ B
+        assert_close(np64(dA), s * (G.T @ X), what=f"{name} dA")
+        assert_close(np64(dB), s * (dY.T @ (X @ A.T)), what=f"{name} dB")
+
+
+def test_argument_errors(q):
+    case = synthetic.linear_case(16, 128, 128, 8, alpha=16.0, seed=13)
+    run = Runner(q, case)
+    Y = torch.empty(16, 128, dtype=torch.float32, device="cuda")
+    small = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(q.QLoraError) as e:
+        q.qlora_linear_fwd(run.w, run.X, 16, run.A, run.B, 8, 2.0, Y, None, small)
+    assert e.value.status == 4
+    with pytest.raises(q.QLoraError) as e:
+        q.qlora_linear_fwd(run.w, run.X, 16, run.A, run.B, 12, 2.0, Y, None, run.ws)
+    assert e.value.status == 2
