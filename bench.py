@@ -1,0 +1,472 @@
+#!/usr/bin/env python
+"""Benchmark of the QLoRA hot path on B200 (one JSON line on rank 0).
+
+Workload (default, "linear7b"): one LLaMA-7B layer's seven QLoRA linears
+(q, k, v, o: 4096x4096; gate, up: 11008x4096; down: 4096x11008), 4096 tokens
+(8 x 512) bf16 ~N(0, 1), r = 64, alpha = 16, NF4 + double-quantized frozen
+weights ~N(0, 0.02) (synthetic, seeded).  One step = forward of the seven
+linears (Y bf16, H saved) then their backward in reverse order (dX bf16, dA,
+dB); with N > 1 processes every rank runs its own 4096 tokens and the adapter
+gradients of the step are summed over ranks with one NCCL all-reduce (weak
+scaling, data parallel).  value = total FLOP / time, FLOP per linear
+4MNK + 6Mr(N+K).
+
+The line also carries "codec": the NF4 + double-quantization round trip
+(quantize then dequantize) over the 224 tensors of LLaMA-7B (6,476,005,376
+bf16 weights ~N(0, 0.02)), algorithmic bytes 2.5159 per weight each way.
+
+--impl reference times the oracle (float64 CPU implementation) on the same
+metric, on a bounded sample per step.
+"""
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "QLoRA linear fwd+bwd TFLOP/s; NF4 (de)quant GB/s; fraction of roofline"
+R, ALPHA, TOKENS = 64, 16.0, 4096
+CODEC_BYTES_PER_WEIGHT = 2 + 0.5 + 1 / 64 + 4 / (64 * 256)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def linear_flops(M, N, K, r):
+    return 4 * M * N * K + 6 * M * r * (N + K)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---- clocks during the timed region -------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.out = None
+
+    def __enter__(self):
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.gpu)], stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        time.sleep(0.2)
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        self.out.flush()
+        rows = []
+        with open(self.out.name) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) == 9:
+                    rows.append(parts)
+        os.unlink(self.out.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---- our arm ---------------------------------------------------------------------------
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import bit_nf4_quantized_16_b200 as q
+    import synthetic
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    peaks, peak_src = load_peaks()
+
+    # ---- set-up (untimed): quantize the seven frozen weights, allocate activations
+    layers = []
+    ws_bytes = 0
+    qws_bytes = max(q.qlora_quantize_workspace_bytes(N, K) for _, N, K in synthetic.LLAMA7B_LINEARS)
+    qws = torch.empty(qws_bytes, dtype=torch.uint8, device=dev)
+    grads = torch.empty(sum(R * K + N * R for _, N, K in synthetic.LLAMA7B_LINEARS), dtype=torch.float32,
+                        device=dev)
+    off = 0
+    for i, (name, N, K) in enumerate(synthetic.LLAMA7B_LINEARS):
+        seed = 1000 * rank + 10 * i
+        W = synthetic.normal((N, K), 0.02, seed, torch.bfloat16, dev)
+        w = q.NF4Weight(N, K, device=dev)
+        q.qlora_quantize_nf4_dq(W, w, qws)
+        del W
+        L = {
+            "name": name, "N": N, "K": K, "w": w,
+            "X": synthetic.normal((TOKENS, K), 1.0, seed + 1, torch.bfloat16, dev),
+            "A": synthetic.normal((R, K), 1.0 / R, seed + 2, torch.bfloat16, dev),
+            "B": synthetic.normal((N, R), 0.01, seed + 3, torch.bfloat16, dev),
+            "dY": synthetic.normal((TOKENS, N), 1.0, seed + 4, torch.bfloat16, dev),
+            "Y": torch.empty(TOKENS, N, dtype=torch.bfloat16, device=dev),
+            "H": torch.empty(TOKENS, R, dtype=torch.float32, device=dev),
+            "dX": torch.empty(TOKENS, K, dtype=torch.bfloat16, device=dev),
+            "dA": grads[off: off + R * K].view(R, K),
+            "dB": grads[off + R * K: off + R * K + N * R].view(N, R),
+        }
+        off += R * K + N * R
+        layers.append(L)
+        ws_bytes = max(ws_bytes, q.qlora_linear_workspace_bytes(TOKENS, N, K, R))
+    del qws
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    scale = ALPHA / R
+    step_flops = sum(linear_flops(TOKENS, L["N"], L["K"], R) for L in layers)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)   # > 126 MB L2
+
+    def step():
+        for L in layers:
+            q.qlora_linear_fwd(L["w"], L["X"], TOKENS, L["A"], L["B"], R, scale, L["Y"], L["H"], ws)
+        for L in reversed(layers):
+            q.qlora_linear_bwd(L["w"], L["X"], L["dY"], TOKENS, L["A"], L["B"], R, scale, L["H"], L["dX"],
+                               L["dA"], L["dB"], ws)
+        if world > 1:
+            dist.all_reduce(grads)
+
+    def timed_steps(k, fn):
+        """Device time of k steps, each after an L2 flush, CUDA events on the
+        launching stream; a sleep kernel lets the host enqueue a whole step
+        before the GPU reaches it."""
+        total = 0.0
+        for _ in range(k):
+            flush.zero_()
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize()
+            torch.cuda._sleep(20_000_000)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            total += e0.elapsed_time(e1)
+        return total
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    q.qlora_check_device_error()
+
+    # ---- timed region
+    launches0 = q.qlora_launch_count()
+    q.qlora_timing_reset()
+    q.qlora_timing_enable(True)
+    with ClockSampler(local_rank) as clk:
+        ms = timed_steps(args.steps, step)
+    q.qlora_timing_enable(False)
+    launches = q.qlora_launch_count() - launches0
+    kern = q.qlora_timing_read()
+    q.qlora_check_device_error()
+    clocks = clk.summary()
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms = ms_t.item()
+    value = step_flops * args.steps * world / (ms * 1e-3) / 1e12
+
+    # ---- end to end through the same API with host buffers
+    pin = {}
+    for L in layers:
+        pin[L["name"]] = {"X": L["X"].cpu().pin_memory(), "dY": L["dY"].cpu().pin_memory()}
+    host_grads = torch.empty(grads.shape, dtype=torch.float32).pin_memory()
+    h2d = sum(L["X"].numel() * 2 + L["dY"].numel() * 2 for L in layers)
+    d2h = grads.numel() * 4
+
+    def e2e_step():
+        for L in layers:
+            L["X"].copy_(pin[L["name"]]["X"], non_blocking=True)
+            q.qlora_linear_fwd(L["w"], L["X"], TOKENS, L["A"], L["B"], R, scale, L["Y"], L["H"], ws)
+        for L in reversed(layers):
+            L["dY"].copy_(pin[L["name"]]["dY"], non_blocking=True)
+            q.qlora_linear_bwd(L["w"], L["X"], L["dY"], TOKENS, L["A"], L["B"], R, scale, L["H"], L["dX"],
+                               L["dA"], L["dB"], ws)
+        if world > 1:
+            dist.all_reduce(grads)
+        host_grads.copy_(grads, non_blocking=True)
+
+    e2e_step()
+    e2e_ms = timed_steps(args.steps, e2e_step)
+    e_t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e_t, op=dist.ReduceOp.MAX)
+    e2e_value = step_flops * args.steps * world / (e_t.item() * 1e-3) / 1e12
+
+    # ---- roofline of the dominant kernel (largest device time in the timed region)
+    kflops = {
+        "fwd_fused": sum(2 * TOKENS * L["N"] * L["K"] + 2 * TOKENS * L["N"] * R for L in layers) * args.steps,
+        "bwd_fused": sum(2 * TOKENS * L["N"] * L["K"] + 2 * TOKENS * L["K"] * R for L in layers) * args.steps,
+    }
+    dom = max(("fwd_fused", "bwd_fused"), key=lambda k: kern[k][0])
+    dom_ms, dom_n = kern[dom]
+    achieved = kflops[dom] / (dom_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    roofline = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                "peak_source": f"{peak_src} bf16_tflops_sustained",
+                "launches": dom_n, "avg_launch_ms": round(dom_ms / max(dom_n, 1), 4)}
+    breakdown = {k: {"ms_per_step": round(v[0] / args.steps, 4), "launches_per_step": v[1] // args.steps}
+                 for k, v in kern.items() if v[1]}
+
+    codec = run_codec(args, q, torch, dev, peaks, peak_src) if (rank == 0 and not args.skip_codec) else None
+
+    if rank != 0:
+        return None
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,0.02) weights quantized to NF4+DQ, N(0,1) activations and gradients)",
+        "config": {"workload": "linear7b: LLaMA-7B layer, 7 QLoRA linears fwd+bwd, 4096 tokens (8x512), "
+                               "r=64, alpha=16, bf16 activations",
+                   "tokens_per_gpu": TOKENS, "rank": R, "alpha": ALPHA, "l2": "flushed (256 MB write) before each step",
+                   "parallelism": f"dp{world}", "flop_per_step_per_gpu": step_flops},
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "roofline": roofline,
+        "kernels": breakdown,
+        "clocks": clocks,
+    }
+    if codec is not None:
+        line["codec"] = codec
+    if world == 1 and not args.skip_cpu:
+        line["cpu_baseline"] = cpu_baseline_linear(budget_s=args.cpu_seconds)
+    return line
+
+
+def run_codec(args, q, torch, dev, peaks, peak_src):
+    """NF4+DQ quantize -> dequantize round trip over the LLaMA-7B tensors,
+    replayed as one CUDA graph per step."""
+    import synthetic
+    shapes = [(N, K) for _ in range(synthetic.LLAMA7B_LAYERS) for _, N, K in synthetic.LLAMA7B_LINEARS]
+    tensors = []
+    for i, (N, K) in enumerate(shapes):
+        W = synthetic.normal((N, K), 0.02, 50_000 + i, torch.bfloat16, dev)
+        tensors.append((W, q.NF4Weight(N, K, device=dev), torch.empty(N, K, dtype=torch.bfloat16, device=dev)))
+    nweights = sum(N * K for N, K in shapes)
+    qws = torch.empty(max(q.qlora_quantize_workspace_bytes(N, K) for N, K in shapes), dtype=torch.uint8, device=dev)
+
+    def round_trip():
+        for W, w, out in tensors:
+            q.qlora_quantize_nf4_dq(W, w, qws)
+        for W, w, out in tensors:
+            q.qlora_dequantize_nf4_dq(w, out)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _ in range(2):
+            round_trip()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        round_trip()
+    for _ in range(args.warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    q.qlora_check_device_error()
+    # the tensors (13 GB in, 13 GB out) are far larger than L2: no flush needed
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    bytes_rt = 2 * CODEC_BYTES_PER_WEIGHT * nweights
+    gbs = bytes_rt / (ms * 1e-3) / 1e9
+    # per-kernel device time, kernels launched directly (events on the stream)
+    q.qlora_timing_reset()
+    q.qlora_timing_enable(True)
+    torch.cuda._sleep(100_000_000)
+    round_trip()
+    q.qlora_timing_enable(False)
+    kern = q.qlora_timing_read()
+    qms = kern["quantize"][0]
+    dms = kern["dequantize"][0]
+    qgbs = CODEC_BYTES_PER_WEIGHT * nweights / (qms * 1e-3) / 1e9
+    dgbs = CODEC_BYTES_PER_WEIGHT * nweights / (dms * 1e-3) / 1e9
+    dom = "quantize" if qms >= dms else "dequantize"
+    ach = qgbs if dom == "quantize" else dgbs
+    peak = peaks["hbm_gbs"]
+    del g
+    return {
+        "workload": "codec7b: NF4+DQ quantize->dequantize round trip, 224 LLaMA-7B tensors, "
+                    f"{nweights} bf16 weights ~N(0,0.02), one CUDA graph per step",
+        "value": round(gbs, 1), "unit": "GB/s", "ms_per_step": round(ms, 4),
+        "weights_per_s": nweights / (ms * 1e-3),
+        "roofline": {"kernel": dom, "bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(ach / peak, 4), "traffic": None, "peak_source": f"{peak_src} hbm_gbs"},
+        "kernels": {"quantize_gbs": round(qgbs, 1), "dequantize_gbs": round(dgbs, 1),
+                    "dq_encode_ms": round(kern["dq_encode"][0], 4),
+                    "quantize_ms": round(qms, 4), "dequantize_ms": round(dms, 4)},
+    }
+
+
+# ---- CPU baselines (the oracle, as it stands) ---------------------------------------
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p.get("num_threads") for p in threadpool_info() if p.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline_linear(budget_s=15.0):
+    """Oracle fwd+bwd of one 4096x4096 QLoRA linear on a token sample sized
+    to about `budget_s` seconds of host time."""
+    import numpy as np
+
+    import synthetic
+    from oracle import linear as olin
+    N = K = 4096
+    case = synthetic.linear_case(64, N, K, R, ALPHA, seed=7)
+    Wd = case["W"].float().numpy().astype(np.float64)   # stands for the dequantized bf16 weight
+    A = case["A"].float().numpy()
+    B = case["B"].float().numpy()
+    rng = np.random.default_rng(0)
+    M = 64
+    spent, flops = 0.0, 0.0
+    while spent < budget_s:
+        X = rng.standard_normal((M, K))
+        dY = rng.standard_normal((M, N))
+        t0 = time.perf_counter()
+        olin.forward(X, Wd, A, B, ALPHA / R)
+        olin.backward(X, Wd, A, B, ALPHA / R, dY)
+        dt = time.perf_counter() - t0
+        spent += dt
+        flops += linear_flops(M, N, K, R)
+        if dt < budget_s / 8 and M < 8192:
+            M *= 2
+    return {"value": round(flops / spent / 1e12, 5), "unit": "TFLOP/s", "cores": _blas_threads(),
+            "kind": "oracle",
+            "sample": f"oracle float64 fwd+bwd of one 4096x4096 linear (r=64), token batches up to {M}, "
+                      f"{spent:.1f} s of host time"}
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the oracle, timed on the host cores, same metric."""
+    if rank != 0:
+        return None
+    import numpy as np
+
+    import synthetic
+    from oracle import linear as olin
+    Ms = 256   # bounded sample: 256 of the 4096 tokens of each linear per step
+    rng = np.random.default_rng(0)
+    mats = []
+    for i, (name, N, K) in enumerate(synthetic.LLAMA7B_LINEARS):
+        Wd = rng.standard_normal((N, K)) * 0.02
+        mats.append((N, K, Wd, rng.standard_normal((R, K)) / R, rng.standard_normal((N, R)) * 0.01))
+    X = {K: rng.standard_normal((Ms, K)) for K in (4096, 11008)}
+    dY = {N: rng.standard_normal((Ms, N)) for N in (4096, 11008)}
+
+    def step():
+        for N, K, Wd, A, B in mats:
+            olin.forward(X[K], Wd, A, B, ALPHA / R)
+            olin.backward(X[K], Wd, A, B, ALPHA / R, dY[N])
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    flops = sum(linear_flops(Ms, N, K, R) for N, K, *_ in mats) * args.steps
+    value = flops / dt / 1e12
+    cores = _blas_threads()
+    sample = f"oracle float64 fwd+bwd of the 7 LLaMA-7B linears on {Ms} of the 4096 tokens per step"
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": "linear7b: LLaMA-7B layer, 7 QLoRA linears fwd+bwd, "
+                                                    "4096 tokens (8x512), r=64, alpha=16, bf16 activations",
+                                        "parallelism": f"dp{world}"},
+        "cpu_baseline": {"value": round(value, 5), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 5), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--skip-codec", action="store_true")
+    ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -30,7 +30,11 @@ EXPORTS = (
     "qlora_build_nf4_codebook", "qlora_quantize_workspace_bytes", "qlora_quantize_nf4_dq",
     "qlora_dequantize_nf4_dq", "qlora_linear_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd",
     "qlora_status_string", "qlora_check_device_error",
+    "qlora_timing_enable", "qlora_timing_reset", "qlora_timing_read", "qlora_launch_count",
 )
+
+KERNEL_KINDS = ("quantize", "dq_encode", "dequantize", "fwd_fused", "bwd_fused", "lowrank", "wgrad",
+                "elementwise")
 
 
 class QLoraError(RuntimeError):
@@ -65,6 +69,10 @@ def _load():
         "qlora_linear_bwd": (ctypes.c_int, [W, P, P, I64, P, P, I32, F, P, P, ctypes.c_int, P, P, P, S, P]),
         "qlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "qlora_check_device_error": (ctypes.c_int, [P]),
+        "qlora_timing_enable": (ctypes.c_int, [ctypes.c_int]),
+        "qlora_timing_reset": (ctypes.c_int, []),
+        "qlora_timing_read": (ctypes.c_int, [P, P]),
+        "qlora_launch_count": (ctypes.c_int64, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -174,3 +182,24 @@ def qlora_status_string(status: int) -> str:
 
 def qlora_check_device_error(stream=None):
     _check(lib.qlora_check_device_error(_stream(stream)), "qlora_check_device_error")
+
+
+def qlora_timing_enable(enable: bool = True):
+    _check(lib.qlora_timing_enable(1 if enable else 0), "qlora_timing_enable")
+
+
+def qlora_timing_reset():
+    _check(lib.qlora_timing_reset(), "qlora_timing_reset")
+
+
+def qlora_timing_read() -> dict:
+    """{kind: (total_ms, launches)} since the last reset (waits for the events)."""
+    ms = (ctypes.c_double * len(KERNEL_KINDS))()
+    n = (ctypes.c_int64 * len(KERNEL_KINDS))()
+    _check(lib.qlora_timing_read(ctypes.cast(ms, ctypes.c_void_p), ctypes.cast(n, ctypes.c_void_p)),
+           "qlora_timing_read")
+    return {k: (ms[i], n[i]) for i, k in enumerate(KERNEL_KINDS)}
+
+
+def qlora_launch_count() -> int:
+    return lib.qlora_launch_count()

@@ -2,7 +2,9 @@
 // strings, device queries and the device error word.
 #include <cuda_runtime.h>
 #include <math.h>
+#include <atomic>
 #include <mutex>
+#include <vector>
 #include <string.h>
 
 #include "common.cuh"
@@ -184,3 +186,115 @@ extern "C" qlora_status qlora_check_device_error(void *stream)
     if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return QLORA_ERR_CUDA;
     return v == kDevTimeout ? QLORA_ERR_TIMEOUT : QLORA_ERR_CUDA;
 }
+
+// ---- kernel timing ------------------------------------------------------------------
+
+namespace qlora {
+namespace {
+struct TimingState {
+    std::mutex mu;
+    bool enabled = false;
+    std::vector<cudaEvent_t> pool;
+    struct Rec {
+        int kind;
+        cudaEvent_t a, b;
+    };
+    std::vector<Rec> pending;
+    double ms[QLORA_NUM_KERNELS] = {};
+    int64_t launches[QLORA_NUM_KERNELS] = {};
+};
+TimingState &timing()
+{
+    static TimingState t;
+    return t;
+}
+std::atomic<int64_t> g_launches{0};
+
+cudaEvent_t take_event(TimingState &t)
+{
+    if (!t.pool.empty()) {
+        cudaEvent_t e = t.pool.back();
+        t.pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+}  // namespace
+
+LaunchScope::LaunchScope(int kind, cudaStream_t s) : kind_(kind), s_(s)
+{
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    TimingState &t = timing();
+    std::lock_guard<std::mutex> lock(t.mu);
+    if (!t.enabled) return;
+    start_ = take_event(t);
+    if (start_) cudaEventRecord(start_, s_);
+}
+
+LaunchScope::~LaunchScope()
+{
+    if (!start_) return;
+    TimingState &t = timing();
+    std::lock_guard<std::mutex> lock(t.mu);
+    cudaEvent_t stop = take_event(t);
+    if (!stop) {
+        t.pool.push_back(start_);
+        return;
+    }
+    cudaEventRecord(stop, s_);
+    t.pending.push_back({kind_, start_, stop});
+}
+
+}  // namespace qlora
+
+extern "C" qlora_status qlora_timing_enable(int enable)
+{
+    TimingState &t = timing();
+    std::lock_guard<std::mutex> lock(t.mu);
+    t.enabled = enable != 0;
+    return QLORA_OK;
+}
+
+extern "C" qlora_status qlora_timing_reset(void)
+{
+    TimingState &t = timing();
+    std::lock_guard<std::mutex> lock(t.mu);
+    for (auto &r : t.pending) {
+        cudaEventSynchronize(r.b);
+        t.pool.push_back(r.a);
+        t.pool.push_back(r.b);
+    }
+    t.pending.clear();
+    for (int i = 0; i < QLORA_NUM_KERNELS; i++) {
+        t.ms[i] = 0.0;
+        t.launches[i] = 0;
+    }
+    return QLORA_OK;
+}
+
+extern "C" qlora_status qlora_timing_read(double ms[QLORA_NUM_KERNELS], int64_t launches[QLORA_NUM_KERNELS])
+{
+    if (!ms || !launches) return QLORA_ERR_INVALID_ARG;
+    TimingState &t = timing();
+    std::lock_guard<std::mutex> lock(t.mu);
+    qlora_status st = QLORA_OK;
+    for (auto &r : t.pending) {
+        float v = 0.0f;
+        if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&v, r.a, r.b) != cudaSuccess)
+            st = QLORA_ERR_CUDA;
+        t.ms[r.kind] += v;
+        t.launches[r.kind] += 1;
+        t.pool.push_back(r.a);
+        t.pool.push_back(r.b);
+    }
+    t.pending.clear();
+    for (int i = 0; i < QLORA_NUM_KERNELS; i++) {
+        ms[i] = t.ms[i];
+        launches[i] = t.launches[i];
+    }
+    return st;
+}
+
+extern "C" int64_t qlora_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

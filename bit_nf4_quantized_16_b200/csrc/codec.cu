@@ -409,10 +409,13 @@ extern "C" qlora_status qlora_quantize_nf4_dq(const void *W, qlora_dtype w_dtype
     qp.nblocks = nblocks;
     memcpy(qp.mkey, mkey, sizeof(mkey));
     int grid = grid_for(qp.nwords, kThreads * kUnroll, dev.sms * 4);
-    if (w_dtype == QLORA_FP32)
-        quantize_blocks_kernel<true><<<grid, kThreads, 0, s>>>(qp);
-    else
-        quantize_blocks_kernel<false><<<grid, kThreads, 0, s>>>(qp);
+    {
+        LaunchScope ls(QLORA_KERNEL_QUANTIZE, s);
+        if (w_dtype == QLORA_FP32)
+            quantize_blocks_kernel<true><<<grid, kThreads, 0, s>>>(qp);
+        else
+            quantize_blocks_kernel<false><<<grid, kThreads, 0, s>>>(qp);
+    }
     QLORA_TRY(launch_status());
 
     DqParams dp;
@@ -422,7 +425,10 @@ extern "C" qlora_status qlora_quantize_nf4_dq(const void *W, qlora_dtype w_dtype
     dp.c2 = out->c2;
     dp.nblocks = nblocks;
     dp.ngroups = (nblocks + QLORA_GROUP - 1) / QLORA_GROUP;
-    dq_encode_kernel<<<grid_for(dp.ngroups, kThreads / 32, dev.sms * 8), kThreads, 0, s>>>(dp);
+    {
+        LaunchScope ls(QLORA_KERNEL_DQ_ENCODE, s);
+        dq_encode_kernel<<<grid_for(dp.ngroups, kThreads / 32, dev.sms * 8), kThreads, 0, s>>>(dp);
+    }
     return launch_status();
 }
 
@@ -442,6 +448,9 @@ extern "C" qlora_status qlora_dequantize_nf4_dq(const qlora_nf4_weight *w, void 
     p.nwords = w->rows * w->cols / 8;
     memcpy(p.q, w->codebook, sizeof(p.q));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    dequantize_kernel<<<grid_for(p.nwords, kThreads * kUnroll, dev.sms * 8), kThreads, 0, s>>>(p);
+    {
+        LaunchScope ls(QLORA_KERNEL_DEQUANTIZE, s);
+        dequantize_kernel<<<grid_for(p.nwords, kThreads * kUnroll, dev.sms * 8), kThreads, 0, s>>>(p);
+    }
     return launch_status();
 }

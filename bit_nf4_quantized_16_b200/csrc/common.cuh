@@ -49,4 +49,17 @@ inline qlora_status launch_status()
 // Checks shared by every entry point that takes a quantized weight.
 qlora_status check_weight(const qlora_nf4_weight *w);
 
+// Brackets one kernel launch for qlora_timing_read (events only while timing
+// is enabled) and counts it for qlora_launch_count.
+class LaunchScope {
+  public:
+    LaunchScope(int kind, cudaStream_t s);
+    ~LaunchScope();
+
+  private:
+    int kind_;
+    cudaStream_t s_;
+    cudaEvent_t start_ = nullptr;
+};
+
 }  // namespace qlora

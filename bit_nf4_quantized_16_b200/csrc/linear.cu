@@ -73,7 +73,7 @@ qlora_status map_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint64_t
 // ---- GEMM launch ------------------------------------------------------------------
 
 template <int BN, int kBMode, int kEpi>
-qlora_status launch_gemm(GemmParams &p, const DeviceInfo &dev, cudaStream_t s)
+qlora_status launch_gemm(GemmParams &p, const DeviceInfo &dev, cudaStream_t s, int kind)
 {
     using Cfg = GemmCfg<BN, kBMode>;
     static bool attr_done[64] = {};
@@ -87,7 +87,10 @@ qlora_status launch_gemm(GemmParams &p, const DeviceInfo &dev, cudaStream_t s)
     p.timeout_ns = kTimeoutNs;
     const int tiles = p.m_tiles * p.n_tiles * p.splits;
     const int grid = tiles < dev.sms ? tiles : dev.sms;
-    kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, s>>>(p);
+    {
+        LaunchScope ls(kind, s);
+        kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, s>>>(p);
+    }
     return launch_status();
 }
 
@@ -237,12 +240,15 @@ qlora_status run_h(const Plan &pl, const DeviceInfo &dev, const void *X, const v
     p.m_total = (int)pl.M;
     p.n_total = pl.r_pad;
     if (pl.r_pad == 64)
-        QLORA_TRY((launch_gemm<64, kBTmaK, kEpiF32>(p, dev, s)));
+        QLORA_TRY((launch_gemm<64, kBTmaK, kEpiF32>(p, dev, s, QLORA_KERNEL_LOWRANK)));
     else
-        QLORA_TRY((launch_gemm<128, kBTmaK, kEpiF32>(p, dev, s)));
-    finalize_lowrank_kernel<<<elementwise_grid(pl.M * pl.r), 256, 0, s>>>(
-        reinterpret_cast<const float *>(ws + pl.off_part), pl.h_splits, pl.M * pl.r_pad, pl.r_pad, pl.M, pl.r, scale,
-        H_out, reinterpret_cast<__nv_bfloat16 *>(ws + pl.off_h2));
+        QLORA_TRY((launch_gemm<128, kBTmaK, kEpiF32>(p, dev, s, QLORA_KERNEL_LOWRANK)));
+    {
+        LaunchScope ls(QLORA_KERNEL_ELEMENTWISE, s);
+        finalize_lowrank_kernel<<<elementwise_grid(pl.M * pl.r), 256, 0, s>>>(
+            reinterpret_cast<const float *>(ws + pl.off_part), pl.h_splits, pl.M * pl.r_pad, pl.r_pad, pl.M, pl.r,
+            scale, H_out, reinterpret_cast<__nv_bfloat16 *>(ws + pl.off_h2));
+    }
     return launch_status();
 }
 
@@ -299,8 +305,8 @@ extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const void *
     p.out_ld = pl.N;
     p.m_total = (int)M;
     p.n_total = (int)pl.N;
-    if (y_dtype == QLORA_BF16) return launch_gemm<256, kBNf4K, kEpiBf16>(p, dev, s);
-    return launch_gemm<256, kBNf4K, kEpiF32>(p, dev, s);
+    if (y_dtype == QLORA_BF16) return launch_gemm<256, kBNf4K, kEpiBf16>(p, dev, s, QLORA_KERNEL_FWD_FUSED);
+    return launch_gemm<256, kBNf4K, kEpiF32>(p, dev, s, QLORA_KERNEL_FWD_FUSED);
 }
 
 extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *X, const void *dY, int64_t M,
@@ -333,7 +339,10 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *
 
     // H (hi/lo) from the saved fp32 H, or recomputed
     if (H_saved) {
-        split_hi_lo_kernel<<<elementwise_grid(M * r), 256, 0, s>>>(H_saved, M, r, H2);
+        {
+            LaunchScope ls(QLORA_KERNEL_ELEMENTWISE, s);
+            split_hi_lo_kernel<<<elementwise_grid(M * r), 256, 0, s>>>(H_saved, M, r, H2);
+        }
         QLORA_TRY(launch_status());
     } else {
         QLORA_TRY(run_h(pl, dev, X, A, scale, nullptr, ws, s));
@@ -355,11 +364,14 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *
         p.m_total = (int)M;
         p.n_total = pl.r_pad;
         if (pl.r_pad == 64)
-            QLORA_TRY((launch_gemm<64, kBTmaMN, kEpiF32>(p, dev, s)));
+            QLORA_TRY((launch_gemm<64, kBTmaMN, kEpiF32>(p, dev, s, QLORA_KERNEL_LOWRANK)));
         else
-            QLORA_TRY((launch_gemm<128, kBTmaMN, kEpiF32>(p, dev, s)));
-        finalize_lowrank_kernel<<<elementwise_grid(M * r), 256, 0, s>>>(part, pl.g_splits, M * pl.r_pad, pl.r_pad, M,
-                                                                         r, scale, nullptr, G2);
+            QLORA_TRY((launch_gemm<128, kBTmaMN, kEpiF32>(p, dev, s, QLORA_KERNEL_LOWRANK)));
+        {
+            LaunchScope ls(QLORA_KERNEL_ELEMENTWISE, s);
+            finalize_lowrank_kernel<<<elementwise_grid(M * r), 256, 0, s>>>(part, pl.g_splits, M * pl.r_pad, pl.r_pad,
+                                                                             M, r, scale, nullptr, G2);
+        }
         QLORA_TRY(launch_status());
     }
 
@@ -388,9 +400,9 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *
         p.m_total = (int)M;
         p.n_total = (int)K;
         if (dx_dtype == QLORA_BF16)
-            QLORA_TRY((launch_gemm<256, kBNf4MN, kEpiBf16>(p, dev, s)));
+            QLORA_TRY((launch_gemm<256, kBNf4MN, kEpiBf16>(p, dev, s, QLORA_KERNEL_BWD_FUSED)));
         else
-            QLORA_TRY((launch_gemm<256, kBNf4MN, kEpiF32>(p, dev, s)));
+            QLORA_TRY((launch_gemm<256, kBNf4MN, kEpiF32>(p, dev, s, QLORA_KERNEL_BWD_FUSED)));
     }
 
     // dA = G^T X  (rows j of [G_hi | G_lo], contraction over tokens)
@@ -409,9 +421,12 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *
         p.split_stride = 2 * r * K;
         p.m_total = 2 * r;
         p.n_total = (int)K;
-        QLORA_TRY((launch_gemm<128, kBTmaMN, kEpiF32>(p, dev, s)));
-        finalize_wgrad_kernel<<<elementwise_grid((int64_t)r * K), 256, 0, s>>>(part, pl.da_splits, 2 * r * K, K, r, K,
-                                                                               r, 0, dA);
+        QLORA_TRY((launch_gemm<128, kBTmaMN, kEpiF32>(p, dev, s, QLORA_KERNEL_WGRAD)));
+        {
+            LaunchScope ls(QLORA_KERNEL_ELEMENTWISE, s);
+            finalize_wgrad_kernel<<<elementwise_grid((int64_t)r * K), 256, 0, s>>>(part, pl.da_splits, 2 * r * K, K, r,
+                                                                                   K, r, 0, dA);
+        }
         QLORA_TRY(launch_status());
     }
 
@@ -432,13 +447,16 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *
         p.m_total = (int)N;
         p.n_total = 2 * r;
         if (pl.db_bn == 64)
-            QLORA_TRY((launch_gemm<64, kBTmaMN, kEpiF32>(p, dev, s)));
+            QLORA_TRY((launch_gemm<64, kBTmaMN, kEpiF32>(p, dev, s, QLORA_KERNEL_WGRAD)));
         else if (pl.db_bn == 128)
-            QLORA_TRY((launch_gemm<128, kBTmaMN, kEpiF32>(p, dev, s)));
+            QLORA_TRY((launch_gemm<128, kBTmaMN, kEpiF32>(p, dev, s, QLORA_KERNEL_WGRAD)));
         else
-            QLORA_TRY((launch_gemm<256, kBTmaMN, kEpiF32>(p, dev, s)));
-        finalize_wgrad_kernel<<<elementwise_grid(N * r), 256, 0, s>>>(part, pl.db_splits, N * 2 * r, 2 * r, N, r, 0,
-                                                                       r, dB);
+            QLORA_TRY((launch_gemm<256, kBTmaMN, kEpiF32>(p, dev, s, QLORA_KERNEL_WGRAD)));
+        {
+            LaunchScope ls(QLORA_KERNEL_ELEMENTWISE, s);
+            finalize_wgrad_kernel<<<elementwise_grid(N * r), 256, 0, s>>>(part, pl.db_splits, N * 2 * r, 2 * r, N, r,
+                                                                           0, r, dB);
+        }
         return launch_status();
     }
 }

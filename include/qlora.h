@@ -214,6 +214,33 @@ QLORA_API const char *qlora_status_string(qlora_status status);
  */
 QLORA_API qlora_status qlora_check_device_error(void *stream);
 
+/*
+ * Kernel timing for benchmarks.  While enabled, every kernel this library
+ * launches is bracketed by two CUDA events recorded on the kernel's own
+ * stream; qlora_timing_read() waits for the recorded events and returns the
+ * summed device time and launch count per kernel kind since the last reset.
+ * Disabled by default; enabling it adds two event records per launch.
+ *   kinds: QLORA_KERNEL_* below; ms and launches have QLORA_NUM_KERNELS
+ *   entries (host arrays, written).
+ * qlora_launch_count() counts every kernel launch of the library since the
+ * process started, whether timing is enabled or not.
+ */
+enum {
+    QLORA_KERNEL_QUANTIZE = 0,    /* first-level quantization pass       */
+    QLORA_KERNEL_DQ_ENCODE = 1,   /* double quantization of constants    */
+    QLORA_KERNEL_DEQUANTIZE = 2,  /* stand-alone dequantizer             */
+    QLORA_KERNEL_FWD_FUSED = 3,   /* fused dequant-GEMM, forward         */
+    QLORA_KERNEL_BWD_FUSED = 4,   /* fused dequant-GEMM, input gradient  */
+    QLORA_KERNEL_LOWRANK = 5,     /* H = X A^T and G = dY B products     */
+    QLORA_KERNEL_WGRAD = 6,       /* dA and dB products                  */
+    QLORA_KERNEL_ELEMENTWISE = 7, /* split-sum / hi-lo finalize kernels  */
+    QLORA_NUM_KERNELS = 8
+};
+QLORA_API qlora_status qlora_timing_enable(int enable);
+QLORA_API qlora_status qlora_timing_reset(void);
+QLORA_API qlora_status qlora_timing_read(double ms[QLORA_NUM_KERNELS], int64_t launches[QLORA_NUM_KERNELS]);
+QLORA_API int64_t qlora_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif
