@@ -117,14 +117,19 @@ def run_ours(args, rank, world, local_rank):
     peaks, peak_src = load_peaks()
 
     # ---- set-up (untimed): quantize the seven frozen weights, allocate activations
+    TOKENS = args.tokens
+    if args.linears == "llama7b":
+        shapes = synthetic.LLAMA7B_LINEARS
+    else:
+        n_, k_ = (int(v) for v in args.linears.lower().split("x"))
+        shapes = [("single", n_, k_)]
     layers = []
     ws_bytes = 0
-    qws_bytes = max(q.qlora_quantize_workspace_bytes(N, K) for _, N, K in synthetic.LLAMA7B_LINEARS)
+    qws_bytes = max(q.qlora_quantize_workspace_bytes(N, K) for _, N, K in shapes)
     qws = torch.empty(qws_bytes, dtype=torch.uint8, device=dev)
-    grads = torch.empty(sum(R * K + N * R for _, N, K in synthetic.LLAMA7B_LINEARS), dtype=torch.float32,
-                        device=dev)
+    grads = torch.empty(sum(R * K + N * R for _, N, K in shapes), dtype=torch.float32, device=dev)
     off = 0
-    for i, (name, N, K) in enumerate(synthetic.LLAMA7B_LINEARS):
+    for i, (name, N, K) in enumerate(shapes):
         seed = 1000 * rank + 10 * i
         W = synthetic.normal((N, K), 0.02, seed, torch.bfloat16, dev)
         w = q.NF4Weight(N, K, device=dev)
@@ -253,8 +258,9 @@ def run_ours(args, rank, world, local_rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,0.02) weights quantized to NF4+DQ, N(0,1) activations and gradients)",
-        "config": {"workload": "linear7b: LLaMA-7B layer, 7 QLoRA linears fwd+bwd, 4096 tokens (8x512), "
-                               "r=64, alpha=16, bf16 activations",
+        "config": {"workload": ("linear7b: LLaMA-7B layer, 7 QLoRA linears fwd+bwd, 4096 tokens (8x512), "
+                                "r=64, alpha=16, bf16 activations") if args.linears == "llama7b" else
+                               f"single QLoRA linear {args.linears} fwd+bwd, {TOKENS} tokens, r=64, alpha=16",
                    "tokens_per_gpu": TOKENS, "rank": R, "alpha": ALPHA, "l2": "flushed (256 MB write) before each step",
                    "parallelism": f"dp{world}", "flop_per_step_per_gpu": step_flops},
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
@@ -438,6 +444,9 @@ def main():
     ap.add_argument("--skip-codec", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--linears", default="llama7b",
+                    help="llama7b (the seven linears of one layer) or NxK for one linear (profiling runs)")
+    ap.add_argument("--tokens", type=int, default=TOKENS)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank = int(os.environ.get("RANK", "0"))

@@ -37,10 +37,66 @@ QLORA_HD void exact_mean_split(uint32_t bits, uint32_t *bucket, uint32_t *sig)
     *sig = E ? (F | 0x800000u) : F;
 }
 
+// Fast path: all non-zero buckets lie within 61 consecutive exponents, so the
+// exact sum fits one 128-bit integer T (units of 2^(lo-150)); the quotient
+// T / count is normalized to at least 26 bits before rounding.  Returns false
+// when the fast path does not apply.
+QLORA_HD bool exact_mean_bits_narrow(const unsigned long long *bucket, uint64_t count, int lo, int hi,
+                                     uint32_t *out)
+{
+    if (hi - lo > 60) return false;
+    unsigned __int128 T = 0;
+    for (int j = lo; j <= hi; j++) T += (unsigned __int128)bucket[j] << (j - lo);
+    int b = lo - 150;                                   // value = T * 2^b / count
+    // normalize so that the quotient has at least 26 significant bits
+    const unsigned __int128 need = (unsigned __int128)count << 26;
+    while (T < need) {
+        T <<= 1;
+        b -= 1;
+    }
+    const unsigned __int128 Q = T / count;
+    const uint64_t rem = (uint64_t)(T - Q * count);
+    int p = 127;
+    while (!((Q >> p) & 1)) p--;
+    // least significant kept bit: 2^(p+b-23) for a normal result, 2^-149 below
+    int L = p + b - 23;
+    if (L < -149) L = -149;
+    const int t = L - b;                                // quotient bits dropped (>= 2)
+    uint32_t mant;
+    bool up;
+    if (t > 127) {
+        mant = 0;
+        up = false;                                     // far below 2^-150: rounds to 0
+    } else {
+        mant = (uint32_t)(Q >> t);
+        const bool round_bit = (Q >> (t - 1)) & 1;
+        const unsigned __int128 low_mask = (((unsigned __int128)1) << (t - 1)) - 1;
+        const bool sticky = (Q & low_mask) != 0 || rem != 0;
+        up = round_bit && (sticky || (mant & 1u));
+    }
+    if (up) mant += 1;
+    // value = mant * 2^L; the same formula covers subnormals (L = -149) and a
+    // carry into the next binade
+    *out = ((uint32_t)(L + 149) << 23) + mant;
+    return true;
+}
+
 // Binary32 bit pattern of RN(sum_j bucket[j] * 2^(j-150) / count).
 // bucket has 256 entries; count >= 1 and < 2^32.
 QLORA_HD uint32_t exact_mean_bits(const unsigned long long *bucket, uint64_t count)
 {
+    int lo = 256, hi = -1;
+#pragma unroll 8
+    for (int j = 1; j < 255; j++) {
+        if (bucket[j]) {
+            lo = j < lo ? j : lo;
+            hi = j;
+        }
+    }
+    if (hi < 0) return 0u;
+    uint32_t fast;
+    if (exact_mean_bits_narrow(bucket, count, lo, hi, &fast)) return fast;
+
     // 1. exact sum as an integer in units of 2^-149: sum_j bucket[j] << (j-1)
     //    held in ten 32-bit digits (320 bits, least significant first).
     uint32_t dig[10];

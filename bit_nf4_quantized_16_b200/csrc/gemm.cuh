@@ -73,7 +73,7 @@ template <int BN, int kBMode>
 struct GemmCfg {
     static constexpr int kStages = (kBMode >= kBNf4K) ? 4 : (BN >= 256 ? 4 : 6);
     static constexpr bool kFused = kBMode >= kBNf4K;
-    static constexpr int kDeqWarps = kFused ? 4 : 0;
+    static constexpr int kDeqWarps = kFused ? 8 : 0;
     static constexpr int kThreads = 256 + 32 * kDeqWarps;
     static constexpr uint32_t kABytes = 128 * 64 * 2;
     static constexpr uint32_t kBBytes = BN * 64 * 2;
@@ -352,9 +352,14 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode>::kThreads, 1)
             if (lane == 0) mbar_arrive(&acc_empty[buf]);
         }
     } else if (kFused && warp >= 8) {
+      if constexpr (kFused) {
         // ---------------- dequantization producer ----------------
+        // One quantization block (64 consecutive k of one row of W) per thread
+        // per stage: forward stages hold BN rows x 64 columns of W, input-
+        // gradient stages hold 64 rows x BN columns (BN / 64 blocks per row).
+        // The block constant of the next stage is fetched one stage ahead.
         const int dt = (warp - 8) * 32 + lane;
-        constexpr int kDeqThreads = 32 * Cfg::kDeqWarps;
+        static_assert(32 * Cfg::kDeqWarps == BN, "one block per thread per stage");
         const float mu = *p.mean;
         uint32_t it = 0;
         for (int t = blockIdx.x; t < num_tiles && !*vabort; t += gridDim.x) {
@@ -362,53 +367,74 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode>::kThreads, 1)
             decode(t, mt, nt, sp);
             stages_of(sp, kb0, nmain);
             const int nst = nmain + (sp == 0 ? p.k_stages_lora : 0);
+            // block (row, column block) of this thread at main stage ks
+            auto block_of = [&](int ks, int64_t &n, int64_t &kb) {
+                if (kBMode == kBNf4K) {
+                    n = (int64_t)nt * BN + dt;
+                    kb = kb0 + ks;
+                } else {
+                    n = (int64_t)(kb0 + ks) * 64 + (dt & 63);
+                    kb = (int64_t)nt * (BN / 64) + (dt >> 6);
+                }
+            };
+            int64_t n, kb;
+            block_of(0, n, kb);
+            float c1p = nmain > 0 ? block_scale(p, n, kb, mu) : 0.0f;
             bool ok = true;
             for (int ks = 0; ks < nst; ks++, it++) {
                 const int s = it % S;
                 const uint32_t use = it / S;
+                // prefetch the next stage's block constant (raw bytes only)
+                uint8_t e_next = 0;
+                float c2_next = 0.0f;
+                bool have_next = false;
+                if (ks + 1 < nmain) {
+                    int64_t n1, kb1;
+                    block_of(ks + 1, n1, kb1);
+                    if (n1 < p.wrows && kb1 < p.kblocks) {
+                        const int64_t b = n1 * p.kblocks + kb1;
+                        e_next = p.code2[b];
+                        c2_next = p.c2[b >> 8];
+                        have_next = true;
+                    }
+                }
                 if (!mbar_wait_bounded(&full_a[s], use & 1, p.timeout_ns)) {
                     record_timeout(p, abort_flag);
                     ok = false;
                     break;
                 }
                 if (ks < nmain) {
-                    const int k0 = (kb0 + ks) * 64;
-                    uint8_t *pb = sP(s);
+                    const uint8_t *pb = sP(s);
                     uint8_t *bb = sB(s);
                     if (kBMode == kBNf4K) {
-                        // stage = rows n0..n0+BN-1 of W, columns k0..k0+63 (one block per row)
-                        for (int nl = dt; nl < BN; nl += kDeqThreads) {
-                            const float c1p = block_scale(p, (int64_t)nt * BN + nl, k0 / 64, mu);
-                            const int sw = (nl >> 2) & 1;   // 32-byte swizzle of the packed tile
-                            const uint4 lo = *reinterpret_cast<const uint4 *>(pb + nl * 32 + (sw << 4));
-                            const uint4 hi = *reinterpret_cast<const uint4 *>(pb + nl * 32 + ((sw ^ 1) << 4));
-                            const uint32_t words[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-                            uint8_t *dst = bb + nl * 128;
+                        const int nl = dt;
+                        const int sw = (nl >> 2) & 1;   // 32-byte swizzle of the packed tile
+                        const uint4 lo = *reinterpret_cast<const uint4 *>(pb + nl * 32 + (sw << 4));
+                        const uint4 hi = *reinterpret_cast<const uint4 *>(pb + nl * 32 + ((sw ^ 1) << 4));
+                        const uint32_t words[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+                        uint8_t *dst = bb + nl * 128;
 #pragma unroll
-                            for (int j = 0; j < 8; j++)
-                                *reinterpret_cast<uint4 *>(dst + ((j ^ (nl & 7)) << 4)) = expand8(words[j], lut, c1p);
-                        }
+                        for (int j = 0; j < 8; j++)
+                            *reinterpret_cast<uint4 *>(dst + ((j ^ (nl & 7)) << 4)) = expand8(words[j], lut, c1p);
                     } else {
-                        // stage = rows k0..k0+63 of W (contraction), columns n0..n0+BN-1
-                        for (int u = dt; u < 64 * (BN / 64); u += kDeqThreads) {
-                            const int r = u & 63, c = u >> 6;
-                            const float c1p = block_scale(p, (int64_t)k0 + r, (int64_t)nt * (BN / 64) + c, mu);
-                            const uint4 lo = *reinterpret_cast<const uint4 *>(pb + r * 128 + (((2 * c) ^ (r & 7)) << 4));
-                            const uint4 hi = *reinterpret_cast<const uint4 *>(pb + r * 128 + (((2 * c + 1) ^ (r & 7)) << 4));
-                            const uint32_t words[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-                            uint8_t *dst = bb + c * 8192 + r * 128;
+                        const int r = dt & 63, c = dt >> 6;
+                        const uint4 lo = *reinterpret_cast<const uint4 *>(pb + r * 128 + (((2 * c) ^ (r & 7)) << 4));
+                        const uint4 hi = *reinterpret_cast<const uint4 *>(pb + r * 128 + (((2 * c + 1) ^ (r & 7)) << 4));
+                        const uint32_t words[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+                        uint8_t *dst = bb + c * 8192 + r * 128;
 #pragma unroll
-                            for (int j = 0; j < 8; j++)
-                                *reinterpret_cast<uint4 *>(dst + ((j ^ (r & 7)) << 4)) = expand8(words[j], lut, c1p);
-                        }
+                        for (int j = 0; j < 8; j++)
+                            *reinterpret_cast<uint4 *>(dst + ((j ^ (r & 7)) << 4)) = expand8(words[j], lut, c1p);
                     }
                     fence_proxy_async_smem();
+                    c1p = have_next ? __fmaf_rn(e4m3_to_float(e_next), c2_next, mu) : 0.0f;
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&full_b[s]);
             }
             if (!ok) break;
         }
+      }
     }
 
     __syncthreads();
