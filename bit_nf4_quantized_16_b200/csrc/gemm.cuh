@@ -1,9 +1,11 @@
 // Warp-specialized tcgen05 GEMM for sm_100a, with an optional on-chip NF4
 // dequantization producer for the B operand.
 //
-// D[128 x BN] tiles accumulate in tensor memory (fp32); operands are staged
-// in shared memory in the 128-byte-swizzled canonical layouts described in
-// sm100.cuh.  Roles (one CTA per SM, persistent over output tiles):
+// D[128*MT x BN] tiles (MT = 1 or 2 accumulators of 128 rows that share one B
+// tile, so every dequantized element feeds MT MMAs) accumulate in tensor
+// memory (fp32); operands are staged in shared memory in the 128-byte-
+// swizzled canonical layouts described in sm100.cuh.  Roles (one CTA per SM,
+// persistent over output tiles):
 //   warp 0       TMA producer: A tiles and either B tiles or packed NF4 tiles
 //   warp 1       MMA issuer (one thread) and TMEM owner
 //   warps 4..7   epilogue: TMEM -> registers -> global (bf16 / fp32)
@@ -69,19 +71,26 @@ struct GemmParams {
     uint64_t timeout_ns;
 };
 
-template <int BN, int kBMode>
+template <int BN, int kBMode, int MT>
 struct GemmCfg {
-    static constexpr int kStages = (kBMode >= kBNf4K) ? 4 : (BN >= 256 ? 4 : 6);
     static constexpr bool kFused = kBMode >= kBNf4K;
     static constexpr int kDeqWarps = kFused ? 8 : 0;
     static constexpr int kThreads = 256 + 32 * kDeqWarps;
-    static constexpr uint32_t kABytes = 128 * 64 * 2;
+    static constexpr uint32_t kABytes = MT * 128 * 64 * 2;
     static constexpr uint32_t kBBytes = BN * 64 * 2;
     static constexpr uint32_t kPBytes = kFused ? BN * 32 : 0;
     static constexpr uint32_t kStageBytes = kABytes + kBBytes + kPBytes;
+    static constexpr int kMaxStages = (232448 - 2048) / kStageBytes;
+    static constexpr int kStages = kMaxStages > 6 ? 6 : kMaxStages;
     static constexpr uint32_t kBarOff = kStages * kStageBytes;
     static constexpr uint32_t kSmemBytes = kBarOff + 512 + 1024;  // barriers etc. + alignment slack
-    static constexpr uint32_t kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;
+    static constexpr uint32_t kAccCols = MT * BN;                  // one accumulator buffer
+    static constexpr uint32_t kTmemCols = 2 * kAccCols < 32 ? 32 : 2 * kAccCols;
+    static_assert(2 * kAccCols <= 512, "two accumulator buffers must fit in TMEM");
+    static_assert(kStages >= 2, "shared memory too small for two stages");
+    // dequantization: blocks per stage (BN rows x 1 block forward, 64 rows x
+    // BN/64 blocks for the input gradient: BN blocks either way), threads per block
+    static constexpr int kTPB = kFused ? (32 * kDeqWarps) / BN : 1;
 };
 
 namespace gemm_detail {
@@ -99,25 +108,35 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return d;
 }
 
+// (a, b) * (s, s), each lane rounded to nearest-even (packed f32x2 multiply)
+__device__ __forceinline__ void mul2(float a, float b, float s, float &ra, float &rb)
+{
+    uint64_t x, y;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a), "f"(b));
+    uint64_t ss;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(ss) : "f"(s));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(y) : "l"(x), "l"(ss));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(ra), "=f"(rb) : "l"(y));
+}
+
 // 8 consecutive codes (one 32-bit word, element 0 in bits 0-3) -> 8 bf16 in a
-// 16-byte vector: w = bf16(RN32(q[code] * c1p)).
+// 16-byte vector: w = bf16(RN32(q[code] * c1p)), the stand-alone dequantizer's
+// arithmetic.
 __device__ __forceinline__ uint4 expand8(uint32_t word, const float *lut, float c1p)
 {
     uint32_t o[4];
 #pragma unroll
     for (int i = 0; i < 4; i++) {
-        float lo = __fmul_rn(lut[(word >> (8 * i)) & 15u], c1p);
-        float hi = __fmul_rn(lut[(word >> (8 * i + 4)) & 15u], c1p);
+        float lo, hi;
+        mul2(lut[(word >> (8 * i)) & 15u], lut[(word >> (8 * i + 4)) & 15u], c1p, lo, hi);
         o[i] = pack_bf16x2(lo, hi);
     }
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-__device__ __forceinline__ float block_scale(const GemmParams &p, int64_t n, int64_t kb, float mu)
+__device__ __forceinline__ float block_scale_raw(uint8_t e, float c2, float mu)
 {
-    if (n >= p.wrows || kb >= p.kblocks) return 0.0f;
-    int64_t b = n * p.kblocks + kb;
-    return __fmaf_rn(e4m3_to_float(p.code2[b]), p.c2[b >> 8], mu);
+    return __fmaf_rn(e4m3_to_float(e), c2, mu);
 }
 
 __device__ __forceinline__ void record_timeout(const GemmParams &p, int *abort_flag)
@@ -128,17 +147,19 @@ __device__ __forceinline__ void record_timeout(const GemmParams &p, int *abort_f
 
 }  // namespace gemm_detail
 
-template <int BN, int kBMode, int kEpi>
-__global__ void __launch_bounds__(GemmCfg<BN, kBMode>::kThreads, 1)
+template <int BN, int kBMode, int kEpi, int MT>
+__global__ void __launch_bounds__(GemmCfg<BN, kBMode, MT>::kThreads, 1)
     qgemm_kernel(const __grid_constant__ GemmParams p)
 {
-    using Cfg = GemmCfg<BN, kBMode>;
+    using Cfg = GemmCfg<BN, kBMode, MT>;
     using namespace sm100;
     using namespace gemm_detail;
     constexpr int S = Cfg::kStages;
     constexpr bool kFused = Cfg::kFused;
+    constexpr int BM = 128 * MT;
 
     extern __shared__ uint8_t smem_raw[];
+    __shared__ float lut[16];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *full_a = reinterpret_cast<uint64_t *>(smem + Cfg::kBarOff);
     uint64_t *full_b = full_a + S;
@@ -148,7 +169,6 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode>::kThreads, 1)
     uint64_t *drain = acc_empty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
-    float *lut = reinterpret_cast<float *>(tmem_slot + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     auto sA = [&](int s) { return smem + s * Cfg::kABytes; };
@@ -223,15 +243,15 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode>::kThreads, 1)
                     break;
                 }
                 if (*vabort) break;
-                const int m0 = mt * 128, n0 = nt * BN;
+                const int m0 = mt * BM, n0 = nt * BN;
                 if (ks < nmain) {
                     const int k0 = (kb0 + ks) * 64;
                     mbar_arrive_expect_tx(&full_a[s], Cfg::kABytes + (kFused ? Cfg::kPBytes : Cfg::kBBytes));
                     if (!p.a_mn) {
-                        tma_load_2d(sA(s), &p.tm_a, &full_a[s], k0, m0);
+                        tma_load_2d(sA(s), &p.tm_a, &full_a[s], k0, m0);                  // [BM rows][64]
                     } else {
-                        tma_load_2d(sA(s), &p.tm_a, &full_a[s], m0, k0);
-                        tma_load_2d(sA(s) + 8192, &p.tm_a, &full_a[s], m0 + 64, k0);
+#pragma unroll
+                        for (int j = 0; j < 2 * MT; j++) tma_load_2d(sA(s) + 8192 * j, &p.tm_a, &full_a[s], m0 + 64 * j, k0);
                     }
                     if (kBMode == kBTmaK) {
                         tma_load_2d(sB(s), &p.tm_b, &full_a[s], k0, n0);
@@ -274,7 +294,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode>::kThreads, 1)
                 break;
             }
             tc_fence_after();
-            const uint32_t d_tmem = tmem_base + buf * BN;
+            const uint32_t d_tmem = tmem_base + buf * Cfg::kAccCols;
             for (int ks = 0; ks < nst; ks++, it++) {
                 const int s = it % S;
                 const uint32_t use = it / S;
@@ -288,11 +308,15 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode>::kThreads, 1)
                 const uint32_t a_addr = smem_u32(sA(s)), b_addr = smem_u32(sB(s));
 #pragma unroll
                 for (int kk = 0; kk < 4; kk++) {
-                    const uint64_t adesc = p.a_mn ? smem_desc_sw128(a_addr + 2048 * kk, 8192, 1024)
-                                                  : smem_desc_sw128(a_addr + 32 * kk, 16, 1024);
                     const uint64_t bdesc = kBMn ? smem_desc_sw128(b_addr + 2048 * kk, 8192, 1024)
                                                 : smem_desc_sw128(b_addr + 32 * kk, 16, 1024);
-                    tc_mma_bf16(d_tmem, adesc, bdesc, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                    for (int m = 0; m < MT; m++) {
+                        const uint32_t a_sub = a_addr + m * 16384;
+                        const uint64_t adesc = p.a_mn ? smem_desc_sw128(a_sub + 2048 * kk, 8192, 1024)
+                                                      : smem_desc_sw128(a_sub + 32 * kk, 16, 1024);
+                        tc_mma_bf16(d_tmem + m * BN, adesc, bdesc, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+                    }
                 }
                 tc_commit(&empty[s]);
             }
@@ -317,33 +341,36 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode>::kThreads, 1)
                 break;
             }
             tc_fence_after();
-            const int row = mt * 128 + 32 * q + lane;
-            const bool row_ok = row < p.m_total;
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; c++) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * q) << 16) + buf * BN + 32 * c, r);
-                tmem_ld_wait();
-                const int col0 = nt * BN + 32 * c;
-                if (!row_ok) continue;
-                if (kEpi == kEpiBf16) {
-                    __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.out) + (int64_t)row * p.out_ld + col0;
+            for (int m = 0; m < MT; m++) {
+                const int row = mt * BM + m * 128 + 32 * q + lane;
+                const bool row_ok = row < p.m_total;
+#pragma unroll 1
+                for (int c = 0; c < BN / 32; c++) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * q) << 16) + buf * Cfg::kAccCols + m * BN + 32 * c, r);
+                    tmem_ld_wait();
+                    const int col0 = nt * BN + 32 * c;
+                    if (!row_ok) continue;
+                    if (kEpi == kEpiBf16) {
+                        __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.out) + (int64_t)row * p.out_ld + col0;
 #pragma unroll
-                    for (int g = 0; g < 4; g++) {
-                        if (col0 + 8 * g >= p.n_total) break;
-                        uint4 v;
-                        v.x = pack_bf16x2(__uint_as_float(r[8 * g + 0]), __uint_as_float(r[8 * g + 1]));
-                        v.y = pack_bf16x2(__uint_as_float(r[8 * g + 2]), __uint_as_float(r[8 * g + 3]));
-                        v.z = pack_bf16x2(__uint_as_float(r[8 * g + 4]), __uint_as_float(r[8 * g + 5]));
-                        v.w = pack_bf16x2(__uint_as_float(r[8 * g + 6]), __uint_as_float(r[8 * g + 7]));
-                        *reinterpret_cast<uint4 *>(o + 8 * g) = v;
-                    }
-                } else {
-                    float *o = static_cast<float *>(p.out) + (int64_t)sp * p.split_stride + (int64_t)row * p.out_ld + col0;
+                        for (int g = 0; g < 4; g++) {
+                            if (col0 + 8 * g >= p.n_total) break;
+                            uint4 v;
+                            v.x = pack_bf16x2(__uint_as_float(r[8 * g + 0]), __uint_as_float(r[8 * g + 1]));
+                            v.y = pack_bf16x2(__uint_as_float(r[8 * g + 2]), __uint_as_float(r[8 * g + 3]));
+                            v.z = pack_bf16x2(__uint_as_float(r[8 * g + 4]), __uint_as_float(r[8 * g + 5]));
+                            v.w = pack_bf16x2(__uint_as_float(r[8 * g + 6]), __uint_as_float(r[8 * g + 7]));
+                            *reinterpret_cast<uint4 *>(o + 8 * g) = v;
+                        }
+                    } else {
+                        float *o = static_cast<float *>(p.out) + (int64_t)sp * p.split_stride + (int64_t)row * p.out_ld + col0;
 #pragma unroll
-                    for (int g = 0; g < 8; g++) {
-                        if (col0 + 4 * g >= p.n_total) break;
-                        *reinterpret_cast<uint4 *>(o + 4 * g) = make_uint4(r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]);
+                        for (int g = 0; g < 8; g++) {
+                            if (col0 + 4 * g >= p.n_total) break;
+                            *reinterpret_cast<uint4 *>(o + 4 * g) = make_uint4(r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]);
+                        }
                     }
                 }
             }
@@ -354,12 +381,15 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode>::kThreads, 1)
     } else if (kFused && warp >= 8) {
       if constexpr (kFused) {
         // ---------------- dequantization producer ----------------
-        // One quantization block (64 consecutive k of one row of W) per thread
-        // per stage: forward stages hold BN rows x 64 columns of W, input-
-        // gradient stages hold 64 rows x BN columns (BN / 64 blocks per row).
-        // The block constant of the next stage is fetched one stage ahead.
+        // A stage holds BN quantization blocks (64 consecutive k of one row of
+        // W): forward stages are BN rows x 64 columns of W, input-gradient
+        // stages are 64 rows x BN columns.  kTPB threads share a block, each
+        // expanding 8 / kTPB words of 8 codes.  The block constant of the next
+        // stage is fetched one stage ahead.
+        constexpr int TPB = Cfg::kTPB;
+        constexpr int WPT = 8 / TPB;   // words per thread
         const int dt = (warp - 8) * 32 + lane;
-        static_assert(32 * Cfg::kDeqWarps == BN, "one block per thread per stage");
+        const int blk = dt / TPB, part = dt % TPB;
         const float mu = *p.mean;
         uint32_t it = 0;
         for (int t = blockIdx.x; t < num_tiles && !*vabort; t += gridDim.x) {
@@ -367,37 +397,34 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode>::kThreads, 1)
             decode(t, mt, nt, sp);
             stages_of(sp, kb0, nmain);
             const int nst = nmain + (sp == 0 ? p.k_stages_lora : 0);
-            // block (row, column block) of this thread at main stage ks
             auto block_of = [&](int ks, int64_t &n, int64_t &kb) {
                 if (kBMode == kBNf4K) {
-                    n = (int64_t)nt * BN + dt;
+                    n = (int64_t)nt * BN + blk;
                     kb = kb0 + ks;
                 } else {
-                    n = (int64_t)(kb0 + ks) * 64 + (dt & 63);
-                    kb = (int64_t)nt * (BN / 64) + (dt >> 6);
+                    n = (int64_t)(kb0 + ks) * 64 + (blk & 63);
+                    kb = (int64_t)nt * (BN / 64) + (blk >> 6);
                 }
             };
-            int64_t n, kb;
-            block_of(0, n, kb);
-            float c1p = nmain > 0 ? block_scale(p, n, kb, mu) : 0.0f;
+            auto load_raw = [&](int ks, uint8_t &e, float &c2) -> bool {
+                int64_t n, kb;
+                block_of(ks, n, kb);
+                if (n >= p.wrows || kb >= p.kblocks) return false;
+                const int64_t b = n * p.kblocks + kb;
+                e = p.code2[b];
+                c2 = p.c2[b >> 8];
+                return true;
+            };
+            uint8_t e0 = 0;
+            float c20 = 0.0f;
+            float c1p = (nmain > 0 && load_raw(0, e0, c20)) ? block_scale_raw(e0, c20, mu) : 0.0f;
             bool ok = true;
             for (int ks = 0; ks < nst; ks++, it++) {
                 const int s = it % S;
                 const uint32_t use = it / S;
-                // prefetch the next stage's block constant (raw bytes only)
                 uint8_t e_next = 0;
                 float c2_next = 0.0f;
-                bool have_next = false;
-                if (ks + 1 < nmain) {
-                    int64_t n1, kb1;
-                    block_of(ks + 1, n1, kb1);
-                    if (n1 < p.wrows && kb1 < p.kblocks) {
-                        const int64_t b = n1 * p.kblocks + kb1;
-                        e_next = p.code2[b];
-                        c2_next = p.c2[b >> 8];
-                        have_next = true;
-                    }
-                }
+                const bool have_next = ks + 1 < nmain && load_raw(ks + 1, e_next, c2_next);
                 if (!mbar_wait_bounded(&full_a[s], use & 1, p.timeout_ns)) {
                     record_timeout(p, abort_flag);
                     ok = false;
@@ -406,28 +433,40 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode>::kThreads, 1)
                 if (ks < nmain) {
                     const uint8_t *pb = sP(s);
                     uint8_t *bb = sB(s);
+                    uint32_t words[WPT];
+                    int r, dst_chunk0;
+                    uint8_t *dst;
                     if (kBMode == kBNf4K) {
-                        const int nl = dt;
-                        const int sw = (nl >> 2) & 1;   // 32-byte swizzle of the packed tile
-                        const uint4 lo = *reinterpret_cast<const uint4 *>(pb + nl * 32 + (sw << 4));
-                        const uint4 hi = *reinterpret_cast<const uint4 *>(pb + nl * 32 + ((sw ^ 1) << 4));
-                        const uint32_t words[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-                        uint8_t *dst = bb + nl * 128;
+                        // packed tile [BN rows][32 B], 32-byte swizzle: chunk h at h ^ ((row >> 2) & 1)
+                        r = blk;
+                        const int sw = (r >> 2) & 1;
 #pragma unroll
-                        for (int j = 0; j < 8; j++)
-                            *reinterpret_cast<uint4 *>(dst + ((j ^ (nl & 7)) << 4)) = expand8(words[j], lut, c1p);
+                        for (int h = 0; h < 2 / TPB; h++) {
+                            const int chunk = part * (2 / TPB) + h;
+                            const uint4 v = *reinterpret_cast<const uint4 *>(pb + r * 32 + ((chunk ^ sw) << 4));
+                            words[4 * h + 0] = v.x; words[4 * h + 1] = v.y; words[4 * h + 2] = v.z; words[4 * h + 3] = v.w;
+                        }
+                        dst = bb + r * 128;
                     } else {
-                        const int r = dt & 63, c = dt >> 6;
-                        const uint4 lo = *reinterpret_cast<const uint4 *>(pb + r * 128 + (((2 * c) ^ (r & 7)) << 4));
-                        const uint4 hi = *reinterpret_cast<const uint4 *>(pb + r * 128 + (((2 * c + 1) ^ (r & 7)) << 4));
-                        const uint32_t words[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-                        uint8_t *dst = bb + c * 8192 + r * 128;
+                        // packed tile [64 rows][BN/2 B]: 128-byte swizzle (BN = 256) or
+                        // 64-byte swizzle (BN = 128) of its 16-byte chunks
+                        r = blk & 63;
+                        const int c = blk >> 6;
 #pragma unroll
-                        for (int j = 0; j < 8; j++)
-                            *reinterpret_cast<uint4 *>(dst + ((j ^ (r & 7)) << 4)) = expand8(words[j], lut, c1p);
+                        for (int h = 0; h < 2 / TPB; h++) {
+                            const int chunk = 2 * c + part * (2 / TPB) + h;
+                            const int pos = BN == 256 ? (chunk ^ (r & 7)) : (chunk ^ ((r >> 1) & 3));
+                            const uint4 v = *reinterpret_cast<const uint4 *>(pb + r * (BN / 2) + (pos << 4));
+                            words[4 * h + 0] = v.x; words[4 * h + 1] = v.y; words[4 * h + 2] = v.z; words[4 * h + 3] = v.w;
+                        }
+                        dst = bb + c * 8192 + r * 128;
                     }
+                    dst_chunk0 = part * WPT;
+#pragma unroll
+                    for (int j = 0; j < WPT; j++)
+                        *reinterpret_cast<uint4 *>(dst + (((dst_chunk0 + j) ^ (r & 7)) << 4)) = expand8(words[j], lut, c1p);
                     fence_proxy_async_smem();
-                    c1p = have_next ? __fmaf_rn(e4m3_to_float(e_next), c2_next, mu) : 0.0f;
+                    c1p = have_next ? block_scale_raw(e_next, c2_next, mu) : 0.0f;
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&full_b[s]);

@@ -72,12 +72,12 @@ qlora_status map_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint64_t
 
 // ---- GEMM launch ------------------------------------------------------------------
 
-template <int BN, int kBMode, int kEpi>
+template <int BN, int kBMode, int kEpi, int MT = 1>
 qlora_status launch_gemm(GemmParams &p, const DeviceInfo &dev, cudaStream_t s, int kind)
 {
-    using Cfg = GemmCfg<BN, kBMode>;
+    using Cfg = GemmCfg<BN, kBMode, MT>;
     static bool attr_done[64] = {};
-    auto kern = qgemm_kernel<BN, kBMode, kEpi>;
+    auto kern = qgemm_kernel<BN, kBMode, kEpi, MT>;
     if (!attr_done[dev.device]) {
         QLORA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes));
         attr_done[dev.device] = true;
@@ -283,20 +283,22 @@ extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const void *
 
     QLORA_TRY(run_h(pl, dev, X, A, scale, H_save, ws, s));
 
+    // fused forward: 256 tokens (two 128-row accumulators) x 128 output features per tile
+    constexpr int kFBN = 128, kFMT = 2;
     GemmParams p{};
-    QLORA_TRY(map_bf16(&p.tm_a, X, pl.K, M, pl.K, 64, 128));
-    QLORA_TRY(make_map(&p.tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->packed, pl.K / 2, pl.N, pl.K / 2, 32, 256,
+    QLORA_TRY(map_bf16(&p.tm_a, X, pl.K, M, pl.K, 64, 128 * kFMT));
+    QLORA_TRY(make_map(&p.tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->packed, pl.K / 2, pl.N, pl.K / 2, 32, kFBN,
                        CU_TENSOR_MAP_SWIZZLE_32B));
-    QLORA_TRY(map_bf16(&p.tm_a2, ws + pl.off_h2, r, M, 2 * r, 64, 128));       // hi half of H
-    QLORA_TRY(map_bf16(&p.tm_b2, B, r, pl.N, r, 64, 256));
+    QLORA_TRY(map_bf16(&p.tm_a2, ws + pl.off_h2, r, M, 2 * r, 64, 128 * kFMT));   // hi half of H
+    QLORA_TRY(map_bf16(&p.tm_b2, B, r, pl.N, r, 64, kFBN));
     p.code2 = w->code2;
     p.c2 = w->c2;
     p.mean = w->mean;
     p.kblocks = pl.K / 64;
     p.wrows = pl.N;
     for (int i = 0; i < 16; i++) p.q[i] = w->codebook[i];
-    p.m_tiles = ceil_div(M, 128);
-    p.n_tiles = ceil_div(pl.N, 256);
+    p.m_tiles = ceil_div(M, 128 * kFMT);
+    p.n_tiles = ceil_div(pl.N, kFBN);
     p.splits = 1;
     p.k_stages_total = (int)(pl.K / 64);
     p.k_stages_split = p.k_stages_total;
@@ -305,8 +307,8 @@ extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const void *
     p.out_ld = pl.N;
     p.m_total = (int)M;
     p.n_total = (int)pl.N;
-    if (y_dtype == QLORA_BF16) return launch_gemm<256, kBNf4K, kEpiBf16>(p, dev, s, QLORA_KERNEL_FWD_FUSED);
-    return launch_gemm<256, kBNf4K, kEpiF32>(p, dev, s, QLORA_KERNEL_FWD_FUSED);
+    if (y_dtype == QLORA_BF16) return launch_gemm<kFBN, kBNf4K, kEpiBf16, kFMT>(p, dev, s, QLORA_KERNEL_FWD_FUSED);
+    return launch_gemm<kFBN, kBNf4K, kEpiF32, kFMT>(p, dev, s, QLORA_KERNEL_FWD_FUSED);
 }
 
 extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *X, const void *dY, int64_t M,
@@ -377,20 +379,22 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *
 
     // dX = dY W' + bf16(G) A  (fused transposed dequant-GEMM)
     if (dX) {
+        // fused input gradient: 256 tokens x 128 input features per tile
+        constexpr int kBBN = 128, kBMT = 2;
         GemmParams p{};
-        QLORA_TRY(map_bf16(&p.tm_a, dY, N, M, N, 64, 128));
-        QLORA_TRY(make_map(&p.tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->packed, K / 2, N, K / 2, 128, 64,
-                           CU_TENSOR_MAP_SWIZZLE_128B));
-        QLORA_TRY(map_bf16(&p.tm_a2, G2, r, M, 2 * r, 64, 128));   // hi half of G
-        QLORA_TRY(map_bf16(&p.tm_b2, A, K, r, K, 64, 64));         // A[j][k]: MN-major operand
+        QLORA_TRY(map_bf16(&p.tm_a, dY, N, M, N, 64, 128 * kBMT));
+        QLORA_TRY(make_map(&p.tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->packed, K / 2, N, K / 2, kBBN / 2, 64,
+                           kBBN == 256 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B));
+        QLORA_TRY(map_bf16(&p.tm_a2, G2, r, M, 2 * r, 64, 128 * kBMT));   // hi half of G
+        QLORA_TRY(map_bf16(&p.tm_b2, A, K, r, K, 64, 64));                // A[j][k]: MN-major operand
         p.code2 = w->code2;
         p.c2 = w->c2;
         p.mean = w->mean;
         p.kblocks = K / 64;
         p.wrows = N;
         for (int i = 0; i < 16; i++) p.q[i] = w->codebook[i];
-        p.m_tiles = ceil_div(M, 128);
-        p.n_tiles = ceil_div(K, 256);
+        p.m_tiles = ceil_div(M, 128 * kBMT);
+        p.n_tiles = ceil_div(K, kBBN);
         p.splits = 1;
         p.k_stages_total = ceil_div(N, 64);
         p.k_stages_split = p.k_stages_total;
@@ -400,9 +404,9 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *
         p.m_total = (int)M;
         p.n_total = (int)K;
         if (dx_dtype == QLORA_BF16)
-            QLORA_TRY((launch_gemm<256, kBNf4MN, kEpiBf16>(p, dev, s, QLORA_KERNEL_BWD_FUSED)));
+            QLORA_TRY((launch_gemm<kBBN, kBNf4MN, kEpiBf16, kBMT>(p, dev, s, QLORA_KERNEL_BWD_FUSED)));
         else
-            QLORA_TRY((launch_gemm<256, kBNf4MN, kEpiF32>(p, dev, s, QLORA_KERNEL_BWD_FUSED)));
+            QLORA_TRY((launch_gemm<kBBN, kBNf4MN, kEpiF32, kBMT>(p, dev, s, QLORA_KERNEL_BWD_FUSED)));
     }
 
     // dA = G^T X  (rows j of [G_hi | G_lo], contraction over tokens)
