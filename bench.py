@@ -282,6 +282,8 @@ def run_codec(args, q, torch, dev, peaks, peak_src):
     replayed as one CUDA graph per step."""
     import synthetic
     shapes = [(N, K) for _ in range(synthetic.LLAMA7B_LAYERS) for _, N, K in synthetic.LLAMA7B_LINEARS]
+    if args.codec_tensors:
+        shapes = shapes[:args.codec_tensors]
     tensors = []
     for i, (N, K) in enumerate(shapes):
         W = synthetic.normal((N, K), 0.02, 50_000 + i, torch.bfloat16, dev)
@@ -447,6 +449,9 @@ def main():
     ap.add_argument("--linears", default="llama7b",
                     help="llama7b (the seven linears of one layer) or NxK for one linear (profiling runs)")
     ap.add_argument("--tokens", type=int, default=TOKENS)
+    ap.add_argument("--codec-tensors", type=int, default=0,
+                    help="limit the codec round trip to the first N LLaMA-7B tensors (profiling runs)")
+    ap.add_argument("--codec-only", action="store_true", help="run only the codec round trip (profiling runs)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank = int(os.environ.get("RANK", "0"))
@@ -467,7 +472,13 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        line = run_ours(args, rank, world, local_rank)
+        if args.codec_only:
+            import bit_nf4_quantized_16_b200 as q
+            torch.cuda.set_device(local_rank)
+            peaks, src = load_peaks()
+            line = {"impl": "ours", "codec": run_codec(args, q, torch, torch.device("cuda", local_rank), peaks, src)}
+        else:
+            line = run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:
             dist.barrier()
