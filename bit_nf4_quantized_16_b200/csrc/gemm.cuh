@@ -415,16 +415,26 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode, MT>::kThreads, 1)
                 c2 = p.c2[b >> 8];
                 return true;
             };
-            uint8_t e0 = 0;
-            float c20 = 0.0f;
-            float c1p = (nmain > 0 && load_raw(0, e0, c20)) ? block_scale_raw(e0, c20, mu) : 0.0f;
+            // block constants of the next kPre main stages, fetched ahead in a
+            // register queue (q[0] = current stage)
+            constexpr int kPre = 4;
+            uint8_t qe[kPre];
+            float qc2[kPre];
+            bool qok[kPre];
+#pragma unroll
+            for (int i = 0; i < kPre; i++) qok[i] = i < nmain && load_raw(i, qe[i], qc2[i]);
             bool ok = true;
             for (int ks = 0; ks < nst; ks++, it++) {
                 const int s = it % S;
                 const uint32_t use = it / S;
-                uint8_t e_next = 0;
-                float c2_next = 0.0f;
-                const bool have_next = ks + 1 < nmain && load_raw(ks + 1, e_next, c2_next);
+                const float c1p = qok[0] ? block_scale_raw(qe[0], qc2[0], mu) : 0.0f;
+#pragma unroll
+                for (int i = 0; i + 1 < kPre; i++) {
+                    qe[i] = qe[i + 1];
+                    qc2[i] = qc2[i + 1];
+                    qok[i] = qok[i + 1];
+                }
+                qok[kPre - 1] = ks + kPre < nmain && load_raw(ks + kPre, qe[kPre - 1], qc2[kPre - 1]);
                 if (!mbar_wait_bounded(&full_a[s], use & 1, p.timeout_ns)) {
                     record_timeout(p, abort_flag);
                     ok = false;
@@ -466,7 +476,6 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode, MT>::kThreads, 1)
                     for (int j = 0; j < WPT; j++)
                         *reinterpret_cast<uint4 *>(dst + (((dst_chunk0 + j) ^ (r & 7)) << 4)) = expand8(words[j], lut, c1p);
                     fence_proxy_async_smem();
-                    c1p = have_next ? block_scale_raw(e_next, c2_next, mu) : 0.0f;
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&full_b[s]);
