@@ -19,8 +19,11 @@
 #include <math.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "exact_mean.cuh"
+#include "nf4_expand.cuh"
 
 namespace qlora {
 
@@ -56,20 +59,6 @@ __device__ __forceinline__ uint32_t ld_stream_u32(const void *p)
     return v;
 }
 
-// Two binary32 values rounded to nearest-even bf16, lo in bits 0-15.
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
-{
-    uint32_t d;
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
-    return d;
-}
-
-__device__ __forceinline__ float e4m3_to_float(uint8_t code)
-{
-    __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)code, __NV_E4M3);
-    return __half2float(__half(h));
-}
-
 // ---- pass 1: absmax, codes, exact-mean buckets -----------------------------------
 
 struct QuantParams {
@@ -81,7 +70,7 @@ struct QuantParams {
     float *mean_out;           // 1 float
     int64_t nwords;            // numel / 8: one word = 8 codes = 32 bits
     int64_t nblocks;
-    uint32_t mkey[15];         // keys of the round-down midpoints, ascending
+    uint32_t lut[4096];        // code lookup table (built on the host, see code_lut_entry)
 };
 
 // Code lookup on the top 12 bits of the key of n = x * (1/c1).  The 15
@@ -92,23 +81,8 @@ struct QuantParams {
 // host checks this), so one table entry plus one carry decides the code:
 //   entry = (midpoints below the interval) << 20, plus 2^20-1 - low20(key_m)
 //   if midpoint m lies inside the interval;  code = (entry + low20(key)) >> 20.
-__device__ __forceinline__ void build_code_lut(uint32_t *lut, const uint32_t (&mkey)[15])
-{
-    for (int idx = threadIdx.x; idx < 4096; idx += blockDim.x) {
-        uint32_t lo = (uint32_t)idx << 20;
-        uint32_t below = 0, inc = 0;
-#pragma unroll
-        for (int j = 0; j < 15; j++) {
-            uint32_t k = mkey[j];
-            if (k < lo)
-                below++;
-            else if ((k >> 20) == (uint32_t)idx)
-                inc = 0xFFFFFu - (k & 0xFFFFFu);
-        }
-        lut[idx] = (below << 20) + inc;
-    }
-}
-
+// The table depends only on the codebook; the host builds it and passes it in
+// the kernel parameters.
 __device__ __forceinline__ uint32_t code_of(const uint32_t *lut, float x, float r)
 {
     uint32_t k = sortable_key(__fmul_rn(x, r));
@@ -116,12 +90,14 @@ __device__ __forceinline__ uint32_t code_of(const uint32_t *lut, float x, float 
 }
 
 template <bool kF32In>
-__global__ void __launch_bounds__(kThreads) quantize_blocks_kernel(QuantParams p)
+__global__ void __launch_bounds__(kThreads) quantize_blocks_kernel(const __grid_constant__ QuantParams p)
 {
-    __shared__ uint32_t lut[4096];
+    __shared__ uint4 lut4[1024];
     __shared__ unsigned long long s_acc[256];
     __shared__ bool s_last;
-    build_code_lut(lut, p.mkey);
+    uint32_t *lut = reinterpret_cast<uint32_t *>(lut4);
+    for (int i = threadIdx.x; i < 1024; i += kThreads)
+        lut4[i] = make_uint4(p.lut[4 * i], p.lut[4 * i + 1], p.lut[4 * i + 2], p.lut[4 * i + 3]);
     s_acc[threadIdx.x] = 0;
     __syncthreads();
 
@@ -304,21 +280,14 @@ __global__ void __launch_bounds__(kThreads) dequantize_kernel(DeqParams p)
             if (w < p.nwords) {
                 word[u] = ld_stream_u32(p.packed + 4 * w);
                 int64_t b = w >> 3;
-                c1p[u] = __fmaf_rn(e4m3_to_float(p.code2[b]), p.c2[b / QLORA_GROUP], mu);
+                c1p[u] = nf4::block_scale(p.code2[b], p.c2[b / QLORA_GROUP], mu);
             }
         }
 #pragma unroll
         for (int u = 0; u < kUnroll; u++) {
             int64_t w = w0 + u * stride;
             if (w >= p.nwords) continue;
-            uint32_t o[4];
-#pragma unroll
-            for (int i = 0; i < 4; i++) {
-                float lo = __fmul_rn(lut[(word[u] >> (8 * i)) & 15u], c1p[u]);
-                float hi = __fmul_rn(lut[(word[u] >> (8 * i + 4)) & 15u], c1p[u]);
-                o[i] = pack_bf16x2(lo, hi);
-            }
-            *reinterpret_cast<uint4 *>(p.out + 8 * w) = make_uint4(o[0], o[1], o[2], o[3]);
+            *reinterpret_cast<uint4 *>(p.out + 8 * w) = nf4::expand8(word[u], lut, c1p[u]);
         }
     }
 }
@@ -354,6 +323,35 @@ qlora_status midpoint_keys(const float q[16], uint32_t out[15])
         if (j > 0 && (out[j] >> 20) == (out[j - 1] >> 20)) return QLORA_ERR_UNSUPPORTED;
     }
     return QLORA_OK;
+}
+
+// Table entry for keys whose top 12 bits are `idx` (see the kernel comment).
+uint32_t code_lut_entry(uint32_t idx, const uint32_t mkey[15])
+{
+    uint32_t lo = idx << 20, below = 0, inc = 0;
+    for (int j = 0; j < 15; j++) {
+        if (mkey[j] < lo)
+            below++;
+        else if ((mkey[j] >> 20) == idx)
+            inc = 0xFFFFFu - (mkey[j] & 0xFFFFFu);
+    }
+    return (below << 20) + inc;
+}
+
+// The code table of a codebook, cached for the last codebook seen.
+void code_lut(const uint32_t mkey[15], uint32_t out[4096])
+{
+    static std::mutex mu;
+    static uint32_t cached_key[15];
+    static uint32_t cached[4096];
+    static bool valid = false;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!valid || memcmp(cached_key, mkey, sizeof(cached_key)) != 0) {
+        for (uint32_t i = 0; i < 4096; i++) cached[i] = code_lut_entry(i, mkey);
+        memcpy(cached_key, mkey, sizeof(cached_key));
+        valid = true;
+    }
+    memcpy(out, cached, sizeof(cached));
 }
 
 int grid_for(int64_t work_items, int items_per_cta, int max_ctas)
@@ -407,7 +405,7 @@ extern "C" qlora_status qlora_quantize_nf4_dq(const void *W, qlora_dtype w_dtype
     qp.mean_out = out->mean;
     qp.nwords = numel / 8;
     qp.nblocks = nblocks;
-    memcpy(qp.mkey, mkey, sizeof(mkey));
+    code_lut(mkey, qp.lut);
     int grid = grid_for(qp.nwords, kThreads * kUnroll, dev.sms * 4);
     {
         LaunchScope ls(QLORA_KERNEL_QUANTIZE, s);

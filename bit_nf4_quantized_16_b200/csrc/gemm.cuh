@@ -37,6 +37,7 @@
 #include <cuda_fp8.h>
 #include <stdint.h>
 
+#include "nf4_expand.cuh"
 #include "sm100.cuh"
 
 namespace qlora {
@@ -95,49 +96,9 @@ struct GemmCfg {
 
 namespace gemm_detail {
 
-__device__ __forceinline__ float e4m3_to_float(uint8_t code)
-{
-    __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)code, __NV_E4M3);
-    return __half2float(__half(h));
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
-{
-    uint32_t d;
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
-    return d;
-}
-
-// (a, b) * (s, s), each lane rounded to nearest-even (packed f32x2 multiply)
-__device__ __forceinline__ void mul2(float a, float b, float s, float &ra, float &rb)
-{
-    uint64_t x, y;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a), "f"(b));
-    uint64_t ss;
-    asm("mov.b64 %0, {%1, %1};" : "=l"(ss) : "f"(s));
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(y) : "l"(x), "l"(ss));
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(ra), "=f"(rb) : "l"(y));
-}
-
-// 8 consecutive codes (one 32-bit word, element 0 in bits 0-3) -> 8 bf16 in a
-// 16-byte vector: w = bf16(RN32(q[code] * c1p)), the stand-alone dequantizer's
-// arithmetic.
-__device__ __forceinline__ uint4 expand8(uint32_t word, const float *lut, float c1p)
-{
-    uint32_t o[4];
-#pragma unroll
-    for (int i = 0; i < 4; i++) {
-        float lo, hi;
-        mul2(lut[(word >> (8 * i)) & 15u], lut[(word >> (8 * i + 4)) & 15u], c1p, lo, hi);
-        o[i] = pack_bf16x2(lo, hi);
-    }
-    return make_uint4(o[0], o[1], o[2], o[3]);
-}
-
-__device__ __forceinline__ float block_scale_raw(uint8_t e, float c2, float mu)
-{
-    return __fmaf_rn(e4m3_to_float(e), c2, mu);
-}
+using nf4::block_scale;
+using nf4::expand8;
+using nf4::pack_bf16x2;
 
 __device__ __forceinline__ void record_timeout(const GemmParams &p, int *abort_flag)
 {
@@ -427,7 +388,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode, MT>::kThreads, 1)
             for (int ks = 0; ks < nst; ks++, it++) {
                 const int s = it % S;
                 const uint32_t use = it / S;
-                const float c1p = qok[0] ? block_scale_raw(qe[0], qc2[0], mu) : 0.0f;
+                const float c1p = qok[0] ? block_scale(qe[0], qc2[0], mu) : 0.0f;
 #pragma unroll
                 for (int i = 0; i + 1 < kPre; i++) {
                     qe[i] = qe[i + 1];
