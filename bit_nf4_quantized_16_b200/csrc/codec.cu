@@ -19,8 +19,6 @@
 #include <math.h>
 #include <string.h>
 
-#include <mutex>
-
 #include "common.cuh"
 #include "exact_mean.cuh"
 #include "nf4_expand.cuh"
@@ -30,7 +28,8 @@ namespace qlora {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kUnroll = 4;
+constexpr int kUnroll = 4;      // words per thread in flight (quantize)
+constexpr int kDeqUnroll = 8;   // words per thread in flight (dequantize)
 
 // ---- small device helpers ----------------------------------------------------
 
@@ -68,9 +67,9 @@ struct QuantParams {
     unsigned long long *acc;   // 256 buckets (workspace, zero on entry)
     unsigned int *ticket;      // CTA arrival counter (workspace, zero on entry)
     float *mean_out;           // 1 float
-    int64_t nwords;            // numel / 8: one word = 8 codes = 32 bits
+    uint32_t nwords;           // numel / 8: one word = 8 codes = 32 bits
     int64_t nblocks;
-    uint32_t lut[4096];        // code lookup table (built on the host, see code_lut_entry)
+    uint32_t mkey[15];         // keys of the round-down midpoints, ascending
 };
 
 // Code lookup on the top 12 bits of the key of n = x * (1/c1).  The 15
@@ -81,40 +80,70 @@ struct QuantParams {
 // host checks this), so one table entry plus one carry decides the code:
 //   entry = (midpoints below the interval) << 20, plus 2^20-1 - low20(key_m)
 //   if midpoint m lies inside the interval;  code = (entry + low20(key)) >> 20.
-// The table depends only on the codebook; the host builds it and passes it in
-// the kernel parameters.
-__device__ __forceinline__ uint32_t code_of(const uint32_t *lut, float x, float r)
+// Every CTA builds the table once: thread t fills entries 16t..16t+15,
+// walking the sorted midpoint keys once.
+__device__ __forceinline__ void build_code_lut(uint32_t *lut, const uint32_t *mkey_smem)
 {
-    uint32_t k = sortable_key(__fmul_rn(x, r));
-    return (lut[k >> 20] + (k & 0xFFFFFu)) >> 20;
+    const uint32_t first = threadIdx.x * 16u;
+    uint32_t j = 0;
+    while (j < 15 && mkey_smem[j] < (first << 20)) j++;
+    uint32_t e[16];
+#pragma unroll
+    for (int i = 0; i < 16; i++) {
+        const uint32_t idx = first + i;
+        while (j < 15 && mkey_smem[j] < (idx << 20)) j++;
+        uint32_t inc = 0;
+        if (j < 15 && (mkey_smem[j] >> 20) == idx) inc = 0xFFFFFu - (mkey_smem[j] & 0xFFFFFu);
+        e[i] = (j << 20) + inc;
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(lut + first);
+#pragma unroll
+    for (int i = 0; i < 4; i++) dst[i] = make_uint4(e[4 * i], e[4 * i + 1], e[4 * i + 2], e[4 * i + 3]);
+}
+
+// Code of element x of a block with reciprocal scale r, already shifted to
+// nibble position 4*i: ((entry + low20(key)) >> 20) << 4i.
+template <int I>
+__device__ __forceinline__ uint32_t code_at(const uint32_t *lut, float n)
+{
+    uint32_t k = sortable_key(n);
+    uint32_t v = lut[k >> 20] + (k & 0xFFFFFu);
+    if constexpr (4 * I <= 20)
+        return (v >> (20 - 4 * I)) & (0xFu << (4 * I));
+    else
+        return (v << (4 * I - 20)) & (0xFu << (4 * I));
 }
 
 template <bool kF32In>
 __global__ void __launch_bounds__(kThreads) quantize_blocks_kernel(const __grid_constant__ QuantParams p)
 {
-    __shared__ uint4 lut4[1024];
+    static_assert(kThreads * 16 == 4096, "one 16-entry slice of the code table per thread");
+    __shared__ __align__(16) uint32_t lut[4096];
     __shared__ unsigned long long s_acc[256];
+    __shared__ uint32_t s_mkey[16];
     __shared__ bool s_last;
-    uint32_t *lut = reinterpret_cast<uint32_t *>(lut4);
-    for (int i = threadIdx.x; i < 1024; i += kThreads)
-        lut4[i] = make_uint4(p.lut[4 * i], p.lut[4 * i + 1], p.lut[4 * i + 2], p.lut[4 * i + 3]);
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int j = 0; j < 15; j++) s_mkey[j] = p.mkey[j];
+    }
     s_acc[threadIdx.x] = 0;
     __syncthreads();
+    build_code_lut(lut, s_mkey);
+    __syncthreads();
 
-    const int lane = threadIdx.x & 31;
-    const int64_t stride = (int64_t)gridDim.x * kThreads;
-    for (int64_t base = (int64_t)blockIdx.x * kThreads + (threadIdx.x & ~31); base < p.nwords;
-         base += stride * kUnroll) {
+    const uint32_t lane = threadIdx.x & 31;
+    const uint32_t stride = gridDim.x * kThreads;
+    for (uint32_t base = blockIdx.x * kThreads + (threadIdx.x & ~31u); base < p.nwords; base += stride * kUnroll) {
         float x[kUnroll][8];
         bool act[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; u++) {
-            int64_t w = base + lane + u * stride;
+            const uint32_t w = base + lane + u * stride;
             act[u] = w < p.nwords;
             if (kF32In) {
                 uint4 a = make_uint4(0, 0, 0, 0), b = a;
                 if (act[u]) {
-                    const float *src = static_cast<const float *>(p.W) + 8 * w;
+                    const float *src = static_cast<const float *>(p.W) + 8ull * w;
                     a = ld_stream_v4(src);
                     b = ld_stream_v4(src + 4);
                 }
@@ -124,7 +153,7 @@ __global__ void __launch_bounds__(kThreads) quantize_blocks_kernel(const __grid_
                 x[u][6] = __uint_as_float(b.z); x[u][7] = __uint_as_float(b.w);
             } else {
                 uint4 a = make_uint4(0, 0, 0, 0);
-                if (act[u]) a = ld_stream_v4(static_cast<const __nv_bfloat16 *>(p.W) + 8 * w);
+                if (act[u]) a = ld_stream_v4(static_cast<const __nv_bfloat16 *>(p.W) + 8ull * w);
                 const uint32_t v[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
                 for (int i = 0; i < 4; i++) {
@@ -133,52 +162,60 @@ __global__ void __launch_bounds__(kThreads) quantize_blocks_kernel(const __grid_
                 }
             }
         }
+        // block absmax: the 8 lanes of one block reduce together
         float c1v[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; u++) {
             float m = 0.0f;
 #pragma unroll
             for (int i = 0; i < 8; i++) m = fmaxf(m, fabsf(x[u][i]));
-            // the 8 lanes of one block reduce together
             m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
             m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
             m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
             c1v[u] = m;
-            // zero block (absmax below the smallest normal): r = 0 sends every
-            // element to n = +-0, whose code is the codebook's zero
-            const float r = m < 1.17549435e-38f ? 0.0f : __frcp_rn(m);
-            uint32_t word = 0;
-#pragma unroll
-            for (int i = 0; i < 8; i++) word |= code_of(lut, x[u][i], r) << (4 * i);
-            if (act[u]) reinterpret_cast<uint32_t *>(p.packed)[base + lane + u * stride] = word;
         }
         // Gather the warp's 4*kUnroll block constants into lanes 0..4*kUnroll-1
-        // (lane 4u+g takes block g of unrolled step u), store them, and add
-        // them to the exponent buckets with one shared atomic per distinct
-        // exponent instead of one per block.
+        // (lane 4u+g takes block g of unrolled step u): one reciprocal per lane,
+        // the stores of c1, and the exponent buckets of the exact mean.
         float cv = 0.0f;
         bool ca = false;
 #pragma unroll
         for (int u = 0; u < kUnroll; u++) {
-            float t = __shfl_sync(0xffffffffu, c1v[u], (lane & 3) * 8);
-            bool a = __shfl_sync(0xffffffffu, (int)act[u], (lane & 3) * 8) != 0;
-            if ((lane >> 2) == u) {
+            const float t = __shfl_sync(0xffffffffu, c1v[u], (lane & 3) * 8);
+            const bool a = __shfl_sync(0xffffffffu, (int)act[u], (lane & 3) * 8) != 0;
+            if ((lane >> 2) == (uint32_t)u) {
                 cv = t;
                 ca = a;
             }
         }
+        // zero block (absmax below the smallest normal): r = 0 sends every
+        // element to n = +-0, whose code is the codebook's zero
+        const float rv = cv < 1.17549435e-38f ? 0.0f : __frcp_rn(cv);
         if (lane < 4 * kUnroll && ca) p.c1[(base + 8 * (lane & 3) + (lane >> 2) * stride) >> 3] = cv;
+        // codes
+#pragma unroll
+        for (int u = 0; u < kUnroll; u++) {
+            const float r = __shfl_sync(0xffffffffu, rv, 4 * u + (lane >> 3));
+            float n[8];
+#pragma unroll
+            for (int i = 0; i < 8; i += 2) nf4::mul2(x[u][i], x[u][i + 1], r, n[i], n[i + 1]);
+            const uint32_t word = code_at<0>(lut, n[0]) | code_at<1>(lut, n[1]) | code_at<2>(lut, n[2]) |
+                                  code_at<3>(lut, n[3]) | code_at<4>(lut, n[4]) | code_at<5>(lut, n[5]) |
+                                  code_at<6>(lut, n[6]) | code_at<7>(lut, n[7]);
+            if (act[u]) reinterpret_cast<uint32_t *>(p.packed)[base + lane + u * stride] = word;
+        }
+        // exact-mean buckets: one shared atomic per distinct exponent
         uint32_t bucket, sig;
         exact_mean_split(__float_as_uint(cv), &bucket, &sig);
         bool pending = lane < 4 * kUnroll && ca;
         for (;;) {
-            unsigned pend = __ballot_sync(0xffffffffu, pending);
+            const unsigned pend = __ballot_sync(0xffffffffu, pending);
             if (!pend) break;
-            int leader = __ffs(pend) - 1;
-            uint32_t lb = __shfl_sync(0xffffffffu, bucket, leader);
-            bool mine = pending && bucket == lb;
-            uint32_t sum = __reduce_add_sync(0xffffffffu, mine ? sig : 0u);   // < 16 * 2^24
-            if (lane == leader) atomicAdd(&s_acc[lb], (unsigned long long)sum);
+            const int leader = __ffs(pend) - 1;
+            const uint32_t lb = __shfl_sync(0xffffffffu, bucket, leader);
+            const bool mine = pending && bucket == lb;
+            const uint32_t sum = __reduce_add_sync(0xffffffffu, mine ? sig : 0u);   // < 16 * 2^24
+            if ((int)lane == leader) atomicAdd(&s_acc[lb], (unsigned long long)sum);
             pending = pending && !mine;
         }
     }
@@ -269,11 +306,11 @@ __global__ void __launch_bounds__(kThreads) dequantize_kernel(DeqParams p)
     __syncthreads();
     const float mu = *p.mean;
     const int64_t stride = (int64_t)gridDim.x * kThreads;
-    for (int64_t w0 = (int64_t)blockIdx.x * kThreads + threadIdx.x; w0 < p.nwords; w0 += stride * kUnroll) {
-        uint32_t word[kUnroll];
-        float c1p[kUnroll];
+    for (int64_t w0 = (int64_t)blockIdx.x * kThreads + threadIdx.x; w0 < p.nwords; w0 += stride * kDeqUnroll) {
+        uint32_t word[kDeqUnroll];
+        float c1p[kDeqUnroll];
 #pragma unroll
-        for (int u = 0; u < kUnroll; u++) {
+        for (int u = 0; u < kDeqUnroll; u++) {
             int64_t w = w0 + u * stride;
             word[u] = 0;
             c1p[u] = 0.0f;
@@ -284,7 +321,7 @@ __global__ void __launch_bounds__(kThreads) dequantize_kernel(DeqParams p)
             }
         }
 #pragma unroll
-        for (int u = 0; u < kUnroll; u++) {
+        for (int u = 0; u < kDeqUnroll; u++) {
             int64_t w = w0 + u * stride;
             if (w >= p.nwords) continue;
             *reinterpret_cast<uint4 *>(p.out + 8 * w) = nf4::expand8(word[u], lut, c1p[u]);
@@ -325,35 +362,6 @@ qlora_status midpoint_keys(const float q[16], uint32_t out[15])
     return QLORA_OK;
 }
 
-// Table entry for keys whose top 12 bits are `idx` (see the kernel comment).
-uint32_t code_lut_entry(uint32_t idx, const uint32_t mkey[15])
-{
-    uint32_t lo = idx << 20, below = 0, inc = 0;
-    for (int j = 0; j < 15; j++) {
-        if (mkey[j] < lo)
-            below++;
-        else if ((mkey[j] >> 20) == idx)
-            inc = 0xFFFFFu - (mkey[j] & 0xFFFFFu);
-    }
-    return (below << 20) + inc;
-}
-
-// The code table of a codebook, cached for the last codebook seen.
-void code_lut(const uint32_t mkey[15], uint32_t out[4096])
-{
-    static std::mutex mu;
-    static uint32_t cached_key[15];
-    static uint32_t cached[4096];
-    static bool valid = false;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!valid || memcmp(cached_key, mkey, sizeof(cached_key)) != 0) {
-        for (uint32_t i = 0; i < 4096; i++) cached[i] = code_lut_entry(i, mkey);
-        memcpy(cached_key, mkey, sizeof(cached_key));
-        valid = true;
-    }
-    memcpy(out, cached, sizeof(cached));
-}
-
 int grid_for(int64_t work_items, int items_per_cta, int max_ctas)
 {
     int64_t g = (work_items + items_per_cta - 1) / items_per_cta;
@@ -385,6 +393,7 @@ extern "C" qlora_status qlora_quantize_nf4_dq(const void *W, qlora_dtype w_dtype
     QLORA_TRY(check_weight(out));
     if (!aligned16(W) || !aligned16(workspace)) return QLORA_ERR_ALIGNMENT;
     if (workspace_bytes < qlora_quantize_workspace_bytes(out->rows, out->cols)) return QLORA_ERR_WORKSPACE;
+    if (out->rows * out->cols / 8 >= ((int64_t)1 << 31)) return QLORA_ERR_SHAPE;   // 32-bit word indices
     uint32_t mkey[15];
     QLORA_TRY(midpoint_keys(out->codebook, mkey));
     DeviceInfo dev;
@@ -403,9 +412,9 @@ extern "C" qlora_status qlora_quantize_nf4_dq(const void *W, qlora_dtype w_dtype
     qp.ticket = reinterpret_cast<unsigned int *>(ws + 256 * sizeof(unsigned long long));
     qp.c1 = reinterpret_cast<float *>(ws + kAccBytes);
     qp.mean_out = out->mean;
-    qp.nwords = numel / 8;
+    qp.nwords = (uint32_t)(numel / 8);
     qp.nblocks = nblocks;
-    code_lut(mkey, qp.lut);
+    memcpy(qp.mkey, mkey, sizeof(mkey));
     int grid = grid_for(qp.nwords, kThreads * kUnroll, dev.sms * 4);
     {
         LaunchScope ls(QLORA_KERNEL_QUANTIZE, s);
@@ -448,7 +457,7 @@ extern "C" qlora_status qlora_dequantize_nf4_dq(const qlora_nf4_weight *w, void 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     {
         LaunchScope ls(QLORA_KERNEL_DEQUANTIZE, s);
-        dequantize_kernel<<<grid_for(p.nwords, kThreads * kUnroll, dev.sms * 8), kThreads, 0, s>>>(p);
+        dequantize_kernel<<<grid_for(p.nwords, kThreads * kDeqUnroll, dev.sms * 8), kThreads, 0, s>>>(p);
     }
     return launch_status();
 }
