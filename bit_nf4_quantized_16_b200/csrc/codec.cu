@@ -29,18 +29,9 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kUnroll = 4;      // words per thread in flight (quantize)
-constexpr int kDeqUnroll = 8;   // words per thread in flight (dequantize)
+constexpr int kDeqUnroll = 4;   // words per thread in flight (dequantize)
 
 // ---- small device helpers ----------------------------------------------------
-
-// Order-preserving map from binary32 to uint32: a < b (as floats, -0 < +0)
-// iff key(a) < key(b).
-__device__ __forceinline__ uint32_t sortable_key(float f)
-{
-    uint32_t b = __float_as_uint(f);
-    uint32_t s = (uint32_t)((int32_t)b >> 31);
-    return b ^ (s | 0x80000000u);
-}
 
 __device__ __forceinline__ uint4 ld_stream_v4(const void *p)
 {
@@ -72,46 +63,50 @@ struct QuantParams {
     uint32_t mkey[15];         // keys of the round-down midpoints, ascending
 };
 
-// Code lookup on the top 12 bits of the key of n = x * (1/c1).  The 15
-// midpoints between neighbouring codebook values are rounded down to binary32,
-// so "n > midpoint_j" holds exactly when n is nearer to value j+1 than to
-// value j (a tie stays with the lower index), and the code is the number of
-// midpoints below n.  Each 2^20-key interval holds at most one midpoint (the
-// host checks this), so one table entry plus one carry decides the code:
-//   entry = (midpoints below the interval) << 20, plus 2^20-1 - low20(key_m)
-//   if midpoint m lies inside the interval;  code = (entry + low20(key)) >> 20.
-// Every CTA builds the table once: thread t fills entries 16t..16t+15,
-// walking the sorted midpoint keys once.
+// Code lookup.  The 15 midpoints between neighbouring codebook values are
+// rounded down to binary32, so "n > midpoint_j" holds exactly when n is nearer
+// to value j+1 than to value j (a tie stays with the lower index), and the
+// code is the number of midpoints below n.
+// Keys: an order-preserving integer key of n has the same top 12 bits as a
+// 2^20-wide interval of keys; each such interval holds at most one midpoint
+// (the host checks this), so with
+//   E(j) = (midpoints below interval j) << 20, plus 2^20-1 - low20(key_m) if
+//          midpoint m lies inside interval j,
+// the code is (E(j) + low20(key)) >> 20 (the carry decides the one midpoint).
+// The kernel uses k = bits(n) with its low 20 bits flipped when n < 0: the
+// top 12 bits of k are the raw sign/exponent/3-bit index i of n, and the low
+// 20 bits of k equal those of the order-preserving key.  Entry i of the
+// table holds E(j(i)) - (i << 20), so that code = (table[i] + k) >> 20 with
+// no masking; every step except one logic op runs on the multiply-add pipe.
+// Every CTA builds the table once: thread t fills the entries of ordered
+// intervals j = 16t..16t+15, walking the sorted midpoint keys once.
 __device__ __forceinline__ void build_code_lut(uint32_t *lut, const uint32_t *mkey_smem)
 {
     const uint32_t first = threadIdx.x * 16u;
     uint32_t j = 0;
     while (j < 15 && mkey_smem[j] < (first << 20)) j++;
-    uint32_t e[16];
 #pragma unroll
-    for (int i = 0; i < 16; i++) {
-        const uint32_t idx = first + i;
+    for (int t = 0; t < 16; t++) {
+        const uint32_t idx = first + t;    // interval of the order-preserving key
         while (j < 15 && mkey_smem[j] < (idx << 20)) j++;
         uint32_t inc = 0;
         if (j < 15 && (mkey_smem[j] >> 20) == idx) inc = 0xFFFFFu - (mkey_smem[j] & 0xFFFFFu);
-        e[i] = (j << 20) + inc;
+        // raw index: positive numbers have key = bits | 2^31, negative ones ~bits
+        const uint32_t raw = idx >= 2048u ? idx - 2048u : 4095u - idx;
+        lut[raw] = (j << 20) + inc - (raw << 20);
     }
-    uint4 *dst = reinterpret_cast<uint4 *>(lut + first);
-#pragma unroll
-    for (int i = 0; i < 4; i++) dst[i] = make_uint4(e[4 * i], e[4 * i + 1], e[4 * i + 2], e[4 * i + 3]);
 }
 
-// Code of element x of a block with reciprocal scale r, already shifted to
-// nibble position 4*i: ((entry + low20(key)) >> 20) << 4i.
+// Code of n shifted to nibble position 4*I and added to acc.
 template <int I>
-__device__ __forceinline__ uint32_t code_at(const uint32_t *lut, float n)
+__device__ __forceinline__ uint32_t add_code(const uint32_t *lut, float n, uint32_t acc)
 {
-    uint32_t k = sortable_key(n);
-    uint32_t v = lut[k >> 20] + (k & 0xFFFFFu);
-    if constexpr (4 * I <= 20)
-        return (v >> (20 - 4 * I)) & (0xFu << (4 * I));
-    else
-        return (v << (4 * I - 20)) & (0xFu << (4 * I));
+    const uint32_t b = __float_as_uint(n);
+    const uint32_t s = (uint32_t)__mulhi((int)b, 2);       // 0 or all ones: the sign mask
+    const uint32_t k = b ^ (s & 0xFFFFFu);                  // low 20 bits flipped for n < 0
+    const uint32_t e = lut[__umulhi(k, 1u << 12)];          // k >> 20
+    const uint32_t code = __umulhi(e + k, 1u << 12);        // (e + k) >> 20
+    return acc + code * (1u << (4 * I));
 }
 
 template <bool kF32In>
@@ -199,9 +194,14 @@ __global__ void __launch_bounds__(kThreads) quantize_blocks_kernel(const __grid_
             float n[8];
 #pragma unroll
             for (int i = 0; i < 8; i += 2) nf4::mul2(x[u][i], x[u][i + 1], r, n[i], n[i + 1]);
-            const uint32_t word = code_at<0>(lut, n[0]) | code_at<1>(lut, n[1]) | code_at<2>(lut, n[2]) |
-                                  code_at<3>(lut, n[3]) | code_at<4>(lut, n[4]) | code_at<5>(lut, n[5]) |
-                                  code_at<6>(lut, n[6]) | code_at<7>(lut, n[7]);
+            uint32_t word = add_code<0>(lut, n[0], 0u);
+            word = add_code<1>(lut, n[1], word);
+            word = add_code<2>(lut, n[2], word);
+            word = add_code<3>(lut, n[3], word);
+            word = add_code<4>(lut, n[4], word);
+            word = add_code<5>(lut, n[5], word);
+            word = add_code<6>(lut, n[6], word);
+            word = add_code<7>(lut, n[7], word);
             if (act[u]) reinterpret_cast<uint32_t *>(p.packed)[base + lane + u * stride] = word;
         }
         // exact-mean buckets: one shared atomic per distinct exponent

@@ -75,7 +75,7 @@ struct GemmParams {
 template <int BN, int kBMode, int MT>
 struct GemmCfg {
     static constexpr bool kFused = kBMode >= kBNf4K;
-    static constexpr int kDeqWarps = kFused ? 8 : 0;
+    static constexpr int kDeqWarps = kFused ? (BN == 128 ? 16 : 8) : 0;
     static constexpr int kThreads = 256 + 32 * kDeqWarps;
     static constexpr uint32_t kABytes = MT * 128 * 64 * 2;
     static constexpr uint32_t kBBytes = BN * 64 * 2;
@@ -405,34 +405,44 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode, MT>::kThreads, 1)
                     const uint8_t *pb = sP(s);
                     uint8_t *bb = sB(s);
                     uint32_t words[WPT];
-                    int r, dst_chunk0;
+                    int r;
                     uint8_t *dst;
+                    // this thread's words part*WPT .. part*WPT+WPT-1 of the block's 8;
+                    // 16-byte chunk h of the block holds words 4h..4h+3
+                    auto load_words = [&](const uint8_t *row, auto chunk_pos) {
+                        if constexpr (WPT == 8) {
+#pragma unroll
+                            for (int h = 0; h < 2; h++) {
+                                const uint4 v = *reinterpret_cast<const uint4 *>(row + (chunk_pos(h) << 4));
+                                words[4 * h + 0] = v.x; words[4 * h + 1] = v.y; words[4 * h + 2] = v.z; words[4 * h + 3] = v.w;
+                            }
+                        } else if constexpr (WPT == 4) {
+                            const uint4 v = *reinterpret_cast<const uint4 *>(row + (chunk_pos(part) << 4));
+                            words[0] = v.x; words[1] = v.y; words[2] = v.z; words[3] = v.w;
+                        } else {
+                            static_assert(WPT == 2, "2, 4 or 8 words per thread");
+                            const uint2 v = *reinterpret_cast<const uint2 *>(row + (chunk_pos(part >> 1) << 4) + ((part & 1) << 3));
+                            words[0] = v.x; words[1] = v.y;
+                        }
+                    };
                     if (kBMode == kBNf4K) {
                         // packed tile [BN rows][32 B], 32-byte swizzle: chunk h at h ^ ((row >> 2) & 1)
                         r = blk;
                         const int sw = (r >> 2) & 1;
-#pragma unroll
-                        for (int h = 0; h < 2 / TPB; h++) {
-                            const int chunk = part * (2 / TPB) + h;
-                            const uint4 v = *reinterpret_cast<const uint4 *>(pb + r * 32 + ((chunk ^ sw) << 4));
-                            words[4 * h + 0] = v.x; words[4 * h + 1] = v.y; words[4 * h + 2] = v.z; words[4 * h + 3] = v.w;
-                        }
+                        load_words(pb + r * 32, [&](int h) { return h ^ sw; });
                         dst = bb + r * 128;
                     } else {
                         // packed tile [64 rows][BN/2 B]: 128-byte swizzle (BN = 256) or
                         // 64-byte swizzle (BN = 128) of its 16-byte chunks
                         r = blk & 63;
                         const int c = blk >> 6;
-#pragma unroll
-                        for (int h = 0; h < 2 / TPB; h++) {
-                            const int chunk = 2 * c + part * (2 / TPB) + h;
-                            const int pos = BN == 256 ? (chunk ^ (r & 7)) : (chunk ^ ((r >> 1) & 3));
-                            const uint4 v = *reinterpret_cast<const uint4 *>(pb + r * (BN / 2) + (pos << 4));
-                            words[4 * h + 0] = v.x; words[4 * h + 1] = v.y; words[4 * h + 2] = v.z; words[4 * h + 3] = v.w;
-                        }
+                        load_words(pb + r * (BN / 2), [&](int h) {
+                            const int chunk = 2 * c + h;
+                            return BN == 256 ? (chunk ^ (r & 7)) : (chunk ^ ((r >> 1) & 3));
+                        });
                         dst = bb + c * 8192 + r * 128;
                     }
-                    dst_chunk0 = part * WPT;
+                    const int dst_chunk0 = part * WPT;
 #pragma unroll
                     for (int j = 0; j < WPT; j++)
                         *reinterpret_cast<uint4 *>(dst + (((dst_chunk0 + j) ^ (r & 7)) << 4)) = expand8(words[j], lut, c1p);
