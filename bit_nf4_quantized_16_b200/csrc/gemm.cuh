@@ -33,6 +33,7 @@
 // 64-deep K steps to split 0 of every tile: the LoRA term of the layer.
 #pragma once
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 #include <stdint.h>
@@ -43,7 +44,18 @@
 namespace qlora {
 
 enum BMode : int { kBTmaK = 0, kBTmaMN = 1, kBNf4K = 2, kBNf4MN = 3 };
-enum Epi : int { kEpiBf16 = 0, kEpiF32 = 1 };
+// Epilogues.  kEpiBf16 / kEpiF32 store the tile.  The split modes store an
+// fp32 partial of the tile for this split of the contraction; each epilogue
+// warp counts the arrivals for its own 32-row quadrant of the tile, and the
+// warp of the last split to arrive adds the partials of those rows in split
+// order -- a fixed order, so results are deterministic -- and writes the
+// final values (no synchronization between warps is needed):
+//   kEpiSplitLowRank   v = scale * sum -> hi/lo bf16 pairs in 64-column chunks
+//                      (the H / G buffers), optionally fp32 v, and optionally
+//                      the hi/lo split of a second fp32 matrix of the same shape
+//   kEpiSplitWgrad     tile columns are [hi 64 | lo 64] of one 64-wide chunk:
+//                      out = hi + lo, stored row-major or transposed
+enum Epi : int { kEpiBf16 = 0, kEpiF32 = 1, kEpiSplitLowRank = 2, kEpiSplitWgrad = 3 };
 
 struct GemmParams {
     CUtensorMap tm_a;    // main A operand
@@ -63,11 +75,22 @@ struct GemmParams {
     int k_stages_split;  // main K steps per split (last split may have fewer)
     int k_stages_lora;   // extra LoRA K steps (split 0 only)
     int a_mn;            // A operand is MN-major
+    int a2_x_step;       // x-coordinate advance of the LoRA A operand per 64-deep step
     // output (row-major, leading dimension out_ld elements)
     void *out;
     int64_t out_ld;
-    int64_t split_stride;  // elements between split planes (partial outputs)
     int m_total, n_total;
+    // split modes: fp32 partial planes, per-tile arrival counters, finalize inputs
+    float *part;
+    int64_t part_ld;
+    int64_t split_stride;  // elements between split planes
+    unsigned *counters;
+    float scale;
+    int r, r_pad;
+    float *out_f32;        // optional fp32 copy (low-rank finalize)
+    int out_transposed;    // weight-gradient finalize: out[j][row] instead of out[row][j]
+    const float *aux_in;   // optional fp32 [m_total][r] to split into hi/lo
+    __nv_bfloat16 *aux_out;
     int *err;            // device error word
     uint64_t timeout_ns;
 };
@@ -75,7 +98,7 @@ struct GemmParams {
 template <int BN, int kBMode, int MT>
 struct GemmCfg {
     static constexpr bool kFused = kBMode >= kBNf4K;
-    static constexpr int kDeqWarps = kFused ? (BN == 128 ? 16 : 8) : 0;
+    static constexpr int kDeqWarps = kFused ? 8 : 0;
     static constexpr int kThreads = 256 + 32 * kDeqWarps;
     static constexpr uint32_t kABytes = MT * 128 * 64 * 2;
     static constexpr uint32_t kBBytes = BN * 64 * 2;
@@ -104,6 +127,61 @@ __device__ __forceinline__ void record_timeout(const GemmParams &p, int *abort_f
 {
     atomicExch(p.err, 1);
     *reinterpret_cast<volatile int *>(abort_flag) = 1;
+}
+
+// Sum of split partials at (row, col), splits in order.
+__device__ __forceinline__ float split_sum(const GemmParams &p, int64_t row, int64_t col)
+{
+    float v = 0.0f;
+    const float *src = p.part + row * p.part_ld + col;
+    for (int sp = 0; sp < p.splits; sp++) v = __fadd_rn(v, __ldcg(src + sp * p.split_stride));
+    return v;
+}
+
+__device__ __forceinline__ void store_hi_lo_chunked(__nv_bfloat16 *dst, int64_t row, int r_pad, int col, float v)
+{
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(__fsub_rn(v, __bfloat162float(hi)));
+    __nv_bfloat16 *d = dst + row * 2 * r_pad + 128 * (col >> 6) + (col & 63);
+    d[0] = hi;
+    d[64] = lo;
+}
+
+// Final values of the rows of one 32-row quadrant of an output tile from the
+// split partials (one warp; lanes run along the columns).
+template <int BN, int MT, int kEpi>
+__device__ void split_finalize(const GemmParams &p, int mt, int nt, int q, int lane)
+{
+#pragma unroll 1
+    for (int m = 0; m < MT; m++) {
+#pragma unroll 1
+        for (int i = 0; i < 32; i++) {
+            const int64_t row = (int64_t)mt * 128 * MT + m * 128 + 32 * q + i;
+            if (row >= p.m_total) break;
+            if constexpr (kEpi == kEpiSplitLowRank) {
+                for (int col = lane; col < BN; col += 32) {
+                    const float v = __fmul_rn(p.scale, split_sum(p, row, col));
+                    const bool in = col < p.r;
+                    store_hi_lo_chunked(static_cast<__nv_bfloat16 *>(p.out), row, p.r_pad, col, in ? v : 0.0f);
+                    if (p.out_f32 && in) p.out_f32[row * p.r + col] = v;
+                    if (p.aux_in)
+                        store_hi_lo_chunked(p.aux_out, row, p.r_pad, col, in ? p.aux_in[row * p.r + col] : 0.0f);
+                }
+            } else {
+                for (int ii = lane; ii < 64; ii += 32) {
+                    const int j = 64 * nt + ii;
+                    if (j >= p.r) continue;
+                    const float hi = split_sum(p, row, 128 * nt + ii);
+                    const float lo = split_sum(p, row, 128 * nt + 64 + ii);
+                    float *o = static_cast<float *>(p.out);
+                    if (p.out_transposed)
+                        o[(int64_t)j * p.out_ld + row] = __fadd_rn(hi, lo);
+                    else
+                        o[row * p.out_ld + j] = __fadd_rn(hi, lo);
+                }
+            }
+        }
+    }
 }
 
 }  // namespace gemm_detail
@@ -227,7 +305,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode, MT>::kThreads, 1)
                 } else {
                     const int r0 = (ks - nmain) * 64;
                     mbar_arrive_expect_tx(&full_a[s], Cfg::kABytes + Cfg::kBBytes);
-                    tma_load_2d(sA(s), &p.tm_a2, &full_a[s], r0, m0);
+                    tma_load_2d(sA(s), &p.tm_a2, &full_a[s], (ks - nmain) * p.a2_x_step, m0);
                     if (kBMode == kBNf4MN || kBMode == kBTmaMN) {
 #pragma unroll
                         for (int j = 0; j < BN / 64; j++) tma_load_2d(sB(s) + 8192 * j, &p.tm_b2, &full_a[s], n0 + 64 * j, r0);
@@ -326,7 +404,9 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode, MT>::kThreads, 1)
                             *reinterpret_cast<uint4 *>(o + 8 * g) = v;
                         }
                     } else {
-                        float *o = static_cast<float *>(p.out) + (int64_t)sp * p.split_stride + (int64_t)row * p.out_ld + col0;
+                        float *o = kEpi == kEpiF32
+                                       ? static_cast<float *>(p.out) + (int64_t)row * p.out_ld + col0
+                                       : p.part + (int64_t)sp * p.split_stride + (int64_t)row * p.part_ld + col0;
 #pragma unroll
                         for (int g = 0; g < 8; g++) {
                             if (col0 + 4 * g >= p.n_total) break;
@@ -338,6 +418,21 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode, MT>::kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[buf]);
+            if constexpr (kEpi >= kEpiSplitLowRank) {
+                // the last split to arrive at this quadrant adds up all partials
+                __threadfence();
+                __syncwarp();
+                unsigned *ctr = &p.counters[(nt * p.m_tiles + mt) * 4 + q];
+                unsigned last = 0;
+                if (lane == 0) last = atomicAdd(ctr, 1u) == (unsigned)(p.splits - 1);
+                last = __shfl_sync(0xffffffffu, last, 0);
+                if (last) {
+                    __threadfence();
+                    split_finalize<BN, MT, kEpi>(p, mt, nt, q, lane);
+                    __syncwarp();
+                    if (lane == 0) *ctr = 0u;   // ready for the next launch
+                }
+            }
         }
     } else if (kFused && warp >= 8) {
       if constexpr (kFused) {

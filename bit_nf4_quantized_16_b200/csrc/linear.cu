@@ -111,72 +111,19 @@ void choose_splits(int tiles, int total, int sms, int min_per_split, int *splits
 int ceil_div(int64_t a, int64_t b) { return (int)((a + b - 1) / b); }
 int pad64(int v) { return (v + 63) / 64 * 64; }
 
-// ---- small elementwise kernels ----------------------------------------------------
-
-__device__ __forceinline__ void store_hi_lo(__nv_bfloat16 *h2, int64_t m, int r, int j, float v)
-{
-    __nv_bfloat16 hi = __float2bfloat16_rn(v);
-    __nv_bfloat16 lo = __float2bfloat16_rn(__fsub_rn(v, __bfloat162float(hi)));
-    h2[m * 2 * r + j] = hi;
-    h2[m * 2 * r + r + j] = lo;
-}
-
-// v[m][j] = scale * sum_s part[s][m][j] (splits in order); writes the hi/lo
-// pair and optionally the fp32 value.
-__global__ void finalize_lowrank_kernel(const float *part, int splits, int64_t split_stride, int ld, int64_t M,
-                                        int r, float scale, float *out_f32, __nv_bfloat16 *out_hi_lo)
-{
-    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= M * r) return;
-    int64_t m = i / r;
-    int j = (int)(i % r);
-    float acc = 0.0f;
-    for (int s = 0; s < splits; s++) acc = __fadd_rn(acc, part[s * split_stride + m * ld + j]);
-    float v = __fmul_rn(scale, acc);
-    if (out_f32) out_f32[m * r + j] = v;
-    store_hi_lo(out_hi_lo, m, r, j, v);
-}
-
-__global__ void split_hi_lo_kernel(const float *h, int64_t M, int r, __nv_bfloat16 *out_hi_lo)
-{
-    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= M * r) return;
-    store_hi_lo(out_hi_lo, i / r, r, (int)(i % r), h[i]);
-}
-
-// out[a][b] = sum_s part[s][a][b] + sum_s part[s][a + da][b + db]: the hi and
-// lo halves of a weight-gradient product, added in a fixed order.
-__global__ void finalize_wgrad_kernel(const float *part, int splits, int64_t split_stride, int64_t ld, int64_t rows,
-                                      int64_t cols, int64_t da, int64_t db, float *out)
-{
-    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= rows * cols) return;
-    int64_t a = i / cols, b = i % cols;
-    float hi = 0.0f, lo = 0.0f;
-    for (int s = 0; s < splits; s++) {
-        hi = __fadd_rn(hi, part[s * split_stride + a * ld + b]);
-        lo = __fadd_rn(lo, part[s * split_stride + (a + da) * ld + b + db]);
-    }
-    out[i] = __fadd_rn(hi, lo);
-}
-
-int elementwise_grid(int64_t n) { return (int)((n + 255) / 256); }
-
 // ---- problem plan -------------------------------------------------------------------
 
+// H2 / G2 buffers: [M][2*r_pad] bf16, 64-column chunks alternating hi | lo
+// (hi of columns 64c..64c+63 at 128c, their lo at 128c+64).
 struct Plan {
     int64_t M, N, K;
     int r, r_pad;
-    // H = X A^T : tiles over M, split over K
-    int h_splits, h_per;
-    // G = dY B  : tiles over M, split over N
-    int g_splits, g_per;
-    // dA = G2^T X : tiles (2r rows) x (K / 128), split over M
-    int da_splits, da_per, da_mtiles;
-    // dB = dY^T H2 : tiles (N / 128) x 1, split over M
-    int db_splits, db_per, db_bn;
-    // workspace offsets
-    size_t off_h2, off_g2, off_part, bytes;
+    int h_splits, h_per;          // H = s X A^T : M tiles, split over K
+    int g_splits, g_per;          // G = s dY B  : M tiles, split over N
+    int da_splits, da_per;        // dA^T = X^T [G_hi|G_lo] : K tiles x chunks, split over M
+    int db_splits, db_per;        // dB = dY^T [H_hi|H_lo]  : N tiles x chunks, split over M
+    int max_tiles;
+    size_t off_h2, off_g2, off_ctr, off_part, bytes;
 };
 
 size_t align256(size_t v) { return (v + 255) / 256 * 256; }
@@ -189,23 +136,24 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int r, int sms)
     pl.K = K;
     pl.r = r;
     pl.r_pad = pad64(r);
-    const int mt = ceil_div(M, 128);
+    const int chunks = pl.r_pad / 64;
+    const int mt = ceil_div(M, 128), kt = ceil_div(K, 128), nt = ceil_div(N, 128);
     choose_splits(mt, ceil_div(K, 64), sms, 4, &pl.h_splits, &pl.h_per);
     choose_splits(mt, ceil_div(N, 64), sms, 4, &pl.g_splits, &pl.g_per);
-    pl.da_mtiles = ceil_div(2 * r, 128);
-    choose_splits(pl.da_mtiles * ceil_div(K, 128), ceil_div(M, 64), sms, 4, &pl.da_splits, &pl.da_per);
-    pl.db_bn = 2 * r <= 64 ? 64 : (2 * r <= 128 ? 128 : 256);
-    choose_splits(ceil_div(N, 128), ceil_div(M, 64), sms, 4, &pl.db_splits, &pl.db_per);
-    size_t hl = align256((size_t)M * 2 * r * 2);
+    choose_splits(kt * chunks, ceil_div(M, 64), sms, 4, &pl.da_splits, &pl.da_per);
+    choose_splits(nt * chunks, ceil_div(M, 64), sms, 4, &pl.db_splits, &pl.db_per);
+    pl.max_tiles = std::max(std::max(mt, kt * chunks), nt * chunks);
+    const size_t hl = align256((size_t)M * 2 * pl.r_pad * 2);
     size_t part = 0;
     part = std::max(part, (size_t)pl.h_splits * M * pl.r_pad * 4);
     part = std::max(part, (size_t)pl.g_splits * M * pl.r_pad * 4);
-    part = std::max(part, (size_t)pl.da_splits * 2 * r * K * 4);
-    part = std::max(part, (size_t)pl.db_splits * N * 2 * r * 4);
+    part = std::max(part, (size_t)pl.da_splits * K * 2 * pl.r_pad * 4);
+    part = std::max(part, (size_t)pl.db_splits * N * 2 * pl.r_pad * 4);
     pl.off_h2 = 0;
     pl.off_g2 = hl;
-    pl.off_part = 2 * hl;
-    pl.bytes = 2 * hl + align256(part);
+    pl.off_ctr = 2 * hl;
+    pl.off_part = pl.off_ctr + align256((size_t)pl.max_tiles * 4 * sizeof(unsigned));
+    pl.bytes = pl.off_part + align256(part);
     return pl;
 }
 
@@ -222,7 +170,22 @@ qlora_status check_linear(const qlora_nf4_weight *w, const void *X, int64_t M, c
     return QLORA_OK;
 }
 
-// H = s X A^T into the hi/lo workspace buffer (and optionally fp32 H_out)
+// Common settings of a split-K product whose last split finalizes in place.
+void set_split(GemmParams &p, const Plan &pl, char *ws, int splits, int per, int total_stages, int64_t part_ld,
+               int64_t plane)
+{
+    p.splits = splits;
+    p.k_stages_total = total_stages;
+    p.k_stages_split = per;
+    p.part = reinterpret_cast<float *>(ws + pl.off_part);
+    p.part_ld = part_ld;
+    p.split_stride = plane;
+    p.counters = reinterpret_cast<unsigned *>(ws + pl.off_ctr);
+    p.r = pl.r;
+    p.r_pad = pl.r_pad;
+}
+
+// H = s X A^T into the hi/lo buffer (and optionally fp32 H_out)
 qlora_status run_h(const Plan &pl, const DeviceInfo &dev, const void *X, const void *A, float scale, float *H_out,
                    char *ws, cudaStream_t s)
 {
@@ -231,25 +194,14 @@ qlora_status run_h(const Plan &pl, const DeviceInfo &dev, const void *X, const v
     QLORA_TRY(map_bf16(&p.tm_b, A, pl.K, pl.r, pl.K, 64, pl.r_pad));
     p.m_tiles = ceil_div(pl.M, 128);
     p.n_tiles = 1;
-    p.splits = pl.h_splits;
-    p.k_stages_total = ceil_div(pl.K, 64);
-    p.k_stages_split = pl.h_per;
-    p.out = ws + pl.off_part;
-    p.out_ld = pl.r_pad;
-    p.split_stride = pl.M * pl.r_pad;
+    set_split(p, pl, ws, pl.h_splits, pl.h_per, ceil_div(pl.K, 64), pl.r_pad, pl.M * pl.r_pad);
+    p.out = ws + pl.off_h2;
     p.m_total = (int)pl.M;
     p.n_total = pl.r_pad;
-    if (pl.r_pad == 64)
-        QLORA_TRY((launch_gemm<64, kBTmaK, kEpiF32>(p, dev, s, QLORA_KERNEL_LOWRANK)));
-    else
-        QLORA_TRY((launch_gemm<128, kBTmaK, kEpiF32>(p, dev, s, QLORA_KERNEL_LOWRANK)));
-    {
-        LaunchScope ls(QLORA_KERNEL_ELEMENTWISE, s);
-        finalize_lowrank_kernel<<<elementwise_grid(pl.M * pl.r), 256, 0, s>>>(
-            reinterpret_cast<const float *>(ws + pl.off_part), pl.h_splits, pl.M * pl.r_pad, pl.r_pad, pl.M, pl.r,
-            scale, H_out, reinterpret_cast<__nv_bfloat16 *>(ws + pl.off_h2));
-    }
-    return launch_status();
+    p.scale = scale;
+    p.out_f32 = H_out;
+    if (pl.r_pad == 64) return launch_gemm<64, kBTmaK, kEpiSplitLowRank>(p, dev, s, QLORA_KERNEL_LOWRANK);
+    return launch_gemm<128, kBTmaK, kEpiSplitLowRank>(p, dev, s, QLORA_KERNEL_LOWRANK);
 }
 
 }  // namespace
@@ -280,6 +232,7 @@ extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const void *
     if (workspace_bytes < pl.bytes) return QLORA_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     char *ws = static_cast<char *>(workspace);
+    QLORA_CUDA_TRY(cudaMemsetAsync(ws + pl.off_ctr, 0, (size_t)pl.max_tiles * 4 * sizeof(unsigned), s));
 
     QLORA_TRY(run_h(pl, dev, X, A, scale, H_save, ws, s));
 
@@ -289,8 +242,9 @@ extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const void *
     QLORA_TRY(map_bf16(&p.tm_a, X, pl.K, M, pl.K, 64, 128 * kFMT));
     QLORA_TRY(make_map(&p.tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->packed, pl.K / 2, pl.N, pl.K / 2, 32, kFBN,
                        CU_TENSOR_MAP_SWIZZLE_32B));
-    QLORA_TRY(map_bf16(&p.tm_a2, ws + pl.off_h2, r, M, 2 * r, 64, 128 * kFMT));   // hi half of H
+    QLORA_TRY(map_bf16(&p.tm_a2, ws + pl.off_h2, 2 * pl.r_pad, M, 2 * pl.r_pad, 64, 128 * kFMT));   // hi chunks of H
     QLORA_TRY(map_bf16(&p.tm_b2, B, r, pl.N, r, 64, kFBN));
+    p.a2_x_step = 128;
     p.code2 = w->code2;
     p.c2 = w->c2;
     p.mean = w->mean;
@@ -302,7 +256,7 @@ extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const void *
     p.splits = 1;
     p.k_stages_total = (int)(pl.K / 64);
     p.k_stages_split = p.k_stages_total;
-    p.k_stages_lora = ceil_div(r, 64);
+    p.k_stages_lora = pl.r_pad / 64;
     p.out = Y;
     p.out_ld = pl.N;
     p.m_total = (int)M;
@@ -335,46 +289,32 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *
     const Plan pl = make_plan(M, N, K, r, dev.sms);
     if (workspace_bytes < pl.bytes) return QLORA_ERR_WORKSPACE;
     char *ws = static_cast<char *>(workspace);
+    QLORA_CUDA_TRY(cudaMemsetAsync(ws + pl.off_ctr, 0, (size_t)pl.max_tiles * 4 * sizeof(unsigned), s));
     __nv_bfloat16 *H2 = reinterpret_cast<__nv_bfloat16 *>(ws + pl.off_h2);
     __nv_bfloat16 *G2 = reinterpret_cast<__nv_bfloat16 *>(ws + pl.off_g2);
-    float *part = reinterpret_cast<float *>(ws + pl.off_part);
+    const int hl_cols = 2 * pl.r_pad;
 
-    // H (hi/lo) from the saved fp32 H, or recomputed
-    if (H_saved) {
-        {
-            LaunchScope ls(QLORA_KERNEL_ELEMENTWISE, s);
-            split_hi_lo_kernel<<<elementwise_grid(M * r), 256, 0, s>>>(H_saved, M, r, H2);
-        }
-        QLORA_TRY(launch_status());
-    } else {
-        QLORA_TRY(run_h(pl, dev, X, A, scale, nullptr, ws, s));
-    }
+    // H (hi/lo) recomputed when no saved H is given
+    if (!H_saved) QLORA_TRY(run_h(pl, dev, X, A, scale, nullptr, ws, s));
 
-    // G = s dY B  (contraction over N)
+    // G = s dY B (contraction over N); its finalize also splits a saved H into hi/lo
     {
         GemmParams p{};
         QLORA_TRY(map_bf16(&p.tm_a, dY, N, M, N, 64, 128));
         QLORA_TRY(map_bf16(&p.tm_b, B, r, N, r, 64, 64));      // B[n][j]: MN-major operand
         p.m_tiles = ceil_div(M, 128);
         p.n_tiles = 1;
-        p.splits = pl.g_splits;
-        p.k_stages_total = ceil_div(N, 64);
-        p.k_stages_split = pl.g_per;
-        p.out = part;
-        p.out_ld = pl.r_pad;
-        p.split_stride = M * pl.r_pad;
+        set_split(p, pl, ws, pl.g_splits, pl.g_per, ceil_div(N, 64), pl.r_pad, M * pl.r_pad);
+        p.out = G2;
         p.m_total = (int)M;
         p.n_total = pl.r_pad;
+        p.scale = scale;
+        p.aux_in = H_saved;
+        p.aux_out = H2;
         if (pl.r_pad == 64)
-            QLORA_TRY((launch_gemm<64, kBTmaMN, kEpiF32>(p, dev, s, QLORA_KERNEL_LOWRANK)));
+            QLORA_TRY((launch_gemm<64, kBTmaMN, kEpiSplitLowRank>(p, dev, s, QLORA_KERNEL_LOWRANK)));
         else
-            QLORA_TRY((launch_gemm<128, kBTmaMN, kEpiF32>(p, dev, s, QLORA_KERNEL_LOWRANK)));
-        {
-            LaunchScope ls(QLORA_KERNEL_ELEMENTWISE, s);
-            finalize_lowrank_kernel<<<elementwise_grid(M * r), 256, 0, s>>>(part, pl.g_splits, M * pl.r_pad, pl.r_pad,
-                                                                             M, r, scale, nullptr, G2);
-        }
-        QLORA_TRY(launch_status());
+            QLORA_TRY((launch_gemm<128, kBTmaMN, kEpiSplitLowRank>(p, dev, s, QLORA_KERNEL_LOWRANK)));
     }
 
     // dX = dY W' + bf16(G) A  (fused transposed dequant-GEMM)
@@ -385,8 +325,9 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *
         QLORA_TRY(map_bf16(&p.tm_a, dY, N, M, N, 64, 128 * kBMT));
         QLORA_TRY(make_map(&p.tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->packed, K / 2, N, K / 2, kBBN / 2, 64,
                            kBBN == 256 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B));
-        QLORA_TRY(map_bf16(&p.tm_a2, G2, r, M, 2 * r, 64, 128 * kBMT));   // hi half of G
-        QLORA_TRY(map_bf16(&p.tm_b2, A, K, r, K, 64, 64));                // A[j][k]: MN-major operand
+        QLORA_TRY(map_bf16(&p.tm_a2, G2, hl_cols, M, hl_cols, 64, 128 * kBMT));   // hi chunks of G
+        QLORA_TRY(map_bf16(&p.tm_b2, A, K, r, K, 64, 64));                        // A[j][k]: MN-major operand
+        p.a2_x_step = 128;
         p.code2 = w->code2;
         p.c2 = w->c2;
         p.mean = w->mean;
@@ -398,7 +339,7 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *
         p.splits = 1;
         p.k_stages_total = ceil_div(N, 64);
         p.k_stages_split = p.k_stages_total;
-        p.k_stages_lora = ceil_div(r, 64);
+        p.k_stages_lora = pl.r_pad / 64;
         p.out = dX;
         p.out_ld = K;
         p.m_total = (int)M;
@@ -409,58 +350,36 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *
             QLORA_TRY((launch_gemm<kBBN, kBNf4MN, kEpiF32, kBMT>(p, dev, s, QLORA_KERNEL_BWD_FUSED)));
     }
 
-    // dA = G^T X  (rows j of [G_hi | G_lo], contraction over tokens)
+    // dA^T = X^T [G_hi | G_lo]  (rows k, chunk columns; contraction over tokens), stored transposed
     {
         GemmParams p{};
-        QLORA_TRY(map_bf16(&p.tm_a, G2, 2 * r, M, 2 * r, 64, 64));   // MN-major A
-        QLORA_TRY(map_bf16(&p.tm_b, X, K, M, K, 64, 64));            // MN-major B
+        QLORA_TRY(map_bf16(&p.tm_a, X, K, M, K, 64, 64));              // MN-major A
+        QLORA_TRY(map_bf16(&p.tm_b, G2, hl_cols, M, hl_cols, 64, 64));  // MN-major B
         p.a_mn = 1;
-        p.m_tiles = pl.da_mtiles;
-        p.n_tiles = ceil_div(K, 128);
-        p.splits = pl.da_splits;
-        p.k_stages_total = ceil_div(M, 64);
-        p.k_stages_split = pl.da_per;
-        p.out = part;
+        p.m_tiles = ceil_div(K, 128);
+        p.n_tiles = pl.r_pad / 64;
+        set_split(p, pl, ws, pl.da_splits, pl.da_per, ceil_div(M, 64), hl_cols, K * hl_cols);
+        p.out = dA;
         p.out_ld = K;
-        p.split_stride = 2 * r * K;
-        p.m_total = 2 * r;
-        p.n_total = (int)K;
-        QLORA_TRY((launch_gemm<128, kBTmaMN, kEpiF32>(p, dev, s, QLORA_KERNEL_WGRAD)));
-        {
-            LaunchScope ls(QLORA_KERNEL_ELEMENTWISE, s);
-            finalize_wgrad_kernel<<<elementwise_grid((int64_t)r * K), 256, 0, s>>>(part, pl.da_splits, 2 * r * K, K, r,
-                                                                                   K, r, 0, dA);
-        }
-        QLORA_TRY(launch_status());
+        p.out_transposed = 1;
+        p.m_total = (int)K;
+        p.n_total = hl_cols;
+        QLORA_TRY((launch_gemm<128, kBTmaMN, kEpiSplitWgrad>(p, dev, s, QLORA_KERNEL_WGRAD)));
     }
 
-    // dB = dY^T H  (rows n, columns [H_hi | H_lo], contraction over tokens)
+    // dB = dY^T [H_hi | H_lo]  (rows n, chunk columns; contraction over tokens)
     {
         GemmParams p{};
-        QLORA_TRY(map_bf16(&p.tm_a, dY, N, M, N, 64, 64));           // MN-major A
-        QLORA_TRY(map_bf16(&p.tm_b, H2, 2 * r, M, 2 * r, 64, 64));   // MN-major B
+        QLORA_TRY(map_bf16(&p.tm_a, dY, N, M, N, 64, 64));              // MN-major A
+        QLORA_TRY(map_bf16(&p.tm_b, H2, hl_cols, M, hl_cols, 64, 64));  // MN-major B
         p.a_mn = 1;
         p.m_tiles = ceil_div(N, 128);
-        p.n_tiles = 1;
-        p.splits = pl.db_splits;
-        p.k_stages_total = ceil_div(M, 64);
-        p.k_stages_split = pl.db_per;
-        p.out = part;
-        p.out_ld = 2 * r;
-        p.split_stride = N * 2 * r;
+        p.n_tiles = pl.r_pad / 64;
+        set_split(p, pl, ws, pl.db_splits, pl.db_per, ceil_div(M, 64), hl_cols, N * hl_cols);
+        p.out = dB;
+        p.out_ld = r;
         p.m_total = (int)N;
-        p.n_total = 2 * r;
-        if (pl.db_bn == 64)
-            QLORA_TRY((launch_gemm<64, kBTmaMN, kEpiF32>(p, dev, s, QLORA_KERNEL_WGRAD)));
-        else if (pl.db_bn == 128)
-            QLORA_TRY((launch_gemm<128, kBTmaMN, kEpiF32>(p, dev, s, QLORA_KERNEL_WGRAD)));
-        else
-            QLORA_TRY((launch_gemm<256, kBTmaMN, kEpiF32>(p, dev, s, QLORA_KERNEL_WGRAD)));
-        {
-            LaunchScope ls(QLORA_KERNEL_ELEMENTWISE, s);
-            finalize_wgrad_kernel<<<elementwise_grid(N * r), 256, 0, s>>>(part, pl.db_splits, N * 2 * r, 2 * r, N, r,
-                                                                           0, r, dB);
-        }
-        return launch_status();
+        p.n_total = hl_cols;
+        return launch_gemm<128, kBTmaMN, kEpiSplitWgrad>(p, dev, s, QLORA_KERNEL_WGRAD);
     }
 }
