@@ -129,55 +129,101 @@ __device__ __forceinline__ void record_timeout(const GemmParams &p, int *abort_f
     *reinterpret_cast<volatile int *>(abort_flag) = 1;
 }
 
-// Sum of split partials at (row, col), splits in order.
-__device__ __forceinline__ float split_sum(const GemmParams &p, int64_t row, int64_t col)
+// Sum of split partials at (row, col..col+3), splits added in order; the
+// loads of up to 8 splits are issued before the adds.
+__device__ __forceinline__ float4 split_sum4(const GemmParams &p, int64_t row, int64_t col)
 {
-    float v = 0.0f;
     const float *src = p.part + row * p.part_ld + col;
-    for (int sp = 0; sp < p.splits; sp++) v = __fadd_rn(v, __ldcg(src + sp * p.split_stride));
-    return v;
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    for (int sp0 = 0; sp0 < p.splits; sp0 += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; u++)
+            if (sp0 + u < p.splits) v[u] = __ldcg(reinterpret_cast<const float4 *>(src + (int64_t)(sp0 + u) * p.split_stride));
+#pragma unroll
+        for (int u = 0; u < 8; u++) {
+            if (sp0 + u < p.splits) {
+                acc.x = __fadd_rn(acc.x, v[u].x);
+                acc.y = __fadd_rn(acc.y, v[u].y);
+                acc.z = __fadd_rn(acc.z, v[u].z);
+                acc.w = __fadd_rn(acc.w, v[u].w);
+            }
+        }
+    }
+    return acc;
 }
 
-__device__ __forceinline__ void store_hi_lo_chunked(__nv_bfloat16 *dst, int64_t row, int r_pad, int col, float v)
+__device__ __forceinline__ uint32_t bf16_bits(float v)
 {
-    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-    const __nv_bfloat16 lo = __float2bfloat16_rn(__fsub_rn(v, __bfloat162float(hi)));
+    return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+
+// hi/lo bf16 of 4 consecutive columns col..col+3 (col % 4 == 0) of one row
+__device__ __forceinline__ void store_hi_lo4(__nv_bfloat16 *dst, int64_t row, int r_pad, int col, float4 v)
+{
+    const float vv[4] = {v.x, v.y, v.z, v.w};
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        hi[i] = bf16_bits(vv[i]);
+        lo[i] = bf16_bits(__fsub_rn(vv[i], __uint_as_float(hi[i] << 16)));
+    }
     __nv_bfloat16 *d = dst + row * 2 * r_pad + 128 * (col >> 6) + (col & 63);
-    d[0] = hi;
-    d[64] = lo;
+    *reinterpret_cast<uint2 *>(d) = make_uint2(hi[0] | (hi[1] << 16), hi[2] | (hi[3] << 16));
+    *reinterpret_cast<uint2 *>(d + 64) = make_uint2(lo[0] | (lo[1] << 16), lo[2] | (lo[3] << 16));
 }
 
 // Final values of the rows of one 32-row quadrant of an output tile from the
-// split partials (one warp; lanes run along the columns).
+// split partials (one warp; 16 lanes x 4 columns cover 64 columns of a row,
+// so the warp handles two rows at a time).
 template <int BN, int MT, int kEpi>
 __device__ void split_finalize(const GemmParams &p, int mt, int nt, int q, int lane)
 {
+    const int half = lane >> 4, c4 = 4 * (lane & 15);
 #pragma unroll 1
     for (int m = 0; m < MT; m++) {
 #pragma unroll 1
-        for (int i = 0; i < 32; i++) {
+        for (int i = half; i < 32; i += 2) {
             const int64_t row = (int64_t)mt * 128 * MT + m * 128 + 32 * q + i;
             if (row >= p.m_total) break;
             if constexpr (kEpi == kEpiSplitLowRank) {
-                for (int col = lane; col < BN; col += 32) {
-                    const float v = __fmul_rn(p.scale, split_sum(p, row, col));
-                    const bool in = col < p.r;
-                    store_hi_lo_chunked(static_cast<__nv_bfloat16 *>(p.out), row, p.r_pad, col, in ? v : 0.0f);
-                    if (p.out_f32 && in) p.out_f32[row * p.r + col] = v;
-                    if (p.aux_in)
-                        store_hi_lo_chunked(p.aux_out, row, p.r_pad, col, in ? p.aux_in[row * p.r + col] : 0.0f);
+#pragma unroll
+                for (int col = c4; col < BN; col += 64) {
+                    float4 v = split_sum4(p, row, col);
+                    v.x = __fmul_rn(p.scale, v.x);
+                    v.y = __fmul_rn(p.scale, v.y);
+                    v.z = __fmul_rn(p.scale, v.z);
+                    v.w = __fmul_rn(p.scale, v.w);
+                    // columns at or beyond r are padding: keep them zero
+                    if (col + 0 >= p.r) v.x = 0.0f;
+                    if (col + 1 >= p.r) v.y = 0.0f;
+                    if (col + 2 >= p.r) v.z = 0.0f;
+                    if (col + 3 >= p.r) v.w = 0.0f;
+                    store_hi_lo4(static_cast<__nv_bfloat16 *>(p.out), row, p.r_pad, col, v);
+                    if (p.out_f32 && col < p.r)   // r % 8 == 0: the 4 columns are all in or all out
+                        *reinterpret_cast<float4 *>(p.out_f32 + row * p.r + col) = v;
+                    if (p.aux_in) {
+                        float4 h = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                        if (col < p.r) h = *reinterpret_cast<const float4 *>(p.aux_in + row * p.r + col);
+                        store_hi_lo4(p.aux_out, row, p.r_pad, col, h);
+                    }
                 }
             } else {
-                for (int ii = lane; ii < 64; ii += 32) {
-                    const int j = 64 * nt + ii;
-                    if (j >= p.r) continue;
-                    const float hi = split_sum(p, row, 128 * nt + ii);
-                    const float lo = split_sum(p, row, 128 * nt + 64 + ii);
+                const int j = 64 * nt + c4;
+                if (j < p.r) {
+                    const float4 hi = split_sum4(p, row, 128 * nt + c4);
+                    const float4 lo = split_sum4(p, row, 128 * nt + 64 + c4);
+                    const float4 v = make_float4(__fadd_rn(hi.x, lo.x), __fadd_rn(hi.y, lo.y), __fadd_rn(hi.z, lo.z),
+                                                 __fadd_rn(hi.w, lo.w));
                     float *o = static_cast<float *>(p.out);
-                    if (p.out_transposed)
-                        o[(int64_t)j * p.out_ld + row] = __fadd_rn(hi, lo);
-                    else
-                        o[row * p.out_ld + j] = __fadd_rn(hi, lo);
+                    if (p.out_transposed) {
+                        o[(int64_t)(j + 0) * p.out_ld + row] = v.x;
+                        o[(int64_t)(j + 1) * p.out_ld + row] = v.y;
+                        o[(int64_t)(j + 2) * p.out_ld + row] = v.z;
+                        o[(int64_t)(j + 3) * p.out_ld + row] = v.w;
+                    } else {
+                        *reinterpret_cast<float4 *>(o + row * p.out_ld + j) = v;
+                    }
                 }
             }
         }
