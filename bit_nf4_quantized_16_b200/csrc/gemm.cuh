@@ -44,18 +44,10 @@
 namespace qlora {
 
 enum BMode : int { kBTmaK = 0, kBTmaMN = 1, kBNf4K = 2, kBNf4MN = 3 };
-// Epilogues.  kEpiBf16 / kEpiF32 store the tile.  The split modes store an
-// fp32 partial of the tile for this split of the contraction; each epilogue
-// warp counts the arrivals for its own 32-row quadrant of the tile, and the
-// warp of the last split to arrive adds the partials of those rows in split
-// order -- a fixed order, so results are deterministic -- and writes the
-// final values (no synchronization between warps is needed):
-//   kEpiSplitLowRank   v = scale * sum -> hi/lo bf16 pairs in 64-column chunks
-//                      (the H / G buffers), optionally fp32 v, and optionally
-//                      the hi/lo split of a second fp32 matrix of the same shape
-//   kEpiSplitWgrad     tile columns are [hi 64 | lo 64] of one 64-wide chunk:
-//                      out = hi + lo, stored row-major or transposed
-enum Epi : int { kEpiBf16 = 0, kEpiF32 = 1, kEpiSplitLowRank = 2, kEpiSplitWgrad = 3 };
+// Epilogues: kEpiBf16 stores the tile as bf16; kEpiF32 stores it as fp32,
+// into plane `split` of a stack of partial products when the contraction is
+// split (out + split * split_stride).
+enum Epi : int { kEpiBf16 = 0, kEpiF32 = 1 };
 
 struct GemmParams {
     CUtensorMap tm_a;    // main A operand
@@ -80,17 +72,7 @@ struct GemmParams {
     void *out;
     int64_t out_ld;
     int m_total, n_total;
-    // split modes: fp32 partial planes, per-tile arrival counters, finalize inputs
-    float *part;
-    int64_t part_ld;
-    int64_t split_stride;  // elements between split planes
-    unsigned *counters;
-    float scale;
-    int r, r_pad;
-    float *out_f32;        // optional fp32 copy (low-rank finalize)
-    int out_transposed;    // weight-gradient finalize: out[j][row] instead of out[row][j]
-    const float *aux_in;   // optional fp32 [m_total][r] to split into hi/lo
-    __nv_bfloat16 *aux_out;
+    int64_t split_stride;  // elements between split planes (partial products)
     int *err;            // device error word
     uint64_t timeout_ns;
 };
@@ -127,107 +109,6 @@ __device__ __forceinline__ void record_timeout(const GemmParams &p, int *abort_f
 {
     atomicExch(p.err, 1);
     *reinterpret_cast<volatile int *>(abort_flag) = 1;
-}
-
-// Sum of split partials at (row, col..col+3), splits added in order; the
-// loads of up to 8 splits are issued before the adds.
-__device__ __forceinline__ float4 split_sum4(const GemmParams &p, int64_t row, int64_t col)
-{
-    const float *src = p.part + row * p.part_ld + col;
-    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    for (int sp0 = 0; sp0 < p.splits; sp0 += 8) {
-        float4 v[8];
-#pragma unroll
-        for (int u = 0; u < 8; u++)
-            if (sp0 + u < p.splits) v[u] = __ldcg(reinterpret_cast<const float4 *>(src + (int64_t)(sp0 + u) * p.split_stride));
-#pragma unroll
-        for (int u = 0; u < 8; u++) {
-            if (sp0 + u < p.splits) {
-                acc.x = __fadd_rn(acc.x, v[u].x);
-                acc.y = __fadd_rn(acc.y, v[u].y);
-                acc.z = __fadd_rn(acc.z, v[u].z);
-                acc.w = __fadd_rn(acc.w, v[u].w);
-            }
-        }
-    }
-    return acc;
-}
-
-__device__ __forceinline__ uint32_t bf16_bits(float v)
-{
-    return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v));
-}
-
-// hi/lo bf16 of 4 consecutive columns col..col+3 (col % 4 == 0) of one row
-__device__ __forceinline__ void store_hi_lo4(__nv_bfloat16 *dst, int64_t row, int r_pad, int col, float4 v)
-{
-    const float vv[4] = {v.x, v.y, v.z, v.w};
-    uint32_t hi[4], lo[4];
-#pragma unroll
-    for (int i = 0; i < 4; i++) {
-        hi[i] = bf16_bits(vv[i]);
-        lo[i] = bf16_bits(__fsub_rn(vv[i], __uint_as_float(hi[i] << 16)));
-    }
-    __nv_bfloat16 *d = dst + row * 2 * r_pad + 128 * (col >> 6) + (col & 63);
-    *reinterpret_cast<uint2 *>(d) = make_uint2(hi[0] | (hi[1] << 16), hi[2] | (hi[3] << 16));
-    *reinterpret_cast<uint2 *>(d + 64) = make_uint2(lo[0] | (lo[1] << 16), lo[2] | (lo[3] << 16));
-}
-
-// Final values of the rows of one 32-row quadrant of an output tile from the
-// split partials (one warp; 16 lanes x 4 columns cover 64 columns of a row,
-// so the warp handles two rows at a time).
-template <int BN, int MT, int kEpi>
-__device__ void split_finalize(const GemmParams &p, int mt, int nt, int q, int lane)
-{
-    const int half = lane >> 4, c4 = 4 * (lane & 15);
-#pragma unroll 1
-    for (int m = 0; m < MT; m++) {
-#pragma unroll 1
-        for (int i = half; i < 32; i += 2) {
-            const int64_t row = (int64_t)mt * 128 * MT + m * 128 + 32 * q + i;
-            if (row >= p.m_total) break;
-            if constexpr (kEpi == kEpiSplitLowRank) {
-#pragma unroll
-                for (int col = c4; col < BN; col += 64) {
-                    float4 v = split_sum4(p, row, col);
-                    v.x = __fmul_rn(p.scale, v.x);
-                    v.y = __fmul_rn(p.scale, v.y);
-                    v.z = __fmul_rn(p.scale, v.z);
-                    v.w = __fmul_rn(p.scale, v.w);
-                    // columns at or beyond r are padding: keep them zero
-                    if (col + 0 >= p.r) v.x = 0.0f;
-                    if (col + 1 >= p.r) v.y = 0.0f;
-                    if (col + 2 >= p.r) v.z = 0.0f;
-                    if (col + 3 >= p.r) v.w = 0.0f;
-                    store_hi_lo4(static_cast<__nv_bfloat16 *>(p.out), row, p.r_pad, col, v);
-                    if (p.out_f32 && col < p.r)   // r % 8 == 0: the 4 columns are all in or all out
-                        *reinterpret_cast<float4 *>(p.out_f32 + row * p.r + col) = v;
-                    if (p.aux_in) {
-                        float4 h = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                        if (col < p.r) h = *reinterpret_cast<const float4 *>(p.aux_in + row * p.r + col);
-                        store_hi_lo4(p.aux_out, row, p.r_pad, col, h);
-                    }
-                }
-            } else {
-                const int j = 64 * nt + c4;
-                if (j < p.r) {
-                    const float4 hi = split_sum4(p, row, 128 * nt + c4);
-                    const float4 lo = split_sum4(p, row, 128 * nt + 64 + c4);
-                    const float4 v = make_float4(__fadd_rn(hi.x, lo.x), __fadd_rn(hi.y, lo.y), __fadd_rn(hi.z, lo.z),
-                                                 __fadd_rn(hi.w, lo.w));
-                    float *o = static_cast<float *>(p.out);
-                    if (p.out_transposed) {
-                        o[(int64_t)(j + 0) * p.out_ld + row] = v.x;
-                        o[(int64_t)(j + 1) * p.out_ld + row] = v.y;
-                        o[(int64_t)(j + 2) * p.out_ld + row] = v.z;
-                        o[(int64_t)(j + 3) * p.out_ld + row] = v.w;
-                    } else {
-                        *reinterpret_cast<float4 *>(o + row * p.out_ld + j) = v;
-                    }
-                }
-            }
-        }
-    }
 }
 
 }  // namespace gemm_detail
@@ -450,9 +331,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode, MT>::kThreads, 1)
                             *reinterpret_cast<uint4 *>(o + 8 * g) = v;
                         }
                     } else {
-                        float *o = kEpi == kEpiF32
-                                       ? static_cast<float *>(p.out) + (int64_t)row * p.out_ld + col0
-                                       : p.part + (int64_t)sp * p.split_stride + (int64_t)row * p.part_ld + col0;
+                        float *o = static_cast<float *>(p.out) + (int64_t)sp * p.split_stride + (int64_t)row * p.out_ld + col0;
 #pragma unroll
                         for (int g = 0; g < 8; g++) {
                             if (col0 + 4 * g >= p.n_total) break;
@@ -464,21 +343,6 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode, MT>::kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[buf]);
-            if constexpr (kEpi >= kEpiSplitLowRank) {
-                // the last split to arrive at this quadrant adds up all partials
-                __threadfence();
-                __syncwarp();
-                unsigned *ctr = &p.counters[(nt * p.m_tiles + mt) * 4 + q];
-                unsigned last = 0;
-                if (lane == 0) last = atomicAdd(ctr, 1u) == (unsigned)(p.splits - 1);
-                last = __shfl_sync(0xffffffffu, last, 0);
-                if (last) {
-                    __threadfence();
-                    split_finalize<BN, MT, kEpi>(p, mt, nt, q, lane);
-                    __syncwarp();
-                    if (lane == 0) *ctr = 0u;   // ready for the next launch
-                }
-            }
         }
     } else if (kFused && warp >= 8) {
       if constexpr (kFused) {

@@ -95,10 +95,11 @@ qlora_status launch_gemm(GemmParams &p, const DeviceInfo &dev, cudaStream_t s, i
 }
 
 // number of splits of a contraction of `total` 64-deep steps over `tiles`
-// output tiles, aiming at about one wave of the GPU; every split non-empty
+// output tiles: as many as fit in one wave of the GPU (tiles * splits <= sms),
+// each with at least `min_per_split` steps; every split non-empty
 void choose_splits(int tiles, int total, int sms, int min_per_split, int *splits, int *per)
 {
-    int sp = (sms + tiles - 1) / tiles;
+    int sp = sms / (tiles > 0 ? tiles : 1);
     int cap = total / min_per_split;
     if (cap < 1) cap = 1;
     if (sp > cap) sp = cap;
@@ -110,6 +111,107 @@ void choose_splits(int tiles, int total, int sms, int min_per_split, int *splits
 
 int ceil_div(int64_t a, int64_t b) { return (int)((a + b - 1) / b); }
 int pad64(int v) { return (v + 63) / 64 * 64; }
+int elementwise_grid(int64_t n) { return (int)((n + 255) / 256); }
+
+// ---- finalize kernels (grid-wide, one thread per 4 outputs) ---------------------------
+
+// Sum of the split partials at (row, col..col+3), splits added in order.
+__device__ __forceinline__ float4 split_sum4(const float *part, int splits, int64_t split_stride, int64_t ld,
+                                             int64_t row, int64_t col)
+{
+    const float *src = part + row * ld + col;
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    for (int sp = 0; sp < splits; sp++) {
+        const float4 v = __ldcg(reinterpret_cast<const float4 *>(src + sp * split_stride));
+        acc.x = __fadd_rn(acc.x, v.x);
+        acc.y = __fadd_rn(acc.y, v.y);
+        acc.z = __fadd_rn(acc.z, v.z);
+        acc.w = __fadd_rn(acc.w, v.w);
+    }
+    return acc;
+}
+
+__device__ __forceinline__ uint32_t bf16_bits(float v) { return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v)); }
+
+// hi = bf16(v), lo = bf16(v - hi) of 4 consecutive columns col..col+3 into the
+// chunked hi/lo layout: [M][2*r_pad], hi of column c at 128*(c/64) + c%64, lo 64 further.
+__device__ __forceinline__ void store_hi_lo4(__nv_bfloat16 *dst, int64_t row, int r_pad, int col, float4 v)
+{
+    const float vv[4] = {v.x, v.y, v.z, v.w};
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        hi[i] = bf16_bits(vv[i]);
+        lo[i] = bf16_bits(__fsub_rn(vv[i], __uint_as_float(hi[i] << 16)));
+    }
+    __nv_bfloat16 *d = dst + row * 2 * r_pad + 128 * (col >> 6) + (col & 63);
+    *reinterpret_cast<uint2 *>(d) = make_uint2(hi[0] | (hi[1] << 16), hi[2] | (hi[3] << 16));
+    *reinterpret_cast<uint2 *>(d + 64) = make_uint2(lo[0] | (lo[1] << 16), lo[2] | (lo[3] << 16));
+}
+
+// v = scale * sum over splits of part[.][m][j]  ->  hi/lo chunked buffer (padding
+// columns j >= r set to zero), optionally fp32 v [M][r]; optionally also the
+// hi/lo split of aux_in [M][r] into aux_out.
+__global__ void finalize_lowrank_kernel(const float *part, int splits, int64_t split_stride, int64_t M, int r,
+                                        int r_pad, float scale, __nv_bfloat16 *out, float *out_f32,
+                                        const float *aux_in, __nv_bfloat16 *aux_out)
+{
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int per_row = r_pad / 4;
+    if (i >= M * per_row) return;
+    const int64_t m = i / per_row;
+    const int col = 4 * (int)(i % per_row);
+    const bool in = col < r;   // r % 8 == 0: 4 columns are all in or all out
+    float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (in) {
+        v = split_sum4(part, splits, split_stride, r_pad, m, col);
+        v = make_float4(__fmul_rn(scale, v.x), __fmul_rn(scale, v.y), __fmul_rn(scale, v.z), __fmul_rn(scale, v.w));
+        if (out_f32) *reinterpret_cast<float4 *>(out_f32 + m * r + col) = v;
+    }
+    store_hi_lo4(out, m, r_pad, col, v);
+    if (aux_in) {
+        float4 h = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        if (in) h = *reinterpret_cast<const float4 *>(aux_in + m * r + col);
+        store_hi_lo4(aux_out, m, r_pad, col, h);
+    }
+}
+
+// Weight gradients from the partial products of the hi and lo halves, two jobs
+// in one launch: job 0 = dA (rows k of X^T [G_hi|G_lo], stored transposed into
+// dA[j][k]), job 1 = dB (rows n of dY^T [H_hi|H_lo], stored as dB[n][j]).
+struct WgradJob {
+    const float *part;
+    int splits;
+    int64_t split_stride;
+    int64_t rows;
+    float *out;
+    int64_t out_ld;
+    int transposed;
+};
+
+__global__ void finalize_wgrad_kernel(WgradJob j0, WgradJob j1, int64_t n0, int r, int r_pad)
+{
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int per_row = r / 4;
+    const WgradJob &J = i < n0 ? j0 : j1;
+    if (i >= n0) i -= n0;
+    if (i >= J.rows * per_row) return;
+    const int64_t row = i / per_row;
+    const int j = 4 * (int)(i % per_row);
+    const int64_t ld = 2 * r_pad;
+    const int64_t chunk = 128 * (j >> 6) + (j & 63);
+    const float4 hi = split_sum4(J.part, J.splits, J.split_stride, ld, row, chunk);
+    const float4 lo = split_sum4(J.part, J.splits, J.split_stride, ld, row, chunk + 64);
+    const float4 v = make_float4(__fadd_rn(hi.x, lo.x), __fadd_rn(hi.y, lo.y), __fadd_rn(hi.z, lo.z), __fadd_rn(hi.w, lo.w));
+    if (J.transposed) {
+        J.out[(int64_t)(j + 0) * J.out_ld + row] = v.x;
+        J.out[(int64_t)(j + 1) * J.out_ld + row] = v.y;
+        J.out[(int64_t)(j + 2) * J.out_ld + row] = v.z;
+        J.out[(int64_t)(j + 3) * J.out_ld + row] = v.w;
+    } else {
+        *reinterpret_cast<float4 *>(J.out + row * J.out_ld + j) = v;
+    }
+}
 
 // ---- problem plan -------------------------------------------------------------------
 
@@ -122,8 +224,7 @@ struct Plan {
     int g_splits, g_per;          // G = s dY B  : M tiles, split over N
     int da_splits, da_per;        // dA^T = X^T [G_hi|G_lo] : K tiles x chunks, split over M
     int db_splits, db_per;        // dB = dY^T [H_hi|H_lo]  : N tiles x chunks, split over M
-    int max_tiles;
-    size_t off_h2, off_g2, off_ctr, off_part, bytes;
+    size_t off_h2, off_g2, off_part, off_part2, bytes;
 };
 
 size_t align256(size_t v) { return (v + 255) / 256 * 256; }
@@ -142,18 +243,15 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int r, int sms)
     choose_splits(mt, ceil_div(N, 64), sms, 4, &pl.g_splits, &pl.g_per);
     choose_splits(kt * chunks, ceil_div(M, 64), sms, 4, &pl.da_splits, &pl.da_per);
     choose_splits(nt * chunks, ceil_div(M, 64), sms, 4, &pl.db_splits, &pl.db_per);
-    pl.max_tiles = std::max(std::max(mt, kt * chunks), nt * chunks);
     const size_t hl = align256((size_t)M * 2 * pl.r_pad * 2);
-    size_t part = 0;
-    part = std::max(part, (size_t)pl.h_splits * M * pl.r_pad * 4);
-    part = std::max(part, (size_t)pl.g_splits * M * pl.r_pad * 4);
+    size_t part = std::max((size_t)pl.h_splits, (size_t)pl.g_splits) * M * pl.r_pad * 4;
     part = std::max(part, (size_t)pl.da_splits * K * 2 * pl.r_pad * 4);
-    part = std::max(part, (size_t)pl.db_splits * N * 2 * pl.r_pad * 4);
+    const size_t part2 = (size_t)pl.db_splits * N * 2 * pl.r_pad * 4;
     pl.off_h2 = 0;
     pl.off_g2 = hl;
-    pl.off_ctr = 2 * hl;
-    pl.off_part = pl.off_ctr + align256((size_t)pl.max_tiles * 4 * sizeof(unsigned));
-    pl.bytes = pl.off_part + align256(part);
+    pl.off_part = 2 * hl;
+    pl.off_part2 = pl.off_part + align256(part);
+    pl.bytes = pl.off_part2 + align256(part2);
     return pl;
 }
 
@@ -170,19 +268,12 @@ qlora_status check_linear(const qlora_nf4_weight *w, const void *X, int64_t M, c
     return QLORA_OK;
 }
 
-// Common settings of a split-K product whose last split finalizes in place.
-void set_split(GemmParams &p, const Plan &pl, char *ws, int splits, int per, int total_stages, int64_t part_ld,
-               int64_t plane)
+void set_split(GemmParams &p, int splits, int per, int total_stages, int64_t plane)
 {
     p.splits = splits;
     p.k_stages_total = total_stages;
     p.k_stages_split = per;
-    p.part = reinterpret_cast<float *>(ws + pl.off_part);
-    p.part_ld = part_ld;
     p.split_stride = plane;
-    p.counters = reinterpret_cast<unsigned *>(ws + pl.off_ctr);
-    p.r = pl.r;
-    p.r_pad = pl.r_pad;
 }
 
 // H = s X A^T into the hi/lo buffer (and optionally fp32 H_out)
@@ -194,14 +285,22 @@ qlora_status run_h(const Plan &pl, const DeviceInfo &dev, const void *X, const v
     QLORA_TRY(map_bf16(&p.tm_b, A, pl.K, pl.r, pl.K, 64, pl.r_pad));
     p.m_tiles = ceil_div(pl.M, 128);
     p.n_tiles = 1;
-    set_split(p, pl, ws, pl.h_splits, pl.h_per, ceil_div(pl.K, 64), pl.r_pad, pl.M * pl.r_pad);
-    p.out = ws + pl.off_h2;
+    set_split(p, pl.h_splits, pl.h_per, ceil_div(pl.K, 64), pl.M * pl.r_pad);
+    p.out = ws + pl.off_part;
+    p.out_ld = pl.r_pad;
     p.m_total = (int)pl.M;
     p.n_total = pl.r_pad;
-    p.scale = scale;
-    p.out_f32 = H_out;
-    if (pl.r_pad == 64) return launch_gemm<64, kBTmaK, kEpiSplitLowRank>(p, dev, s, QLORA_KERNEL_LOWRANK);
-    return launch_gemm<128, kBTmaK, kEpiSplitLowRank>(p, dev, s, QLORA_KERNEL_LOWRANK);
+    if (pl.r_pad == 64)
+        QLORA_TRY((launch_gemm<64, kBTmaK, kEpiF32>(p, dev, s, QLORA_KERNEL_LOWRANK)));
+    else
+        QLORA_TRY((launch_gemm<128, kBTmaK, kEpiF32>(p, dev, s, QLORA_KERNEL_LOWRANK)));
+    {
+        LaunchScope ls(QLORA_KERNEL_ELEMENTWISE, s);
+        finalize_lowrank_kernel<<<elementwise_grid(pl.M * pl.r_pad / 4), 256, 0, s>>>(
+            reinterpret_cast<const float *>(ws + pl.off_part), pl.h_splits, pl.M * pl.r_pad, pl.M, pl.r, pl.r_pad,
+            scale, reinterpret_cast<__nv_bfloat16 *>(ws + pl.off_h2), H_out, nullptr, nullptr);
+    }
+    return launch_status();
 }
 
 }  // namespace
@@ -232,7 +331,6 @@ extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const void *
     if (workspace_bytes < pl.bytes) return QLORA_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     char *ws = static_cast<char *>(workspace);
-    QLORA_CUDA_TRY(cudaMemsetAsync(ws + pl.off_ctr, 0, (size_t)pl.max_tiles * 4 * sizeof(unsigned), s));
 
     QLORA_TRY(run_h(pl, dev, X, A, scale, H_save, ws, s));
 
@@ -289,7 +387,6 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *
     const Plan pl = make_plan(M, N, K, r, dev.sms);
     if (workspace_bytes < pl.bytes) return QLORA_ERR_WORKSPACE;
     char *ws = static_cast<char *>(workspace);
-    QLORA_CUDA_TRY(cudaMemsetAsync(ws + pl.off_ctr, 0, (size_t)pl.max_tiles * 4 * sizeof(unsigned), s));
     __nv_bfloat16 *H2 = reinterpret_cast<__nv_bfloat16 *>(ws + pl.off_h2);
     __nv_bfloat16 *G2 = reinterpret_cast<__nv_bfloat16 *>(ws + pl.off_g2);
     const int hl_cols = 2 * pl.r_pad;
@@ -304,17 +401,22 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *
         QLORA_TRY(map_bf16(&p.tm_b, B, r, N, r, 64, 64));      // B[n][j]: MN-major operand
         p.m_tiles = ceil_div(M, 128);
         p.n_tiles = 1;
-        set_split(p, pl, ws, pl.g_splits, pl.g_per, ceil_div(N, 64), pl.r_pad, M * pl.r_pad);
-        p.out = G2;
+        set_split(p, pl.g_splits, pl.g_per, ceil_div(N, 64), M * pl.r_pad);
+        p.out = ws + pl.off_part;
+        p.out_ld = pl.r_pad;
         p.m_total = (int)M;
         p.n_total = pl.r_pad;
-        p.scale = scale;
-        p.aux_in = H_saved;
-        p.aux_out = H2;
         if (pl.r_pad == 64)
-            QLORA_TRY((launch_gemm<64, kBTmaMN, kEpiSplitLowRank>(p, dev, s, QLORA_KERNEL_LOWRANK)));
+            QLORA_TRY((launch_gemm<64, kBTmaMN, kEpiF32>(p, dev, s, QLORA_KERNEL_LOWRANK)));
         else
-            QLORA_TRY((launch_gemm<128, kBTmaMN, kEpiSplitLowRank>(p, dev, s, QLORA_KERNEL_LOWRANK)));
+            QLORA_TRY((launch_gemm<128, kBTmaMN, kEpiF32>(p, dev, s, QLORA_KERNEL_LOWRANK)));
+        {
+            LaunchScope ls(QLORA_KERNEL_ELEMENTWISE, s);
+            finalize_lowrank_kernel<<<elementwise_grid(M * pl.r_pad / 4), 256, 0, s>>>(
+                reinterpret_cast<const float *>(ws + pl.off_part), pl.g_splits, M * pl.r_pad, M, r, pl.r_pad, scale, G2,
+                nullptr, H_saved, H_saved ? H2 : nullptr);
+        }
+        QLORA_TRY(launch_status());
     }
 
     // dX = dY W' + bf16(G) A  (fused transposed dequant-GEMM)
@@ -350,7 +452,10 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *
             QLORA_TRY((launch_gemm<kBBN, kBNf4MN, kEpiF32, kBMT>(p, dev, s, QLORA_KERNEL_BWD_FUSED)));
     }
 
-    // dA^T = X^T [G_hi | G_lo]  (rows k, chunk columns; contraction over tokens), stored transposed
+    // dA^T = X^T [G_hi | G_lo]  and  dB = dY^T [H_hi | H_lo]: rows k (resp. n), chunked
+    // hi | lo columns, contraction over tokens; one finalize adds the halves
+    float *part_a = reinterpret_cast<float *>(ws + pl.off_part);
+    float *part_b = reinterpret_cast<float *>(ws + pl.off_part2);
     {
         GemmParams p{};
         QLORA_TRY(map_bf16(&p.tm_a, X, K, M, K, 64, 64));              // MN-major A
@@ -358,16 +463,13 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *
         p.a_mn = 1;
         p.m_tiles = ceil_div(K, 128);
         p.n_tiles = pl.r_pad / 64;
-        set_split(p, pl, ws, pl.da_splits, pl.da_per, ceil_div(M, 64), hl_cols, K * hl_cols);
-        p.out = dA;
-        p.out_ld = K;
-        p.out_transposed = 1;
+        set_split(p, pl.da_splits, pl.da_per, ceil_div(M, 64), K * hl_cols);
+        p.out = part_a;
+        p.out_ld = hl_cols;
         p.m_total = (int)K;
         p.n_total = hl_cols;
-        QLORA_TRY((launch_gemm<128, kBTmaMN, kEpiSplitWgrad>(p, dev, s, QLORA_KERNEL_WGRAD)));
+        QLORA_TRY((launch_gemm<128, kBTmaMN, kEpiF32>(p, dev, s, QLORA_KERNEL_WGRAD)));
     }
-
-    // dB = dY^T [H_hi | H_lo]  (rows n, chunk columns; contraction over tokens)
     {
         GemmParams p{};
         QLORA_TRY(map_bf16(&p.tm_a, dY, N, M, N, 64, 64));              // MN-major A
@@ -375,11 +477,19 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *
         p.a_mn = 1;
         p.m_tiles = ceil_div(N, 128);
         p.n_tiles = pl.r_pad / 64;
-        set_split(p, pl, ws, pl.db_splits, pl.db_per, ceil_div(M, 64), hl_cols, N * hl_cols);
-        p.out = dB;
-        p.out_ld = r;
+        set_split(p, pl.db_splits, pl.db_per, ceil_div(M, 64), N * hl_cols);
+        p.out = part_b;
+        p.out_ld = hl_cols;
         p.m_total = (int)N;
         p.n_total = hl_cols;
-        return launch_gemm<128, kBTmaMN, kEpiSplitWgrad>(p, dev, s, QLORA_KERNEL_WGRAD);
+        QLORA_TRY((launch_gemm<128, kBTmaMN, kEpiF32>(p, dev, s, QLORA_KERNEL_WGRAD)));
     }
+    {
+        WgradJob ja{part_a, pl.da_splits, K * hl_cols, K, dA, K, 1};
+        WgradJob jb{part_b, pl.db_splits, N * hl_cols, N, dB, r, 0};
+        const int64_t n0 = K * (r / 4), n1 = N * (r / 4);
+        LaunchScope ls(QLORA_KERNEL_ELEMENTWISE, s);
+        finalize_wgrad_kernel<<<elementwise_grid(n0 + n1), 256, 0, s>>>(ja, jb, n0, r, pl.r_pad);
+    }
+    return launch_status();
 }
