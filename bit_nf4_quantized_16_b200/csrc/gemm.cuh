@@ -86,14 +86,10 @@ struct GemmCfg {
     static constexpr uint32_t kBBytes = BN * 64 * 2;
     static constexpr uint32_t kPBytes = kFused ? BN * 32 : 0;
     static constexpr uint32_t kStageBytes = kABytes + kBBytes + kPBytes;
-    static constexpr int kMaxStages = (232448 - 2048 - (kFused ? 4 * 32 * 8 * 16 : 0)) / kStageBytes;
+    static constexpr int kMaxStages = (232448 - 2048) / kStageBytes;
     static constexpr int kStages = kMaxStages > 6 ? 6 : kMaxStages;
     static constexpr uint32_t kBarOff = kStages * kStageBytes;
-    // dequantization: per-thread ring of the block constants of the next stages
-    static constexpr int kPre = 4;
-    static constexpr uint32_t kRingOff = kBarOff + 512;
-    static constexpr uint32_t kRingBytes = kFused ? kPre * 32 * kDeqWarps * 16 : 0;
-    static constexpr uint32_t kSmemBytes = kRingOff + kRingBytes + 1024;  // + alignment slack
+    static constexpr uint32_t kSmemBytes = kBarOff + 512 + 1024;  // barriers etc. + alignment slack
     static constexpr uint32_t kAccCols = MT * BN;                  // one accumulator buffer
     static constexpr uint32_t kTmemCols = 2 * kAccCols < 32 ? 32 : 2 * kAccCols;
     static_assert(2 * kAccCols <= 512, "two accumulator buffers must fit in TMEM");
@@ -376,56 +372,35 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode, MT>::kThreads, 1)
                     kb = (int64_t)nt * (BN / 64) + (blk >> 6);
                 }
             };
-            // Block constants of the next kPre main stages are copied ahead
-            // into a per-thread shared-memory ring with cp.async (one group per
-            // stage, always committed so the group count stays uniform).
-            constexpr int kPre = Cfg::kPre;
-            constexpr int kDeqThreads = 32 * Cfg::kDeqWarps;
-            // ring entry (16 B): [0] word of code2 holding the code (async),
-            // [1] c2 (async), [2] how to read the code (written directly):
-            // ~0 = no block (zero scale), 0x100 | i = byte i of word [0],
-            // 0x200 | byte = the code itself (the last word of code2 is not
-            // copied as a whole, so nothing is read past the array)
-            uint32_t *ring = reinterpret_cast<uint32_t *>(smem + Cfg::kRingOff);
-            auto issue = [&](int ks) {
-                const int slot = ks % kPre;
-                uint32_t *dst = ring + (slot * kDeqThreads + dt) * 4;
-                uint32_t how = 0xFFFFFFFFu;
-                if (ks < nmain) {
-                    int64_t n, kb;
-                    block_of(ks, n, kb);
-                    if (n < p.wrows && kb < p.kblocks) {
-                        const int64_t b = n * p.kblocks + kb;
-                        if ((b | 3) < p.wrows * p.kblocks) {
-                            cp_async_4(dst, p.code2 + (b & ~(int64_t)3));
-                            how = 0x100u | (uint32_t)(b & 3);
-                        } else {
-                            how = 0x200u | p.code2[b];
-                        }
-                        cp_async_4(dst + 1, p.c2 + (b >> 8));
-                    }
-                }
-                dst[2] = how;
-                cp_async_commit();
+            auto load_raw = [&](int ks, uint8_t &e, float &c2) -> bool {
+                int64_t n, kb;
+                block_of(ks, n, kb);
+                if (n >= p.wrows || kb >= p.kblocks) return false;
+                const int64_t b = n * p.kblocks + kb;
+                e = p.code2[b];
+                c2 = p.c2[b >> 8];
+                return true;
             };
+            // block constants of the next kPre main stages, fetched ahead in a
+            // register queue (q[0] = current stage)
+            constexpr int kPre = 4;
+            uint8_t qe[kPre];
+            float qc2[kPre];
+            bool qok[kPre];
 #pragma unroll
-            for (int i = 0; i < kPre; i++) issue(i);
+            for (int i = 0; i < kPre; i++) qok[i] = i < nmain && load_raw(i, qe[i], qc2[i]);
             bool ok = true;
             for (int ks = 0; ks < nst; ks++, it++) {
                 const int s = it % S;
                 const uint32_t use = it / S;
-                // constants of stage ks: its group is the oldest of the kPre in flight
-                cp_async_wait<kPre - 1>();
-                float c1p = 0.0f;
-                {
-                    const uint32_t *src = ring + ((ks % kPre) * kDeqThreads + dt) * 4;
-                    const uint32_t d = src[2];
-                    if (d != 0xFFFFFFFFu) {
-                        const uint8_t e = (d & 0x200u) ? (uint8_t)(d & 0xFFu) : (uint8_t)(src[0] >> (8 * (d & 3u)));
-                        c1p = block_scale(e, __uint_as_float(src[1]), mu);
-                    }
+                const float c1p = qok[0] ? block_scale(qe[0], qc2[0], mu) : 0.0f;
+#pragma unroll
+                for (int i = 0; i + 1 < kPre; i++) {
+                    qe[i] = qe[i + 1];
+                    qc2[i] = qc2[i + 1];
+                    qok[i] = qok[i + 1];
                 }
-                issue(ks + kPre);
+                qok[kPre - 1] = ks + kPre < nmain && load_raw(ks + kPre, qe[kPre - 1], qc2[kPre - 1]);
                 if (!mbar_wait_bounded(&full_a[s], use & 1, p.timeout_ns)) {
                     record_timeout(p, abort_flag);
                     ok = false;

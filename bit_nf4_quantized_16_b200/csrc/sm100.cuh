@@ -113,21 +113,6 @@ __device__ __forceinline__ void fence_proxy_async_smem()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// 4-byte asynchronous global -> shared copy (no register round trip) and its
-// group bookkeeping.
-__device__ __forceinline__ void cp_async_4(void *smem_dst, const void *gmem_src)
-{
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
-}
-
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-
-template <int N>
-__device__ __forceinline__ void cp_async_wait()
-{
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
 // ---- tcgen05 / TMEM ---------------------------------------------------------------
 
 // Allocates `ncols` TMEM columns (power of two >= 32); one full warp calls it.
