@@ -25,6 +25,7 @@
 
 #include "common.cuh"
 #include "gemm.cuh"
+#include "gemm_pair.cuh"
 
 namespace qlora {
 namespace {
@@ -90,6 +91,39 @@ qlora_status launch_gemm(GemmParams &p, const DeviceInfo &dev, cudaStream_t s, i
     {
         LaunchScope ls(kind, s);
         kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, s>>>(p);
+    }
+    return launch_status();
+}
+
+// Fused dequant-GEMM on CTA pairs: p.m_tiles / p.n_tiles count pair tiles
+// (2 * 128 * MT tokens x 256 features); one cluster of two CTAs per tile,
+// persistent over tiles, at most as many clusters as can be resident at once.
+template <int kBMode, int kEpi, int MT>
+qlora_status launch_gemm_pair(GemmParams &p, const DeviceInfo &dev, cudaStream_t s, int kind)
+{
+    using Cfg = PairCfg<kBMode, MT>;
+    static int max_clusters[64] = {};
+    auto kern = qgemm_pair_kernel<kBMode, kEpi, MT>;
+    if (!max_clusters[dev.device]) {
+        QLORA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes));
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3(2 * (dev.sms / 2));
+        cfg.blockDim = dim3(Cfg::kThreads);
+        cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+        int n = 0;
+        QLORA_CUDA_TRY(cudaOccupancyMaxActiveClusters(&n, kern, &cfg));
+        if (n < 1) return QLORA_ERR_CUDA;
+        max_clusters[dev.device] = n;
+    }
+    p.err = device_error_word();
+    if (!p.err) return QLORA_ERR_CUDA;
+    p.timeout_ns = kTimeoutNs;
+    p.splits = 1;
+    const int tiles = p.m_tiles * p.n_tiles;
+    const int clusters = tiles < max_clusters[dev.device] ? tiles : max_clusters[dev.device];
+    {
+        LaunchScope ls(kind, s);
+        kern<<<2 * clusters, Cfg::kThreads, Cfg::kSmemBytes, s>>>(p);
     }
     return launch_status();
 }
@@ -359,6 +393,13 @@ extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const void *
     p.out_ld = pl.N;
     p.m_total = (int)M;
     p.n_total = (int)pl.N;
+    if (M > 128 * kFMT) {
+        // more than one tile of tokens: CTA pairs, 512 tokens x 256 features per pair
+        p.m_tiles = ceil_div(M, 2 * 128 * kFMT);
+        p.n_tiles = ceil_div(pl.N, 2 * kFBN);
+        if (y_dtype == QLORA_BF16) return launch_gemm_pair<kBNf4K, kEpiBf16, kFMT>(p, dev, s, QLORA_KERNEL_FWD_FUSED);
+        return launch_gemm_pair<kBNf4K, kEpiF32, kFMT>(p, dev, s, QLORA_KERNEL_FWD_FUSED);
+    }
     if (y_dtype == QLORA_BF16) return launch_gemm<kFBN, kBNf4K, kEpiBf16, kFMT>(p, dev, s, QLORA_KERNEL_FWD_FUSED);
     return launch_gemm<kFBN, kBNf4K, kEpiF32, kFMT>(p, dev, s, QLORA_KERNEL_FWD_FUSED);
 }
@@ -446,7 +487,15 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *
         p.out_ld = K;
         p.m_total = (int)M;
         p.n_total = (int)K;
-        if (dx_dtype == QLORA_BF16)
+        if (M > 128 * kBMT) {
+            // CTA pairs: 512 tokens x 256 input features per pair
+            p.m_tiles = ceil_div(M, 2 * 128 * kBMT);
+            p.n_tiles = ceil_div(K, 2 * kBBN);
+            if (dx_dtype == QLORA_BF16)
+                QLORA_TRY((launch_gemm_pair<kBNf4MN, kEpiBf16, kBMT>(p, dev, s, QLORA_KERNEL_BWD_FUSED)));
+            else
+                QLORA_TRY((launch_gemm_pair<kBNf4MN, kEpiF32, kBMT>(p, dev, s, QLORA_KERNEL_BWD_FUSED)));
+        } else if (dx_dtype == QLORA_BF16)
             QLORA_TRY((launch_gemm<kBBN, kBNf4MN, kEpiBf16, kBMT>(p, dev, s, QLORA_KERNEL_BWD_FUSED)));
         else
             QLORA_TRY((launch_gemm<kBBN, kBNf4MN, kEpiF32, kBMT>(p, dev, s, QLORA_KERNEL_BWD_FUSED)));
