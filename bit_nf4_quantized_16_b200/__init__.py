@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(_HERE, "libqlora_b200.so")
 
 QLORA_BLOCK = 64
 QLORA_GROUP = 256
+QLORA_NOALLOC_MAX_BLOCKS = 1 << 20   # largest rows*cols/64 of qlora_quantize_nf4_dq_noalloc
 QLORA_BF16 = 0
 QLORA_FP32 = 1
 
@@ -28,6 +29,7 @@ STATUS = {
 # every symbol the header declares
 EXPORTS = (
     "qlora_build_nf4_codebook", "qlora_quantize_workspace_bytes", "qlora_quantize_nf4_dq",
+    "qlora_quantize_nf4_dq_noalloc",
     "qlora_dequantize_nf4_dq", "qlora_linear_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd",
     "qlora_status_string", "qlora_check_device_error",
     "qlora_timing_enable", "qlora_timing_reset", "qlora_timing_read", "qlora_launch_count",
@@ -63,6 +65,7 @@ def _load():
         "qlora_build_nf4_codebook": (ctypes.c_int, [ctypes.c_double, P]),
         "qlora_quantize_workspace_bytes": (S, [I64, I64]),
         "qlora_quantize_nf4_dq": (ctypes.c_int, [P, ctypes.c_int, W, P, S, P]),
+        "qlora_quantize_nf4_dq_noalloc": (ctypes.c_int, [P, ctypes.c_int, W, P]),
         "qlora_dequantize_nf4_dq": (ctypes.c_int, [W, P, P]),
         "qlora_linear_workspace_bytes": (S, [I64, I64, I64, I32]),
         "qlora_linear_fwd": (ctypes.c_int, [W, P, I64, P, P, I32, F, P, ctypes.c_int, P, P, S, P]),
@@ -147,6 +150,14 @@ def qlora_quantize_nf4_dq(W: torch.Tensor, out: NF4Weight, workspace: torch.Tens
     _check(lib.qlora_quantize_nf4_dq(_ptr(W), _dtype_code(W), ctypes.byref(out.desc), _ptr(workspace),
                                      workspace.numel() * workspace.element_size(), _stream(stream)),
            "qlora_quantize_nf4_dq")
+
+
+def qlora_quantize_nf4_dq_noalloc(W: torch.Tensor, out: NF4Weight, stream=None):
+    """qlora_quantize_nf4_dq with the library's fixed scratch array instead of a
+    workspace (at most QLORA_NOALLOC_MAX_BLOCKS blocks of 64; calls must not
+    overlap in time)."""
+    _check(lib.qlora_quantize_nf4_dq_noalloc(_ptr(W), _dtype_code(W), ctypes.byref(out.desc), _stream(stream)),
+           "qlora_quantize_nf4_dq_noalloc")
 
 
 def qlora_dequantize_nf4_dq(w: NF4Weight, out_bf16: torch.Tensor, stream=None):

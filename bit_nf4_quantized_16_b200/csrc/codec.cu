@@ -19,6 +19,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "exact_mean.cuh"
 #include "nf4_expand.cuh"
@@ -458,6 +460,105 @@ extern "C" qlora_status qlora_dequantize_nf4_dq(const qlora_nf4_weight *w, void 
     {
         LaunchScope ls(QLORA_KERNEL_DEQUANTIZE, s);
         dequantize_kernel<<<grid_for(p.nwords, kThreads * kDeqUnroll, dev.sms * 8), kThreads, 0, s>>>(p);
+    }
+    return launch_status();
+}
+
+// ---- quantization without allocation ------------------------------------------------
+//
+// Same kernels and results as qlora_quantize_nf4_dq, but the scratch memory
+// (reduction slots and the first-level constants c1) lives in a fixed
+// module-level device array instead of a caller-provided workspace.  For
+// callers that cannot hand over device memory at quantization time: a process
+// whose memory is already fully reserved for a pool or cache, or code that
+// quantizes weights while other streams are busy and must not call cudaMalloc
+// or cudaFree, which synchronize the device.  The array is shared by every
+// call on a device, so calls that overlap in time (two streams, two host
+// threads) race on it; the caller must order them.
+
+namespace qlora {
+namespace {
+
+constexpr size_t kStaticAccBytes = 2304;   // kAccBytes rounded up to 256 bytes
+static_assert(kStaticAccBytes >= kAccBytes, "reduction slots must fit");
+constexpr size_t kStaticScratchBytes = kStaticAccBytes + (size_t)QLORA_NOALLOC_MAX_BLOCKS * 4;
+
+// [acc 256 u64][ticket][pad][c1: QLORA_NOALLOC_MAX_BLOCKS floats], about 4 MiB per device
+static __device__ __align__(256) unsigned char g_quant_scratch[kStaticScratchBytes];
+
+constexpr int kMaxScratchDevices = 64;
+unsigned char *g_scratch_ptr[kMaxScratchDevices] = {};
+std::mutex g_scratch_mutex;
+
+// Device address of this device's scratch array; the first call per device
+// looks it up (with that device current) and caches it.
+qlora_status static_scratch(int device, unsigned char **out)
+{
+    if (device < 0 || device >= kMaxScratchDevices) return QLORA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (!g_scratch_ptr[device]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_quant_scratch) != cudaSuccess || !p) return QLORA_ERR_CUDA;
+        g_scratch_ptr[device] = static_cast<unsigned char *>(p);
+    }
+    *out = g_scratch_ptr[device];
+    return QLORA_OK;
+}
+
+}  // namespace
+}  // namespace qlora
+
+extern "C" qlora_status qlora_quantize_nf4_dq_noalloc(const void *W, qlora_dtype w_dtype,
+                                                      const qlora_nf4_weight *out, void *stream)
+{
+    if (!W || !out) return QLORA_ERR_INVALID_ARG;
+    if (w_dtype != QLORA_BF16 && w_dtype != QLORA_FP32) return QLORA_ERR_INVALID_ARG;
+    QLORA_TRY(check_weight(out));
+    if (!aligned16(W)) return QLORA_ERR_ALIGNMENT;
+    const int64_t numel = out->rows * out->cols;
+    const int64_t nblocks = numel / QLORA_BLOCK;
+    if (nblocks > QLORA_NOALLOC_MAX_BLOCKS) return QLORA_ERR_SHAPE;   // larger than the fixed scratch
+    uint32_t mkey[15];
+    QLORA_TRY(midpoint_keys(out->codebook, mkey));
+    DeviceInfo dev;
+    QLORA_TRY(device_info(&dev));
+    unsigned char *ws = nullptr;
+    QLORA_TRY(static_scratch(dev.device, &ws));
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the reduction slots and the arrival ticket start at zero on every call
+    QLORA_CUDA_TRY(cudaMemsetAsync(ws, 0, kAccBytes, s));
+
+    QuantParams qp;
+    qp.W = W;
+    qp.packed = out->packed;
+    qp.acc = reinterpret_cast<unsigned long long *>(ws);
+    qp.ticket = reinterpret_cast<unsigned int *>(ws + 256 * sizeof(unsigned long long));
+    qp.c1 = reinterpret_cast<float *>(ws + kStaticAccBytes);
+    qp.mean_out = out->mean;
+    qp.nwords = (uint32_t)(numel / 8);
+    qp.nblocks = nblocks;
+    memcpy(qp.mkey, mkey, sizeof(mkey));
+    const int grid = grid_for(qp.nwords, kThreads * kUnroll, dev.sms * 4);
+    {
+        LaunchScope ls(QLORA_KERNEL_QUANTIZE, s);
+        if (w_dtype == QLORA_FP32)
+            quantize_blocks_kernel<true><<<grid, kThreads, 0, s>>>(qp);
+        else
+            quantize_blocks_kernel<false><<<grid, kThreads, 0, s>>>(qp);
+    }
+    QLORA_TRY(launch_status());
+
+    DqParams dp;
+    dp.c1 = qp.c1;
+    dp.mean = out->mean;
+    dp.code2 = out->code2;
+    dp.c2 = out->c2;
+    dp.nblocks = nblocks;
+    dp.ngroups = (nblocks + QLORA_GROUP - 1) / QLORA_GROUP;
+    {
+        LaunchScope ls(QLORA_KERNEL_DQ_ENCODE, s);
+        dq_encode_kernel<<<grid_for(dp.ngroups, kThreads / 32, dev.sms * 8), kThreads, 0, s>>>(dp);
     }
     return launch_status();
 }

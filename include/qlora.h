@@ -144,6 +144,42 @@ QLORA_API qlora_status qlora_quantize_nf4_dq(const void *W, qlora_dtype w_dtype,
                                    void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Largest number of 64-weight blocks qlora_quantize_nf4_dq_noalloc accepts
+ * (rows * cols / 64): 2^20 blocks, i.e. 67,108,864 weights, such as 8192 x
+ * 8192.  Its fixed scratch array takes about 4 MiB of device memory per
+ * device, reserved when the library's device code is loaded.
+ */
+#define QLORA_NOALLOC_MAX_BLOCKS (1 << 20)
+
+/*
+ * qlora_quantize_nf4_dq_noalloc -- qlora_quantize_nf4_dq without a workspace.
+ * The papers describe no such variant; it is a library convenience.  It
+ * writes the same bytes as qlora_quantize_nf4_dq, but its scratch memory
+ * (reduction slots and the first-level constants) is a fixed array inside
+ * the library, so the call allocates nothing and needs no buffer from the
+ * caller: for callers that have no device memory to spare at quantization
+ * time (memory already reserved for a pool or a cache) or that must not
+ * call cudaMalloc / cudaFree, which synchronize the whole device, while
+ * other streams are running.
+ *   W, w_dtype, out  as for qlora_quantize_nf4_dq.
+ *   stream           cudaStream_t the kernels run on (NULL: legacy default).
+ * Limits and caveats:
+ *   - rows * cols / 64 must not exceed QLORA_NOALLOC_MAX_BLOCKS; larger
+ *     weights are rejected with QLORA_ERR_SHAPE before any CUDA call.
+ *   - The scratch array is one per device and shared by all calls: two calls
+ *     whose kernels may run at the same time (different streams or host
+ *     threads without ordering between them) race and corrupt each other's
+ *     results.  Order them, e.g. on one stream.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture begins.  Each call then clears the reduction
+ *     slots with cudaMemsetAsync on `stream` and launches two kernels.
+ * Errors: INVALID_ARG, SHAPE, ALIGNMENT, CUDA, UNSUPPORTED.
+ */
+QLORA_API qlora_status qlora_quantize_nf4_dq_noalloc(const void *W, qlora_dtype w_dtype,
+                                                     const qlora_nf4_weight *out, void *stream);
+
+/*
  * qlora_dequantize_nf4_dq -- expand a quantized weight to BFloat16 ("Method":
  * the tensor is dequantized to BFloat16 whenever it is used).  Per block:
  * c1' = fmaf(E4M3value(code2), c2, mean) (one rounding); per element
