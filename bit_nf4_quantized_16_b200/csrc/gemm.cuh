@@ -54,6 +54,7 @@ struct GemmParams {
     CUtensorMap tm_b;    // main B operand, or packed NF4 codes (uint8 [N][K/2])
     CUtensorMap tm_a2;   // LoRA A operand (K-major)
     CUtensorMap tm_b2;   // LoRA B operand (same majorness as the main B)
+    CUtensorMap tm_out;  // bf16 output, box 32 x 32, 64-byte swizzle (CTA-pair kernel's bf16 epilogue)
     // quantized weight constants (fused modes)
     const uint8_t *code2;
     const float *c2;

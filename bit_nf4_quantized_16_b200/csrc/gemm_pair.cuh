@@ -21,7 +21,11 @@
 //   full_b[s]   leader; expansion finished in both CTAs (16 warp arrivals)
 //   empty[s]    per CTA; the pair's MMAs that read stage s completed (multicast commit)
 //   acc_full    per CTA; accumulators ready (multicast commit)
-//   acc_empty   leader; both CTAs' epilogues drained the accumulators (8 warp arrivals)
+//   acc_empty   leader; both CTAs' epilogues drained the accumulators (16 warp arrivals)
+// Roles per CTA: warp 0 TMA, warp 1 MMA (leader only) and TMEM allocation,
+// warps 8..15 dequantization, warps 4..7 and 16..19 epilogue (two warps per
+// TMEM lane quadrant, each half of the columns; bf16 results leave through a
+// shared-memory box and a TMA store).
 // No load uses cluster multicast.
 #pragma once
 #include "gemm.cuh"
@@ -34,7 +38,8 @@ struct PairCfg {
     static constexpr int BNC = 128;   // weight columns of B per CTA
     static constexpr int NP = 2 * BNC; // MMA N of the pair
     static constexpr int kDeqWarps = 8;
-    static constexpr int kThreads = 256 + 32 * kDeqWarps;
+    static constexpr int kEpiWarps = 8;  // warps 4..7 and 16..19: two per TMEM lane quadrant
+    static constexpr int kThreads = 256 + 32 * kDeqWarps + 32 * (kEpiWarps - 4);
     static constexpr uint32_t kABytes = MT * 128 * 64 * 2;
     static constexpr uint32_t kBBytes = BNC * 64 * 2;
     static constexpr uint32_t kPBytes = BNC * 32;
@@ -42,13 +47,18 @@ struct PairCfg {
     static constexpr int kMaxStages = (232448 - 2048) / kStageBytes;
     static constexpr int kStages = kMaxStages > 6 ? 6 : kMaxStages;
     static constexpr uint32_t kBarOff = kStages * kStageBytes;
-    static constexpr uint32_t kSmemBytes = kBarOff + 512 + 1024;
+    // bf16 epilogue staging: one 32 x 32 bf16 box (2 KB) per epilogue warp
+    static constexpr uint32_t kEpiOff = kBarOff + 1024;
+    static constexpr uint32_t kEpiBoxBytes = 32 * 32 * 2;
+    static constexpr uint32_t kEpiBytes = kEpiWarps * kEpiBoxBytes;
+    static constexpr uint32_t kSmemBytes = kEpiOff + kEpiBytes + 1024;
     static constexpr uint32_t kAccCols = MT * NP;
     static constexpr int kAccBufs = 2 * kAccCols <= 512 ? 2 : 1;
     static constexpr uint32_t kTmemCols = kAccBufs * kAccCols;
     static constexpr int kTPB = (32 * kDeqWarps) / BNC;   // threads per quantization block
     static_assert(kTmemCols <= 512, "accumulators must fit in TMEM");
     static_assert(kStages >= 2, "shared memory too small");
+    static_assert(kSmemBytes + 64 <= 232448, "shared memory per block");
 };
 
 template <int kBMode, int kEpi, int MT>
@@ -95,7 +105,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<kBMode, MT>:
         }
         for (int b = 0; b < 2; b++) {
             mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], 2 * 4);
+            mbar_init(&acc_empty[b], 2 * Cfg::kEpiWarps);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -108,6 +118,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<kBMode, MT>:
             tma_prefetch_desc(&p.tm_a2);
             tma_prefetch_desc(&p.tm_b2);
         }
+        if (kEpi == kEpiBf16) tma_prefetch_desc(&p.tm_out);
     }
     if (warp == 1) {
         tmem_alloc_pair(tmem_slot, Cfg::kTmemCols);
@@ -220,10 +231,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<kBMode, MT>:
             tc_commit_pair(drain, 0x1);
             mbar_wait_bounded(drain, 0, p.timeout_ns);
         }
-    } else if (warp >= 4 && warp < 8) {
+    } else if ((warp >= 4 && warp < 8) || warp >= 16) {
         // ---------------- epilogue (both CTAs) ----------------
+        // warp (q, h): TMEM lanes 32q..32q+31, columns [h * NP/2, (h+1) * NP/2) of each accumulator
         const int q = warp & 3;
+        const int h = warp >= 16 ? 1 : 0;
         const uint32_t acc_empty_leader = at_leader(&acc_empty[0]);
+        uint8_t *box = smem + Cfg::kEpiOff + (h * 4 + q) * Cfg::kEpiBoxBytes;
+        uint32_t epi_it = 0;   // boxes stored by this warp
         uint32_t local = 0;
         for (int t = cluster_id; t < num_tiles && !*vabort; t += num_clusters, local++) {
             int mt, nt;
@@ -236,28 +251,43 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<kBMode, MT>:
             tc_fence_after();
 #pragma unroll 1
             for (int m = 0; m < MT; m++) {
-                const int row = mt * 2 * BMC + (int)rank * BMC + m * 128 + 32 * q + lane;
+                const int row0 = mt * 2 * BMC + (int)rank * BMC + m * 128 + 32 * q;
+                const int row = row0 + lane;
                 const bool row_ok = row < p.m_total;
 #pragma unroll 1
-                for (int c = 0; c < NP / 32; c++) {
+                for (int c = h * (NP / 64); c < (h + 1) * (NP / 64); c++) {
                     uint32_t r[32];
                     tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * q) << 16) + buf * Cfg::kAccCols + m * NP + 32 * c, r);
                     tmem_ld_wait();
                     const int col0 = nt * NP + 32 * c;
-                    if (!row_ok) continue;
                     if (kEpi == kEpiBf16) {
-                        __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.out) + (int64_t)row * p.out_ld + col0;
+                        // stage the warp's 32 x 32 box in shared memory (64-byte swizzle:
+                        // 16-byte chunk j of row i at j ^ ((i >> 1) & 3)), then one TMA
+                        // store; the tensor map clips rows and columns past the end
+                        if (row0 >= p.m_total || col0 >= p.n_total) continue;
+                        if (epi_it >= 1) {
+                            // the previous box's store must have read the staging buffer
+                            if (lane == 0) bulk_wait_group_read<0>();
+                            __syncwarp();
+                        }
 #pragma unroll
                         for (int g = 0; g < 4; g++) {
-                            if (col0 + 8 * g >= p.n_total) break;
                             uint4 v;
                             v.x = pack_bf16x2(__uint_as_float(r[8 * g + 0]), __uint_as_float(r[8 * g + 1]));
                             v.y = pack_bf16x2(__uint_as_float(r[8 * g + 2]), __uint_as_float(r[8 * g + 3]));
                             v.z = pack_bf16x2(__uint_as_float(r[8 * g + 4]), __uint_as_float(r[8 * g + 5]));
                             v.w = pack_bf16x2(__uint_as_float(r[8 * g + 6]), __uint_as_float(r[8 * g + 7]));
-                            *reinterpret_cast<uint4 *>(o + 8 * g) = v;
+                            *reinterpret_cast<uint4 *>(box + lane * 64 + ((g ^ ((lane >> 1) & 3)) << 4)) = v;
                         }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&p.tm_out, box, col0, row0);
+                            bulk_commit_group();
+                        }
+                        epi_it++;
                     } else {
+                        if (!row_ok) continue;
                         float *o = static_cast<float *>(p.out) + (int64_t)row * p.out_ld + col0;
 #pragma unroll
                         for (int g = 0; g < 8; g++) {
@@ -271,7 +301,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<kBMode, MT>:
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(acc_empty_leader + buf * 8u);
         }
-    } else if (warp >= 8) {
+        // the staging buffers must stay valid until the last stores have read them
+        if (kEpi == kEpiBf16 && lane == 0) bulk_wait_group_all();
+    } else if (warp >= 8 && warp < 16) {
         // ---------------- dequantization producer (both CTAs) ----------------
         // This CTA expands BNC of the pair's 256 weight columns: forward stages
         // are BNC rows of W x 64 columns, input-gradient stages 64 rows x BNC

@@ -395,6 +395,9 @@ extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const void *
     p.n_total = (int)pl.N;
     if (M > 128 * kFMT) {
         // more than one tile of tokens: CTA pairs, 512 tokens x 256 features per pair
+        if (y_dtype == QLORA_BF16)
+            QLORA_TRY(make_map(&p.tm_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, pl.N, M, pl.N * 2, 32, 32,
+                               CU_TENSOR_MAP_SWIZZLE_64B));
         p.m_tiles = ceil_div(M, 2 * 128 * kFMT);
         p.n_tiles = ceil_div(pl.N, 2 * kFBN);
         if (y_dtype == QLORA_BF16) return launch_gemm_pair<kBNf4K, kEpiBf16, kFMT>(p, dev, s, QLORA_KERNEL_FWD_FUSED);
@@ -489,6 +492,9 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *
         p.n_total = (int)K;
         if (M > 128 * kBMT) {
             // CTA pairs: 512 tokens x 256 input features per pair
+            if (dx_dtype == QLORA_BF16)
+                QLORA_TRY(make_map(&p.tm_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dX, K, M, K * 2, 32, 32,
+                                   CU_TENSOR_MAP_SWIZZLE_64B));
             p.m_tiles = ceil_div(M, 2 * 128 * kBMT);
             p.n_tiles = ceil_div(K, 2 * kBBN);
             if (dx_dtype == QLORA_BF16)
