@@ -189,14 +189,19 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     q.qlora_check_device_error()
 
-    # ---- timed region
+    # ---- timed region (headline): no per-launch events, so that consecutive
+    # kernels overlap set-up and tail as they do for a user
     launches0 = q.qlora_launch_count()
-    q.qlora_timing_reset()
-    q.qlora_timing_enable(True)
     with ClockSampler(local_rank) as clk:
         ms = timed_steps(args.steps, step)
-    q.qlora_timing_enable(False)
     launches = q.qlora_launch_count() - launches0
+    q.qlora_check_device_error()
+    # ---- per-kernel device times: the same steps again with CUDA events around
+    # every launch (on the launching stream)
+    q.qlora_timing_reset()
+    q.qlora_timing_enable(True)
+    ms_events = timed_steps(args.steps, step)
+    q.qlora_timing_enable(False)
     kern = q.qlora_timing_read()
     q.qlora_check_device_error()
     clocks = clk.summary()
@@ -241,10 +246,12 @@ def run_ours(args, rank, world, local_rank):
     dom = max(("fwd_fused", "bwd_fused"), key=lambda k: kern[k][0])
     dom_ms, dom_n = kern[dom]
     achieved = kflops[dom] / (dom_ms * 1e-3) / 1e12
-    peak = peaks["bf16_tflops_sustained"]
+    # burst peak: the timed region lasts tens of milliseconds and the SM clock
+    # stays at its maximum (the sustained figure is for seconds under the power cap)
+    peak = peaks["bf16_tflops"]
     roofline = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
                 "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
-                "peak_source": f"{peak_src} bf16_tflops_sustained",
+                "peak_source": f"{peak_src} bf16_tflops (burst)",
                 "launches": dom_n, "avg_launch_ms": round(dom_ms / max(dom_n, 1), 4)}
     breakdown = {k: {"ms_per_step": round(v[0] / args.steps, 4), "launches_per_step": v[1] // args.steps}
                  for k, v in kern.items() if v[1]}

@@ -171,6 +171,9 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode, MT>::kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // everything above overlaps the previous kernel's tail; inputs are read below
+    pdl_wait();
+    pdl_trigger();
     const uint32_t tmem_base = *tmem_slot;
     const int num_tiles = p.m_tiles * p.n_tiles * p.splits;
     volatile int *vabort = abort_flag;

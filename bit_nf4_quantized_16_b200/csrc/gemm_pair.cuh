@@ -128,6 +128,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<kBMode, MT>:
     __syncthreads();
     cluster_sync();   // barriers of both CTAs initialized before any remote arrive
     tc_fence_after();
+    // everything above overlaps the previous kernel's tail; inputs are read below
+    pdl_wait();
+    pdl_trigger();
     const uint32_t tmem_base = *tmem_slot;
     const int num_tiles = p.m_tiles * p.n_tiles;
     const int cluster_id = blockIdx.x >> 1, num_clusters = gridDim.x >> 1;

@@ -22,6 +22,7 @@
 #include <cuda_bf16.h>
 #include <algorithm>
 #include <mutex>
+#include <utility>
 
 #include "common.cuh"
 #include "gemm.cuh"
@@ -71,6 +72,28 @@ qlora_status map_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint64_t
                     CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+// ---- launches ------------------------------------------------------------------------
+
+// Every kernel of the linear path is launched with programmatic stream
+// serialization: its set-up (barrier init, TMEM allocation, descriptor
+// prefetch) overlaps the tail of the kernel before it, and it waits
+// (griddepcontrol.wait) before reading anything that kernel produced.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args &&...args)
+{
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // ---- GEMM launch ------------------------------------------------------------------
 
 template <int BN, int kBMode, int kEpi, int MT = 1>
@@ -90,7 +113,7 @@ qlora_status launch_gemm(GemmParams &p, const DeviceInfo &dev, cudaStream_t s, i
     const int grid = tiles < dev.sms ? tiles : dev.sms;
     {
         LaunchScope ls(kind, s);
-        kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, s>>>(p);
+        QLORA_CUDA_TRY(launch_pdl(kern, dim3(grid), dim3(Cfg::kThreads), Cfg::kSmemBytes, s, p));
     }
     return launch_status();
 }
@@ -123,7 +146,7 @@ qlora_status launch_gemm_pair(GemmParams &p, const DeviceInfo &dev, cudaStream_t
     const int clusters = tiles < max_clusters[dev.device] ? tiles : max_clusters[dev.device];
     {
         LaunchScope ls(kind, s);
-        kern<<<2 * clusters, Cfg::kThreads, Cfg::kSmemBytes, s>>>(p);
+        QLORA_CUDA_TRY(launch_pdl(kern, dim3(2 * clusters), dim3(Cfg::kThreads), Cfg::kSmemBytes, s, p));
     }
     return launch_status();
 }
@@ -190,6 +213,8 @@ __global__ void finalize_lowrank_kernel(const float *part, int splits, int64_t s
                                         int r_pad, float scale, __nv_bfloat16 *out, float *out_f32,
                                         const float *aux_in, __nv_bfloat16 *aux_out)
 {
+    sm100::pdl_wait();
+    sm100::pdl_trigger();
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int per_row = r_pad / 4;
     if (i >= M * per_row) return;
@@ -225,6 +250,8 @@ struct WgradJob {
 
 __global__ void finalize_wgrad_kernel(WgradJob j0, WgradJob j1, int64_t n0, int r, int r_pad)
 {
+    sm100::pdl_wait();
+    sm100::pdl_trigger();
     int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int per_row = r / 4;
     const WgradJob &J = i < n0 ? j0 : j1;
@@ -330,9 +357,11 @@ qlora_status run_h(const Plan &pl, const DeviceInfo &dev, const void *X, const v
         QLORA_TRY((launch_gemm<128, kBTmaK, kEpiF32>(p, dev, s, QLORA_KERNEL_LOWRANK)));
     {
         LaunchScope ls(QLORA_KERNEL_ELEMENTWISE, s);
-        finalize_lowrank_kernel<<<elementwise_grid(pl.M * pl.r_pad / 4), 256, 0, s>>>(
-            reinterpret_cast<const float *>(ws + pl.off_part), pl.h_splits, pl.M * pl.r_pad, pl.M, pl.r, pl.r_pad,
-            scale, reinterpret_cast<__nv_bfloat16 *>(ws + pl.off_h2), H_out, nullptr, nullptr);
+        QLORA_CUDA_TRY(launch_pdl(finalize_lowrank_kernel, dim3(elementwise_grid(pl.M * pl.r_pad / 4)), dim3(256), 0,
+                                  s, reinterpret_cast<const float *>(ws + pl.off_part), pl.h_splits,
+                                  (int64_t)(pl.M * pl.r_pad), pl.M, pl.r, pl.r_pad, scale,
+                                  reinterpret_cast<__nv_bfloat16 *>(ws + pl.off_h2), H_out, (const float *)nullptr,
+                                  (__nv_bfloat16 *)nullptr));
     }
     return launch_status();
 }
@@ -456,9 +485,10 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *
             QLORA_TRY((launch_gemm<128, kBTmaMN, kEpiF32>(p, dev, s, QLORA_KERNEL_LOWRANK)));
         {
             LaunchScope ls(QLORA_KERNEL_ELEMENTWISE, s);
-            finalize_lowrank_kernel<<<elementwise_grid(M * pl.r_pad / 4), 256, 0, s>>>(
-                reinterpret_cast<const float *>(ws + pl.off_part), pl.g_splits, M * pl.r_pad, M, r, pl.r_pad, scale, G2,
-                nullptr, H_saved, H_saved ? H2 : nullptr);
+            QLORA_CUDA_TRY(launch_pdl(finalize_lowrank_kernel, dim3(elementwise_grid(M * pl.r_pad / 4)), dim3(256), 0,
+                                      s, reinterpret_cast<const float *>(ws + pl.off_part), pl.g_splits,
+                                      (int64_t)(M * pl.r_pad), M, r, pl.r_pad, scale, G2, (float *)nullptr, H_saved,
+                                      H_saved ? H2 : (__nv_bfloat16 *)nullptr));
         }
         QLORA_TRY(launch_status());
     }
@@ -544,7 +574,8 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *
         WgradJob jb{part_b, pl.db_splits, N * hl_cols, N, dB, r, 0};
         const int64_t n0 = K * (r / 4), n1 = N * (r / 4);
         LaunchScope ls(QLORA_KERNEL_ELEMENTWISE, s);
-        finalize_wgrad_kernel<<<elementwise_grid(n0 + n1), 256, 0, s>>>(ja, jb, n0, r, pl.r_pad);
+        QLORA_CUDA_TRY(launch_pdl(finalize_wgrad_kernel, dim3(elementwise_grid(n0 + n1)), dim3(256), 0, s, ja, jb,
+                                  (int64_t)n0, r, pl.r_pad));
     }
     return launch_status();
 }

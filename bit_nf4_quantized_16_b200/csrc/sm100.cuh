@@ -28,6 +28,17 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p)
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// ---- programmatic dependent launch -----------------------------------------------
+// A kernel launched with programmatic stream serialization may start while the
+// previous kernel in the stream is still running.  pdl_wait() blocks until
+// that kernel has completed and its memory operations are visible (a no-op for
+// an ordinary launch); pdl_trigger() lets the next such kernel start once
+// every CTA of this grid has issued it or exited.
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---- mbarrier ---------------------------------------------------------------------
 
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
