@@ -43,6 +43,37 @@ def linear_flops(M, N, K, r):
     return 4 * M * N * K + 6 * M * r * (N + K)
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch from one
+# ncu capture of the bench workloads, averaged over the launches of one step
+# (profiles/dram_traffic_linear7b_codec.md).  Each set describes the kernel
+# sources whose SHA-256 it names and is reported only while they are unchanged.
+_CSRC = os.path.join("bit_nf4_quantized_16_b200", "csrc")
+MEASURED_TRAFFIC = {
+    "linear": {
+        "sources": ["gemm_pair.cuh", "gemm.cuh", "sm100.cuh", "nf4_expand.cuh", "linear.cu"],
+        "sha256": "14a786a9c05fc602d83381985c4830f790a52311e45e2c841b553636136d8ea4",
+        "bytes": {"fwd_fused": 98.8e6, "bwd_fused": 112.2e6},
+    },
+    "codec": {
+        "sources": ["codec.cu", "nf4_expand.cuh", "exact_mean.cuh"],
+        "sha256": "fe37e1bdd9262e07231195263c9a179e0d91d21c79794e843349bae541510c2f",
+        "bytes": {"quantize": 59.3e6, "dequantize": 27.1e6},
+    },
+}
+
+
+def measured_traffic(group, kernel):
+    import hashlib
+    t = MEASURED_TRAFFIC[group]
+    h = hashlib.sha256()
+    for f in t["sources"]:
+        with open(os.path.join(ROOT, _CSRC, f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest() != t["sha256"]:
+        return None   # the kernels changed since the capture
+    return t["bytes"].get(kernel)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -250,7 +281,7 @@ def run_ours(args, rank, world, local_rank):
     # stays at its maximum (the sustained figure is for seconds under the power cap)
     peak = peaks["bf16_tflops"]
     roofline = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
-                "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": measured_traffic("linear", dom),
                 "peak_source": f"{peak_src} bf16_tflops (burst)",
                 "launches": dom_n, "avg_launch_ms": round(dom_ms / max(dom_n, 1), 4)}
     breakdown = {k: {"ms_per_step": round(v[0] / args.steps, 4), "launches_per_step": v[1] // args.steps}
@@ -349,7 +380,8 @@ def run_codec(args, q, torch, dev, peaks, peak_src):
         "value": round(gbs, 1), "unit": "GB/s", "ms_per_step": round(ms, 4),
         "weights_per_s": nweights / (ms * 1e-3),
         "roofline": {"kernel": dom, "bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(ach / peak, 4), "traffic": None, "peak_source": f"{peak_src} hbm_gbs"},
+                     "frac": round(ach / peak, 4), "traffic": measured_traffic("codec", dom),
+                     "peak_source": f"{peak_src} hbm_gbs"},
         "kernels": {"quantize_gbs": round(qgbs, 1), "dequantize_gbs": round(dgbs, 1),
                     "dq_encode_ms": round(kern["dq_encode"][0], 4),
                     "quantize_ms": round(qms, 4), "dequantize_ms": round(dms, 4)},
