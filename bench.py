@@ -288,6 +288,7 @@ def run_ours(args, rank, world, local_rank):
                  for k, v in kern.items() if v[1]}
 
     codec = run_codec(args, q, torch, dev, peaks, peak_src) if (rank == 0 and not args.skip_codec) else None
+    decode = run_decode65b(args, q, torch, dev, peaks, peak_src) if (rank == 0 and not args.skip_decode) else None
 
     if rank != 0:
         return None
@@ -310,6 +311,8 @@ def run_ours(args, rank, world, local_rank):
     }
     if codec is not None:
         line["codec"] = codec
+    if decode is not None:
+        line["decode65b"] = decode
     if world == 1 and not args.skip_cpu:
         line["cpu_baseline"] = cpu_baseline_linear(budget_s=args.cpu_seconds)
     return line
@@ -386,6 +389,84 @@ def run_codec(args, q, torch, dev, peaks, peak_src):
                     "dq_encode_ms": round(kern["dq_encode"][0], 4),
                     "quantize_ms": round(qms, 4), "dequantize_ms": round(dms, 4)},
     }
+
+
+def weight_bytes(N, K):
+    """Bytes of one quantized weight: packed codes, E4M3 block codes, group scales."""
+    nblocks = N * K // 64
+    return N * K // 2 + nblocks + 4 * (-(-nblocks // 256))
+
+
+def run_decode65b(args, q, torch, dev, peaks, peak_src):
+    """Decode-shaped forward of the seven LLaMA-65B linears at 1, 4 and 16
+    tokens: every call streams its packed weight from HBM once.  One step is
+    the seven linears; the 437 MB of weights per step exceed L2, so nothing
+    needs flushing."""
+    import synthetic
+    shapes = synthetic.LLAMA65B_LINEARS
+    qws = torch.empty(max(q.qlora_quantize_workspace_bytes(N, K) for _, N, K in shapes), dtype=torch.uint8,
+                      device=dev)
+    layers = []
+    for i, (name, N, K) in enumerate(shapes):
+        W = synthetic.normal((N, K), 0.02, 70_000 + i, torch.bfloat16, dev)
+        w = q.NF4Weight(N, K, device=dev)
+        q.qlora_quantize_nf4_dq(W, w, qws)
+        del W
+        layers.append({"N": N, "K": K, "w": w,
+                       "A": synthetic.normal((R, K), 1.0 / R, 70_100 + i, torch.bfloat16, dev),
+                       "B": synthetic.normal((N, R), 0.01, 70_200 + i, torch.bfloat16, dev)})
+    del qws
+    scale = ALPHA / R
+    out = {"workload": "decode65b: forward of the 7 LLaMA-65B linears (8192x8192 x4, 22016x8192 x2, 8192x22016), "
+                       "r=64, bf16 activations, tokens 1/4/16", "unit": "GB/s", "tokens": {}}
+    for M in (1, 4, 16):
+        ws = torch.empty(max(q.qlora_linear_workspace_bytes(M, L["N"], L["K"], R) for L in layers),
+                         dtype=torch.uint8, device=dev)
+        for L in layers:
+            L["X"] = synthetic.normal((M, L["K"]), 1.0, 70_300 + M, torch.bfloat16, dev)
+            L["Y"] = torch.empty(M, L["N"], dtype=torch.bfloat16, device=dev)
+
+        def step():
+            for L in layers:
+                q.qlora_linear_fwd(L["w"], L["X"], M, L["A"], L["B"], R, scale, L["Y"], None, ws)
+
+        for _ in range(max(args.warmup, 3)):
+            step()
+        torch.cuda.synchronize()
+        q.qlora_check_device_error()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = max(args.steps, 10)
+        torch.cuda._sleep(20_000_000)
+        e0.record()
+        for _ in range(reps):
+            step()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        # algorithmic bytes: quantized weights, adapters, activations in and out
+        nbytes = sum(weight_bytes(L["N"], L["K"]) + 2 * R * (L["N"] + L["K"]) + 2 * M * (L["N"] + L["K"])
+                     for L in layers)
+        q.qlora_timing_reset()
+        q.qlora_timing_enable(True)
+        torch.cuda._sleep(20_000_000)
+        for _ in range(reps):
+            step()
+        q.qlora_timing_enable(False)
+        kern = q.qlora_timing_read()
+        q.qlora_check_device_error()
+        gemv_ms = kern["fwd_fused"][0] / reps
+        gemv_bytes = sum(weight_bytes(L["N"], L["K"]) + 2 * R * L["K"] + 2 * M * L["K"] + 4 * M * L["N"]
+                         for L in layers)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        ach = gemv_bytes / (gemv_ms * 1e-3) / 1e9
+        out["tokens"][str(M)] = {
+            "value": round(gbs, 1), "us_per_layer": round(ms * 1e3, 2), "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
+            "roofline": {"kernel": "decode_gemv", "bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": None,
+                         "peak_source": f"{peak_src} hbm_gbs"},
+            "kernels_us": {k: round(v[0] / reps * 1e3, 2) for k, v in kern.items() if v[1]},
+        }
+    return out
 
 
 # ---- CPU baselines (the oracle, as it stands) ---------------------------------------
@@ -484,6 +565,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--skip-codec", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--skip-decode", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--linears", default="llama7b",
                     help="llama7b (the seven linears of one layer) or NxK for one linear (profiling runs)")

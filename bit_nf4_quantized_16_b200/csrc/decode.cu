@@ -1,0 +1,378 @@
+// QLoRA forward for a handful of tokens (M <= 16) on sm_100a: the decode
+// shape, where the product is bound by streaming the packed 4-bit weight
+// from HBM (0.516 B per weight against 2 M FLOP).
+//
+//   Y = X W'^T + H B^T,  H = s X A^T
+//
+// ("QLoRA: Efficient Finetuning of Quantized LLMs", section "Method": the
+// 4-bit weight is dequantized to BFloat16 and multiplied in 16-bit; the LoRA
+// term x_out = (W + BA) x_in from the mbrenndoerfer.com essay, section
+// "Low-Rank Adaptation (LoRA)").
+//
+// decode_gemv_kernel: each warp owns 16 rows of W (or of A) and a range of the
+// contraction.  Every lane streams the packed codes of its two rows with
+// 16-byte loads (32 codes = 32 consecutive k per row), expands them with the
+// dequantizer's own arithmetic (nf4::expand8, bit-identical bf16) straight
+// into the A fragments of mma.sync m16n8k16, and multiplies them with X.  The
+// contraction index is permuted the same way on both operands (a fragment's
+// k slots map to the lane's 32 consecutive k), so no shared-memory transpose
+// is needed; the tensor cores only replace the 2 M FMAs per weight that CUDA
+// cores could not keep up with at 16 tokens.  Rows of A (the LoRA down
+// projection) run through the same loop without expansion.  Partial products
+// of each contraction split are written in fp32.
+//
+// decode_finalize_kernel: sums the splits in a fixed order (deterministic),
+// forms H = s X A^T (fp32, optionally saved for the backward pass), adds
+// H B^T and stores Y in bf16 or fp32.
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "decode.cuh"
+#include "nf4_expand.cuh"
+#include "sm100.cuh"
+
+namespace qlora {
+namespace {
+
+constexpr int kDecWarps = 8;                    // 16 rows each: 128 rows per CTA
+constexpr int kDecThreads = 32 * kDecWarps;
+constexpr int kDecRows = 16 * kDecWarps;
+constexpr int kDecCtasPerSm = 2;   // resident CTAs per SM (registers: the prefetched steps)
+
+struct DecodeParams {
+    const uint8_t *packed;
+    const uint8_t *code2;
+    const float *c2;
+    const float *mean;
+    float q[16];
+    const __nv_bfloat16 *X;   // [M][K]
+    const __nv_bfloat16 *A;   // [r][K]
+    int64_t N, K, kblocks;
+    int M, r;
+    int row_tiles;            // CTAs along the rows of W; the CTAs after them take the rows of A
+    int dblk_per_split;       // 128-wide contraction steps per split
+    int n_dblk;               // total 128-wide steps (the last may hold only 64)
+    float *part;              // [splits][M][N]: partial products of W
+    float *part_h;            // [kAPieces][M][r]: partial products of A
+};
+
+// The rows of A are bf16 already (4x the bytes of a packed row): their whole
+// contraction is cut into kAPieces ranges, one warp per (16 rows, range), all
+// in the CTAs of split 0.
+constexpr int kAPieces = 8;
+// 128-wide steps of W in flight per warp (fewer with two token tiles, whose
+// accumulators and X fragments take the registers)
+template <int NT>
+constexpr int prefetch_depth() { return NT == 1 ? 4 : 3; }
+
+__device__ __forceinline__ uint4 ld_stream_v4(const void *p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint4 ld_cached_v4(const void *p)
+{
+    return __ldg(reinterpret_cast<const uint4 *>(p));
+}
+
+// D += A B, m16n8k16, bf16 inputs, fp32 accumulators.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// One 128-wide step of this lane's two rows: packed codes and block constants.
+// Loads only: nothing computed from a loaded value until the step is used,
+// so issuing the next step's loads never waits for them.
+struct WStage {
+    uint4 pg, pg8;
+    uint32_t eg, eg8;   // E4M3 block codes of rows g and g+8
+    float c2g, c2g8;
+};
+
+// Fragment layout (lane = 4 g + c): A regs {a0a1, a2a3, a4a5, a6a7} hold rows
+// g, g+8, g, g+8 at k slots {2c, 2c+1}, {2c, 2c+1}, {2c+8, 2c+9}, {2c+8, 2c+9};
+// B regs {b0b1, b2b3} hold token g at the same two slot pairs.  Slot pair
+// {2c, 2c+1} of step t is real k = base + 32 c + 4 t + {0, 1}, pair {2c+8,
+// 2c+9} is + {2, 3}: lane c's 32 consecutive k feed 8 steps, four per step.
+// mma.sync is warp-collective: every lane calls this; lanes whose k is past the
+// end pass kin = false and multiply zeros.
+template <int NT>
+__device__ __forceinline__ void mma_step(float (&acc)[NT][2][4], const uint4 (&ea)[4], const uint4 (&eb)[4],
+                                         const __nv_bfloat16 *const (&xrow)[NT], const bool (&xok)[NT], int64_t k,
+                                         bool kin)
+{
+#pragma unroll
+    for (int w = 0; w < 4; w++) {
+#pragma unroll
+        for (int t = 0; t < NT; t++) {
+            const uint4 xb = (xok[t] && kin) ? ld_cached_v4(xrow[t] + k + 8 * w) : make_uint4(0, 0, 0, 0);
+            mma_bf16_16816(acc[t][0], ea[w].x, eb[w].x, ea[w].y, eb[w].y, xb.x, xb.y);
+            mma_bf16_16816(acc[t][0], ea[w].z, eb[w].z, ea[w].w, eb[w].w, xb.z, xb.w);
+        }
+    }
+}
+
+template <int NT>
+__global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm) decode_gemv_kernel(const __grid_constant__ DecodeParams p)
+{
+    __shared__ float lut[16];
+    sm100::pdl_wait();
+    sm100::pdl_trigger();
+    if (threadIdx.x < 16) lut[threadIdx.x] = p.q[threadIdx.x];
+    __syncthreads();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, c = lane & 3;
+    const int sp = blockIdx.y;
+    int d0 = sp * p.dblk_per_split;
+    int d1 = min(d0 + p.dblk_per_split, p.n_dblk);
+
+    float acc[NT][2][4];
+#pragma unroll
+    for (int t = 0; t < NT; t++)
+#pragma unroll
+        for (int i = 0; i < 4; i++) acc[t][0][i] = acc[t][1][i] = 0.0f;
+    const __nv_bfloat16 *xrow[NT];
+    bool xok[NT];
+#pragma unroll
+    for (int t = 0; t < NT; t++) {
+        const int tok = 8 * t + g;
+        xok[t] = tok < p.M;
+        xrow[t] = p.X + (int64_t)(xok[t] ? tok : 0) * p.K;
+    }
+
+    if ((int)blockIdx.x >= p.row_tiles) {
+        // ---- rows of A: warp task = (16-row group, piece of the contraction)
+        if (sp != 0) return;
+        const int groups = (p.r + 15) / 16;
+        const int task = ((int)blockIdx.x - p.row_tiles) * kDecWarps + warp;
+        const int grp = task % groups, qtr = task / groups;
+        if (qtr >= kAPieces) return;
+        const int qper = (p.n_dblk + kAPieces - 1) / kAPieces;
+        d0 = qtr * qper;
+        d1 = min(p.n_dblk, d0 + qper);
+        const int64_t rg = 16 * grp + g, rg8 = rg + 8;
+        const bool ok_g = rg < p.r, ok_g8 = rg8 < p.r;
+        for (int d = d0; d < d1; d++) {
+            const int64_t k = (int64_t)d * 128 + 32 * c;
+            const bool k_ok = k < p.K;
+            uint4 ea[4], eb[4];
+#pragma unroll
+            for (int w = 0; w < 4; w++) {
+                ea[w] = (ok_g && k_ok) ? ld_cached_v4(p.A + rg * p.K + k + 8 * w) : make_uint4(0, 0, 0, 0);
+                eb[w] = (ok_g8 && k_ok) ? ld_cached_v4(p.A + rg8 * p.K + k + 8 * w) : make_uint4(0, 0, 0, 0);
+            }
+            mma_step<NT>(acc, ea, eb, xrow, xok, k, k_ok);
+        }
+        float *part = p.part_h + (int64_t)qtr * p.M * p.r;
+#pragma unroll
+        for (int t = 0; t < NT; t++) {
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                const int tok = 8 * t + 2 * c + (i & 1);
+                const int64_t row = (i < 2) ? rg : rg8;
+                if (tok < p.M && row < p.r) part[(int64_t)tok * p.r + row] = __fadd_rn(acc[t][0][i], acc[t][1][i]);
+            }
+        }
+        return;
+    }
+
+    // ---- rows of W: packed codes streamed kPrefetch steps ahead
+    constexpr int kPrefetch = prefetch_depth<NT>();
+    const int64_t row0 = (int64_t)blockIdx.x * kDecRows + 16 * warp;
+    if (row0 >= p.N) return;
+    const int64_t rg = row0 + g, rg8 = row0 + g + 8;
+    const bool ok_g = rg < p.N, ok_g8 = rg8 < p.N;
+    const float mu = *p.mean;
+    const int64_t half_k = p.K / 2;
+    auto load = [&](int d, WStage &st) {
+        const int64_t k = (int64_t)d * 128 + 32 * c;
+        const bool in = d < d1 && k < p.K;
+        const uint4 z = make_uint4(0, 0, 0, 0);
+        st.pg = (in && ok_g) ? ld_stream_v4(p.packed + rg * half_k + k / 2) : z;
+        st.pg8 = (in && ok_g8) ? ld_stream_v4(p.packed + rg8 * half_k + k / 2) : z;
+        const int64_t b = rg * p.kblocks + k / 64, b8 = rg8 * p.kblocks + k / 64;
+        st.eg = (in && ok_g) ? (uint32_t)__ldg(p.code2 + b) : 0u;
+        st.c2g = (in && ok_g) ? __ldg(p.c2 + (b >> 8)) : 0.0f;
+        st.eg8 = (in && ok_g8) ? (uint32_t)__ldg(p.code2 + b8) : 0u;
+        st.c2g8 = (in && ok_g8) ? __ldg(p.c2 + (b8 >> 8)) : 0.0f;
+    };
+    WStage st[kPrefetch];
+#pragma unroll
+    for (int i = 0; i < kPrefetch; i++) load(d0 + i, st[i]);
+    for (int d = d0; d < d1; d += kPrefetch) {
+#pragma unroll
+        for (int i = 0; i < kPrefetch; i++) {
+            if (d + i < d1) {
+                const int64_t k = (int64_t)(d + i) * 128 + 32 * c;
+                const bool kin = k < p.K;   // false only for the upper half of a final 64-wide step
+                {
+                    const float sg = (ok_g && kin) ? nf4::block_scale((uint8_t)st[i].eg, st[i].c2g, mu) : 0.0f;
+                    const float sg8 = (ok_g8 && kin) ? nf4::block_scale((uint8_t)st[i].eg8, st[i].c2g8, mu) : 0.0f;
+                    uint4 ea[4], eb[4];
+                    ea[0] = nf4::expand8(st[i].pg.x, lut, sg);
+                    ea[1] = nf4::expand8(st[i].pg.y, lut, sg);
+                    ea[2] = nf4::expand8(st[i].pg.z, lut, sg);
+                    ea[3] = nf4::expand8(st[i].pg.w, lut, sg);
+                    eb[0] = nf4::expand8(st[i].pg8.x, lut, sg8);
+                    eb[1] = nf4::expand8(st[i].pg8.y, lut, sg8);
+                    eb[2] = nf4::expand8(st[i].pg8.z, lut, sg8);
+                    eb[3] = nf4::expand8(st[i].pg8.w, lut, sg8);
+                    mma_step<NT>(acc, ea, eb, xrow, xok, k, kin);
+                }
+                load(d + i + kPrefetch, st[i]);
+            }
+        }
+    }
+
+    // acc[t] = {(row g, token 8t+2c), (row g, 8t+2c+1), (row g+8, 8t+2c), (row g+8, 8t+2c+1)}
+    float *part = p.part + (int64_t)sp * p.M * p.N;
+#pragma unroll
+    for (int t = 0; t < NT; t++) {
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const int tok = 8 * t + 2 * c + (i & 1);
+            const int64_t row = (i < 2) ? rg : rg8;
+            if (tok < p.M && row < p.N) part[(int64_t)tok * p.N + row] = __fadd_rn(acc[t][0][i], acc[t][1][i]);
+        }
+    }
+}
+
+// One CTA per 256 outputs n (all tokens): the H rows of every token from the
+// A partials (fixed order) in shared memory, B[n] in registers, then
+// y[m][n] = sum of the W splits + H[m] . B[n].
+__global__ void __launch_bounds__(256) decode_finalize_kernel(const float *part, const float *part_h, int splits,
+                                                            int M, int64_t N, int r, float scale,
+                                                            const __nv_bfloat16 *B, void *Y, int y_f32,
+                                                            float *H_save)
+{
+    __shared__ float h[kDecodeMaxTokens * 128];
+    sm100::pdl_wait();
+    sm100::pdl_trigger();
+    for (int i = threadIdx.x; i < M * r; i += blockDim.x) {
+        float v = 0.0f;
+#pragma unroll
+        for (int s = 0; s < kAPieces; s++) v = __fadd_rn(v, part_h[(int64_t)s * M * r + i]);
+        v = __fmul_rn(scale, v);
+        h[i] = v;
+        if (H_save && blockIdx.x == 0) H_save[i] = v;
+    }
+    __syncthreads();
+    const int64_t n = (int64_t)blockIdx.x * 256 + threadIdx.x;
+    if (n >= N) return;
+    uint4 bv[16];   // B[n][0 .. r), r <= 128
+    const __nv_bfloat16 *bn = B + n * r;
+#pragma unroll
+    for (int j = 0; j < 16; j++) bv[j] = (8 * j < r) ? *reinterpret_cast<const uint4 *>(bn + 8 * j) : make_uint4(0, 0, 0, 0);
+    for (int m = 0; m < M; m++) {
+        float y = 0.0f;
+        for (int s = 0; s < splits; s++) y = __fadd_rn(y, part[((int64_t)s * M + m) * N + n]);
+        const float *hm = h + m * r;
+        float l = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 16; j++) {
+            if (8 * j >= r) break;
+            const uint32_t w[4] = {bv[j].x, bv[j].y, bv[j].z, bv[j].w};
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                l = __fmaf_rn(hm[8 * j + 2 * i], __uint_as_float(w[i] << 16), l);
+                l = __fmaf_rn(hm[8 * j + 2 * i + 1], __uint_as_float(w[i] & 0xFFFF0000u), l);
+            }
+        }
+        y = __fadd_rn(y, l);
+        if (y_f32)
+            static_cast<float *>(Y)[(int64_t)m * N + n] = y;
+        else
+            static_cast<__nv_bfloat16 *>(Y)[(int64_t)m * N + n] = __float2bfloat16_rn(y);
+    }
+}
+
+int ceil_div_i(int64_t a, int64_t b) { return (int)((a + b - 1) / b); }
+
+struct DecodePlan {
+    int row_tiles, a_ctas, n_dblk, splits, per;
+    size_t part_bytes, part_h_bytes;
+};
+
+DecodePlan decode_plan(int64_t M, int64_t N, int64_t K, int r, int sms)
+{
+    DecodePlan d;
+    d.row_tiles = ceil_div_i(N, kDecRows);
+    d.a_ctas = ceil_div_i((int64_t)((r + 15) / 16) * kAPieces, kDecWarps);
+    d.n_dblk = ceil_div_i(K, 128);
+    // about three CTAs per SM in all (1.5 waves at two resident per SM: measured
+    // faster than a single wave), at least two 128-wide steps per split
+    int want = ceil_div_i((int64_t)3 * sms, d.row_tiles + d.a_ctas);
+    want = std::max(1, std::min(want, std::max(1, d.n_dblk / 2)));
+    d.per = ceil_div_i(d.n_dblk, want);
+    d.splits = ceil_div_i(d.n_dblk, d.per);
+    d.part_bytes = ((size_t)d.splits * M * N * 4 + 255) / 256 * 256;
+    d.part_h_bytes = (size_t)kAPieces * M * r * 4;
+    return d;
+}
+
+}  // namespace
+
+size_t decode_workspace_bytes(int64_t M, int64_t N, int64_t K, int r, int sms)
+{
+    const DecodePlan d = decode_plan(M, N, K, r, sms);
+    return d.part_bytes + d.part_h_bytes;
+}
+
+qlora_status run_decode_fwd(const qlora_nf4_weight *w, const void *X, int64_t M, const void *A, const void *B, int r,
+                            float scale, void *Y, qlora_dtype y_dtype, float *H_save, void *ws, size_t ws_bytes,
+                            const DeviceInfo &dev, cudaStream_t s)
+{
+    if (M < 1 || M > kDecodeMaxTokens) return QLORA_ERR_SHAPE;
+    const DecodePlan d = decode_plan(M, w->rows, w->cols, r, dev.sms);
+    if (ws_bytes < d.part_bytes + d.part_h_bytes) return QLORA_ERR_WORKSPACE;
+    DecodeParams p;
+    p.packed = w->packed;
+    p.code2 = w->code2;
+    p.c2 = w->c2;
+    p.mean = w->mean;
+    for (int i = 0; i < 16; i++) p.q[i] = w->codebook[i];
+    p.X = static_cast<const __nv_bfloat16 *>(X);
+    p.A = static_cast<const __nv_bfloat16 *>(A);
+    p.N = w->rows;
+    p.K = w->cols;
+    p.kblocks = w->cols / QLORA_BLOCK;
+    p.M = (int)M;
+    p.r = r;
+    p.row_tiles = d.row_tiles;
+    p.dblk_per_split = d.per;
+    p.n_dblk = d.n_dblk;
+    p.part = static_cast<float *>(ws);
+    p.part_h = reinterpret_cast<float *>(static_cast<char *>(ws) + d.part_bytes);
+    const dim3 grid(d.row_tiles + d.a_ctas, d.splits);
+    {
+        LaunchScope ls(QLORA_KERNEL_FWD_FUSED, s);
+        if (M <= 8)
+            QLORA_CUDA_TRY(launch_pdl(decode_gemv_kernel<1>, grid, dim3(kDecThreads), 0, s, p));
+        else
+            QLORA_CUDA_TRY(launch_pdl(decode_gemv_kernel<2>, grid, dim3(kDecThreads), 0, s, p));
+    }
+    {
+        LaunchScope ls(QLORA_KERNEL_ELEMENTWISE, s);
+        QLORA_CUDA_TRY(launch_pdl(decode_finalize_kernel, dim3(ceil_div_i(w->rows, 256)), dim3(256), 0, s,
+                                  (const float *)p.part, (const float *)p.part_h, d.splits, (int)M,
+                                  (int64_t)w->rows, r, scale, static_cast<const __nv_bfloat16 *>(B), Y,
+                                  y_dtype == QLORA_FP32 ? 1 : 0, H_save));
+    }
+    return launch_status();
+}
+
+}  // namespace qlora

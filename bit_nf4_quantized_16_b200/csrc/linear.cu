@@ -25,6 +25,7 @@
 #include <utility>
 
 #include "common.cuh"
+#include "decode.cuh"
 #include "gemm.cuh"
 #include "gemm_pair.cuh"
 
@@ -73,26 +74,6 @@ qlora_status map_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint64_t
 }
 
 // ---- launches ------------------------------------------------------------------------
-
-// Every kernel of the linear path is launched with programmatic stream
-// serialization: its set-up (barrier init, TMEM allocation, descriptor
-// prefetch) overlaps the tail of the kernel before it, and it waits
-// (griddepcontrol.wait) before reading anything that kernel produced.
-template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args &&...args)
-{
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
-}
 
 // ---- GEMM launch ------------------------------------------------------------------
 
@@ -313,6 +294,8 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int r, int sms)
     pl.off_part = 2 * hl;
     pl.off_part2 = pl.off_part + align256(part);
     pl.bytes = pl.off_part2 + align256(part2);
+    // the decode forward (M <= kDecodeMaxTokens) uses the start of the workspace for its partials
+    if (M <= kDecodeMaxTokens) pl.bytes = std::max(pl.bytes, align256(decode_workspace_bytes(M, N, K, r, sms)));
     return pl;
 }
 
@@ -394,6 +377,10 @@ extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const void *
     if (workspace_bytes < pl.bytes) return QLORA_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     char *ws = static_cast<char *>(workspace);
+
+    // a handful of tokens: stream the packed weight once (bound by HBM, not the tensor cores)
+    if (M <= kDecodeMaxTokens)
+        return run_decode_fwd(w, X, M, A, B, r, scale, Y, y_dtype, H_save, ws, workspace_bytes, dev, s);
 
     QLORA_TRY(run_h(pl, dev, X, A, scale, H_save, ws, s));
 
