@@ -289,6 +289,8 @@ def run_ours(args, rank, world, local_rank):
 
     codec = run_codec(args, q, torch, dev, peaks, peak_src) if (rank == 0 and not args.skip_codec) else None
     decode = run_decode65b(args, q, torch, dev, peaks, peak_src) if (rank == 0 and not args.skip_decode) else None
+    del layers, ws, grads, flush
+    stack = run_stack65b(args, q, torch, dev, peaks, peak_src) if (rank == 0 and not args.skip_stack) else None
 
     if rank != 0:
         return None
@@ -313,6 +315,8 @@ def run_ours(args, rank, world, local_rank):
         line["codec"] = codec
     if decode is not None:
         line["decode65b"] = decode
+    if stack is not None:
+        line["stack65b"] = stack
     if world == 1 and not args.skip_cpu:
         line["cpu_baseline"] = cpu_baseline_linear(budget_s=args.cpu_seconds)
     return line
@@ -469,6 +473,91 @@ def run_decode65b(args, q, torch, dev, peaks, peak_src):
     return out
 
 
+def run_stack65b(args, q, torch, dev, peaks, peak_src, layers_n=None, tokens=2048):
+    """Forward then backward through a stack of 80 LLaMA-65B layers of 7 QLoRA
+    linears each (no attention) at 2048 tokens.  Every linear has its own
+    quantized weight buffers (about 33 GB in all), adapters and gradients;
+    the seven quantized weights of one layer are generated and copied into
+    the other layers' buffers (same values, distinct memory), and the
+    activation buffers are shared per shape."""
+    import synthetic
+    shapes = synthetic.LLAMA65B_LINEARS
+    n_layers = layers_n or synthetic.LLAMA65B_LAYERS
+    qws = torch.empty(max(q.qlora_quantize_workspace_bytes(N, K) for _, N, K in shapes), dtype=torch.uint8,
+                      device=dev)
+    proto = []
+    for i, (name, N, K) in enumerate(shapes):
+        W = synthetic.normal((N, K), 0.02, 80_000 + i, torch.bfloat16, dev)
+        w = q.NF4Weight(N, K, device=dev)
+        q.qlora_quantize_nf4_dq(W, w, qws)
+        del W
+        proto.append(w)
+    del qws
+    act = {}
+    for _, N, K in shapes:
+        act.setdefault(("X", K), synthetic.normal((tokens, K), 1.0, 80_100 + K, torch.bfloat16, dev))
+        act.setdefault(("dY", N), synthetic.normal((tokens, N), 1.0, 80_200 + N, torch.bfloat16, dev))
+        act.setdefault(("Y", N), torch.empty(tokens, N, dtype=torch.bfloat16, device=dev))
+        act.setdefault(("dX", K), torch.empty(tokens, K, dtype=torch.bfloat16, device=dev))
+    lin = []
+    for layer in range(n_layers):
+        for i, (name, N, K) in enumerate(shapes):
+            w = q.NF4Weight(N, K, codebook=proto[i].codebook, device=dev)
+            for dst, src in ((w.packed, proto[i].packed), (w.code2, proto[i].code2), (w.c2, proto[i].c2),
+                             (w.mean, proto[i].mean)):
+                dst.copy_(src)
+            lin.append({"N": N, "K": K, "w": w,
+                        "A": synthetic.normal((R, K), 1.0 / R, 80_300 + i, torch.bfloat16, dev),
+                        "B": synthetic.normal((N, R), 0.01, 80_400 + i, torch.bfloat16, dev),
+                        "H": torch.empty(tokens, R, dtype=torch.float32, device=dev),
+                        "dA": torch.empty(R, K, dtype=torch.float32, device=dev),
+                        "dB": torch.empty(N, R, dtype=torch.float32, device=dev)})
+    del proto
+    wbytes = sum(L["w"].nbytes for L in lin)
+    ws = torch.empty(max(q.qlora_linear_workspace_bytes(tokens, N, K, R) for _, N, K in shapes), dtype=torch.uint8,
+                     device=dev)
+    scale = ALPHA / R
+
+    def step():
+        for L in lin:
+            q.qlora_linear_fwd(L["w"], act[("X", L["K"])], tokens, L["A"], L["B"], R, scale, act[("Y", L["N"])],
+                               L["H"], ws)
+        for L in reversed(lin):
+            q.qlora_linear_bwd(L["w"], act[("X", L["K"])], act[("dY", L["N"])], tokens, L["A"], L["B"], R, scale,
+                               L["H"], act[("dX", L["K"])], L["dA"], L["dB"], ws)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    q.qlora_check_device_error()
+    steps = max(1, min(args.steps, 5))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = q.qlora_launch_count()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        e0.record()
+        for _ in range(steps):
+            step()
+        e1.record()
+        torch.cuda.synchronize()
+    q.qlora_check_device_error()
+    ms = e0.elapsed_time(e1) / steps
+    flops = sum(linear_flops(tokens, L["N"], L["K"], R) for L in lin)
+    value = flops / (ms * 1e-3) / 1e12
+    return {
+        "workload": f"stack65b: {n_layers} LLaMA-65B layers x 7 QLoRA linears fwd+bwd, {tokens} tokens, r=64, "
+                    "alpha=16, no attention",
+        "value": round(value, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 3), "steps": steps,
+        "flop_per_step": flops, "nf4_weight_gb": round(wbytes / 1e9, 2),
+        # a step lasts about half a second at the power limit: the sustained peak applies
+        "roofline": {"bound": "tensor", "achieved": round(value, 1), "peak": peaks["bf16_tflops_sustained"],
+                     "unit": "TFLOP/s", "frac": round(value / peaks["bf16_tflops_sustained"], 4),
+                     "frac_of_burst_peak": round(value / peaks["bf16_tflops"], 4), "traffic": None,
+                     "peak_source": f"{peak_src} bf16_tflops_sustained"},
+        "gpu_launches_per_step": (q.qlora_launch_count() - launches0) // steps,
+        "clocks": clk.summary(),
+    }
+
+
 # ---- CPU baselines (the oracle, as it stands) ---------------------------------------
 
 def _blas_threads():
@@ -566,6 +655,7 @@ def main():
     ap.add_argument("--skip-codec", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-decode", action="store_true")
+    ap.add_argument("--skip-stack", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--linears", default="llama7b",
                     help="llama7b (the seven linears of one layer) or NxK for one linear (profiling runs)")

@@ -208,6 +208,26 @@ def test_llama7b_shapes_sampled(q):
         assert_close(np64(dB), s * (dY.T @ (X @ A.T)), what=f"{name} dB")
 
 
+def test_llama65b_shapes_sampled(q):
+    """65B-shaped linears at 2048 tokens (the stack configuration): Y and dX on
+    sampled rows, dA and dB in full."""
+    rng = np.random.default_rng(1)
+    for i, (name, N, K) in enumerate([("q", 8192, 8192), ("gate", 22016, 8192), ("down", 8192, 22016)]):
+        case = synthetic.linear_case(2048, N, K, 64, alpha=16.0, seed=500 + i, device="cpu")
+        run = Runner(q, case)
+        Wd = oracle_weight(case["W"])
+        X, A, B, dY = (np64(case[k]) for k in ("X", "A", "B", "dY"))
+        s = case["scale"]
+        rows = np.sort(rng.choice(2048, 32, replace=False))
+        Y, H = run.fwd(save_h=True)
+        assert_close(np64(Y)[rows], olin.forward_rows(X, Wd, A, B, s, rows), what=f"{name} Y")
+        dX, dA, dB = run.bwd(H=H)
+        assert_close(np64(dX)[rows], olin.backward_dx_rows(Wd, A, B, s, dY, rows), what=f"{name} dX")
+        G = dY @ B
+        assert_close(np64(dA), s * (G.T @ X), what=f"{name} dA")
+        assert_close(np64(dB), s * (dY.T @ (X @ A.T)), what=f"{name} dB")
+
+
 def test_argument_errors(q):
     case = synthetic.linear_case(16, 128, 128, 8, alpha=16.0, seed=13)
     run = Runner(q, case)
