@@ -324,7 +324,7 @@ def run_ours(args, rank, world, local_rank):
 
 def run_codec(args, q, torch, dev, peaks, peak_src):
     """NF4+DQ quantize -> dequantize round trip over the LLaMA-7B tensors,
-    replayed as one CUDA graph per step."""
+    replayed as one CUDA graph per step (four streams of independent tensors)."""
     import synthetic
     shapes = [(N, K) for _ in range(synthetic.LLAMA7B_LAYERS) for _, N, K in synthetic.LLAMA7B_LINEARS]
     if args.codec_tensors:
@@ -334,13 +334,24 @@ def run_codec(args, q, torch, dev, peaks, peak_src):
         W = synthetic.normal((N, K), 0.02, 50_000 + i, torch.bfloat16, dev)
         tensors.append((W, q.NF4Weight(N, K, device=dev), torch.empty(N, K, dtype=torch.bfloat16, device=dev)))
     nweights = sum(N * K for N, K in shapes)
-    qws = torch.empty(max(q.qlora_quantize_workspace_bytes(N, K) for N, K in shapes), dtype=torch.uint8, device=dev)
+    # the tensors are independent: they are spread over a few streams (one
+    # quantize workspace each) so that one tensor's launch and tail overlap
+    # another's streaming
+    n_streams = 4
+    qws_bytes = max(q.qlora_quantize_workspace_bytes(N, K) for N, K in shapes)
+    qws = [torch.empty(qws_bytes, dtype=torch.uint8, device=dev) for _ in range(n_streams)]
+    side = [torch.cuda.Stream() for _ in range(n_streams)]
 
     def round_trip():
-        for W, w, out in tensors:
-            q.qlora_quantize_nf4_dq(W, w, qws)
-        for W, w, out in tensors:
-            q.qlora_dequantize_nf4_dq(w, out)
+        main = torch.cuda.current_stream()
+        for st in side:
+            st.wait_stream(main)
+        for i, (W, w, out) in enumerate(tensors):
+            with torch.cuda.stream(side[i % n_streams]):
+                q.qlora_quantize_nf4_dq(W, w, qws[i % n_streams])
+                q.qlora_dequantize_nf4_dq(w, out)
+        for st in side:
+            main.wait_stream(st)
 
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
@@ -366,11 +377,14 @@ def run_codec(args, q, torch, dev, peaks, peak_src):
     ms = e0.elapsed_time(e1) / args.steps
     bytes_rt = 2 * CODEC_BYTES_PER_WEIGHT * nweights
     gbs = bytes_rt / (ms * 1e-3) / 1e9
-    # per-kernel device time, kernels launched directly (events on the stream)
+    # per-kernel device time: the same work on one stream, each kernel bracketed
+    # by CUDA events
     q.qlora_timing_reset()
     q.qlora_timing_enable(True)
     torch.cuda._sleep(100_000_000)
-    round_trip()
+    for i, (W, w, out) in enumerate(tensors):
+        q.qlora_quantize_nf4_dq(W, w, qws[0])
+        q.qlora_dequantize_nf4_dq(w, out)
     q.qlora_timing_enable(False)
     kern = q.qlora_timing_read()
     qms = kern["quantize"][0]

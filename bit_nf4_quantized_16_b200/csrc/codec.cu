@@ -30,7 +30,6 @@ namespace qlora {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kUnroll = 4;      // words per thread in flight (quantize)
 constexpr int kDeqUnroll = 4;   // words per thread in flight (dequantize)
 
 // ---- small device helpers ----------------------------------------------------
@@ -42,6 +41,14 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void *p)
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "l"(p));
     return v;
+}
+
+// 32-byte load (sm_100).
+__device__ __forceinline__ void ld_v8(const void *p, uint4 &a, uint4 &b)
+{
+    asm volatile("ld.global.nc.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+                 : "l"(p));
 }
 
 __device__ __forceinline__ uint32_t ld_stream_u32(const void *p)
@@ -111,6 +118,33 @@ __device__ __forceinline__ uint32_t add_code(const uint32_t *lut, float n, uint3
     return acc + code * (1u << (4 * I));
 }
 
+// Absolute maximum of 8 bf16 values held as 4 packed pairs: the magnitudes'
+// bit patterns compare like the values, so a 16-bit unsigned SIMD max does it.
+__device__ __forceinline__ uint32_t absmax8_bf16(uint4 v, uint32_t m)
+{
+    const uint32_t a = __vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu);
+    const uint32_t b = __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu);
+    return __vmaxu2(m, __vmaxu2(a, b));
+}
+
+// 8 codes of 8 consecutive values (already multiplied by r), element 0 in bits 0-3.
+__device__ __forceinline__ uint32_t codes8(const uint32_t *lut, const float (&n)[8])
+{
+    uint32_t word = add_code<0>(lut, n[0], 0u);
+    word = add_code<1>(lut, n[1], word);
+    word = add_code<2>(lut, n[2], word);
+    word = add_code<3>(lut, n[3], word);
+    word = add_code<4>(lut, n[4], word);
+    word = add_code<5>(lut, n[5], word);
+    word = add_code<6>(lut, n[6], word);
+    return add_code<7>(lut, n[7], word);
+}
+
+// One lane per block of 64 weights, 32 consecutive blocks per warp and step:
+// the loads of a warp cover 4 KB (bf16) of contiguous input and its stores 1 KB
+// of packed codes; the block absmax, the reciprocal and the block constant are
+// lane-local.  A lane's 8 (bf16) or 16 (fp32) 16-byte loads are issued
+// together; fp32 input is read twice (the second time from L1).
 template <bool kF32In>
 __global__ void __launch_bounds__(kThreads) quantize_blocks_kernel(const __grid_constant__ QuantParams p)
 {
@@ -119,6 +153,7 @@ __global__ void __launch_bounds__(kThreads) quantize_blocks_kernel(const __grid_
     __shared__ unsigned long long s_acc[256];
     __shared__ uint32_t s_mkey[16];
     __shared__ bool s_last;
+    __shared__ int s_lohi[kThreads / 32][2];
     if (threadIdx.x == 0) {
 #pragma unroll
         for (int j = 0; j < 15; j++) s_mkey[j] = p.mkey[j];
@@ -129,94 +164,80 @@ __global__ void __launch_bounds__(kThreads) quantize_blocks_kernel(const __grid_
     __syncthreads();
 
     const uint32_t lane = threadIdx.x & 31;
-    const uint32_t stride = gridDim.x * kThreads;
-    for (uint32_t base = blockIdx.x * kThreads + (threadIdx.x & ~31u); base < p.nwords; base += stride * kUnroll) {
-        float x[kUnroll][8];
-        bool act[kUnroll];
+    const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
+    for (int64_t b0 = ((int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5)) * 32; b0 < p.nblocks;
+         b0 += nwarps * 32) {
+        const int64_t b = b0 + lane;
+        const bool act = b < p.nblocks;
+        uint32_t words[8];
+        float cv;
+        if (!kF32In) {
+            const uint4 *src = static_cast<const uint4 *>(p.W) + 8 * b;   // 64 bf16 = 4 x 32 B
+            uint4 v[8];
 #pragma unroll
-        for (int u = 0; u < kUnroll; u++) {
-            const uint32_t w = base + lane + u * stride;
-            act[u] = w < p.nwords;
-            if (kF32In) {
-                uint4 a = make_uint4(0, 0, 0, 0), b = a;
-                if (act[u]) {
-                    const float *src = static_cast<const float *>(p.W) + 8ull * w;
-                    a = ld_stream_v4(src);
-                    b = ld_stream_v4(src + 4);
-                }
-                x[u][0] = __uint_as_float(a.x); x[u][1] = __uint_as_float(a.y);
-                x[u][2] = __uint_as_float(a.z); x[u][3] = __uint_as_float(a.w);
-                x[u][4] = __uint_as_float(b.x); x[u][5] = __uint_as_float(b.y);
-                x[u][6] = __uint_as_float(b.z); x[u][7] = __uint_as_float(b.w);
-            } else {
-                uint4 a = make_uint4(0, 0, 0, 0);
-                if (act[u]) a = ld_stream_v4(static_cast<const __nv_bfloat16 *>(p.W) + 8ull * w);
-                const uint32_t v[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-                for (int i = 0; i < 4; i++) {
-                    x[u][2 * i] = __uint_as_float(v[i] << 16);
-                    x[u][2 * i + 1] = __uint_as_float(v[i] & 0xFFFF0000u);
+            for (int i = 0; i < 8; i += 2) {
+                if (act) {
+                    ld_v8(src + i, v[i], v[i + 1]);
+                } else {
+                    v[i] = v[i + 1] = make_uint4(0, 0, 0, 0);
                 }
             }
-        }
-        // block absmax: the 8 lanes of one block reduce together
-        float c1v[kUnroll];
+            uint32_t m = 0;
 #pragma unroll
-        for (int u = 0; u < kUnroll; u++) {
+            for (int i = 0; i < 8; i++) m = absmax8_bf16(v[i], m);
+            cv = __uint_as_float(__vmaxu2(m, m >> 16) << 16);   // larger half, as binary32
+            // zero block (absmax below the smallest normal): r = 0 sends every
+            // element to n = +-0, whose code is the codebook's zero
+            const float r = cv < 1.17549435e-38f ? 0.0f : __frcp_rn(cv);
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+                const uint32_t u[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+                float n[8];
+#pragma unroll
+                for (int j = 0; j < 4; j++)
+                    nf4::mul2(__uint_as_float(u[j] << 16), __uint_as_float(u[j] & 0xFFFF0000u), r, n[2 * j], n[2 * j + 1]);
+                words[i] = codes8(lut, n);
+            }
+        } else {
+            const uint4 *src = static_cast<const uint4 *>(p.W) + 16 * b;  // 64 fp32 = 16 x 16 B
             float m = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 8; i++) m = fmaxf(m, fabsf(x[u][i]));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-            c1v[u] = m;
-        }
-        // Gather the warp's 4*kUnroll block constants into lanes 0..4*kUnroll-1
-        // (lane 4u+g takes block g of unrolled step u): one reciprocal per lane,
-        // the stores of c1, and the exponent buckets of the exact mean.
-        float cv = 0.0f;
-        bool ca = false;
+            for (int i = 0; i < 16; i++) {
+                const uint4 v = act ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+                m = fmaxf(fmaxf(m, fmaxf(fabsf(__uint_as_float(v.x)), fabsf(__uint_as_float(v.y)))),
+                          fmaxf(fabsf(__uint_as_float(v.z)), fabsf(__uint_as_float(v.w))));
+            }
+            cv = m;
+            const float r = cv < 1.17549435e-38f ? 0.0f : __frcp_rn(cv);
 #pragma unroll
-        for (int u = 0; u < kUnroll; u++) {
-            const float t = __shfl_sync(0xffffffffu, c1v[u], (lane & 3) * 8);
-            const bool a = __shfl_sync(0xffffffffu, (int)act[u], (lane & 3) * 8) != 0;
-            if ((lane >> 2) == (uint32_t)u) {
-                cv = t;
-                ca = a;
+            for (int i = 0; i < 8; i++) {
+                const uint4 v0 = act ? __ldg(src + 2 * i) : make_uint4(0, 0, 0, 0);
+                const uint4 v1 = act ? __ldg(src + 2 * i + 1) : make_uint4(0, 0, 0, 0);
+                float n[8];
+                nf4::mul2(__uint_as_float(v0.x), __uint_as_float(v0.y), r, n[0], n[1]);
+                nf4::mul2(__uint_as_float(v0.z), __uint_as_float(v0.w), r, n[2], n[3]);
+                nf4::mul2(__uint_as_float(v1.x), __uint_as_float(v1.y), r, n[4], n[5]);
+                nf4::mul2(__uint_as_float(v1.z), __uint_as_float(v1.w), r, n[6], n[7]);
+                words[i] = codes8(lut, n);
             }
         }
-        // zero block (absmax below the smallest normal): r = 0 sends every
-        // element to n = +-0, whose code is the codebook's zero
-        const float rv = cv < 1.17549435e-38f ? 0.0f : __frcp_rn(cv);
-        if (lane < 4 * kUnroll && ca) p.c1[(base + 8 * (lane & 3) + (lane >> 2) * stride) >> 3] = cv;
-        // codes
-#pragma unroll
-        for (int u = 0; u < kUnroll; u++) {
-            const float r = __shfl_sync(0xffffffffu, rv, 4 * u + (lane >> 3));
-            float n[8];
-#pragma unroll
-            for (int i = 0; i < 8; i += 2) nf4::mul2(x[u][i], x[u][i + 1], r, n[i], n[i + 1]);
-            uint32_t word = add_code<0>(lut, n[0], 0u);
-            word = add_code<1>(lut, n[1], word);
-            word = add_code<2>(lut, n[2], word);
-            word = add_code<3>(lut, n[3], word);
-            word = add_code<4>(lut, n[4], word);
-            word = add_code<5>(lut, n[5], word);
-            word = add_code<6>(lut, n[6], word);
-            word = add_code<7>(lut, n[7], word);
-            if (act[u]) reinterpret_cast<uint32_t *>(p.packed)[base + lane + u * stride] = word;
+        if (act) {
+            uint4 *dst = reinterpret_cast<uint4 *>(p.packed) + 2 * b;          // 64 codes = 2 x 16 B
+            dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
+            dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
+            p.c1[b] = cv;
         }
-        // exact-mean buckets: one shared atomic per distinct exponent
+        // exact-mean buckets: one shared atomic per distinct exponent in the warp
         uint32_t bucket, sig;
         exact_mean_split(__float_as_uint(cv), &bucket, &sig);
-        bool pending = lane < 4 * kUnroll && ca;
+        bool pending = act;
         for (;;) {
             const unsigned pend = __ballot_sync(0xffffffffu, pending);
             if (!pend) break;
             const int leader = __ffs(pend) - 1;
             const uint32_t lb = __shfl_sync(0xffffffffu, bucket, leader);
             const bool mine = pending && bucket == lb;
-            const uint32_t sum = __reduce_add_sync(0xffffffffu, mine ? sig : 0u);   // < 16 * 2^24
+            const uint32_t sum = __reduce_add_sync(0xffffffffu, mine ? sig : 0u);   // < 32 * 2^24
             if ((int)lane == leader) atomicAdd(&s_acc[lb], (unsigned long long)sum);
             pending = pending && !mine;
         }
@@ -231,10 +252,24 @@ __global__ void __launch_bounds__(kThreads) quantize_blocks_kernel(const __grid_
     __syncthreads();
     if (s_last) {
         __threadfence();
-        s_acc[threadIdx.x] = atomicAdd(&p.acc[threadIdx.x], 0ull);
+        const unsigned long long mine = atomicAdd(&p.acc[threadIdx.x], 0ull);
+        s_acc[threadIdx.x] = mine;
+        // lowest and highest non-zero bucket (1..254), found by the whole block
+        const bool nz = mine != 0 && threadIdx.x >= 1 && threadIdx.x <= 254;
+        const unsigned bal = __ballot_sync(0xffffffffu, nz);
+        if ((threadIdx.x & 31) == 0) {
+            s_lohi[threadIdx.x >> 5][0] = bal ? (int)(threadIdx.x + __ffs(bal) - 1) : 256;
+            s_lohi[threadIdx.x >> 5][1] = bal ? (int)(threadIdx.x + 31 - __clz(bal)) : -1;
+        }
         __syncthreads();
-        if (threadIdx.x == 0)
-            *p.mean_out = __uint_as_float(exact_mean_bits(s_acc, (uint64_t)p.nblocks));
+        if (threadIdx.x == 0) {
+            int lo = 256, hi = -1;
+            for (int w = 0; w < kThreads / 32; w++) {
+                lo = min(lo, s_lohi[w][0]);
+                hi = max(hi, s_lohi[w][1]);
+            }
+            *p.mean_out = __uint_as_float(exact_mean_bits_range(s_acc, (uint64_t)p.nblocks, lo, hi));
+        }
     }
 }
 
@@ -417,7 +452,7 @@ extern "C" qlora_status qlora_quantize_nf4_dq(const void *W, qlora_dtype w_dtype
     qp.nwords = (uint32_t)(numel / 8);
     qp.nblocks = nblocks;
     memcpy(qp.mkey, mkey, sizeof(mkey));
-    int grid = grid_for(qp.nwords, kThreads * kUnroll, dev.sms * 4);
+    int grid = grid_for(qp.nblocks, kThreads * 4, dev.sms * 4);
     {
         LaunchScope ls(QLORA_KERNEL_QUANTIZE, s);
         if (w_dtype == QLORA_FP32)
@@ -539,7 +574,7 @@ extern "C" qlora_status qlora_quantize_nf4_dq_noalloc(const void *W, qlora_dtype
     qp.nwords = (uint32_t)(numel / 8);
     qp.nblocks = nblocks;
     memcpy(qp.mkey, mkey, sizeof(mkey));
-    const int grid = grid_for(qp.nwords, kThreads * kUnroll, dev.sms * 4);
+    const int grid = grid_for(qp.nblocks, kThreads * 4, dev.sms * 4);
     {
         LaunchScope ls(QLORA_KERNEL_QUANTIZE, s);
         if (w_dtype == QLORA_FP32)

@@ -37,6 +37,16 @@ QLORA_HD void exact_mean_split(uint32_t bits, uint32_t *bucket, uint32_t *sig)
     *sig = E ? (F | 0x800000u) : F;
 }
 
+// Count of leading zero bits of a non-zero 64-bit value.
+QLORA_HD int clz64(uint64_t v)
+{
+#if defined(__CUDA_ARCH__)
+    return __clzll((long long)v);
+#else
+    return __builtin_clzll(v);
+#endif
+}
+
 // Fast path: all non-zero buckets lie within 61 consecutive exponents, so the
 // exact sum fits one 128-bit integer T (units of 2^(lo-150)); the quotient
 // T / count is normalized to at least 26 bits before rounding.  Returns false
@@ -54,10 +64,20 @@ QLORA_HD bool exact_mean_bits_narrow(const unsigned long long *bucket, uint64_t 
         T <<= 1;
         b -= 1;
     }
-    const unsigned __int128 Q = T / count;
-    const uint64_t rem = (uint64_t)(T - Q * count);
-    int p = 127;
-    while (!((Q >> p) & 1)) p--;
+    // Q = T / count by long division in 32-bit digits (count < 2^32), which
+    // avoids a generic 128-bit division
+    uint32_t qd[4];
+    uint64_t rem = 0;
+    for (int i = 3; i >= 0; i--) {
+        const uint64_t cur = (rem << 32) | (uint32_t)(T >> (32 * i));
+        qd[i] = (uint32_t)(cur / count);
+        rem = cur % count;
+    }
+    const unsigned __int128 Q = ((unsigned __int128)(((uint64_t)qd[3] << 32) | qd[2]) << 64) |
+                                (((uint64_t)qd[1] << 32) | qd[0]);
+    // position of the most significant set bit (Q >= 2^26 after normalization)
+    const uint64_t qhi = (uint64_t)(Q >> 64), qlo = (uint64_t)Q;
+    int p = qhi ? 127 - clz64(qhi) : 63 - clz64(qlo);
     // least significant kept bit: 2^(p+b-23) for a normal result, 2^-149 below
     int L = p + b - 23;
     if (L < -149) L = -149;
@@ -81,6 +101,8 @@ QLORA_HD bool exact_mean_bits_narrow(const unsigned long long *bucket, uint64_t 
     return true;
 }
 
+QLORA_HD uint32_t exact_mean_bits_range(const unsigned long long *bucket, uint64_t count, int lo, int hi);
+
 // Binary32 bit pattern of RN(sum_j bucket[j] * 2^(j-150) / count).
 // bucket has 256 entries; count >= 1 and < 2^32.
 QLORA_HD uint32_t exact_mean_bits(const unsigned long long *bucket, uint64_t count)
@@ -93,6 +115,13 @@ QLORA_HD uint32_t exact_mean_bits(const unsigned long long *bucket, uint64_t cou
             hi = j;
         }
     }
+    return exact_mean_bits_range(bucket, count, lo, hi);
+}
+
+// The same, given the lowest (lo) and highest (hi) non-zero bucket in 1..254
+// (hi < 0 when every bucket is zero).
+QLORA_HD uint32_t exact_mean_bits_range(const unsigned long long *bucket, uint64_t count, int lo, int hi)
+{
     if (hi < 0) return 0u;
     uint32_t fast;
     if (exact_mean_bits_narrow(bucket, count, lo, hi, &fast)) return fast;
