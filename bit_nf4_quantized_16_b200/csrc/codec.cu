@@ -24,6 +24,7 @@
 #include "common.cuh"
 #include "exact_mean.cuh"
 #include "nf4_expand.cuh"
+#include "sm100.cuh"
 
 namespace qlora {
 
@@ -41,6 +42,14 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void *p)
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "l"(p));
     return v;
+}
+
+// 32-byte store (sm_100).
+__device__ __forceinline__ void st_v8(void *p, uint4 a, uint4 b)
+{
+    asm volatile("st.global.v8.u32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(a.x), "r"(a.y), "r"(a.z),
+                 "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+                 : "memory");
 }
 
 // 32-byte load (sm_100).
@@ -70,7 +79,17 @@ struct QuantParams {
     uint32_t nwords;           // numel / 8: one word = 8 codes = 32 bits
     int64_t nblocks;
     uint32_t mkey[15];         // keys of the round-down midpoints, ascending
+    CUtensorMap tm_w;          // bf16 input as [nblocks][64], box 64 x 32, 128-byte swizzle
+    int *err;                  // device error word (a bounded wait gave up)
+    uint64_t timeout_ns;
 };
+
+// bf16 input: every warp streams its 32 blocks (4 KB) per step through a
+// two-stage shared-memory ring filled by TMA (lane 0 issues the copy of the
+// next step before the current one is processed).
+constexpr int kQStages = 2;
+constexpr uint32_t kQStageBytes = 32 * 128;
+constexpr uint32_t kQDynSmem = (kThreads / 32) * kQStages * kQStageBytes + 1024;
 
 // Code lookup.  The 15 midpoints between neighbouring codebook values are
 // rounded down to binary32, so "n > midpoint_j" holds exactly when n is nearer
@@ -164,24 +183,55 @@ __global__ void __launch_bounds__(kThreads) quantize_blocks_kernel(const __grid_
     __syncthreads();
 
     const uint32_t lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
     const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
-    for (int64_t b0 = ((int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5)) * 32; b0 < p.nblocks;
-         b0 += nwarps * 32) {
+    const int64_t first = ((int64_t)blockIdx.x * (kThreads / 32) + warp) * 32;
+    // bf16: this warp's TMA ring (stages of 32 rows x 128 B, 128-byte swizzle)
+    extern __shared__ uint8_t q_dyn[];
+    uint8_t *ring = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(q_dyn) + 1023) & ~uintptr_t(1023)) +
+                    warp * kQStages * kQStageBytes;
+    __shared__ uint64_t s_bar[kThreads / 32][kQStages];
+    if (!kF32In) {
+        if (lane == 0) {
+            for (int st = 0; st < kQStages; st++) sm100::mbar_init(&s_bar[warp][st], 1);
+            sm100::fence_barrier_init();
+            if (first < p.nblocks) {
+                sm100::mbar_arrive_expect_tx(&s_bar[warp][0], kQStageBytes);
+                sm100::tma_load_2d(ring, &p.tm_w, &s_bar[warp][0], 0, (int32_t)first);
+            }
+        }
+        __syncwarp();
+    }
+    uint32_t it = 0;
+    for (int64_t b0 = first; b0 < p.nblocks; b0 += nwarps * 32, it++) {
         const int64_t b = b0 + lane;
         const bool act = b < p.nblocks;
         uint32_t words[8];
         float cv;
         if (!kF32In) {
-            const uint4 *src = static_cast<const uint4 *>(p.W) + 8 * b;   // 64 bf16 = 4 x 32 B
+            const int st = it & 1;
+            const int64_t nb = b0 + nwarps * 32;
+            if (lane == 0 && nb < p.nblocks) {
+                // the other stage was read by every lane in the previous step
+                sm100::fence_proxy_async_smem();
+                sm100::mbar_arrive_expect_tx(&s_bar[warp][st ^ 1], kQStageBytes);
+                sm100::tma_load_2d(ring + (st ^ 1) * kQStageBytes, &p.tm_w, &s_bar[warp][st ^ 1], 0, (int32_t)nb);
+            }
+            const bool landed = sm100::mbar_wait_bounded(&s_bar[warp][st], (it >> 1) & 1, p.timeout_ns);
+            if (!__all_sync(0xffffffffu, landed)) {
+                // a copy did not arrive: record it and stop; the copy of the next
+                // step (if issued) is waited for below, bounded, before leaving
+                if (lane == 0) {
+                    atomicExch(p.err, 1);
+                    if (nb < p.nblocks) sm100::mbar_wait_bounded(&s_bar[warp][st ^ 1], ((it + 1) >> 1) & 1, p.timeout_ns);
+                }
+                break;
+            }
+            // row `lane` of the stage: 16-byte chunk c sits at c ^ (lane & 7)
+            const uint8_t *row = ring + st * kQStageBytes + lane * 128;
             uint4 v[8];
 #pragma unroll
-            for (int i = 0; i < 8; i += 2) {
-                if (act) {
-                    ld_v8(src + i, v[i], v[i + 1]);
-                } else {
-                    v[i] = v[i + 1] = make_uint4(0, 0, 0, 0);
-                }
-            }
+            for (int i = 0; i < 8; i++) v[i] = *reinterpret_cast<const uint4 *>(row + ((i ^ (lane & 7)) << 4));
             uint32_t m = 0;
 #pragma unroll
             for (int i = 0; i < 8; i++) m = absmax8_bf16(v[i], m);
@@ -222,11 +272,11 @@ __global__ void __launch_bounds__(kThreads) quantize_blocks_kernel(const __grid_
             }
         }
         if (act) {
-            uint4 *dst = reinterpret_cast<uint4 *>(p.packed) + 2 * b;          // 64 codes = 2 x 16 B
-            dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
-            dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
+            st_v8(reinterpret_cast<uint4 *>(p.packed) + 2 * b, make_uint4(words[0], words[1], words[2], words[3]),
+                  make_uint4(words[4], words[5], words[6], words[7]));   // 64 codes = 32 B
             p.c1[b] = cv;
         }
+        if (!kF32In) __syncwarp();   // every lane has read its row before the stage is refilled
         // exact-mean buckets: one shared atomic per distinct exponent in the warp
         uint32_t bucket, sig;
         exact_mean_split(__float_as_uint(cv), &bucket, &sig);
@@ -399,6 +449,27 @@ qlora_status midpoint_keys(const float q[16], uint32_t out[15])
     return QLORA_OK;
 }
 
+// Tensor map of a bf16 input, error word, timeout and the kernel's dynamic
+// shared-memory limit (once per device).
+qlora_status prepare_quantize(QuantParams &qp, const void *W, qlora_dtype w_dtype, int64_t numel,
+                              const DeviceInfo &dev)
+{
+    qp.err = device_error_word();
+    if (!qp.err) return QLORA_ERR_CUDA;
+    qp.timeout_ns = 2000000000ull;
+    if (w_dtype == QLORA_BF16) {
+        QLORA_TRY(make_map(&qp.tm_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, 64, (uint64_t)(numel / 64), 128, 64, 32,
+                           CU_TENSOR_MAP_SWIZZLE_128B));
+        static bool attr_done[64] = {};
+        if (dev.device >= 0 && dev.device < 64 && !attr_done[dev.device]) {
+            QLORA_CUDA_TRY(cudaFuncSetAttribute(quantize_blocks_kernel<false>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize, kQDynSmem));
+            attr_done[dev.device] = true;
+        }
+    }
+    return QLORA_OK;
+}
+
 int grid_for(int64_t work_items, int items_per_cta, int max_ctas)
 {
     int64_t g = (work_items + items_per_cta - 1) / items_per_cta;
@@ -452,13 +523,14 @@ extern "C" qlora_status qlora_quantize_nf4_dq(const void *W, qlora_dtype w_dtype
     qp.nwords = (uint32_t)(numel / 8);
     qp.nblocks = nblocks;
     memcpy(qp.mkey, mkey, sizeof(mkey));
-    int grid = grid_for(qp.nblocks, kThreads * 4, dev.sms * 4);
+    QLORA_TRY(prepare_quantize(qp, W, w_dtype, numel, dev));
+    int grid = grid_for(qp.nblocks, kThreads * 4, dev.sms * 2);
     {
         LaunchScope ls(QLORA_KERNEL_QUANTIZE, s);
         if (w_dtype == QLORA_FP32)
             quantize_blocks_kernel<true><<<grid, kThreads, 0, s>>>(qp);
         else
-            quantize_blocks_kernel<false><<<grid, kThreads, 0, s>>>(qp);
+            quantize_blocks_kernel<false><<<grid, kThreads, kQDynSmem, s>>>(qp);
     }
     QLORA_TRY(launch_status());
 
@@ -574,13 +646,14 @@ extern "C" qlora_status qlora_quantize_nf4_dq_noalloc(const void *W, qlora_dtype
     qp.nwords = (uint32_t)(numel / 8);
     qp.nblocks = nblocks;
     memcpy(qp.mkey, mkey, sizeof(mkey));
-    const int grid = grid_for(qp.nblocks, kThreads * 4, dev.sms * 4);
+    QLORA_TRY(prepare_quantize(qp, W, w_dtype, numel, dev));
+    const int grid = grid_for(qp.nblocks, kThreads * 4, dev.sms * 2);
     {
         LaunchScope ls(QLORA_KERNEL_QUANTIZE, s);
         if (w_dtype == QLORA_FP32)
             quantize_blocks_kernel<true><<<grid, kThreads, 0, s>>>(qp);
         else
-            quantize_blocks_kernel<false><<<grid, kThreads, 0, s>>>(qp);
+            quantize_blocks_kernel<false><<<grid, kThreads, kQDynSmem, s>>>(qp);
     }
     QLORA_TRY(launch_status());
 

@@ -1,6 +1,7 @@
 // Shared host-side plumbing of the QLoRA library: status handling, argument
 // checks, device properties and the device error word.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -66,6 +67,11 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
+
+// 2-D row-major tensor map: `inner` elements per row (contiguous), `rows` rows,
+// `pitch_bytes` between rows; box = box_inner x box_rows elements.
+qlora_status make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t rows,
+                      uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw);
 
 // Checks shared by every entry point that takes a quantized weight.
 qlora_status check_weight(const qlora_nf4_weight *w);
