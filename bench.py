@@ -141,6 +141,7 @@ def run_ours(args, rank, world, local_rank):
     import torch.distributed as dist
 
     import bit_nf4_quantized_16_b200 as q
+    from bit_nf4_quantized_16_b200 import dp
     import synthetic
 
     torch.cuda.set_device(local_rank)
@@ -194,7 +195,7 @@ def run_ours(args, rank, world, local_rank):
             q.qlora_linear_bwd(L["w"], L["X"], L["dY"], TOKENS, L["A"], L["B"], R, scale, L["H"], L["dX"],
                                L["dA"], L["dB"], ws)
         if world > 1:
-            dist.all_reduce(grads)
+            dp.allreduce_adapter_grads(grads)
 
     def timed_steps(k, fn):
         """Device time of k steps, each after an L2 flush, CUDA events on the
@@ -236,10 +237,7 @@ def run_ours(args, rank, world, local_rank):
     kern = q.qlora_timing_read()
     q.qlora_check_device_error()
     clocks = clk.summary()
-    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms = ms_t.item()
+    ms = dp.max_over_ranks(ms, dev)
     value = step_flops * args.steps * world / (ms * 1e-3) / 1e12
 
     # ---- end to end through the same API with host buffers
@@ -259,15 +257,13 @@ def run_ours(args, rank, world, local_rank):
             q.qlora_linear_bwd(L["w"], L["X"], L["dY"], TOKENS, L["A"], L["B"], R, scale, L["H"], L["dX"],
                                L["dA"], L["dB"], ws)
         if world > 1:
-            dist.all_reduce(grads)
+            dp.allreduce_adapter_grads(grads)
         host_grads.copy_(grads, non_blocking=True)
 
     e2e_step()
     e2e_ms = timed_steps(args.steps, e2e_step)
-    e_t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e_t, op=dist.ReduceOp.MAX)
-    e2e_value = step_flops * args.steps * world / (e_t.item() * 1e-3) / 1e12
+    e2e_ms = dp.max_over_ranks(e2e_ms, dev)
+    e2e_value = step_flops * args.steps * world / (e2e_ms * 1e-3) / 1e12
 
     # ---- roofline of the dominant kernel (largest device time in the timed region)
     kflops = {
