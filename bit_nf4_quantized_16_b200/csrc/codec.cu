@@ -35,29 +35,12 @@ constexpr int kDeqUnroll = 4;   // words per thread in flight (dequantize)
 
 // ---- small device helpers ----------------------------------------------------
 
-__device__ __forceinline__ uint4 ld_stream_v4(const void *p)
-{
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
-
 // 32-byte store (sm_100).
 __device__ __forceinline__ void st_v8(void *p, uint4 a, uint4 b)
 {
     asm volatile("st.global.v8.u32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(a.x), "r"(a.y), "r"(a.z),
                  "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
                  : "memory");
-}
-
-// 32-byte load (sm_100).
-__device__ __forceinline__ void ld_v8(const void *p, uint4 &a, uint4 &b)
-{
-    asm volatile("ld.global.nc.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
-                 : "l"(p));
 }
 
 __device__ __forceinline__ uint32_t ld_stream_u32(const void *p)
@@ -89,7 +72,8 @@ struct QuantParams {
 // next step before the current one is processed).
 constexpr int kQStages = 2;
 constexpr uint32_t kQStageBytes = 32 * 128;
-constexpr uint32_t kQDynSmem = (kThreads / 32) * kQStages * kQStageBytes + 1024;
+constexpr int kQThreads = 768;   // quantizer: one CTA of 24 warps per SM (the TMA rings fill shared memory)
+constexpr uint32_t kQDynSmem = (kQThreads / 32) * kQStages * kQStageBytes + 1024;
 
 // Code lookup.  The 15 midpoints between neighbouring codebook values are
 // rounded down to binary32, so "n > midpoint_j" holds exactly when n is nearer
@@ -165,32 +149,32 @@ __device__ __forceinline__ uint32_t codes8(const uint32_t *lut, const float (&n)
 // lane-local.  A lane's 8 (bf16) or 16 (fp32) 16-byte loads are issued
 // together; fp32 input is read twice (the second time from L1).
 template <bool kF32In>
-__global__ void __launch_bounds__(kThreads) quantize_blocks_kernel(const __grid_constant__ QuantParams p)
+__global__ void __launch_bounds__(kQThreads, 1) quantize_blocks_kernel(const __grid_constant__ QuantParams p)
 {
-    static_assert(kThreads * 16 == 4096, "one 16-entry slice of the code table per thread");
+    static_assert(kQThreads >= 256, "the first 256 threads build the code table and own the buckets");
     __shared__ __align__(16) uint32_t lut[4096];
     __shared__ unsigned long long s_acc[256];
     __shared__ uint32_t s_mkey[16];
     __shared__ bool s_last;
-    __shared__ int s_lohi[kThreads / 32][2];
+    __shared__ int s_lohi[8][2];
     if (threadIdx.x == 0) {
 #pragma unroll
         for (int j = 0; j < 15; j++) s_mkey[j] = p.mkey[j];
     }
-    s_acc[threadIdx.x] = 0;
+    if (threadIdx.x < 256) s_acc[threadIdx.x] = 0;
     __syncthreads();
-    build_code_lut(lut, s_mkey);
+    if (threadIdx.x < 256) build_code_lut(lut, s_mkey);
     __syncthreads();
 
     const uint32_t lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-    const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
-    const int64_t first = ((int64_t)blockIdx.x * (kThreads / 32) + warp) * 32;
+    const int64_t nwarps = (int64_t)gridDim.x * (kQThreads / 32);
+    const int64_t first = ((int64_t)blockIdx.x * (kQThreads / 32) + warp) * 32;
     // bf16: this warp's TMA ring (stages of 32 rows x 128 B, 128-byte swizzle)
     extern __shared__ uint8_t q_dyn[];
     uint8_t *ring = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(q_dyn) + 1023) & ~uintptr_t(1023)) +
                     warp * kQStages * kQStageBytes;
-    __shared__ uint64_t s_bar[kThreads / 32][kQStages];
+    __shared__ uint64_t s_bar[kQThreads / 32][kQStages];
     if (!kF32In) {
         if (lane == 0) {
             for (int st = 0; st < kQStages; st++) sm100::mbar_init(&s_bar[warp][st], 1);
@@ -293,8 +277,10 @@ __global__ void __launch_bounds__(kThreads) quantize_blocks_kernel(const __grid_
         }
     }
     __syncthreads();
-    unsigned long long v = s_acc[threadIdx.x];
-    if (v) atomicAdd(&p.acc[threadIdx.x], v);
+    if (threadIdx.x < 256) {
+        const unsigned long long v = s_acc[threadIdx.x];
+        if (v) atomicAdd(&p.acc[threadIdx.x], v);
+    }
     // the last CTA to finish turns the buckets into the mean
     __threadfence();
     __syncthreads();
@@ -302,19 +288,20 @@ __global__ void __launch_bounds__(kThreads) quantize_blocks_kernel(const __grid_
     __syncthreads();
     if (s_last) {
         __threadfence();
-        const unsigned long long mine = atomicAdd(&p.acc[threadIdx.x], 0ull);
-        s_acc[threadIdx.x] = mine;
-        // lowest and highest non-zero bucket (1..254), found by the whole block
+        // the first 256 threads own the buckets
+        const unsigned long long mine = threadIdx.x < 256 ? atomicAdd(&p.acc[threadIdx.x], 0ull) : 0ull;
+        if (threadIdx.x < 256) s_acc[threadIdx.x] = mine;
+        // lowest and highest non-zero bucket (1..254)
         const bool nz = mine != 0 && threadIdx.x >= 1 && threadIdx.x <= 254;
         const unsigned bal = __ballot_sync(0xffffffffu, nz);
-        if ((threadIdx.x & 31) == 0) {
+        if ((threadIdx.x & 31) == 0 && threadIdx.x < 256) {
             s_lohi[threadIdx.x >> 5][0] = bal ? (int)(threadIdx.x + __ffs(bal) - 1) : 256;
             s_lohi[threadIdx.x >> 5][1] = bal ? (int)(threadIdx.x + 31 - __clz(bal)) : -1;
         }
         __syncthreads();
         if (threadIdx.x == 0) {
             int lo = 256, hi = -1;
-            for (int w = 0; w < kThreads / 32; w++) {
+            for (int w = 0; w < 8; w++) {
                 lo = min(lo, s_lohi[w][0]);
                 hi = max(hi, s_lohi[w][1]);
             }
@@ -524,13 +511,13 @@ extern "C" qlora_status qlora_quantize_nf4_dq(const void *W, qlora_dtype w_dtype
     qp.nblocks = nblocks;
     memcpy(qp.mkey, mkey, sizeof(mkey));
     QLORA_TRY(prepare_quantize(qp, W, w_dtype, numel, dev));
-    int grid = grid_for(qp.nblocks, kThreads * 4, dev.sms * 2);
+    int grid = grid_for(qp.nblocks, kQThreads * 2, dev.sms);
     {
         LaunchScope ls(QLORA_KERNEL_QUANTIZE, s);
         if (w_dtype == QLORA_FP32)
-            quantize_blocks_kernel<true><<<grid, kThreads, 0, s>>>(qp);
+            quantize_blocks_kernel<true><<<grid, kQThreads, 0, s>>>(qp);
         else
-            quantize_blocks_kernel<false><<<grid, kThreads, kQDynSmem, s>>>(qp);
+            quantize_blocks_kernel<false><<<grid, kQThreads, kQDynSmem, s>>>(qp);
     }
     QLORA_TRY(launch_status());
 
@@ -647,13 +634,13 @@ extern "C" qlora_status qlora_quantize_nf4_dq_noalloc(const void *W, qlora_dtype
     qp.nblocks = nblocks;
     memcpy(qp.mkey, mkey, sizeof(mkey));
     QLORA_TRY(prepare_quantize(qp, W, w_dtype, numel, dev));
-    const int grid = grid_for(qp.nblocks, kThreads * 4, dev.sms * 2);
+    const int grid = grid_for(qp.nblocks, kQThreads * 2, dev.sms);
     {
         LaunchScope ls(QLORA_KERNEL_QUANTIZE, s);
         if (w_dtype == QLORA_FP32)
-            quantize_blocks_kernel<true><<<grid, kThreads, 0, s>>>(qp);
+            quantize_blocks_kernel<true><<<grid, kQThreads, 0, s>>>(qp);
         else
-            quantize_blocks_kernel<false><<<grid, kThreads, kQDynSmem, s>>>(qp);
+            quantize_blocks_kernel<false><<<grid, kQThreads, kQDynSmem, s>>>(qp);
     }
     QLORA_TRY(launch_status());
 

@@ -278,8 +278,16 @@ __global__ void __launch_bounds__(256) decode_finalize_kernel(const float *part,
 #pragma unroll
     for (int j = 0; j < 16; j++) bv[j] = (8 * j < r) ? *reinterpret_cast<const uint4 *>(bn + 8 * j) : make_uint4(0, 0, 0, 0);
     for (int m = 0; m < M; m++) {
+        // four splits' loads ahead of their in-order additions
         float y = 0.0f;
-        for (int s = 0; s < splits; s++) y = __fadd_rn(y, part[((int64_t)s * M + m) * N + n]);
+        for (int s0 = 0; s0 < splits; s0 += 4) {
+            float v[4];
+#pragma unroll
+            for (int i = 0; i < 4; i++) v[i] = s0 + i < splits ? __ldcg(part + ((int64_t)(s0 + i) * M + m) * N + n) : 0.0f;
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+                if (s0 + i < splits) y = __fadd_rn(y, v[i]);
+        }
         const float *hm = h + m * r;
         float l = 0.0f;
 #pragma unroll

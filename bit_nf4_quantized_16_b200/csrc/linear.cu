@@ -127,12 +127,22 @@ __device__ __forceinline__ float4 split_sum4(const float *part, int splits, int6
 {
     const float *src = part + row * ld + col;
     float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    for (int sp = 0; sp < splits; sp++) {
-        const float4 v = __ldcg(reinterpret_cast<const float4 *>(src + sp * split_stride));
-        acc.x = __fadd_rn(acc.x, v.x);
-        acc.y = __fadd_rn(acc.y, v.y);
-        acc.z = __fadd_rn(acc.z, v.z);
-        acc.w = __fadd_rn(acc.w, v.w);
+    // four splits' loads are issued before their in-order additions (issue is
+    // in order, so an addition waiting on a load would hold back the next load)
+    for (int sp0 = 0; sp0 < splits; sp0 += 4) {
+        float4 v[4];
+#pragma unroll
+        for (int i = 0; i < 4; i++)
+            v[i] = sp0 + i < splits ? __ldcg(reinterpret_cast<const float4 *>(src + (sp0 + i) * split_stride))
+                                    : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            if (sp0 + i >= splits) break;
+            acc.x = __fadd_rn(acc.x, v[i].x);
+            acc.y = __fadd_rn(acc.y, v[i].y);
+            acc.z = __fadd_rn(acc.z, v[i].z);
+            acc.w = __fadd_rn(acc.w, v[i].w);
+        }
     }
     return acc;
 }
