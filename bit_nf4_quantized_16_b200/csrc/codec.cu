@@ -162,6 +162,27 @@ __global__ void __maxnreg__(64) quantize_blocks_kernel(const __grid_constant__ Q
     __shared__ uint32_t s_mkey[16];
     __shared__ bool s_last;
     __shared__ int s_lohi[8][2];
+    const uint32_t lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int64_t nwarps = (int64_t)gridDim.x * (kQThreads / 32);
+    // warp w of CTA c is global warp w * gridDim.x + c: the steps a few warps
+    // take beyond an equal share are spread over all SMs instead of landing
+    // on the first CTAs
+    const int64_t first = ((int64_t)warp * gridDim.x + blockIdx.x) * 32;
+    // bf16: this warp's TMA ring (stages of 32 rows x 128 B, 128-byte swizzle);
+    // the first copy is issued before the code table is built
+    extern __shared__ uint8_t q_dyn[];
+    uint8_t *ring = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(q_dyn) + 1023) & ~uintptr_t(1023)) +
+                    warp * kQStages * kQStageBytes;
+    __shared__ uint64_t s_bar[kQThreads / 32][kQStages];
+    if (!kF32In && lane == 0) {
+        for (int st = 0; st < kQStages; st++) sm100::mbar_init(&s_bar[warp][st], 1);
+        sm100::fence_barrier_init();
+        if (first < p.nblocks) {
+            sm100::mbar_arrive_expect_tx(&s_bar[warp][0], kQStageBytes);
+            sm100::tma_load_2d(ring, &p.tm_w, &s_bar[warp][0], 0, (int32_t)first);
+        }
+    }
     if (threadIdx.x == 0) {
 #pragma unroll
         for (int j = 0; j < 15; j++) s_mkey[j] = p.mkey[j];
@@ -170,27 +191,6 @@ __global__ void __maxnreg__(64) quantize_blocks_kernel(const __grid_constant__ Q
     __syncthreads();
     if (threadIdx.x < 256) build_code_lut(lut, s_mkey);
     __syncthreads();
-
-    const uint32_t lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const int64_t nwarps = (int64_t)gridDim.x * (kQThreads / 32);
-    const int64_t first = ((int64_t)blockIdx.x * (kQThreads / 32) + warp) * 32;
-    // bf16: this warp's TMA ring (stages of 32 rows x 128 B, 128-byte swizzle)
-    extern __shared__ uint8_t q_dyn[];
-    uint8_t *ring = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(q_dyn) + 1023) & ~uintptr_t(1023)) +
-                    warp * kQStages * kQStageBytes;
-    __shared__ uint64_t s_bar[kQThreads / 32][kQStages];
-    if (!kF32In) {
-        if (lane == 0) {
-            for (int st = 0; st < kQStages; st++) sm100::mbar_init(&s_bar[warp][st], 1);
-            sm100::fence_barrier_init();
-            if (first < p.nblocks) {
-                sm100::mbar_arrive_expect_tx(&s_bar[warp][0], kQStageBytes);
-                sm100::tma_load_2d(ring, &p.tm_w, &s_bar[warp][0], 0, (int32_t)first);
-            }
-        }
-        __syncwarp();
-    }
     uint32_t it = 0;
     for (int64_t b0 = first; b0 < p.nblocks; b0 += nwarps * 32, it++) {
         const int64_t b = b0 + lane;
@@ -286,10 +286,14 @@ __global__ void __maxnreg__(64) quantize_blocks_kernel(const __grid_constant__ Q
         const unsigned long long v = s_acc[threadIdx.x];
         if (v) atomicAdd(&p.acc[threadIdx.x], v);
     }
-    // the last CTA to finish turns the buckets into the mean
-    __threadfence();
+    // the last CTA to finish turns the buckets into the mean.  The barrier
+    // orders this CTA's bucket atomics before thread 0's fence, which is
+    // cumulative over them, and the fence before the ticket.
     __syncthreads();
-    if (threadIdx.x == 0) s_last = atomicAdd(p.ticket, 1u) == gridDim.x - 1;
+    if (threadIdx.x == 0) {
+        __threadfence();
+        s_last = atomicAdd(p.ticket, 1u) == gridDim.x - 1;
+    }
     __syncthreads();
     if (s_last) {
         __threadfence();
