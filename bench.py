@@ -656,6 +656,45 @@ def run_reference(args, rank, world):
     }
 
 
+def run_codec_shape(args, q, torch, dev):
+    """Quantize and dequantize one N(0, 0.02) bf16 tensor of the shape given by
+    --codec-shape NxK: `warmup` untimed calls, then `steps` calls of each, every
+    call after an L2 flush and bracketed by CUDA events (a per-shape view of the
+    codec, small enough for a full ncu capture)."""
+    import synthetic
+    N, K = (int(v) for v in args.codec_shape.lower().split("x"))
+    W = synthetic.normal((N, K), 0.02, 77, torch.bfloat16, dev)
+    w = q.NF4Weight(N, K, device=dev)
+    ws = torch.empty(q.qlora_quantize_workspace_bytes(N, K), dtype=torch.uint8, device=dev)
+    out = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)   # > 126 MB L2
+    for _ in range(args.warmup):
+        q.qlora_quantize_nf4_dq(W, w, ws)
+        q.qlora_dequantize_nf4_dq(w, out)
+    torch.cuda.synchronize()
+    q.qlora_check_device_error()
+    times = {"quantize": [], "dequantize": []}
+    for _ in range(args.steps):
+        for kind in ("quantize", "dequantize"):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            if kind == "quantize":
+                q.qlora_quantize_nf4_dq(W, w, ws)
+            else:
+                q.qlora_dequantize_nf4_dq(w, out)
+            e1.record()
+            torch.cuda.synchronize()
+            times[kind].append(e0.elapsed_time(e1) * 1e3)
+    q.qlora_check_device_error()
+    res = {"workload": f"codec shape {N}x{K}: one bf16 tensor ~N(0,0.02), L2 flushed before each call",
+           "unit": "GB/s", "bytes_per_weight": CODEC_BYTES_PER_WEIGHT}
+    for kind, ts in times.items():
+        us = sorted(ts)[len(ts) // 2]
+        res[kind] = {"us_median": round(us, 2), "value": round(CODEC_BYTES_PER_WEIGHT * N * K / (us * 1e-6) / 1e9, 1)}
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -673,6 +712,8 @@ def main():
     ap.add_argument("--codec-tensors", type=int, default=0,
                     help="limit the codec round trip to the first N LLaMA-7B tensors (profiling runs)")
     ap.add_argument("--codec-only", action="store_true", help="run only the codec round trip (profiling runs)")
+    ap.add_argument("--codec-shape", default=None,
+                    help="NxK: time quantize and dequantize of one tensor of this shape only (profiling runs)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank = int(os.environ.get("RANK", "0"))
@@ -693,7 +734,11 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        if args.codec_only:
+        if args.codec_shape:
+            import bit_nf4_quantized_16_b200 as q
+            torch.cuda.set_device(local_rank)
+            line = {"impl": "ours", "codec_shape": run_codec_shape(args, q, torch, torch.device("cuda", local_rank))}
+        elif args.codec_only:
             import bit_nf4_quantized_16_b200 as q
             torch.cuda.set_device(local_rank)
             peaks, src = load_peaks()
