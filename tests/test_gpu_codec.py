@@ -75,6 +75,13 @@ def test_llama_7b_shapes_bf16(q):
         check_parity(q, synthetic.normal((rows, cols), 0.02, seed=40 + i, dtype=torch.bfloat16))
 
 
+def test_llama_65b_shapes_bf16(q):
+    """The largest tensors of the 65B configurations, compared in full: 8192²
+    (attention) and 22016 x 8192 (2.8 M blocks, about 25 warp-steps per warp)."""
+    for i, (rows, cols) in enumerate([(8192, 8192), (22016, 8192)]):
+        check_parity(q, synthetic.normal((rows, cols), 0.02, seed=60 + i, dtype=torch.bfloat16))
+
+
 def test_edge_blocks(q):
     """Zero blocks, a subnormal block, values exactly on the round-down
     midpoints (ties go to the lower code), and +-absmax."""
