@@ -251,41 +251,56 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm) decode_gemv_kernel
     }
 }
 
+// Up to 8 split partials of token m at outputs n, splits s0 .. s0+7.
+__device__ __forceinline__ void load_splits8(float (&v)[8], const float *part, int s0, int splits, int m, int M,
+                                             int64_t N, int64_t n)
+{
+#pragma unroll
+    for (int i = 0; i < 8; i++)
+        v[i] = s0 + i < splits ? __ldcg(part + ((int64_t)(s0 + i) * M + m) * N + n) : 0.0f;
+}
+
 // One CTA per 256 outputs n (all tokens): the H rows of every token from the
 // A partials (fixed order) in shared memory, B[n] in registers, then
-// y[m][n] = sum of the W splits + H[m] . B[n].
+// y[m][n] = sum of the W splits + H[m] . B[n].  The chain of dependent
+// memory waits is kept short: B[n] is read before the dependency wait (it is
+// not written by the GEMV; everything before the GEMV in the stream completed
+// before the GEMV let this kernel start, and the loads go through L2 only),
+// and the first token's split partials are in flight during the H reduction.
 __global__ void __launch_bounds__(256) decode_finalize_kernel(const float *part, const float *part_h, int splits,
                                                             int M, int64_t N, int r, float scale,
                                                             const __nv_bfloat16 *B, void *Y, int y_f32,
                                                             float *H_save)
 {
     __shared__ float h[kDecodeMaxTokens * 128];
+    const int64_t n = (int64_t)blockIdx.x * 256 + threadIdx.x;
+    const bool has_row = n < N;
+    uint4 bv[16];   // B[n][0 .. r), r <= 128
+    const __nv_bfloat16 *bn = B + (has_row ? n : 0) * r;
+#pragma unroll
+    for (int j = 0; j < 16; j++)
+        bv[j] = (has_row && 8 * j < r) ? __ldcg(reinterpret_cast<const uint4 *>(bn + 8 * j)) : make_uint4(0, 0, 0, 0);
     sm100::pdl_wait();
     sm100::pdl_trigger();
+    float v[8];
+    load_splits8(v, part, 0, has_row ? splits : 0, 0, M, N, n);
     for (int i = threadIdx.x; i < M * r; i += blockDim.x) {
-        float v = 0.0f;
+        float hv = 0.0f;
 #pragma unroll
-        for (int s = 0; s < kAPieces; s++) v = __fadd_rn(v, part_h[(int64_t)s * M * r + i]);
-        v = __fmul_rn(scale, v);
-        h[i] = v;
-        if (H_save && blockIdx.x == 0) H_save[i] = v;
+        for (int s = 0; s < kAPieces; s++) hv = __fadd_rn(hv, part_h[(int64_t)s * M * r + i]);
+        hv = __fmul_rn(scale, hv);
+        h[i] = hv;
+        if (H_save && blockIdx.x == 0) H_save[i] = hv;
     }
     __syncthreads();
-    const int64_t n = (int64_t)blockIdx.x * 256 + threadIdx.x;
-    if (n >= N) return;
-    uint4 bv[16];   // B[n][0 .. r), r <= 128
-    const __nv_bfloat16 *bn = B + n * r;
-#pragma unroll
-    for (int j = 0; j < 16; j++) bv[j] = (8 * j < r) ? *reinterpret_cast<const uint4 *>(bn + 8 * j) : make_uint4(0, 0, 0, 0);
+    if (!has_row) return;
     for (int m = 0; m < M; m++) {
-        // four splits' loads ahead of their in-order additions
+        // eight splits' loads ahead of their in-order additions
         float y = 0.0f;
-        for (int s0 = 0; s0 < splits; s0 += 4) {
-            float v[4];
+        for (int s0 = 0; s0 < splits; s0 += 8) {
+            if (m > 0 || s0 > 0) load_splits8(v, part, s0, splits, m, M, N, n);
 #pragma unroll
-            for (int i = 0; i < 4; i++) v[i] = s0 + i < splits ? __ldcg(part + ((int64_t)(s0 + i) * M + m) * N + n) : 0.0f;
-#pragma unroll
-            for (int i = 0; i < 4; i++)
+            for (int i = 0; i < 8; i++)
                 if (s0 + i < splits) y = __fadd_rn(y, v[i]);
         }
         const float *hm = h + m * r;
