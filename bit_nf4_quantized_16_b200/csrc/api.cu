@@ -193,6 +193,18 @@ extern "C" qlora_status qlora_build_nf4_codebook(double delta, float codebook_ou
     return QLORA_OK;
 }
 
+// Int4 as an absmax code ("QLoRA: Efficient Finetuning of Quantized LLMs",
+// section "Introduction", item (1), compares NF4 with 4-bit integers without
+// defining them): the 16 two's-complement integers -8 .. 7 divided by 7, so
+// that +-7 carry the block's absmax.  -8/7 lies beyond -1 and is never the
+// nearest value to a scaled element.
+extern "C" qlora_status qlora_build_int4_codebook(float codebook_out[16])
+{
+    if (!codebook_out) return QLORA_ERR_INVALID_ARG;
+    for (int j = 0; j < 16; j++) codebook_out[j] = (float)((double)(j - 8) / 7.0);
+    return QLORA_OK;
+}
+
 extern "C" const char *qlora_status_string(qlora_status status)
 {
     switch (status) {

@@ -117,6 +117,18 @@ typedef struct {
 QLORA_API qlora_status qlora_build_nf4_codebook(double delta, float codebook_out[16]);
 
 /*
+ * qlora_build_int4_codebook -- a 4-bit integer table for the same codec and
+ * GEMMs ("Introduction", item (1), names 4-bit integers as the baseline NF4
+ * is compared with, without defining them).  Reading: the two's-complement
+ * integers -8 .. 7 divided by 7, q_j = RN32((j - 8) / 7), so that +-7 carry
+ * the block's absmax; -8/7 is never the nearest value to a scaled element.
+ * Strictly ascending with its one zero at index 8.  Host-only, no CUDA call.
+ *   codebook_out   host, 16 floats.
+ * Errors: QLORA_ERR_INVALID_ARG for a null pointer.
+ */
+QLORA_API qlora_status qlora_build_int4_codebook(float codebook_out[16]);
+
+/*
  * Workspace in bytes that qlora_quantize_nf4_dq needs for a rows x cols
  * weight (first-level constants plus a few reduction slots).
  */

@@ -74,3 +74,12 @@ def nfk_codebook_f64(k: int = 4, delta: float = DEFAULT_DELTA) -> np.ndarray:
 def nf4_codebook(delta: float = DEFAULT_DELTA) -> np.ndarray:
     """NF4 as the 16 binary32 values the codec stores (rounded once)."""
     return nfk_codebook_f64(4, delta).astype(np.float32)
+
+
+def int4_codebook() -> np.ndarray:
+    """4-bit integers as an absmax code.  The paper's introduction, item (1),
+    names 4-bit integers as the data type NF4 is compared with but does not
+    define them.  Reading: the sixteen two's-complement values -8 .. 7 over
+    the level count 7, so that +-7 carry the block's absmax (one binary32
+    rounding of each exact quotient).  -8/7 lies below -1 and never wins."""
+    return np.array([np.float32(float(j) / 7.0) for j in range(-8, 8)], dtype=np.float32)

@@ -27,9 +27,9 @@ def q():
     return q
 
 
-def gpu_quantize(q, W: torch.Tensor):
+def gpu_quantize(q, W: torch.Tensor, codebook=None):
     rows, cols = W.shape
-    w = q.NF4Weight(rows, cols, device="cuda")
+    w = q.NF4Weight(rows, cols, codebook=codebook, device="cuda")
     ws = torch.empty(q.qlora_quantize_workspace_bytes(rows, cols), dtype=torch.uint8, device="cuda")
     q.qlora_quantize_nf4_dq(W.cuda().contiguous(), w, ws)
     torch.cuda.synchronize()
@@ -43,15 +43,16 @@ def gpu_dequantize(q, w):
     return out.view(torch.int16).cpu().numpy().view(np.uint16).ravel()
 
 
-def check_parity(q, W: torch.Tensor):
-    w = gpu_quantize(q, W)
-    ref = occ.quantize(W.float().numpy(), Q)
+def check_parity(q, W: torch.Tensor, codebook=None):
+    table = Q if codebook is None else np.asarray(codebook, np.float32)
+    w = gpu_quantize(q, W, codebook)
+    ref = occ.quantize(W.float().numpy(), table)
     assert np.array_equal(w.packed.cpu().numpy(), ref["packed"]), "packed codes"
     assert np.array_equal(w.code2.cpu().numpy(), ref["e"]), "E4M3 codes"
     assert np.array_equal(w.c2.cpu().numpy().view(np.uint32), ref["c2"].view(np.uint32)), "group scales"
     assert w.mean[0].item() == float(ref["mean"]), "mean"
     got = gpu_dequantize(q, w)
-    want = occ.dequantize(ref["packed"], ref["e"], ref["c2"], ref["mean"], Q)
+    want = occ.dequantize(ref["packed"], ref["e"], ref["c2"], ref["mean"], table)
     assert np.array_equal(got, want), "dequantized bf16"
     return w, ref
 
@@ -80,6 +81,26 @@ def test_llama_65b_shapes_bf16(q):
     (attention) and 22016 x 8192 (2.8 M blocks, about 25 warp-steps per warp)."""
     for i, (rows, cols) in enumerate([(8192, 8192), (22016, 8192)]):
         check_parity(q, synthetic.normal((rows, cols), 0.02, seed=60 + i, dtype=torch.bfloat16))
+
+
+def test_int4_codebook(q):
+    """The Int4 table through the same quantizer and dequantizer: ragged and
+    full-size tensors, a zero block (the table's zero is index 8) and exact
+    midpoints."""
+    table = q.qlora_build_int4_codebook()
+    for i, (rows, cols) in enumerate([(3, 192), (257, 320), (4096, 4096)]):
+        check_parity(q, synthetic.normal((rows, cols), 0.02, seed=80 + i, dtype=torch.bfloat16), table)
+    W = synthetic.normal((4, 256), 0.02, seed=83)
+    W[0, :64] = 0.0
+    t = np.asarray(table, np.float64)
+    mids = np.float32((t[1:] + t[:-1]) / 2)
+    row = np.zeros(64, np.float32)
+    row[0] = 1.0
+    row[1:15] = mids[1:]
+    row[15:29] = np.nextafter(mids[1:], np.float32(2))
+    W[1, :64] = torch.from_numpy(row)
+    w, ref = check_parity(q, W, table)
+    assert np.all(occ.unpack(w.packed.cpu().numpy())[:64] == 8)
 
 
 def test_edge_blocks(q):

@@ -54,19 +54,19 @@ def assert_close(got, ref, bf16_out=False, what=""):
     assert np.all(err <= bound), f"{what}: max abs {err.max():.3e} at {worst}"
 
 
-def oracle_weight(W):
-    ref = occ.quantize(W.float().numpy(), Q)
-    Wd = occ.dequantize(ref["packed"], ref["e"], ref["c2"], ref["mean"], Q)
+def oracle_weight(W, codebook=Q):
+    ref = occ.quantize(W.float().numpy(), codebook)
+    Wd = occ.dequantize(ref["packed"], ref["e"], ref["c2"], ref["mean"], codebook)
     return occ.bf16_bits_to_f32(Wd).reshape(W.shape).astype(np.float64)
 
 
 class Runner:
     """Quantizes W on the GPU and runs the layer through the C ABI."""
 
-    def __init__(self, q, case):
+    def __init__(self, q, case, codebook=None):
         self.q, self.c = q, case
         N, K = case["W"].shape
-        self.w = q.NF4Weight(N, K)
+        self.w = q.NF4Weight(N, K, codebook=codebook)
         ws = torch.empty(q.qlora_quantize_workspace_bytes(N, K), dtype=torch.uint8, device="cuda")
         q.qlora_quantize_nf4_dq(case["W"].cuda(), self.w, ws)
         self.X = case["X"].cuda()
@@ -100,9 +100,9 @@ def np64(t):
     return t.float().cpu().numpy().astype(np.float64)
 
 
-def full_check(q, case, ydt=torch.float32):
-    run = Runner(q, case)
-    Wd = oracle_weight(case["W"])
+def full_check(q, case, ydt=torch.float32, codebook=None):
+    run = Runner(q, case, codebook)
+    Wd = oracle_weight(case["W"], Q if codebook is None else np.asarray(codebook, np.float32))
     X, A, B, dY = (np64(case[k]) for k in ("X", "A", "B", "dY"))
     s = case["scale"]
     Y, _ = run.fwd(ydt)
@@ -132,6 +132,16 @@ def test_tiny_config_bf16_outputs(q):
 ])
 def test_ragged_shapes(q, M, N, K, r):
     full_check(q, synthetic.linear_case(M, N, K, r, alpha=16.0, seed=M + N + K + r))
+
+
+@pytest.mark.parametrize("M", [16, 200, 512])
+def test_int4_codebook(q, M):
+    """The Int4 table through the same kernels: the decode forward (16
+    tokens), the single-CTA fused GEMMs (200) and the CTA-pair GEMMs (512)."""
+    case = synthetic.linear_case(M, 384, 320, 16, alpha=16.0, seed=70 + M)
+    table = q.qlora_build_int4_codebook()
+    assert np.array_equal(np.array(table, np.float32).view(np.uint32), ocb.int4_codebook().view(np.uint32))
+    full_check(q, case, codebook=table)
 
 
 def test_saved_h_equals_recomputed_h(q):

@@ -66,3 +66,20 @@ def test_nfk_general_k(k):
     assert np.count_nonzero(q == 0.0) == 1
     assert np.count_nonzero(q < 0) == 2 ** (k - 1) - 1
     assert np.all(np.diff(q) > 0)
+
+
+def test_int4_table_structure():
+    """Int4 as an absmax code: sixteen strictly increasing values, the zero at
+    index 8 (two's-complement order), +-1 exactly at the levels +-7, one
+    level below -1, and every value within a binary32 rounding of an integer
+    multiple of 1/7 (checked in exact rationals)."""
+    from fractions import Fraction
+    q = codebook.int4_codebook()
+    assert q.dtype == np.float32 and q.size == 16
+    assert np.all(np.diff(q) > 0)
+    assert np.count_nonzero(q == 0.0) == 1 and q[8] == 0.0
+    assert q[1] == -1.0 and q[15] == 1.0 and q[0] < -1.0
+    for j, v in enumerate(q):
+        level = Fraction(j - 8, 7)
+        ulp = Fraction(float(np.spacing(np.float32(abs(v)) if v else np.float32(1e-38))))
+        assert abs(Fraction(float(v)) - level) <= ulp / 2, (j, float(v))

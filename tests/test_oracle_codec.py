@@ -123,6 +123,41 @@ def test_zero_and_subnormal_blocks_take_the_zero_code():
     assert c1[1] == np.float32(1e-40)
 
 
+def test_int4_table_nearest_code_and_zero_blocks():
+    """The same first level with the Int4 table: values on, just below and
+    just above every midpoint of the table take the nearest value (ties to
+    the lower index), a zero block takes the table's zero (index 8), and
+    bf16(q_j * a) inputs come back exactly."""
+    q4 = codebook.int4_codebook()
+    xs = []
+    for j in range(15):
+        m32 = np.float32((float(q4[j]) + float(q4[j + 1])) / 2)
+        xs += [m32, np.nextafter(m32, np.float32(-2)), np.nextafter(m32, np.float32(2))]
+    xs = [x for x in xs if abs(x) <= 1.0]
+    xs = np.array(xs, np.float32)
+    pad = (-xs.size) % 63
+    body = np.concatenate([xs, np.zeros(pad, np.float32)]).reshape(-1, 63)
+    W = np.concatenate([np.ones((body.shape[0], 1), np.float32), body], axis=1)
+    c1, codes = codec.quantize_first_level(W, q4)
+    assert np.all(c1 == 1.0)
+    codes = codes.reshape(W.shape)
+    for i in range(W.shape[0]):
+        for k in range(64):
+            assert codes[i, k] == _nearest_exact(W[i, k], q4), (W[i, k], codes[i, k])
+    assert not np.any(codes == 0), "-8/7 is never the nearest value"
+    _, zc = codec.quantize_first_level(np.zeros((2, 64), np.float32), q4)
+    assert np.all(zc == 8)
+    rng = np.random.default_rng(19)
+    a = np.float32(0.0625)
+    idx = rng.integers(1, 16, (16, 256)).astype(np.uint8)
+    idx[:, ::64] = rng.choice([1, 15], (16, 4))
+    Wr = codec.bf16_bits_to_f32(codec.bf16_rne((q4[idx] * a).astype(np.float32)))
+    d = codec.quantize(Wr, q4)
+    assert np.array_equal(d["codes"].reshape(idx.shape), idx)
+    w = codec.dequantize(d["packed"], d["e"], d["c2"], d["mean"], q4)
+    assert np.array_equal(codec.bf16_bits_to_f32(w), Wr.ravel())
+
+
 def test_first_level_error_bound():
     """|x - q[code] c1| <= c1 * (largest half-gap of the codebook) + rounding."""
     rng = np.random.default_rng(8)
