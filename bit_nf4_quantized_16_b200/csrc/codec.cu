@@ -3,13 +3,15 @@
 // "QLoRA: Efficient Finetuning of Quantized LLMs", section "Method":
 //   - "4-bit NormalFloat Quantization", step (3): each block of 64 weights is
 //     rescaled by its absolute maximum into [-1, 1] and rounded to the nearest
-//     value of the 16-entry NF4 table;
+//     value of the 16-entry table (NF4, or any strictly increasing 16-value
+//     table with one zero, such as the Int4 one);
 //   - "Double Quantization": the per-block 32-bit constants are quantized
 //     again (8-bit floats, groups of 256, mean subtracted);
 //   - storage vs. compute type: the weight is dequantized to BFloat16 when
 //     used.
 //
-// Three kernels, all HBM-bound streaming passes with 16-byte accesses:
+// Three kernels, all streaming passes (bf16 input through per-warp TMA rings,
+// 16- and 32-byte global accesses elsewhere):
 //   quantize_blocks_kernel  W -> packed codes, c1 (workspace), exact mean
 //   dq_encode_kernel        c1, mean -> code2 (E4M3), c2
 //   dequantize_kernel       packed, code2, c2, mean -> bf16 W'
