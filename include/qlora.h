@@ -14,9 +14,8 @@
  *     essay, "Low-Rank Adaptation (LoRA)"), in row-vector form
  *         Y = X W'^T + s (X A^T) B^T,      W' = dequant(W_q),
  *     with its backward pass dX, dA, dB; the quantized weight is frozen, so
- *     there is no dW (abstract: gradients are backpropagated "through a
- *     frozen, 4-bit quantized pretrained language model into Low Rank
- *     Adapters").
+ *     there is no dW (abstract: the gradients pass through the frozen 4-bit
+ *     base model and update only the low-rank adapters).
  *
  * Conventions common to every entry point
  *   - Pointers named "device" must point to memory of the current CUDA device;
@@ -54,7 +53,7 @@ extern "C" {
 #endif
 
 /* Blocksize of the first quantization level: 64 consecutive elements of one
- * row ("Method", "Double Quantization": "a blocksize of 64 for W"). */
+ * row ("Method", paragraph "Double Quantization": W uses blocks of 64). */
 #define QLORA_BLOCK 64
 /* Number of first-level constants per second-level (double-quantization)
  * group: 256 consecutive blocks in row-major block order. */

@@ -21,8 +21,8 @@ Modules
 
 Parity status: every function has a pin in tests/test_oracle_*.py except the
 individual NF4 codebook values beyond the structural invariants, and the
-"equal expected number of values per bin" property, which the pages state
-but never print numbers for ("parity unpinned" for those two).
+claim that every bin holds the same expected share of values, which the
+pages make but never back with numbers ("parity unpinned" for those two).
 """
 
 from . import codebook, exact, codec, linear  # noqa: F401
