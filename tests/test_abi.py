@@ -107,3 +107,90 @@ def test_validation_happens_before_any_cuda_call(lib):
     assert f(fake, 0, ctypes.byref(w), fake, 16, None) == 4                 # workspace too small
     unsorted = Weight(64, 128, fake, fake, fake, fake, (ctypes.c_float * 16)(*q[::-1]))
     assert f(fake, 0, ctypes.byref(unsorted), fake, 1 << 20, None) == 1     # codebook not ascending
+
+
+def _no_gpu():
+    # the fake pointers below are never dereferenced because every call fails
+    # validation first; still, never hand them to a library that sees a GPU
+    try:
+        import torch
+        return not torch.cuda.is_available()
+    except Exception:
+        return True
+
+
+@pytest.mark.skipif(not _no_gpu(), reason="host-only validation test with placeholder pointers")
+def test_validation_of_tables_dequantize_and_noalloc(lib):
+    q = ocb.nf4_codebook()
+    fake = 0x10000
+    quant = lib.qlora_quantize_nf4_dq
+    quant.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(Weight), ctypes.c_void_p, ctypes.c_size_t,
+                      ctypes.c_void_p]
+    two_zeros = q.copy()
+    two_zeros[8] = 0.0
+    two_zeros[7] = np.float32(-1e-30)
+    two_zeros[6] = 0.0
+    w = Weight(64, 128, fake, fake, fake, fake, (ctypes.c_float * 16)(*two_zeros))
+    assert quant(fake, 0, ctypes.byref(w), fake, 1 << 20, None) == 1          # not strictly ascending
+    close = q.copy()
+    close[12] = np.nextafter(close[11], np.float32(2))                        # 11, 12 almost equal:
+    close[13] = np.nextafter(close[12], np.float32(2))                        # two midpoints, one interval
+    w = Weight(64, 128, fake, fake, fake, fake, (ctypes.c_float * 16)(*close))
+    assert quant(fake, 0, ctypes.byref(w), fake, 1 << 20, None) == 6          # QLORA_ERR_UNSUPPORTED
+    noz = np.linspace(-1, 1, 17)[np.arange(17) != 8].astype(np.float32)       # no zero at all
+    w = Weight(64, 128, fake, fake, fake, fake, (ctypes.c_float * 16)(*noz))
+    assert quant(fake, 0, ctypes.byref(w), fake, 1 << 20, None) == 1
+
+    deq = lib.qlora_dequantize_nf4_dq
+    deq.argtypes = [ctypes.POINTER(Weight), ctypes.c_void_p, ctypes.c_void_p]
+    w = Weight(64, 128, fake, fake, fake, fake, (ctypes.c_float * 16)(*q))
+    assert deq(None, fake, None) == 1
+    assert deq(ctypes.byref(w), None, None) == 1
+    assert deq(ctypes.byref(w), fake + 2, None) == 3
+    w_mis = Weight(64, 128, fake + 8, fake, fake, fake, (ctypes.c_float * 16)(*q))
+    assert deq(ctypes.byref(w_mis), fake, None) == 3
+
+    na = lib.qlora_quantize_nf4_dq_noalloc
+    na.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(Weight), ctypes.c_void_p]
+    big = Weight(1 << 14, 1 << 13, fake, fake, fake, fake, (ctypes.c_float * 16)(*q))   # 2^21 blocks
+    assert na(fake, 0, ctypes.byref(big), None) == 2
+    assert na(fake, 3, ctypes.byref(w), None) == 1
+
+
+@pytest.mark.skipif(not _no_gpu(), reason="host-only validation test with placeholder pointers")
+def test_validation_of_the_linear_layer(lib):
+    q = ocb.nf4_codebook()
+    fake = 0x10000
+    P, I64, I32, F, S, I = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t,
+                            ctypes.c_int)
+    W = ctypes.POINTER(Weight)
+    fwd = lib.qlora_linear_fwd
+    fwd.argtypes = [W, P, I64, P, P, I32, F, P, I, P, P, S, P]
+    bwd = lib.qlora_linear_bwd
+    bwd.argtypes = [W, P, P, I64, P, P, I32, F, P, P, I, P, P, P, S, P]
+    w = Weight(256, 256, fake, fake, fake, fake, (ctypes.c_float * 16)(*q))
+    ok = dict(X=fake, M=16, A=fake, B=fake, r=16, Y=fake, ydt=1, H=None, ws=fake)
+
+    def f(**kw):
+        a = dict(ok, **kw)
+        return fwd(kw.get("w", ctypes.byref(w)), a["X"], a["M"], a["A"], a["B"], a["r"], 1.0, a["Y"], a["ydt"],
+                   a["H"], a["ws"], 1 << 30, None)
+
+    assert f(M=-1) == 1
+    assert f(r=0) == 2 and f(r=4) == 2 and f(r=12) == 2 and f(r=136) == 2
+    assert f(X=None) == 1 and f(A=None) == 1 and f(B=None) == 1 and f(ws=None) == 1 and f(Y=None) == 1
+    assert f(X=fake + 2) == 3 and f(B=fake + 8) == 3 and f(Y=fake + 4) == 3 and f(H=fake + 4) == 3
+    assert f(ydt=5) == 1
+    odd = Weight(250, 256, fake, fake, fake, fake, (ctypes.c_float * 16)(*q))
+    assert f(w=ctypes.byref(odd)) == 2                                   # rows % 8
+    assert f(w=None) == 1
+
+    def b(**kw):
+        a = dict(dict(ok, dY=fake, dX=fake, dA=fake, dB=fake, dxdt=1), **kw)
+        return bwd(ctypes.byref(w), a["X"], a["dY"], a["M"], a["A"], a["B"], a["r"], 1.0, a["H"], a["dX"], a["dxdt"],
+                   a["dA"], a["dB"], a["ws"], 1 << 30, None)
+
+    assert b(dY=None) == 1 and b(dA=None) == 1 and b(dB=None) == 1
+    assert b(dxdt=9) == 1
+    assert b(dY=fake + 2) == 3 and b(dX=fake + 4) == 3 and b(dA=fake + 8) == 3 and b(H=fake + 4) == 3
+    assert b(r=200) == 2
