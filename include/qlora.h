@@ -86,8 +86,9 @@ typedef enum { QLORA_BF16 = 0, QLORA_FP32 = 1 } qlora_dtype;
  *           [256g, 256g+256).
  *   mean    device, 1 float: mean of all first-level constants of W.
  *   codebook  host values q[0..15], strictly ascending, containing exactly
- *           one 0; the NF4 table from qlora_build_nf4_codebook() or any other
- *           4-bit table with the same properties.
+ *           one 0; the NF4 table from qlora_build_nf4_codebook(), the Int4
+ *           table from qlora_build_int4_codebook(), or any other 16-value
+ *           table with the same properties that the quantizer accepts.
  */
 typedef struct {
     int64_t rows;
@@ -148,7 +149,13 @@ QLORA_API size_t qlora_quantize_workspace_bytes(int64_t rows, int64_t cols);
  *              the codebook (read).  rows >= 1, cols % 64 == 0.
  *   workspace  device, at least qlora_quantize_workspace_bytes(rows, cols)
  *              bytes; contents on entry do not matter; clobbered.
- * Errors: INVALID_ARG, SHAPE, ALIGNMENT, WORKSPACE, CUDA, UNSUPPORTED.
+ * Errors: INVALID_ARG (null pointer, unknown dtype, a codebook that is not
+ * strictly increasing or does not hold exactly one zero), SHAPE, ALIGNMENT,
+ * WORKSPACE, CUDA, UNSUPPORTED (not a B200, or a codebook the code lookup
+ * cannot serve: two midpoints between neighbouring values that share the top
+ * 12 bits of their order-preserving binary32 keys, or a pair of neighbours
+ * whose sum is not exact in binary64; neither happens for the NF4 and Int4
+ * tables of the builders above).
  * Deterministic: the same input gives the same bytes on every call.
  */
 QLORA_API qlora_status qlora_quantize_nf4_dq(const void *W, qlora_dtype w_dtype, const qlora_nf4_weight *out,
