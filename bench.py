@@ -45,8 +45,8 @@ def linear_flops(M, N, K, r):
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch from one
 # ncu capture of the bench workloads, averaged over the launches of one step
-# (profiles/dram_traffic_linear7b_codec.md).  Each set describes the kernel
-# sources whose SHA-256 it names and is reported only while they are unchanged.
+# (the committed DRAM-traffic capture).  Each set describes the kernel sources
+# whose SHA-256 it names and is reported only while they are unchanged.
 _CSRC = os.path.join("bit_nf4_quantized_16_b200", "csrc")
 MEASURED_TRAFFIC = {
     "linear": {
@@ -285,6 +285,7 @@ def run_ours(args, rank, world, local_rank):
 
     codec = run_codec(args, q, torch, dev, peaks, peak_src) if (rank == 0 and not args.skip_codec) else None
     decode = run_decode65b(args, q, torch, dev, peaks, peak_src) if (rank == 0 and not args.skip_decode) else None
+    adamw = run_adamw7b(args, q, torch, dev, peaks, peak_src) if (rank == 0 and not args.skip_optim) else None
     del layers, ws, grads, flush
     stack = run_stack65b(args, q, torch, dev, peaks, peak_src) if (rank == 0 and not args.skip_stack) else None
 
@@ -311,6 +312,8 @@ def run_ours(args, rank, world, local_rank):
         line["codec"] = codec
     if decode is not None:
         line["decode65b"] = decode
+    if adamw is not None:
+        line["adamw7b"] = adamw
     if stack is not None:
         line["stack65b"] = stack
     if world == 1 and not args.skip_cpu:
@@ -374,7 +377,7 @@ def run_codec(args, q, torch, dev, peaks, peak_src):
     bytes_rt = 2 * CODEC_BYTES_PER_WEIGHT * nweights
     gbs = bytes_rt / (ms * 1e-3) / 1e9
     # per-kernel device time: the same work on one stream, each kernel bracketed
-    # by CUDA events
+    # by CUDA events (the breakdown: brackets separate the kernels)
     q.qlora_timing_reset()
     q.qlora_timing_enable(True)
     torch.cuda._sleep(100_000_000)
@@ -383,10 +386,29 @@ def run_codec(args, q, torch, dev, peaks, peak_src):
         q.qlora_dequantize_nf4_dq(w, out)
     q.qlora_timing_enable(False)
     kern = q.qlora_timing_read()
-    qms = kern["quantize"][0]
-    dms = kern["dequantize"][0]
+    # per-call device time: each API call bracketed by CUDA events, its own
+    # kernels chained as a user sees them (quantize = workspace reset, the
+    # first-level pass and the double quantization of its constants, whose
+    # E4M3 codes and scales are part of the 2.5159 B per weight)
+    marks = []
+    torch.cuda._sleep(100_000_000)
+    for W, w, out in tensors:
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        ev[0].record()
+        q.qlora_quantize_nf4_dq(W, w, qws[0])
+        ev[1].record()
+        q.qlora_dequantize_nf4_dq(w, out)
+        ev[2].record()
+        marks.append(ev)
+    torch.cuda.synchronize()
+    q.qlora_check_device_error()
+    qms = sum(ev[0].elapsed_time(ev[1]) for ev in marks)
+    dms = sum(ev[1].elapsed_time(ev[2]) for ev in marks)
     qgbs = CODEC_BYTES_PER_WEIGHT * nweights / (qms * 1e-3) / 1e9
     dgbs = CODEC_BYTES_PER_WEIGHT * nweights / (dms * 1e-3) / 1e9
+    big = [i for i, (N, K) in enumerate(shapes) if N * K == max(a * b for a, b in shapes)]
+    big_us = sorted(marks[i][0].elapsed_time(marks[i][1]) * 1e3 for i in big)
+    big_n = shapes[big[0]][0] * shapes[big[0]][1]
     dom = "quantize" if qms >= dms else "dequantize"
     ach = qgbs if dom == "quantize" else dgbs
     peak = peaks["hbm_gbs"]
@@ -400,8 +422,15 @@ def run_codec(args, q, torch, dev, peaks, peak_src):
                      "frac": round(ach / peak, 4), "traffic": measured_traffic("codec", dom),
                      "peak_source": f"{peak_src} hbm_gbs"},
         "kernels": {"quantize_gbs": round(qgbs, 1), "dequantize_gbs": round(dgbs, 1),
-                    "dq_encode_ms": round(kern["dq_encode"][0], 4),
-                    "quantize_ms": round(qms, 4), "dequantize_ms": round(dms, 4)},
+                    "quantize_ms": round(qms, 4), "dequantize_ms": round(dms, 4),
+                    "quantize_largest_tensor": {"shape": list(shapes[big[0]]), "us_median": round(big_us[len(big_us) // 2], 2),
+                                                "gbs": round(CODEC_BYTES_PER_WEIGHT * big_n / (big_us[len(big_us) // 2] * 1e-6) / 1e9, 1)},
+                    "per_kernel_ms_bracketed": {"quantize_blocks": round(kern["quantize"][0], 4),
+                                                "dq_encode": round(kern["dq_encode"][0], 4),
+                                                "dequantize": round(kern["dequantize"][0], 4)},
+                    "note": "quantize_ms / dequantize_ms: each API call bracketed by CUDA events on one stream "
+                            "(quantize = workspace reset + first-level pass + double quantization); "
+                            "per_kernel_ms_bracketed: every kernel bracketed separately (no overlap)"},
     }
 
 
@@ -568,6 +597,75 @@ def run_stack65b(args, q, torch, dev, peaks, peak_src, layers_n=None, tokens=204
     }
 
 
+def run_adamw7b(args, q, torch, dev, peaks, peak_src):
+    """Paged AdamW over every LoRA adapter of a 32-layer LLaMA-7B (r = 64: the
+    A and B of the seven linears of each layer, flattened), with the moments m
+    and v in unified memory.  Timed twice: with the state resident on the GPU
+    (the roofline: 30 bytes per parameter), and after evicting the state to
+    host memory, so that the update pages it back on demand."""
+    import synthetic
+    n = synthetic.LLAMA7B_LAYERS * sum(R * (N + K) for _, N, K in synthetic.LLAMA7B_LINEARS)
+    p = synthetic.normal((n,), 0.02, 90_001, torch.float32, dev)
+    p16 = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    g = synthetic.normal((n,), 1e-3, 90_002, torch.float32, dev)
+    m, v = q.PagedBuffer(n), q.PagedBuffer(n)
+    hp = dict(lr=2e-4, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0)
+    step_no = [0]
+
+    def step():
+        step_no[0] += 1
+        q.qlora_adamw_step(p, p16, g, m.tensor, v.tensor, hp["lr"], hp["beta1"], hp["beta2"], hp["eps"],
+                           hp["weight_decay"], step_no[0])
+
+    for b in (m, v):
+        q.qlora_paged_prefetch(b, to_device=True)
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    reps = max(args.steps, 10)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms_res = e0.elapsed_time(e1) / reps
+    bytes_per_step = 30 * n
+    gbs = bytes_per_step / (ms_res * 1e-3) / 1e9
+    # evicted state: every step first pushes m and v out to the host, then the
+    # update faults them back (timed: the update alone, and prefetch + update)
+    paged_ms, prefetch_ms = [], []
+    for mode in ("demand", "prefetch"):
+        for _ in range(3):
+            for b in (m, v):
+                q.qlora_paged_prefetch(b, to_device=False)
+            torch.cuda.synchronize()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record()
+            if mode == "prefetch":
+                for b in (m, v):
+                    q.qlora_paged_prefetch(b, to_device=True)
+            step()
+            a1.record()
+            torch.cuda.synchronize()
+            (paged_ms if mode == "demand" else prefetch_ms).append(a0.elapsed_time(a1))
+    q.qlora_check_device_error()
+    state_bytes = m.nbytes + v.nbytes
+    m.free()
+    v.free()
+    return {
+        "workload": f"adamw7b: AdamW over the LoRA adapters of 32 LLaMA-7B layers (r=64), {n} parameters, "
+                    "m and v in unified (paged) memory",
+        "value": round(gbs, 1), "unit": "GB/s", "ms_per_step_resident": round(ms_res, 4),
+        "params": n, "bytes_per_param": 30, "paged_state_bytes": state_bytes,
+        "ms_per_step_after_eviction": {"demand_paging": round(sorted(paged_ms)[1], 3),
+                                       "prefetch_then_update": round(sorted(prefetch_ms)[1], 3)},
+        "roofline": {"kernel": "adamw", "bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                     "peak_source": f"{peak_src} hbm_gbs"},
+    }
+
+
 # ---- CPU baselines (the oracle, as it stands) ---------------------------------------
 
 def _blas_threads():
@@ -705,6 +803,8 @@ def main():
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-decode", action="store_true")
     ap.add_argument("--skip-stack", action="store_true")
+    ap.add_argument("--skip-optim", action="store_true")
+    ap.add_argument("--optim-only", action="store_true", help="run only the paged AdamW object (profiling runs)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--linears", default="llama7b",
                     help="llama7b (the seven linears of one layer) or NxK for one linear (profiling runs)")
@@ -738,6 +838,11 @@ def main():
             import bit_nf4_quantized_16_b200 as q
             torch.cuda.set_device(local_rank)
             line = {"impl": "ours", "codec_shape": run_codec_shape(args, q, torch, torch.device("cuda", local_rank))}
+        elif args.optim_only:
+            import bit_nf4_quantized_16_b200 as q
+            torch.cuda.set_device(local_rank)
+            peaks, src = load_peaks()
+            line = {"impl": "ours", "adamw7b": run_adamw7b(args, q, torch, torch.device("cuda", local_rank), peaks, src)}
         elif args.codec_only:
             import bit_nf4_quantized_16_b200 as q
             torch.cuda.set_device(local_rank)

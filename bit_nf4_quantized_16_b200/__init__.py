@@ -34,16 +34,23 @@ EXPORTS = (
     "qlora_dequantize_nf4_dq", "qlora_linear_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd",
     "qlora_status_string", "qlora_check_device_error",
     "qlora_timing_enable", "qlora_timing_reset", "qlora_timing_read", "qlora_launch_count",
+    "qlora_debug_inject_stall",
+    "qlora_paged_alloc", "qlora_paged_free", "qlora_paged_prefetch", "qlora_adamw_step",
 )
 
 KERNEL_KINDS = ("quantize", "dq_encode", "dequantize", "fwd_fused", "bwd_fused", "lowrank", "wgrad",
-                "elementwise")
+                "elementwise", "optimizer")
 
 
 class QLoraError(RuntimeError):
     def __init__(self, status: int, where: str):
         super().__init__(f"{where}: {STATUS.get(status, status)}")
         self.status = status
+
+
+class qlora_adamw_hparams(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
+                ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float), ("step", ctypes.c_int64)]
 
 
 class qlora_nf4_weight(ctypes.Structure):
@@ -78,6 +85,11 @@ def _load():
         "qlora_timing_reset": (ctypes.c_int, []),
         "qlora_timing_read": (ctypes.c_int, [P, P]),
         "qlora_launch_count": (ctypes.c_int64, []),
+        "qlora_debug_inject_stall": (ctypes.c_int, [ctypes.c_int, ctypes.c_uint64]),
+        "qlora_paged_alloc": (ctypes.c_int, [S, ctypes.POINTER(ctypes.c_void_p)]),
+        "qlora_paged_free": (ctypes.c_int, [P]),
+        "qlora_paged_prefetch": (ctypes.c_int, [P, S, ctypes.c_int, P]),
+        "qlora_adamw_step": (ctypes.c_int, [P, P, P, P, P, I64, ctypes.POINTER(qlora_adamw_hparams), P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -222,3 +234,64 @@ def qlora_timing_read() -> dict:
 
 def qlora_launch_count() -> int:
     return lib.qlora_launch_count()
+
+
+def qlora_debug_inject_stall(kind: str, timeout_ns: int = 1_000_000):
+    """Failure-detection test hook: arms a one-shot stall in the next launch of
+    kernel family `kind` ("quantize", "fwd_fused" or "bwd_fused"; None disarms)."""
+    code = -1 if kind is None else KERNEL_KINDS.index(kind)
+    _check(lib.qlora_debug_inject_stall(code, timeout_ns), "qlora_debug_inject_stall")
+
+
+# ---- paged optimizer -----------------------------------------------------------------
+
+class PagedBuffer:
+    """A unified-memory allocation from qlora_paged_alloc, viewed as a float32
+    torch tensor on the current device (zero-filled).  Freed with free() or
+    when the object is collected."""
+
+    def __init__(self, numel: int, device="cuda"):
+        ptr = ctypes.c_void_p()
+        self.nbytes = 4 * numel
+        _check(lib.qlora_paged_alloc(self.nbytes, ctypes.byref(ptr)), "qlora_paged_alloc")
+        self.ptr = ptr.value
+        dev = torch.device(device)
+        if dev.index is None:
+            dev = torch.device("cuda", torch.cuda.current_device())
+        # a DLPack-free view: torch wraps the raw pointer without owning it
+        self.tensor = _wrap_device_pointer(self.ptr, numel, dev)
+
+    def free(self):
+        if self.ptr:
+            self.tensor = None
+            _check(lib.qlora_paged_free(ctypes.c_void_p(self.ptr)), "qlora_paged_free")
+            self.ptr = None
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
+
+
+def _wrap_device_pointer(ptr: int, numel: int, device):
+    class _Arr:
+        __cuda_array_interface__ = {"shape": (numel,), "typestr": "<f4", "data": (ptr, False), "version": 3,
+                                    "strides": None}
+    with torch.cuda.device(device):
+        return torch.as_tensor(_Arr(), device=device)
+
+
+def qlora_paged_prefetch(buf, to_device: bool, stream=None, nbytes=None):
+    ptr = buf.ptr if isinstance(buf, PagedBuffer) else buf.data_ptr()
+    n = nbytes if nbytes is not None else (buf.nbytes if isinstance(buf, PagedBuffer) else buf.numel() * buf.element_size())
+    _check(lib.qlora_paged_prefetch(ctypes.c_void_p(ptr), n, 1 if to_device else 0, _stream(stream)),
+           "qlora_paged_prefetch")
+
+
+def qlora_adamw_step(param, param_bf16, grad, exp_avg, exp_avg_sq, lr, beta1, beta2, eps, weight_decay, step,
+                     stream=None):
+    h = qlora_adamw_hparams(lr, beta1, beta2, eps, weight_decay, step)
+    _check(lib.qlora_adamw_step(_ptr(param), _ptr(param_bf16), _ptr(grad), _ptr(exp_avg), _ptr(exp_avg_sq),
+                                param.numel(), ctypes.byref(h), _stream(stream)),
+           "qlora_adamw_step")

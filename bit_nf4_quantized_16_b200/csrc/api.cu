@@ -17,7 +17,6 @@ namespace qlora {
 static __device__ int g_device_error = 0;
 
 namespace {
-constexpr int kMaxDevices = 64;
 int *g_error_ptr[kMaxDevices] = {};
 DeviceInfo g_info[kMaxDevices];
 bool g_info_ok[kMaxDevices] = {};
@@ -94,6 +93,7 @@ qlora_status check_weight(const qlora_nf4_weight *w)
 {
     if (!w) return QLORA_ERR_INVALID_ARG;
     if (w->rows <= 0 || w->cols <= 0 || w->cols % QLORA_BLOCK != 0) return QLORA_ERR_SHAPE;
+    if (w->rows > ((int64_t)1 << 40) / w->cols) return QLORA_ERR_SHAPE;   // rows * cols stays far from overflow
     if (!w->packed || !w->code2 || !w->c2 || !w->mean) return QLORA_ERR_INVALID_ARG;
     if (!aligned16(w->packed) || !aligned16(w->code2) || !aligned16(w->c2) || !aligned16(w->mean))
         return QLORA_ERR_ALIGNMENT;
@@ -229,6 +229,40 @@ extern "C" qlora_status qlora_check_device_error(void *stream)
     int zero = 0;
     if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return QLORA_ERR_CUDA;
     return v == kDevTimeout ? QLORA_ERR_TIMEOUT : QLORA_ERR_CUDA;
+}
+
+// ---- failure-detection test hook -----------------------------------------------------
+
+namespace qlora {
+namespace {
+std::mutex g_stall_mutex;
+int g_stall_kind = -1;
+uint64_t g_stall_ns = 0;
+}  // namespace
+
+bool take_stall_injection(int kind, uint64_t *timeout_ns)
+{
+    std::lock_guard<std::mutex> lock(g_stall_mutex);
+    if (g_stall_kind != kind) return false;
+    g_stall_kind = -1;
+    *timeout_ns = g_stall_ns;
+    return true;
+}
+}  // namespace qlora
+
+extern "C" qlora_status qlora_debug_inject_stall(int kind, uint64_t timeout_ns)
+{
+    std::lock_guard<std::mutex> lock(g_stall_mutex);
+    if (kind == -1) {
+        g_stall_kind = -1;
+        return QLORA_OK;
+    }
+    if (kind != QLORA_KERNEL_QUANTIZE && kind != QLORA_KERNEL_FWD_FUSED && kind != QLORA_KERNEL_BWD_FUSED)
+        return QLORA_ERR_INVALID_ARG;
+    if (timeout_ns < 1000ull || timeout_ns > 2000000000ull) return QLORA_ERR_INVALID_ARG;
+    g_stall_kind = kind;
+    g_stall_ns = timeout_ns;
+    return QLORA_OK;
 }
 
 // ---- kernel timing ------------------------------------------------------------------

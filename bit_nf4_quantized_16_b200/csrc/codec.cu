@@ -67,6 +67,7 @@ struct QuantParams {
     CUtensorMap tm_w;          // bf16 input as [nblocks][64], box 64 x 32, 128-byte swizzle
     int *err;                  // device error word (a bounded wait gave up)
     uint64_t timeout_ns;
+    int stall_inject;          // failure-detection test hook: warp 0 of CTA 0 skips its first copy (bf16)
 };
 
 // bf16 input: every warp streams its 32 blocks (4 KB) per step through a
@@ -95,8 +96,11 @@ constexpr uint32_t kQDynSmem = (kQThreads / 32) * kQStages * kQStageBytes + 1024
 // The kernel uses k = bits(n) with its low 20 bits flipped when n < 0: the
 // top 12 bits of k are the raw sign/exponent/3-bit index i of n, and the low
 // 20 bits of k equal those of the order-preserving key.  Entry i of the
-// table holds E(j(i)) - (i << 20), so that code = (table[i] + k) >> 20 with
-// no masking; every step except one logic op runs on the multiply-add pipe.
+// table holds E(j(i)) - (i << 20), so that t = table[i] + k holds the code in
+// bits 20..23 and zeros above.
+// The steps are plain shifts and logic ops that the compiler spreads over
+// the integer and multiply-add pipes (forcing them onto the multiply-add
+// pipe, through multiply-high, saturated it and measured 14% slower).
 // Every CTA builds the table once: thread t fills the entries of ordered
 // intervals j = 16t..16t+15, walking the sorted midpoint keys once.
 __device__ __forceinline__ void build_code_lut(uint32_t *lut, const uint32_t *mkey_smem)
@@ -116,25 +120,26 @@ __device__ __forceinline__ void build_code_lut(uint32_t *lut, const uint32_t *mk
     }
 }
 
-// Code of n shifted to nibble position 4*I and added to acc.
+// Code of n inserted at nibble position 4*I of acc (whose nibble I is zero).
 template <int I>
 __device__ __forceinline__ uint32_t add_code(const uint32_t *lut, float n, uint32_t acc)
 {
     const uint32_t b = __float_as_uint(n);
-    const uint32_t s = (uint32_t)__mulhi((int)b, 2);       // 0 or all ones: the sign mask
+    const uint32_t s = (uint32_t)((int32_t)b >> 31);        // 0 or all ones: the sign mask
     const uint32_t k = b ^ (s & 0xFFFFFu);                  // low 20 bits flipped for n < 0
-    const uint32_t e = lut[__umulhi(k, 1u << 12)];          // k >> 20
-    const uint32_t code = __umulhi(e + k, 1u << 12);        // (e + k) >> 20
-    return acc + code * (1u << (4 * I));
+    const uint32_t t = lut[k >> 20] + k;                    // code in bits 20..23, zero above
+    const uint32_t part = (4 * I <= 20) ? (t >> (20 - 4 * I)) : (t << (4 * I - 20));
+    return acc | (part & (0xFu << (4 * I)));
 }
 
-// Absolute maximum of 8 bf16 values held as 4 packed pairs: the magnitudes'
-// bit patterns compare like the values, so a 16-bit unsigned SIMD max does it.
-__device__ __forceinline__ uint32_t absmax8_bf16(uint4 v, uint32_t m)
+// Magnitude maximum of two bf16 pairs, lane by lane (max.xorsign.abs: the
+// result's magnitude is max(|a|, |b|); its sign bit is meaningless and masked
+// off by the caller).
+__device__ __forceinline__ uint32_t maxabs_bf16x2(uint32_t a, uint32_t b)
 {
-    const uint32_t a = __vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu);
-    const uint32_t b = __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu);
-    return __vmaxu2(m, __vmaxu2(a, b));
+    uint32_t d;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
 }
 
 // 8 codes of 8 consecutive values (already multiplied by r), element 0 in bits 0-3.
@@ -177,10 +182,16 @@ __global__ void __maxnreg__(64) quantize_blocks_kernel(const __grid_constant__ Q
     uint8_t *ring = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(q_dyn) + 1023) & ~uintptr_t(1023)) +
                     warp * kQStages * kQStageBytes;
     __shared__ uint64_t s_bar[kQThreads / 32][kQStages];
+    // launched with programmatic serialization: the input may come from the
+    // kernel before this one; the double-quantization kernel after it may
+    // become resident now and wait for this grid's completion
+    sm100::pdl_wait();
+    sm100::pdl_trigger();
     if (!kF32In && lane == 0) {
         for (int st = 0; st < kQStages; st++) sm100::mbar_init(&s_bar[warp][st], 1);
         sm100::fence_barrier_init();
-        if (first < p.nblocks) {
+        const bool skip = p.stall_inject && blockIdx.x == 0 && warp == 0;
+        if (first < p.nblocks && !skip) {
             sm100::mbar_arrive_expect_tx(&s_bar[warp][0], kQStageBytes);
             sm100::tma_load_2d(ring, &p.tm_w, &s_bar[warp][0], 0, (int32_t)first);
         }
@@ -223,9 +234,16 @@ __global__ void __maxnreg__(64) quantize_blocks_kernel(const __grid_constant__ Q
             uint4 v[8];
 #pragma unroll
             for (int i = 0; i < 8; i++) v[i] = *reinterpret_cast<const uint4 *>(row + ((i ^ (lane & 7)) << 4));
-            uint32_t m = 0;
+            // block absmax: magnitudes of the 64 values in two lanes of bf16
+            // pairs, then the larger half; magnitude bit patterns compare like
+            // the values
+            uint32_t m0 = maxabs_bf16x2(v[0].x, v[0].y), m1 = maxabs_bf16x2(v[0].z, v[0].w);
 #pragma unroll
-            for (int i = 0; i < 8; i++) m = absmax8_bf16(v[i], m);
+            for (int i = 1; i < 8; i++) {
+                m0 = maxabs_bf16x2(m0, maxabs_bf16x2(v[i].x, v[i].y));
+                m1 = maxabs_bf16x2(m1, maxabs_bf16x2(v[i].z, v[i].w));
+            }
+            const uint32_t m = maxabs_bf16x2(m0, m1) & 0x7FFF7FFFu;
             cv = __uint_as_float(__vmaxu2(m, m >> 16) << 16);   // larger half, as binary32
             // zero block (absmax below the smallest normal): r = 0 sends every
             // element to n = +-0, whose code is the codebook's zero
@@ -336,6 +354,9 @@ struct DqParams {
 __global__ void __launch_bounds__(kThreads) dq_encode_kernel(DqParams p)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // resident while the quantizer runs; c1 and the mean are read after it completed
+    sm100::pdl_wait();
+    sm100::pdl_trigger();
     const float mu = *p.mean;
     for (int64_t g = (int64_t)blockIdx.x * (kThreads / 32) + warp; g < p.ngroups;
          g += (int64_t)gridDim.x * (kThreads / 32)) {
@@ -389,6 +410,8 @@ __global__ void __launch_bounds__(kThreads) dequantize_kernel(DeqParams p)
         for (int i = 0; i < 16; i++) lut[i] = p.q[i];   // static indices keep p in the parameter bank
     }
     __syncthreads();
+    sm100::pdl_wait();   // the quantized weight may come from the kernel before this one
+    sm100::pdl_trigger();
     const float mu = *p.mean;
     const int64_t stride = (int64_t)gridDim.x * kThreads;
     for (int64_t w0 = (int64_t)blockIdx.x * kThreads + threadIdx.x; w0 < p.nwords; w0 += stride * kDeqUnroll) {
@@ -455,15 +478,17 @@ qlora_status prepare_quantize(QuantParams &qp, const void *W, qlora_dtype w_dtyp
     qp.err = device_error_word();
     if (!qp.err) return QLORA_ERR_CUDA;
     qp.timeout_ns = 2000000000ull;
+    qp.stall_inject = 0;
     if (w_dtype == QLORA_BF16) {
         QLORA_TRY(make_map(&qp.tm_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, 64, (uint64_t)(numel / 64), 128, 64, 32,
                            CU_TENSOR_MAP_SWIZZLE_128B));
-        static bool attr_done[64] = {};
-        if (dev.device >= 0 && dev.device < 64 && !attr_done[dev.device]) {
+        static PerDeviceOnce attr;
+        QLORA_TRY(attr.run(dev.device, []() -> qlora_status {
             QLORA_CUDA_TRY(cudaFuncSetAttribute(quantize_blocks_kernel<false>,
                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kQDynSmem));
-            attr_done[dev.device] = true;
-        }
+            return QLORA_OK;
+        }));
+        qp.stall_inject = take_stall_injection(QLORA_KERNEL_QUANTIZE, &qp.timeout_ns) ? 1 : 0;
     }
     return QLORA_OK;
 }
@@ -526,9 +551,9 @@ extern "C" qlora_status qlora_quantize_nf4_dq(const void *W, qlora_dtype w_dtype
     {
         LaunchScope ls(QLORA_KERNEL_QUANTIZE, s);
         if (w_dtype == QLORA_FP32)
-            quantize_blocks_kernel<true><<<grid, kQThreads, 0, s>>>(qp);
+            QLORA_CUDA_TRY(launch_pdl(quantize_blocks_kernel<true>, dim3(grid), dim3(kQThreads), 0, s, qp));
         else
-            quantize_blocks_kernel<false><<<grid, kQThreads, kQDynSmem, s>>>(qp);
+            QLORA_CUDA_TRY(launch_pdl(quantize_blocks_kernel<false>, dim3(grid), dim3(kQThreads), kQDynSmem, s, qp));
     }
     QLORA_TRY(launch_status());
 
@@ -541,7 +566,8 @@ extern "C" qlora_status qlora_quantize_nf4_dq(const void *W, qlora_dtype w_dtype
     dp.ngroups = (nblocks + QLORA_GROUP - 1) / QLORA_GROUP;
     {
         LaunchScope ls(QLORA_KERNEL_DQ_ENCODE, s);
-        dq_encode_kernel<<<grid_for(dp.ngroups, kThreads / 32, dev.sms * 8), kThreads, 0, s>>>(dp);
+        QLORA_CUDA_TRY(launch_pdl(dq_encode_kernel, dim3(grid_for(dp.ngroups, kThreads / 32, dev.sms * 8)),
+                                  dim3(kThreads), 0, s, dp));
     }
     return launch_status();
 }
@@ -564,7 +590,8 @@ extern "C" qlora_status qlora_dequantize_nf4_dq(const qlora_nf4_weight *w, void 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     {
         LaunchScope ls(QLORA_KERNEL_DEQUANTIZE, s);
-        dequantize_kernel<<<grid_for(p.nwords, kThreads * kDeqUnroll, dev.sms * 8), kThreads, 0, s>>>(p);
+        QLORA_CUDA_TRY(launch_pdl(dequantize_kernel, dim3(grid_for(p.nwords, kThreads * kDeqUnroll, dev.sms * 8)),
+                                  dim3(kThreads), 0, s, p));
     }
     return launch_status();
 }
@@ -591,7 +618,7 @@ constexpr size_t kStaticScratchBytes = kStaticAccBytes + (size_t)QLORA_NOALLOC_M
 // [acc 256 u64][ticket][pad][c1: QLORA_NOALLOC_MAX_BLOCKS floats], about 4 MiB per device
 static __device__ __align__(256) unsigned char g_quant_scratch[kStaticScratchBytes];
 
-constexpr int kMaxScratchDevices = 64;
+constexpr int kMaxScratchDevices = kMaxDevices;
 unsigned char *g_scratch_ptr[kMaxScratchDevices] = {};
 std::mutex g_scratch_mutex;
 
@@ -620,9 +647,11 @@ extern "C" qlora_status qlora_quantize_nf4_dq_noalloc(const void *W, qlora_dtype
     if (w_dtype != QLORA_BF16 && w_dtype != QLORA_FP32) return QLORA_ERR_INVALID_ARG;
     QLORA_TRY(check_weight(out));
     if (!aligned16(W)) return QLORA_ERR_ALIGNMENT;
+    // larger than the fixed scratch (compared before multiplying)
+    if (out->rows > (int64_t)QLORA_NOALLOC_MAX_BLOCKS * QLORA_BLOCK / out->cols) return QLORA_ERR_SHAPE;
     const int64_t numel = out->rows * out->cols;
     const int64_t nblocks = numel / QLORA_BLOCK;
-    if (nblocks > QLORA_NOALLOC_MAX_BLOCKS) return QLORA_ERR_SHAPE;   // larger than the fixed scratch
+    if (nblocks > QLORA_NOALLOC_MAX_BLOCKS) return QLORA_ERR_SHAPE;
     uint32_t mkey[15];
     QLORA_TRY(midpoint_keys(out->codebook, mkey));
     DeviceInfo dev;
@@ -649,9 +678,9 @@ extern "C" qlora_status qlora_quantize_nf4_dq_noalloc(const void *W, qlora_dtype
     {
         LaunchScope ls(QLORA_KERNEL_QUANTIZE, s);
         if (w_dtype == QLORA_FP32)
-            quantize_blocks_kernel<true><<<grid, kQThreads, 0, s>>>(qp);
+            QLORA_CUDA_TRY(launch_pdl(quantize_blocks_kernel<true>, dim3(grid), dim3(kQThreads), 0, s, qp));
         else
-            quantize_blocks_kernel<false><<<grid, kQThreads, kQDynSmem, s>>>(qp);
+            QLORA_CUDA_TRY(launch_pdl(quantize_blocks_kernel<false>, dim3(grid), dim3(kQThreads), kQDynSmem, s, qp));
     }
     QLORA_TRY(launch_status());
 
@@ -664,7 +693,8 @@ extern "C" qlora_status qlora_quantize_nf4_dq_noalloc(const void *W, qlora_dtype
     dp.ngroups = (nblocks + QLORA_GROUP - 1) / QLORA_GROUP;
     {
         LaunchScope ls(QLORA_KERNEL_DQ_ENCODE, s);
-        dq_encode_kernel<<<grid_for(dp.ngroups, kThreads / 32, dev.sms * 8), kThreads, 0, s>>>(dp);
+        QLORA_CUDA_TRY(launch_pdl(dq_encode_kernel, dim3(grid_for(dp.ngroups, kThreads / 32, dev.sms * 8)),
+                                  dim3(kThreads), 0, s, dp));
     }
     return launch_status();
 }

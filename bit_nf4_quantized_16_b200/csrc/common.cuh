@@ -5,11 +5,15 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
 #include <utility>
 
 #include "../../include/qlora.h"
 
 namespace qlora {
+
+constexpr int kMaxDevices = 64;
 
 // Kernel-side error codes written into the device error word.
 enum DeviceError : int {
@@ -75,6 +79,34 @@ qlora_status make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, 
 
 // Checks shared by every entry point that takes a quantized weight.
 qlora_status check_weight(const qlora_nf4_weight *w);
+
+// Per-device one-time set-up (kernel attributes, occupancy queries): the first
+// successful run of `fn` on a device happens under a lock; later calls on that
+// device return at once.  The results of `fn` are published by the release
+// store of the done flag.
+class PerDeviceOnce {
+  public:
+    template <typename F>
+    qlora_status run(int device, F &&fn)
+    {
+        if (device < 0 || device >= kMaxDevices) return QLORA_ERR_CUDA;
+        if (done_[device].load(std::memory_order_acquire)) return QLORA_OK;
+        std::lock_guard<std::mutex> lock(mu_);
+        if (done_[device].load(std::memory_order_relaxed)) return QLORA_OK;
+        const qlora_status st = fn();
+        if (st == QLORA_OK) done_[device].store(true, std::memory_order_release);
+        return st;
+    }
+
+  private:
+    std::mutex mu_;
+    std::atomic<bool> done_[kMaxDevices] = {};
+};
+
+// Failure-detection test hook (qlora_debug_inject_stall): true, once, for the
+// first launch of kernel family `kind` after the hook was armed; *timeout_ns
+// then receives the armed wait limit.
+bool take_stall_injection(int kind, uint64_t *timeout_ns);
 
 // Brackets one kernel launch for qlora_timing_read (events only while timing
 // is enabled) and counts it for qlora_launch_count.

@@ -75,7 +75,10 @@ struct GemmParams {
     int m_total, n_total;
     int64_t split_stride;  // elements between split planes (partial products)
     int *err;            // device error word
-    uint64_t timeout_ns;
+    uint64_t timeout_ns; // limit of every pipeline wait
+    uint64_t drain_ns;   // limit of the waits for copies and MMAs already in flight after an abort
+    int stall_inject;    // failure-detection test hook: the first dequantization warp of CTA 0
+                         // (of cluster 0) skips its first arrival, so the MMA's wait runs out
 };
 
 template <int BN, int kBMode, int MT>
@@ -198,7 +201,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode, MT>::kThreads, 1)
         auto drain_loads = [&]() {
             // after an abort: wait (bounded) for the loads still in flight
             for (uint32_t j = it > (uint32_t)S ? it - S : 0; j < it; j++)
-                mbar_wait_bounded(&full_a[j % S], (j / S) & 1, p.timeout_ns);
+                mbar_wait_bounded(&full_a[j % S], (j / S) & 1, p.drain_ns);
         };
         for (int t = blockIdx.x; t < num_tiles && !*vabort; t += gridDim.x) {
             int mt, nt, sp, kb0, nmain;
@@ -296,7 +299,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode, MT>::kThreads, 1)
         if (*vabort) {
             // after an abort: wait (bounded) until the MMAs already issued finish
             tc_commit(drain);
-            mbar_wait_bounded(drain, 0, p.timeout_ns);
+            mbar_wait_bounded(drain, 0, p.drain_ns);
         }
     } else if (warp >= 4 && warp < 8) {
         // ---------------- epilogue ----------------
@@ -458,7 +461,8 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode, MT>::kThreads, 1)
                     fence_proxy_async_smem();
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&full_b[s]);
+                const bool skip = p.stall_inject && blockIdx.x == 0 && warp == 8 && it == 0;
+                if (lane == 0 && !skip) mbar_arrive(&full_b[s]);
             }
             if (!ok) break;
         }

@@ -187,8 +187,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<kBMode, MT>:
             // after an abort: wait (bounded) for the loads still in flight; the
             // leader's full_a also counts the other CTA's bytes
             for (uint32_t j = it > (uint32_t)S ? it - S : 0; j < it; j++) {
-                mbar_wait_bounded(&pk_full[j % S], (j / S) & 1, p.timeout_ns);
-                if (leader) mbar_wait_bounded(&full_a[j % S], (j / S) & 1, p.timeout_ns);
+                mbar_wait_bounded(&pk_full[j % S], (j / S) & 1, p.drain_ns);
+                if (leader) mbar_wait_bounded(&full_a[j % S], (j / S) & 1, p.drain_ns);
             }
         }
     } else if (warp == 1 && lane == 0 && leader) {
@@ -232,7 +232,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<kBMode, MT>:
         }
         if (*vabort) {
             tc_commit_pair(drain, 0x1);
-            mbar_wait_bounded(drain, 0, p.timeout_ns);
+            mbar_wait_bounded(drain, 0, p.drain_ns);
         }
     } else if ((warp >= 4 && warp < 8) || warp >= 16) {
         // ---------------- epilogue (both CTAs) ----------------
@@ -401,7 +401,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<kBMode, MT>:
                     fence_proxy_async_smem();
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(full_b_leader0 + (uint32_t)s * 8u);
+                const bool skip = p.stall_inject && blockIdx.x == 0 && warp == 8 && it == 0;
+                if (lane == 0 && !skip) mbar_arrive_cluster(full_b_leader0 + (uint32_t)s * 8u);
             }
             if (!ok) break;
         }

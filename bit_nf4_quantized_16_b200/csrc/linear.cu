@@ -45,19 +45,27 @@ qlora_status map_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint64_t
 
 // ---- GEMM launch ------------------------------------------------------------------
 
+// Wait limits, and the failure-detection test hook when it is armed for `kind`.
+void set_limits(GemmParams &p, int kind)
+{
+    p.timeout_ns = kTimeoutNs;
+    p.drain_ns = kTimeoutNs;
+    p.stall_inject = take_stall_injection(kind, &p.timeout_ns) ? 1 : 0;
+}
+
 template <int BN, int kBMode, int kEpi, int MT = 1>
 qlora_status launch_gemm(GemmParams &p, const DeviceInfo &dev, cudaStream_t s, int kind)
 {
     using Cfg = GemmCfg<BN, kBMode, MT>;
-    static bool attr_done[64] = {};
+    static PerDeviceOnce attr;
     auto kern = qgemm_kernel<BN, kBMode, kEpi, MT>;
-    if (!attr_done[dev.device]) {
+    QLORA_TRY(attr.run(dev.device, [&]() -> qlora_status {
         QLORA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes));
-        attr_done[dev.device] = true;
-    }
+        return QLORA_OK;
+    }));
     p.err = device_error_word();
     if (!p.err) return QLORA_ERR_CUDA;
-    p.timeout_ns = kTimeoutNs;
+    set_limits(p, kind);
     const int tiles = p.m_tiles * p.n_tiles * p.splits;
     const int grid = tiles < dev.sms ? tiles : dev.sms;
     {
@@ -74,9 +82,10 @@ template <int kBMode, int kEpi, int MT>
 qlora_status launch_gemm_pair(GemmParams &p, const DeviceInfo &dev, cudaStream_t s, int kind)
 {
     using Cfg = PairCfg<kBMode, MT>;
-    static int max_clusters[64] = {};
+    static PerDeviceOnce setup;
+    static int max_clusters[kMaxDevices] = {};
     auto kern = qgemm_pair_kernel<kBMode, kEpi, MT>;
-    if (!max_clusters[dev.device]) {
+    QLORA_TRY(setup.run(dev.device, [&]() -> qlora_status {
         QLORA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes));
         cudaLaunchConfig_t cfg{};
         cfg.gridDim = dim3(2 * (dev.sms / 2));
@@ -86,10 +95,11 @@ qlora_status launch_gemm_pair(GemmParams &p, const DeviceInfo &dev, cudaStream_t
         QLORA_CUDA_TRY(cudaOccupancyMaxActiveClusters(&n, kern, &cfg));
         if (n < 1) return QLORA_ERR_CUDA;
         max_clusters[dev.device] = n;
-    }
+        return QLORA_OK;
+    }));
     p.err = device_error_word();
     if (!p.err) return QLORA_ERR_CUDA;
-    p.timeout_ns = kTimeoutNs;
+    set_limits(p, kind);
     p.splits = 1;
     const int tiles = p.m_tiles * p.n_tiles;
     const int clusters = tiles < max_clusters[dev.device] ? tiles : max_clusters[dev.device];

@@ -20,7 +20,9 @@
  * Conventions common to every entry point
  *   - Pointers named "device" must point to memory of the current CUDA device;
  *     the caller allocates and frees every buffer.  The library never
- *     allocates device memory and never frees what it is given.
+ *     allocates device memory and never frees what it is given, except
+ *     through the paged-memory helpers qlora_paged_alloc / qlora_paged_free,
+ *     which exist to hand out unified memory for optimizer states.
  *   - Every device pointer must be 16-byte aligned (tensor-memory-access
  *     copies require it); QLORA_ERR_ALIGNMENT otherwise.
  *   - All work is enqueued on `stream` (a cudaStream_t; NULL = the legacy
@@ -35,6 +37,12 @@
  *     device error word, read back by qlora_check_device_error().
  *   - The library requires a compute capability 10.0 device (B200);
  *     QLORA_ERR_UNSUPPORTED otherwise.  There is no CPU fallback.
+ *   - Per-device state is set up on first use and kept for the life of the
+ *     process: device properties, kernel attributes, and the device addresses
+ *     of the library's own __device__ variables (the error word, the fixed
+ *     scratch of qlora_quantize_nf4_dq_noalloc).  cudaDeviceReset() destroys
+ *     what that state refers to: do not use the library on a device again
+ *     after resetting it in the same process.
  */
 #ifndef QLORA_H
 #define QLORA_H
@@ -257,6 +265,64 @@ QLORA_API qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *X
                               const float *H_saved, void *dX, qlora_dtype dx_dtype, float *dA,
                               float *dB, void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * Paged optimizer ("QLoRA: Efficient Finetuning of Quantized LLMs",
+ * Introduction item (3) and "Method", opening paragraph; mbrenndoerfer.com
+ * essay, "Paged Optimizers"): the optimizer states are allocated in NVIDIA
+ * unified memory, so the driver evicts them to CPU RAM when the GPU runs out
+ * of memory and pages them back in when the update step touches them.
+ *
+ * qlora_paged_alloc -- `bytes` of unified (managed) memory, zero-filled on the
+ * host (the pages start in CPU memory).  The one place where the library
+ * allocates: paging is the point of these buffers.  The caller owns the
+ * allocation and releases it with qlora_paged_free (a synchronizing call).
+ * Errors: INVALID_ARG (null ptr, bytes == 0), CUDA, UNSUPPORTED.
+ */
+QLORA_API qlora_status qlora_paged_alloc(size_t bytes, void **ptr);
+QLORA_API qlora_status qlora_paged_free(void *ptr);
+
+/*
+ * qlora_paged_prefetch -- migrate [ptr, ptr + bytes) of a paged allocation to
+ * the current device (to_device = 1) or to host memory (to_device = 0),
+ * asynchronously on `stream`.  Without it, pages move on demand when a kernel
+ * or the host touches them.
+ * Errors: INVALID_ARG, CUDA, UNSUPPORTED.
+ */
+QLORA_API qlora_status qlora_paged_prefetch(const void *ptr, size_t bytes, int to_device, void *stream);
+
+/* Hyperparameters of one AdamW step; `step` counts from 1. */
+typedef struct {
+    float lr;
+    float beta1;
+    float beta2;
+    float eps;
+    float weight_decay;
+    int64_t step;
+} qlora_adamw_hparams;
+
+/*
+ * qlora_adamw_step -- one AdamW update (Adam with decoupled weight decay) of
+ * n parameters, element by element, in float32:
+ *     p <- p * (1 - lr * wd)
+ *     m <- beta1 m + (1 - beta1) g
+ *     v <- beta2 v + (1 - beta2) g^2
+ *     p <- p - (lr / (1 - beta1^t)) * m / (sqrt(v) / sqrt(1 - beta2^t) + eps)
+ * The pages name paged optimizers and optimizer states but no optimizer; AdamW
+ * is the reading used here.
+ *   param       device float [n], updated in place (the master copy).
+ *   param_bf16  device bf16 [n] or NULL: receives bf16(p) after the update,
+ *               e.g. a flat buffer holding the adapters A and B that the
+ *               linear layer reads; 8-byte aligned.
+ *   grad        device float [n] (dA and dB of qlora_linear_bwd, flattened).
+ *   exp_avg, exp_avg_sq  float [n], the moments m and v: device memory or a
+ *               qlora_paged_alloc buffer (zero before the first step).
+ *   h           host struct, lr >= 0, 0 <= beta < 1, eps > 0, wd >= 0, step >= 1.
+ * Errors: INVALID_ARG, ALIGNMENT (param, grad, m, v not 16-byte aligned), CUDA,
+ * UNSUPPORTED.
+ */
+QLORA_API qlora_status qlora_adamw_step(float *param, void *param_bf16, const float *grad, float *exp_avg,
+                                        float *exp_avg_sq, int64_t n, const qlora_adamw_hparams *h, void *stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 QLORA_API const char *qlora_status_string(qlora_status status);
 
@@ -288,12 +354,37 @@ enum {
     QLORA_KERNEL_LOWRANK = 5,     /* H = X A^T and G = dY B products     */
     QLORA_KERNEL_WGRAD = 6,       /* dA and dB products                  */
     QLORA_KERNEL_ELEMENTWISE = 7, /* split-sum / hi-lo finalize kernels  */
-    QLORA_NUM_KERNELS = 8
+    QLORA_KERNEL_OPTIMIZER = 8,   /* AdamW update of the adapters        */
+    QLORA_NUM_KERNELS = 9
 };
 QLORA_API qlora_status qlora_timing_enable(int enable);
 QLORA_API qlora_status qlora_timing_reset(void);
 QLORA_API qlora_status qlora_timing_read(double ms[QLORA_NUM_KERNELS], int64_t launches[QLORA_NUM_KERNELS]);
 QLORA_API int64_t qlora_launch_count(void);
+
+/*
+ * qlora_debug_inject_stall -- failure-detection test hook (the pages describe
+ * no such facility; it exists so that tests can drive the bounded-wait path
+ * without faulting the GPU).  Arms a one-shot fault in the next launch of
+ * one kernel family in this process:
+ *   kind  QLORA_KERNEL_QUANTIZE (quantizer, bf16 input: the first warp of the
+ *         first CTA does not issue its first tensor copy),
+ *         QLORA_KERNEL_FWD_FUSED or QLORA_KERNEL_BWD_FUSED (the tcgen05 fused
+ *         dequant-GEMMs, which run from 17 tokens on: the first
+ *         dequantization warp of the first CTA skips its first arrival on the
+ *         stage barrier the MMA issuer waits on),
+ *         or -1 to disarm.
+ *   timeout_ns  wait limit of that one launch, 1e3 .. 2e9 (the normal limit
+ *         is 2 s).
+ * In the armed launch the consumer's wait runs out after timeout_ns; the
+ * kernel records QLORA_ERR_TIMEOUT in the device error word, tells its other
+ * roles to stop, waits (bounded by the normal 2 s) for the copies and MMAs it
+ * already issued, frees its tensor memory and returns.  The outputs of that
+ * one call are unspecified; qlora_check_device_error() reports the timeout;
+ * later calls are unaffected.  Host-only, no CUDA call.
+ * Errors: QLORA_ERR_INVALID_ARG (unknown kind, limit out of range).
+ */
+QLORA_API qlora_status qlora_debug_inject_stall(int kind, uint64_t timeout_ns);
 
 #ifdef __cplusplus
 }

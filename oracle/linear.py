@@ -56,6 +56,14 @@ def backward_dx_rows(Wd, A, B, s: float, dY, rows) -> np.ndarray:
     return dYr @ Wd + s * ((dYr @ B) @ A)
 
 
+def backward_weight_grads(X, A, B, s: float, dY):
+    """(dA, dB) alone, the same products as backward() without the input
+    gradient (whose dY W' term dominates the cost at LLaMA sizes)."""
+    X, A, B, dY = map(_f64, (X, A, B, dY))
+    G = dY @ B
+    return s * (G.T @ X), s * (dY.T @ (X @ A.T))
+
+
 def rel_frobenius(got, ref) -> float:
     got, ref = _f64(got), _f64(ref)
     den = np.linalg.norm(ref)

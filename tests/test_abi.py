@@ -194,3 +194,30 @@ def test_validation_of_the_linear_layer(lib):
     assert b(dxdt=9) == 1
     assert b(dY=fake + 2) == 3 and b(dX=fake + 4) == 3 and b(dA=fake + 8) == 3 and b(H=fake + 4) == 3
     assert b(r=200) == 2
+
+
+def test_stall_hook_validation(lib):
+    """The failure-detection test hook only arms the kernel families that have
+    pipeline waits, with a limit in range; it makes no CUDA call."""
+    f = lib.qlora_debug_inject_stall
+    f.argtypes = [ctypes.c_int, ctypes.c_uint64]
+    assert f(5, 1_000_000) == 1             # low-rank products: not a hook site
+    assert f(0, 10) == 1                    # limit below 1 us
+    assert f(3, 3_000_000_000) == 1         # limit above 2 s
+    assert f(-1, 0) == 0                    # disarm
+    assert f(0, 1_000_000) == 0 and f(-1, 0) == 0
+
+
+@pytest.mark.skipif(not _no_gpu(), reason="host-only validation test with placeholder pointers")
+def test_shape_overflow_is_rejected(lib):
+    """rows * cols that would overflow 64-bit arithmetic is rejected before use."""
+    q = ocb.nf4_codebook()
+    fake = 0x10000
+    na = lib.qlora_quantize_nf4_dq_noalloc
+    na.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(Weight), ctypes.c_void_p]
+    huge = Weight(1 << 40, 1 << 30, fake, fake, fake, fake, (ctypes.c_float * 16)(*q))
+    assert na(fake, 0, ctypes.byref(huge), None) == 2
+    f = lib.qlora_quantize_nf4_dq
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(Weight), ctypes.c_void_p, ctypes.c_size_t,
+                  ctypes.c_void_p]
+    assert f(fake, 0, ctypes.byref(huge), fake, 1 << 62, None) == 2

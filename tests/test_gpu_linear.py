@@ -134,6 +134,24 @@ def test_ragged_shapes(q, M, N, K, r):
     full_check(q, synthetic.linear_case(M, N, K, r, alpha=16.0, seed=M + N + K + r))
 
 
+@pytest.mark.parametrize("M,N,K,r", [
+    (300, 320, 448, 16),     # CTA pairs, ragged in every dimension
+    (600, 264, 576, 64),     # two pair tiles of tokens, N not a multiple of the 256-wide pair tile
+    (513, 512, 256, 128),    # one token into the second pair tile, largest rank
+])
+def test_ragged_shapes_bf16_outputs(q, M, N, K, r):
+    """bf16 Y and dX through the CTA-pair kernels' TMA-store epilogue (the
+    tensor map clips the ragged edges)."""
+    full_check(q, synthetic.linear_case(M, N, K, r, alpha=16.0, seed=2 * M + N + K + r), ydt=torch.bfloat16)
+
+
+@pytest.mark.parametrize("M", [17, 200, 256])
+def test_single_cta_fused_bf16_outputs(q, M):
+    """17..256 tokens: the single-CTA fused forward and input-gradient GEMMs
+    with bf16 outputs (one 256-token tile)."""
+    full_check(q, synthetic.linear_case(M, 384, 512, 64, alpha=16.0, seed=300 + M), ydt=torch.bfloat16)
+
+
 @pytest.mark.parametrize("M", [16, 200, 512])
 def test_int4_codebook(q, M):
     """The Int4 table through the same kernels: the decode forward (16
@@ -198,10 +216,14 @@ def test_deterministic(q):
         assert torch.equal(a, b)
 
 
-def test_llama7b_shapes_sampled(q):
+@pytest.mark.parametrize("ydt", [torch.bfloat16, torch.float32])
+def test_llama7b_shapes_sampled(q, ydt):
     """7B-shaped linears at 4096 tokens: Y and dX on sampled rows, dA and dB in
-    full (they contract over every token)."""
+    full (they contract over every token).  With bf16 outputs and the saved H
+    this is exactly the call sequence the benchmark times (the CTA-pair
+    kernels with the TMA-store epilogue)."""
     rng = np.random.default_rng(0)
+    bf = ydt == torch.bfloat16
     for i, (name, N, K) in enumerate([("q", 4096, 4096), ("gate", 11008, 4096), ("down", 4096, 11008)]):
         case = synthetic.linear_case(4096, N, K, 64, alpha=16.0, seed=100 + i, device="cpu")
         run = Runner(q, case)
@@ -209,18 +231,19 @@ def test_llama7b_shapes_sampled(q):
         X, A, B, dY = (np64(case[k]) for k in ("X", "A", "B", "dY"))
         s = case["scale"]
         rows = np.sort(rng.choice(4096, 48, replace=False))
-        Y, _ = run.fwd()
-        assert_close(np64(Y)[rows], olin.forward_rows(X, Wd, A, B, s, rows), what=f"{name} Y")
-        dX, dA, dB = run.bwd()
-        assert_close(np64(dX)[rows], olin.backward_dx_rows(Wd, A, B, s, dY, rows), what=f"{name} dX")
-        G = dY @ B
-        assert_close(np64(dA), s * (G.T @ X), what=f"{name} dA")
-        assert_close(np64(dB), s * (dY.T @ (X @ A.T)), what=f"{name} dB")
+        Y, H = run.fwd(ydt, save_h=bf)
+        assert_close(np64(Y)[rows], olin.forward_rows(X, Wd, A, B, s, rows), bf16_out=bf, what=f"{name} Y")
+        dX, dA, dB = run.bwd(ydt, H=H)
+        assert_close(np64(dX)[rows], olin.backward_dx_rows(Wd, A, B, s, dY, rows), bf16_out=bf, what=f"{name} dX")
+        rdA, rdB = olin.backward_weight_grads(X, A, B, s, dY)
+        assert_close(np64(dA), rdA, what=f"{name} dA")
+        assert_close(np64(dB), rdB, what=f"{name} dB")
 
 
 def test_llama65b_shapes_sampled(q):
-    """65B-shaped linears at 2048 tokens (the stack configuration): Y and dX on
-    sampled rows, dA and dB in full."""
+    """65B-shaped linears at 2048 tokens with bf16 Y and dX and the saved H, as
+    the 80-layer stack benchmark calls them: Y and dX on sampled rows, dA and
+    dB in full."""
     rng = np.random.default_rng(1)
     for i, (name, N, K) in enumerate([("q", 8192, 8192), ("gate", 22016, 8192), ("down", 8192, 22016)]):
         case = synthetic.linear_case(2048, N, K, 64, alpha=16.0, seed=500 + i, device="cpu")
@@ -229,13 +252,13 @@ def test_llama65b_shapes_sampled(q):
         X, A, B, dY = (np64(case[k]) for k in ("X", "A", "B", "dY"))
         s = case["scale"]
         rows = np.sort(rng.choice(2048, 32, replace=False))
-        Y, H = run.fwd(save_h=True)
-        assert_close(np64(Y)[rows], olin.forward_rows(X, Wd, A, B, s, rows), what=f"{name} Y")
-        dX, dA, dB = run.bwd(H=H)
-        assert_close(np64(dX)[rows], olin.backward_dx_rows(Wd, A, B, s, dY, rows), what=f"{name} dX")
-        G = dY @ B
-        assert_close(np64(dA), s * (G.T @ X), what=f"{name} dA")
-        assert_close(np64(dB), s * (dY.T @ (X @ A.T)), what=f"{name} dB")
+        Y, H = run.fwd(torch.bfloat16, save_h=True)
+        assert_close(np64(Y)[rows], olin.forward_rows(X, Wd, A, B, s, rows), bf16_out=True, what=f"{name} Y")
+        dX, dA, dB = run.bwd(torch.bfloat16, H=H)
+        assert_close(np64(dX)[rows], olin.backward_dx_rows(Wd, A, B, s, dY, rows), bf16_out=True, what=f"{name} dX")
+        rdA, rdB = olin.backward_weight_grads(X, A, B, s, dY)
+        assert_close(np64(dA), rdA, what=f"{name} dA")
+        assert_close(np64(dB), rdB, what=f"{name} dB")
 
 
 def test_argument_errors(q):

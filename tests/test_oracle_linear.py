@@ -79,6 +79,22 @@ def test_row_helpers_match_full_products():
                                linear.backward(X, W, A, B, s, dY)[0][rows], atol=1e-12)
 
 
+def test_weight_grad_helper_matches_full_backward():
+    rng = np.random.default_rng(16)
+    M, K, N, r, s = 11, 64, 24, 8, 0.25
+    X, W, A, B, dY = (_rand(rng, M, K), _rand(rng, N, K), _rand(rng, r, K),
+                      _rand(rng, N, r), _rand(rng, M, N))
+    _, dA, dB = linear.backward(X, W, A, B, s, dY)
+    gA, gB = linear.backward_weight_grads(X, A, B, s, dY)
+    np.testing.assert_allclose(gA, dA, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(gB, dB, rtol=0, atol=1e-12)
+    # and against brute-force sums over tokens: dA[j,k] = s sum_m (sum_n dY[m,n] B[n,j]) X[m,k]
+    for j in range(r):
+        for k in (0, 17, 63):
+            ref = s * sum(sum(dY[m, n] * B[n, j] for n in range(N)) * X[m, k] for m in range(M))
+            assert abs(gA[j, k] - ref) < 1e-10
+
+
 def test_error_metrics():
     ref = np.array([[3.0, 4.0]])
     assert linear.rel_frobenius(ref, ref) == 0.0
