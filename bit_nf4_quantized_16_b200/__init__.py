@@ -28,7 +28,8 @@ STATUS = {
 
 # every symbol the header declares
 EXPORTS = (
-    "qlora_build_nf4_codebook", "qlora_build_int4_codebook", "qlora_quantize_workspace_bytes",
+    "qlora_build_nf4_codebook", "qlora_build_int4_codebook", "qlora_build_fp4_codebook",
+    "qlora_quantize_workspace_bytes",
     "qlora_quantize_nf4_dq",
     "qlora_quantize_nf4_dq_noalloc",
     "qlora_dequantize_nf4_dq", "qlora_linear_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd",
@@ -72,6 +73,7 @@ def _load():
     sig = {
         "qlora_build_nf4_codebook": (ctypes.c_int, [ctypes.c_double, P]),
         "qlora_build_int4_codebook": (ctypes.c_int, [P]),
+        "qlora_build_fp4_codebook": (ctypes.c_int, [P]),
         "qlora_quantize_workspace_bytes": (S, [I64, I64]),
         "qlora_quantize_nf4_dq": (ctypes.c_int, [P, ctypes.c_int, W, P, S, P]),
         "qlora_quantize_nf4_dq_noalloc": (ctypes.c_int, [P, ctypes.c_int, W, P]),
@@ -159,6 +161,12 @@ def qlora_build_nf4_codebook(delta: float = 0.0):
 def qlora_build_int4_codebook():
     out = (ctypes.c_float * 16)()
     _check(lib.qlora_build_int4_codebook(ctypes.cast(out, ctypes.c_void_p)), "qlora_build_int4_codebook")
+    return [float(v) for v in out]
+
+
+def qlora_build_fp4_codebook():
+    out = (ctypes.c_float * 16)()
+    _check(lib.qlora_build_fp4_codebook(ctypes.cast(out, ctypes.c_void_p)), "qlora_build_fp4_codebook")
     return [float(v) for v in out]
 
 

@@ -205,6 +205,23 @@ extern "C" qlora_status qlora_build_int4_codebook(float codebook_out[16])
     return QLORA_OK;
 }
 
+// 4-bit float as an absmax code ("QLoRA: Efficient Finetuning of Quantized
+// LLMs", section "Introduction", item (1), compares NF4 with 4-bit floats
+// without defining them): the values of the E2M1 element type (sign, two
+// exponent bits with bias 1, one mantissa bit: magnitudes 0, 0.5, 1, 1.5, 2,
+// 3, 4, 6) over the largest magnitude 6.  +0 and -0 are one table value, so
+// the sixteenth entry is -8/6 (one exponent step beyond 6), below -1 and never
+// the nearest value to a scaled element.
+extern "C" qlora_status qlora_build_fp4_codebook(float codebook_out[16])
+{
+    if (!codebook_out) return QLORA_ERR_INVALID_ARG;
+    static const double mags[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+    codebook_out[0] = (float)(-8.0 / 6.0);
+    for (int i = 0; i < 7; i++) codebook_out[1 + i] = (float)(-mags[7 - i] / 6.0);   // -1 .. -1/12
+    for (int i = 0; i < 8; i++) codebook_out[8 + i] = (float)(mags[i] / 6.0);        // 0 .. 1
+    return QLORA_OK;
+}
+
 extern "C" const char *qlora_status_string(qlora_status status)
 {
     switch (status) {

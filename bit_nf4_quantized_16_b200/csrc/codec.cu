@@ -98,9 +98,9 @@ constexpr uint32_t kQDynSmem = (kQThreads / 32) * kQStages * kQStageBytes + 1024
 // 20 bits of k equal those of the order-preserving key.  Entry i of the
 // table holds E(j(i)) - (i << 20), so that t = table[i] + k holds the code in
 // bits 20..23 and zeros above.
-// The steps are plain shifts and logic ops that the compiler spreads over
-// the integer and multiply-add pipes (forcing them onto the multiply-add
-// pipe, through multiply-high, saturated it and measured 14% slower).
+// The steps are split between the integer and the multiply-add pipes (all of
+// them on the multiply-add pipe, through multiply-high, saturated it and
+// measured 20% slower; all of them on the integer pipe saturated that one).
 // Every CTA builds the table once: thread t fills the entries of ordered
 // intervals j = 16t..16t+15, walking the sorted midpoint keys once.
 __device__ __forceinline__ void build_code_lut(uint32_t *lut, const uint32_t *mkey_smem)
@@ -121,14 +121,20 @@ __device__ __forceinline__ void build_code_lut(uint32_t *lut, const uint32_t *mk
 }
 
 // Code of n inserted at nibble position 4*I of acc (whose nibble I is zero).
+// The sign mask and the move of the code to its nibble are multiplications
+// (multiply-add pipe), the table index, the add and the logic ops integer-pipe
+// instructions: the two pipes carry about equal shares.
 template <int I>
 __device__ __forceinline__ uint32_t add_code(const uint32_t *lut, float n, uint32_t acc)
 {
     const uint32_t b = __float_as_uint(n);
-    const uint32_t s = (uint32_t)((int32_t)b >> 31);        // 0 or all ones: the sign mask
+    const uint32_t s = (uint32_t)__mulhi((int)b, 2);        // 0 or all ones: the sign mask
     const uint32_t k = b ^ (s & 0xFFFFFu);                  // low 20 bits flipped for n < 0
     const uint32_t t = lut[k >> 20] + k;                    // code in bits 20..23, zero above
-    const uint32_t part = (4 * I <= 20) ? (t >> (20 - 4 * I)) : (t << (4 * I - 20));
+    uint32_t part;
+    if constexpr (4 * I < 20) part = __umulhi(t, 1u << (12 + 4 * I));  // t >> (20 - 4I)
+    else if constexpr (4 * I == 20) part = t;
+    else part = t * (1u << (4 * I - 20));                              // t << (4I - 20)
     return acc | (part & (0xFu << (4 * I)));
 }
 
@@ -350,7 +356,33 @@ struct DqParams {
     int64_t ngroups;
 };
 
-// One warp per group of 256 constants, 8 per lane.
+// E4M3 code (saturating, round to nearest even) of RN32(d / c2) for c2 > 0.
+// Fast path: q = RN32(d * RN32(1/c2)) lies within 3 units in the last place
+// of RN32(d / c2) (two roundings of relative size 2^-24 each); E4M3 rounding
+// is monotone, so when the values 4 units below and above q encode to the
+// same code, that code is the one of RN32(d / c2).  Otherwise (q within a few
+// units of an E4M3 rounding boundary, about once in 10^5 values) the quotient
+// is formed with the IEEE division, as it is for c2 < 2^-100 (rc2 = 0 then).
+__device__ __forceinline__ uint8_t e4m3_of_quotient(float d, float c2, float rc2)
+{
+    if (rc2 == 0.0f)   // c2 below 2^-100: the reciprocal could overflow; divide
+        return (uint8_t)__nv_cvt_float_to_fp8(__fdiv_rn(d, c2), __NV_SATFINITE, __NV_E4M3);
+    const float q = __fmul_rn(d, rc2);
+    const uint32_t b = __float_as_uint(q);
+    const uint32_t mag = b & 0x7FFFFFFFu;
+    float lo = q, hi = q;
+    if (mag >= 4u) {   // |q| far below every E4M3 boundary otherwise
+        lo = __uint_as_float(b - 4u);
+        hi = __uint_as_float(b + 4u);
+    }
+    const __nv_fp8x2_storage_t two = __nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
+    const uint8_t e_lo = (uint8_t)(two & 0xFF), e_hi = (uint8_t)(two >> 8);
+    if (e_lo == e_hi) return e_lo;
+    return (uint8_t)__nv_cvt_float_to_fp8(__fdiv_rn(d, c2), __NV_SATFINITE, __NV_E4M3);
+}
+
+// One warp per group of 256 constants, 8 consecutive ones per lane (two
+// 16-byte loads).
 __global__ void __launch_bounds__(kThreads) dq_encode_kernel(DqParams p)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -361,23 +393,31 @@ __global__ void __launch_bounds__(kThreads) dq_encode_kernel(DqParams p)
     for (int64_t g = (int64_t)blockIdx.x * (kThreads / 32) + warp; g < p.ngroups;
          g += (int64_t)gridDim.x * (kThreads / 32)) {
         const int64_t b0 = g * QLORA_GROUP + lane * 8;
+        float c[8];
+        if (b0 + 8 <= p.nblocks) {
+            const float4 v0 = *reinterpret_cast<const float4 *>(p.c1 + b0);
+            const float4 v1 = *reinterpret_cast<const float4 *>(p.c1 + b0 + 4);
+            c[0] = v0.x; c[1] = v0.y; c[2] = v0.z; c[3] = v0.w;
+            c[4] = v1.x; c[5] = v1.y; c[6] = v1.z; c[7] = v1.w;
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; i++) c[i] = b0 + i < p.nblocks ? p.c1[b0 + i] : mu;   // d = 0 past the end
+        }
         float d[8];
         float amax = 0.0f;
 #pragma unroll
         for (int i = 0; i < 8; i++) {
-            bool ok = b0 + i < p.nblocks;
-            d[i] = ok ? __fsub_rn(p.c1[b0 + i], mu) : 0.0f;
+            d[i] = __fsub_rn(c[i], mu);
             amax = fmaxf(amax, fabsf(d[i]));
         }
 #pragma unroll
         for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
         const float s = __fdiv_rn(amax, 448.0f);
         if (lane == 0) p.c2[g] = s;
+        const float rs = s >= 0x1p-100f ? __frcp_rn(s) : 0.0f;
         uint8_t e[8];
 #pragma unroll
-        for (int i = 0; i < 8; i++)
-            e[i] = s == 0.0f ? (uint8_t)0
-                             : (uint8_t)__nv_cvt_float_to_fp8(__fdiv_rn(d[i], s), __NV_SATFINITE, __NV_E4M3);
+        for (int i = 0; i < 8; i++) e[i] = s == 0.0f ? (uint8_t)0 : e4m3_of_quotient(d[i], s, rs);
         if (b0 + 8 <= p.nblocks) {
             uint2 v;
             v.x = e[0] | (e[1] << 8) | (e[2] << 16) | ((uint32_t)e[3] << 24);

@@ -7,12 +7,18 @@
 // multiply in 16-bit) and abstract (gradients flow through the frozen 4-bit
 // weight into the adapters).
 //
-// Launch sequence (all on the caller's stream):
-//   forward : H-partials (tcgen05, split-K) -> finalize H (x s, hi/lo bf16)
+// Launch sequence (all on the caller's stream, chained by programmatic
+// dependent launch):
+//   forward : H = s X A^T (cluster split-K, hi/lo bf16 + optional fp32 H)
 //             -> fused dequant-GEMM with the LoRA up-projection as extra K steps
-//   backward: H (recomputed, or split from the saved fp32 H) -> G-partials ->
-//             finalize G -> fused transposed dequant-GEMM for dX (+ G A)
-//             -> dA partials (G^T X) -> dB partials (dY^T H) -> finalize both
+//   backward: [H recomputed when no saved H is given]
+//             -> G = s dY B (cluster split-K, hi/lo bf16; a saved H is split
+//                into hi/lo in the same kernel)
+//             -> fused transposed dequant-GEMM for dX (+ G A)
+//             -> dA = G^T X and dB = dY^T H in one launch (cluster split over
+//                the tokens); its inputs were all written at least two
+//                launches earlier, so it starts without waiting for the dX
+//                GEMM and fills the SMs that GEMM's last wave leaves idle
 // H and G are carried as hi + lo bf16 pairs (hi = bf16(v), lo = bf16(v - hi)):
 // the weight gradients contract over all M tokens and need about 16 bits of
 // each factor to stay at the level of fp32 accumulation; the fused GEMMs use
@@ -28,6 +34,7 @@
 #include "decode.cuh"
 #include "gemm.cuh"
 #include "gemm_pair.cuh"
+#include "gemm_skinny.cuh"
 
 namespace qlora {
 namespace {
@@ -110,137 +117,92 @@ qlora_status launch_gemm_pair(GemmParams &p, const DeviceInfo &dev, cudaStream_t
     return launch_status();
 }
 
-// number of splits of a contraction of `total` 64-deep steps over `tiles`
-// output tiles: as many as fit in one wave of the GPU (tiles * splits <= sms),
-// each with at least `min_per_split` steps; every split non-empty
-void choose_splits(int tiles, int total, int sms, int min_per_split, int *splits, int *per)
-{
-    int sp = sms / (tiles > 0 ? tiles : 1);
-    int cap = total / min_per_split;
-    if (cap < 1) cap = 1;
-    if (sp > cap) sp = cap;
-    if (sp < 1) sp = 1;
-    int pr = (total + sp - 1) / sp;
-    *per = pr;
-    *splits = (total + pr - 1) / pr;
-}
-
 int ceil_div(int64_t a, int64_t b) { return (int)((a + b - 1) / b); }
 int pad64(int v) { return (v + 63) / 64 * 64; }
-int elementwise_grid(int64_t n) { return (int)((n + 255) / 256); }
 
-// ---- finalize kernels (grid-wide, one thread per 4 outputs) ---------------------------
+// ---- skinny products (gemm_skinny.cuh) ------------------------------------------
 
-// Sum of the split partials at (row, col..col+3), splits added in order.
-__device__ __forceinline__ float4 split_sum4(const float *part, int splits, int64_t split_stride, int64_t ld,
-                                             int64_t row, int64_t col)
+// Launches one skinny-product grid: `clusters` output tiles, `csize` CTAs per
+// cluster (the contraction split).
+template <int BN, int A_MN, int B_MN>
+qlora_status launch_skinny(SkinnyParams &p, int clusters, int csize, const DeviceInfo &dev, cudaStream_t s, int kind)
 {
-    const float *src = part + row * ld + col;
-    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    // four splits' loads are issued before their in-order additions (issue is
-    // in order, so an addition waiting on a load would hold back the next load)
-    for (int sp0 = 0; sp0 < splits; sp0 += 4) {
-        float4 v[4];
-#pragma unroll
-        for (int i = 0; i < 4; i++)
-            v[i] = sp0 + i < splits ? __ldcg(reinterpret_cast<const float4 *>(src + (sp0 + i) * split_stride))
-                                    : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-#pragma unroll
+    using Cfg = SkinnyCfg<BN, A_MN, B_MN>;
+    auto kern = qgemm_skinny_kernel<BN, A_MN, B_MN>;
+    p.err = device_error_word();
+    if (!p.err) return QLORA_ERR_CUDA;
+    p.timeout_ns = kTimeoutNs;
+    p.drain_ns = kTimeoutNs;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)(clusters * csize));
+    cfg.blockDim = dim3(Cfg::kThreads);
+    cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)csize;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    {
+        LaunchScope ls(kind, s);
+        QLORA_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, p));
+    }
+    return launch_status();
+}
+
+// Kernel attributes and the number of co-resident clusters for each cluster
+// size 1, 2, 4, 8 (once per device and instantiation).
+template <int BN, int A_MN, int B_MN>
+qlora_status skinny_setup(const DeviceInfo &dev, const int **max_clusters)
+{
+    using Cfg = SkinnyCfg<BN, A_MN, B_MN>;
+    static PerDeviceOnce once;
+    static int maxc[kMaxDevices][4] = {};
+    auto kern = qgemm_skinny_kernel<BN, A_MN, B_MN>;
+    QLORA_TRY(once.run(dev.device, [&]() -> qlora_status {
+        QLORA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes));
         for (int i = 0; i < 4; i++) {
-            if (sp0 + i >= splits) break;
-            acc.x = __fadd_rn(acc.x, v[i].x);
-            acc.y = __fadd_rn(acc.y, v[i].y);
-            acc.z = __fadd_rn(acc.z, v[i].z);
-            acc.w = __fadd_rn(acc.w, v[i].w);
+            const int c = 1 << i;
+            cudaLaunchConfig_t cfg{};
+            cfg.gridDim = dim3((unsigned)(c * (dev.sms / c)));
+            cfg.blockDim = dim3(Cfg::kThreads);
+            cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = (unsigned)c;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int n = 0;
+            QLORA_CUDA_TRY(cudaOccupancyMaxActiveClusters(&n, kern, &cfg));
+            maxc[dev.device][i] = n;
         }
-    }
-    return acc;
+        return QLORA_OK;
+    }));
+    *max_clusters = maxc[dev.device];
+    return QLORA_OK;
 }
 
-__device__ __forceinline__ uint32_t bf16_bits(float v) { return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v)); }
-
-// hi = bf16(v), lo = bf16(v - hi) of 4 consecutive columns col..col+3 into the
-// chunked hi/lo layout: [M][2*r_pad], hi of column c at 128*(c/64) + c%64, lo 64 further.
-__device__ __forceinline__ void store_hi_lo4(__nv_bfloat16 *dst, int64_t row, int r_pad, int col, float4 v)
+// Contraction split (cluster size): the largest of 8, 4, 2 for which all
+// tiles' clusters are co-resident in one wave and every CTA keeps at least
+// four 64-deep steps; else 1.
+int choose_csize(int tiles, int k_total, const int *max_clusters)
 {
-    const float vv[4] = {v.x, v.y, v.z, v.w};
-    uint32_t hi[4], lo[4];
-#pragma unroll
-    for (int i = 0; i < 4; i++) {
-        hi[i] = bf16_bits(vv[i]);
-        lo[i] = bf16_bits(__fsub_rn(vv[i], __uint_as_float(hi[i] << 16)));
+    for (int i = 3; i >= 1; i--) {
+        const int c = 1 << i;
+        if (tiles <= max_clusters[i] && k_total >= 4 * c) return c;
     }
-    __nv_bfloat16 *d = dst + row * 2 * r_pad + 128 * (col >> 6) + (col & 63);
-    *reinterpret_cast<uint2 *>(d) = make_uint2(hi[0] | (hi[1] << 16), hi[2] | (hi[3] << 16));
-    *reinterpret_cast<uint2 *>(d + 64) = make_uint2(lo[0] | (lo[1] << 16), lo[2] | (lo[3] << 16));
+    return 1;
 }
 
-// v = scale * sum over splits of part[.][m][j]  ->  hi/lo chunked buffer (padding
-// columns j >= r set to zero), optionally fp32 v [M][r]; optionally also the
-// hi/lo split of aux_in [M][r] into aux_out.
-__global__ void finalize_lowrank_kernel(const float *part, int splits, int64_t split_stride, int64_t M, int r,
-                                        int r_pad, float scale, __nv_bfloat16 *out, float *out_f32,
-                                        const float *aux_in, __nv_bfloat16 *aux_out)
+qlora_status map_k_major(CUtensorMap *m, const void *base, int64_t inner, int64_t rows, uint32_t box_rows)
 {
-    sm100::pdl_wait();
-    sm100::pdl_trigger();
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int per_row = r_pad / 4;
-    if (i >= M * per_row) return;
-    const int64_t m = i / per_row;
-    const int col = 4 * (int)(i % per_row);
-    const bool in = col < r;   // r % 8 == 0: 4 columns are all in or all out
-    float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    if (in) {
-        v = split_sum4(part, splits, split_stride, r_pad, m, col);
-        v = make_float4(__fmul_rn(scale, v.x), __fmul_rn(scale, v.y), __fmul_rn(scale, v.z), __fmul_rn(scale, v.w));
-        if (out_f32) *reinterpret_cast<float4 *>(out_f32 + m * r + col) = v;
-    }
-    store_hi_lo4(out, m, r_pad, col, v);
-    if (aux_in) {
-        float4 h = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-        if (in) h = *reinterpret_cast<const float4 *>(aux_in + m * r + col);
-        store_hi_lo4(aux_out, m, r_pad, col, h);
-    }
-}
-
-// Weight gradients from the partial products of the hi and lo halves, two jobs
-// in one launch: job 0 = dA (rows k of X^T [G_hi|G_lo], stored transposed into
-// dA[j][k]), job 1 = dB (rows n of dY^T [H_hi|H_lo], stored as dB[n][j]).
-struct WgradJob {
-    const float *part;
-    int splits;
-    int64_t split_stride;
-    int64_t rows;
-    float *out;
-    int64_t out_ld;
-    int transposed;
-};
-
-__global__ void finalize_wgrad_kernel(WgradJob j0, WgradJob j1, int64_t n0, int r, int r_pad)
-{
-    sm100::pdl_wait();
-    sm100::pdl_trigger();
-    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int per_row = r / 4;
-    const WgradJob &J = i < n0 ? j0 : j1;
-    if (i >= n0) i -= n0;
-    if (i >= J.rows * per_row) return;
-    const int64_t row = i / per_row;
-    const int j = 4 * (int)(i % per_row);
-    const int64_t ld = 2 * r_pad;
-    const int64_t chunk = 128 * (j >> 6) + (j & 63);
-    const float4 hi = split_sum4(J.part, J.splits, J.split_stride, ld, row, chunk);
-    const float4 lo = split_sum4(J.part, J.splits, J.split_stride, ld, row, chunk + 64);
-    const float4 v = make_float4(__fadd_rn(hi.x, lo.x), __fadd_rn(hi.y, lo.y), __fadd_rn(hi.z, lo.z), __fadd_rn(hi.w, lo.w));
-    if (J.transposed) {
-        J.out[(int64_t)(j + 0) * J.out_ld + row] = v.x;
-        J.out[(int64_t)(j + 1) * J.out_ld + row] = v.y;
-        J.out[(int64_t)(j + 2) * J.out_ld + row] = v.z;
-        J.out[(int64_t)(j + 3) * J.out_ld + row] = v.w;
-    } else {
-        *reinterpret_cast<float4 *>(J.out + row * J.out_ld + j) = v;
-    }
+    return map_bf16(m, base, (uint64_t)inner, (uint64_t)rows, (uint64_t)inner, 64, box_rows);
 }
 
 // ---- problem plan -------------------------------------------------------------------
@@ -250,11 +212,7 @@ __global__ void finalize_wgrad_kernel(WgradJob j0, WgradJob j1, int64_t n0, int 
 struct Plan {
     int64_t M, N, K;
     int r, r_pad;
-    int h_splits, h_per;          // H = s X A^T : M tiles, split over K
-    int g_splits, g_per;          // G = s dY B  : M tiles, split over N
-    int da_splits, da_per;        // dA^T = X^T [G_hi|G_lo] : K tiles x chunks, split over M
-    int db_splits, db_per;        // dB = dY^T [H_hi|H_lo]  : N tiles x chunks, split over M
-    size_t off_h2, off_g2, off_part, off_part2, bytes;
+    size_t off_h2, off_g2, bytes;
 };
 
 size_t align256(size_t v) { return (v + 255) / 256 * 256; }
@@ -267,21 +225,10 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int r, int sms)
     pl.K = K;
     pl.r = r;
     pl.r_pad = pad64(r);
-    const int chunks = pl.r_pad / 64;
-    const int mt = ceil_div(M, 128), kt = ceil_div(K, 128), nt = ceil_div(N, 128);
-    choose_splits(mt, ceil_div(K, 64), sms, 4, &pl.h_splits, &pl.h_per);
-    choose_splits(mt, ceil_div(N, 64), sms, 4, &pl.g_splits, &pl.g_per);
-    choose_splits(kt * chunks, ceil_div(M, 64), sms, 4, &pl.da_splits, &pl.da_per);
-    choose_splits(nt * chunks, ceil_div(M, 64), sms, 4, &pl.db_splits, &pl.db_per);
     const size_t hl = align256((size_t)M * 2 * pl.r_pad * 2);
-    size_t part = std::max((size_t)pl.h_splits, (size_t)pl.g_splits) * M * pl.r_pad * 4;
-    part = std::max(part, (size_t)pl.da_splits * K * 2 * pl.r_pad * 4);
-    const size_t part2 = (size_t)pl.db_splits * N * 2 * pl.r_pad * 4;
     pl.off_h2 = 0;
     pl.off_g2 = hl;
-    pl.off_part = 2 * hl;
-    pl.off_part2 = pl.off_part + align256(part);
-    pl.bytes = pl.off_part2 + align256(part2);
+    pl.bytes = 2 * hl;
     // the decode forward (M <= kDecodeMaxTokens) uses the start of the workspace for its partials
     if (M <= kDecodeMaxTokens) pl.bytes = std::max(pl.bytes, align256(decode_workspace_bytes(M, N, K, r, sms)));
     return pl;
@@ -300,41 +247,48 @@ qlora_status check_linear(const qlora_nf4_weight *w, const void *X, int64_t M, c
     return QLORA_OK;
 }
 
-void set_split(GemmParams &p, int splits, int per, int total_stages, int64_t plane)
+// Low-rank factor v = scale * P Q^T (P [M][Kc] bf16, Q given as the B operand)
+// into the hi/lo buffer `hl`, with an optional fp32 copy and an optional
+// hi/lo split of aux_in into aux_out.
+template <int BN, int B_MN>
+qlora_status run_lowrank(const Plan &pl, const DeviceInfo &dev, const void *P, int64_t Kc, const void *Q,
+                         float scale, __nv_bfloat16 *hl, float *f32_out, const float *aux_in, __nv_bfloat16 *aux_out,
+                         cudaStream_t s)
 {
-    p.splits = splits;
-    p.k_stages_total = total_stages;
-    p.k_stages_split = per;
-    p.split_stride = plane;
+    const int *maxc = nullptr;
+    QLORA_TRY((skinny_setup<BN, 0, B_MN>(dev, &maxc)));
+    SkinnyParams p{};
+    SkinnyJob &J = p.job[0];
+    QLORA_TRY(map_k_major(&J.tm_a, P, Kc, pl.M, 128));
+    if (B_MN)
+        QLORA_TRY(map_k_major(&J.tm_b, Q, pl.r, Kc, 64));       // B [Kc][r]: 64-column chunks
+    else
+        QLORA_TRY(map_k_major(&J.tm_b, Q, Kc, pl.r, pl.r_pad));  // A [r][Kc]
+    J.m_tiles = ceil_div(pl.M, 128);
+    J.k_total = ceil_div(Kc, 64);
+    J.fin = kFinLowRank;
+    J.m_total = (int)pl.M;
+    J.scale = scale;
+    J.r = pl.r;
+    J.r_pad = pl.r_pad;
+    J.hl_out = hl;
+    J.f32_out = f32_out;
+    J.aux_in = aux_in;
+    J.aux_out = aux_out;
+    p.clusters0 = J.m_tiles;
+    p.wait_at_end = 0;
+    const int cs = choose_csize(J.m_tiles, J.k_total, maxc);
+    return launch_skinny<BN, 0, B_MN>(p, J.m_tiles, cs, dev, s, QLORA_KERNEL_LOWRANK);
 }
 
 // H = s X A^T into the hi/lo buffer (and optionally fp32 H_out)
 qlora_status run_h(const Plan &pl, const DeviceInfo &dev, const void *X, const void *A, float scale, float *H_out,
                    char *ws, cudaStream_t s)
 {
-    GemmParams p{};
-    QLORA_TRY(map_bf16(&p.tm_a, X, pl.K, pl.M, pl.K, 64, 128));
-    QLORA_TRY(map_bf16(&p.tm_b, A, pl.K, pl.r, pl.K, 64, pl.r_pad));
-    p.m_tiles = ceil_div(pl.M, 128);
-    p.n_tiles = 1;
-    set_split(p, pl.h_splits, pl.h_per, ceil_div(pl.K, 64), pl.M * pl.r_pad);
-    p.out = ws + pl.off_part;
-    p.out_ld = pl.r_pad;
-    p.m_total = (int)pl.M;
-    p.n_total = pl.r_pad;
+    __nv_bfloat16 *H2 = reinterpret_cast<__nv_bfloat16 *>(ws + pl.off_h2);
     if (pl.r_pad == 64)
-        QLORA_TRY((launch_gemm<64, kBTmaK, kEpiF32>(p, dev, s, QLORA_KERNEL_LOWRANK)));
-    else
-        QLORA_TRY((launch_gemm<128, kBTmaK, kEpiF32>(p, dev, s, QLORA_KERNEL_LOWRANK)));
-    {
-        LaunchScope ls(QLORA_KERNEL_ELEMENTWISE, s);
-        QLORA_CUDA_TRY(launch_pdl(finalize_lowrank_kernel, dim3(elementwise_grid(pl.M * pl.r_pad / 4)), dim3(256), 0,
-                                  s, reinterpret_cast<const float *>(ws + pl.off_part), pl.h_splits,
-                                  (int64_t)(pl.M * pl.r_pad), pl.M, pl.r, pl.r_pad, scale,
-                                  reinterpret_cast<__nv_bfloat16 *>(ws + pl.off_h2), H_out, (const float *)nullptr,
-                                  (__nv_bfloat16 *)nullptr));
-    }
-    return launch_status();
+        return run_lowrank<64, 0>(pl, dev, X, pl.K, A, scale, H2, H_out, nullptr, nullptr, s);
+    return run_lowrank<128, 0>(pl, dev, X, pl.K, A, scale, H2, H_out, nullptr, nullptr, s);
 }
 
 }  // namespace
@@ -442,31 +396,11 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *
     // H (hi/lo) recomputed when no saved H is given
     if (!H_saved) QLORA_TRY(run_h(pl, dev, X, A, scale, nullptr, ws, s));
 
-    // G = s dY B (contraction over N); its finalize also splits a saved H into hi/lo
-    {
-        GemmParams p{};
-        QLORA_TRY(map_bf16(&p.tm_a, dY, N, M, N, 64, 128));
-        QLORA_TRY(map_bf16(&p.tm_b, B, r, N, r, 64, 64));      // B[n][j]: MN-major operand
-        p.m_tiles = ceil_div(M, 128);
-        p.n_tiles = 1;
-        set_split(p, pl.g_splits, pl.g_per, ceil_div(N, 64), M * pl.r_pad);
-        p.out = ws + pl.off_part;
-        p.out_ld = pl.r_pad;
-        p.m_total = (int)M;
-        p.n_total = pl.r_pad;
-        if (pl.r_pad == 64)
-            QLORA_TRY((launch_gemm<64, kBTmaMN, kEpiF32>(p, dev, s, QLORA_KERNEL_LOWRANK)));
-        else
-            QLORA_TRY((launch_gemm<128, kBTmaMN, kEpiF32>(p, dev, s, QLORA_KERNEL_LOWRANK)));
-        {
-            LaunchScope ls(QLORA_KERNEL_ELEMENTWISE, s);
-            QLORA_CUDA_TRY(launch_pdl(finalize_lowrank_kernel, dim3(elementwise_grid(M * pl.r_pad / 4)), dim3(256), 0,
-                                      s, reinterpret_cast<const float *>(ws + pl.off_part), pl.g_splits,
-                                      (int64_t)(M * pl.r_pad), M, r, pl.r_pad, scale, G2, (float *)nullptr, H_saved,
-                                      H_saved ? H2 : (__nv_bfloat16 *)nullptr));
-        }
-        QLORA_TRY(launch_status());
-    }
+    // G = s dY B (contraction over N); the same kernel splits a saved H into hi/lo
+    if (pl.r_pad == 64)
+        QLORA_TRY((run_lowrank<64, 1>(pl, dev, dY, N, B, scale, G2, nullptr, H_saved, H_saved ? H2 : nullptr, s)));
+    else
+        QLORA_TRY((run_lowrank<128, 1>(pl, dev, dY, N, B, scale, G2, nullptr, H_saved, H_saved ? H2 : nullptr, s)));
 
     // dX = dY W' + bf16(G) A  (fused transposed dequant-GEMM)
     if (dX) {
@@ -512,45 +446,38 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *
             QLORA_TRY((launch_gemm<kBBN, kBNf4MN, kEpiF32, kBMT>(p, dev, s, QLORA_KERNEL_BWD_FUSED)));
     }
 
-    // dA^T = X^T [G_hi | G_lo]  and  dB = dY^T [H_hi | H_lo]: rows k (resp. n), chunked
-    // hi | lo columns, contraction over tokens; one finalize adds the halves
-    float *part_a = reinterpret_cast<float *>(ws + pl.off_part);
-    float *part_b = reinterpret_cast<float *>(ws + pl.off_part2);
+    // dA = (X^T [G_hi | G_lo])^T and dB = dY^T [H_hi | H_lo] in one launch: output rows k
+    // (resp. n), 128-column tiles = the hi and lo halves of one 64-column chunk,
+    // contraction over the tokens; the reduction adds the halves
     {
-        GemmParams p{};
-        QLORA_TRY(map_bf16(&p.tm_a, X, K, M, K, 64, 64));              // MN-major A
-        QLORA_TRY(map_bf16(&p.tm_b, G2, hl_cols, M, hl_cols, 64, 64));  // MN-major B
-        p.a_mn = 1;
-        p.m_tiles = ceil_div(K, 128);
-        p.n_tiles = pl.r_pad / 64;
-        set_split(p, pl.da_splits, pl.da_per, ceil_div(M, 64), K * hl_cols);
-        p.out = part_a;
-        p.out_ld = hl_cols;
-        p.m_total = (int)K;
-        p.n_total = hl_cols;
-        QLORA_TRY((launch_gemm<128, kBTmaMN, kEpiF32>(p, dev, s, QLORA_KERNEL_WGRAD)));
-    }
-    {
-        GemmParams p{};
-        QLORA_TRY(map_bf16(&p.tm_a, dY, N, M, N, 64, 64));              // MN-major A
-        QLORA_TRY(map_bf16(&p.tm_b, H2, hl_cols, M, hl_cols, 64, 64));  // MN-major B
-        p.a_mn = 1;
-        p.m_tiles = ceil_div(N, 128);
-        p.n_tiles = pl.r_pad / 64;
-        set_split(p, pl.db_splits, pl.db_per, ceil_div(M, 64), N * hl_cols);
-        p.out = part_b;
-        p.out_ld = hl_cols;
-        p.m_total = (int)N;
-        p.n_total = hl_cols;
-        QLORA_TRY((launch_gemm<128, kBTmaMN, kEpiF32>(p, dev, s, QLORA_KERNEL_WGRAD)));
-    }
-    {
-        WgradJob ja{part_a, pl.da_splits, K * hl_cols, K, dA, K, 1};
-        WgradJob jb{part_b, pl.db_splits, N * hl_cols, N, dB, r, 0};
-        const int64_t n0 = K * (r / 4), n1 = N * (r / 4);
-        LaunchScope ls(QLORA_KERNEL_ELEMENTWISE, s);
-        QLORA_CUDA_TRY(launch_pdl(finalize_wgrad_kernel, dim3(elementwise_grid(n0 + n1)), dim3(256), 0, s, ja, jb,
-                                  (int64_t)n0, r, pl.r_pad));
+        const int *maxc = nullptr;
+        QLORA_TRY((skinny_setup<128, 1, 1>(dev, &maxc)));
+        SkinnyParams p{};
+        SkinnyJob &Ja = p.job[0], &Jb = p.job[1];
+        QLORA_TRY(map_bf16(&Ja.tm_a, X, K, M, K, 64, 64));               // MN-major: rows k, contraction m
+        QLORA_TRY(map_bf16(&Ja.tm_b, G2, hl_cols, M, hl_cols, 64, 64));
+        QLORA_TRY(map_bf16(&Jb.tm_a, dY, N, M, N, 64, 64));
+        QLORA_TRY(map_bf16(&Jb.tm_b, H2, hl_cols, M, hl_cols, 64, 64));
+        const int chunks = pl.r_pad / 64;
+        Ja.m_tiles = ceil_div(K, 128);
+        Jb.m_tiles = ceil_div(N, 128);
+        Ja.k_total = Jb.k_total = ceil_div(M, 64);
+        Ja.fin = kFinWgradT;
+        Jb.fin = kFinWgrad;
+        Ja.m_total = (int)K;
+        Jb.m_total = (int)N;
+        Ja.r = Jb.r = r;
+        Ja.r_pad = Jb.r_pad = pl.r_pad;
+        Ja.f32_out = dA;
+        Ja.out_ld = K;
+        Jb.f32_out = dB;
+        Jb.out_ld = r;
+        const int tiles_a = Ja.m_tiles * chunks, tiles_b = Jb.m_tiles * chunks;
+        p.clusters0 = tiles_a;
+        // after the dX GEMM nothing read here comes from the kernel just before
+        p.wait_at_end = dX ? 1 : 0;
+        const int cs = choose_csize(tiles_a + tiles_b, Ja.k_total, maxc);
+        QLORA_TRY((launch_skinny<128, 1, 1>(p, tiles_a + tiles_b, cs, dev, s, QLORA_KERNEL_WGRAD)));
     }
     return launch_status();
 }

@@ -95,8 +95,9 @@ typedef enum { QLORA_BF16 = 0, QLORA_FP32 = 1 } qlora_dtype;
  *   mean    device, 1 float: mean of all first-level constants of W.
  *   codebook  host values q[0..15], strictly ascending, containing exactly
  *           one 0; the NF4 table from qlora_build_nf4_codebook(), the Int4
- *           table from qlora_build_int4_codebook(), or any other 16-value
- *           table with the same properties that the quantizer accepts.
+ *           table from qlora_build_int4_codebook(), the FP4 table from
+ *           qlora_build_fp4_codebook(), or any other 16-value table with the
+ *           same properties that the quantizer accepts.
  */
 typedef struct {
     int64_t rows;
@@ -135,6 +136,20 @@ QLORA_API qlora_status qlora_build_nf4_codebook(double delta, float codebook_out
  * Errors: QLORA_ERR_INVALID_ARG for a null pointer.
  */
 QLORA_API qlora_status qlora_build_int4_codebook(float codebook_out[16]);
+
+/*
+ * qlora_build_fp4_codebook -- a 4-bit float table for the same codec and
+ * GEMMs ("Introduction", item (1), names 4-bit floats as the other data type
+ * NF4 is compared with, without defining them).  Reading: the E2M1 element
+ * type (1 sign bit, 2 exponent bits with bias 1, 1 mantissa bit; magnitudes
+ * 0, 0.5, 1, 1.5, 2, 3, 4, 6) divided by 6, each value RN32(v / 6).  E2M1's
+ * +0 and -0 are one table value, so index 0 holds -8/6, which lies below -1
+ * and is never the nearest value; -1 .. 1 follow at indices 1 .. 15 with the
+ * zero at index 8.  Host-only, no CUDA call.
+ *   codebook_out   host, 16 floats.
+ * Errors: QLORA_ERR_INVALID_ARG for a null pointer.
+ */
+QLORA_API qlora_status qlora_build_fp4_codebook(float codebook_out[16]);
 
 /*
  * Workspace in bytes that qlora_quantize_nf4_dq needs for a rows x cols

@@ -83,3 +83,28 @@ def int4_codebook() -> np.ndarray:
     the level count 7, so that +-7 carry the block's absmax (one binary32
     rounding of each exact quotient).  -8/7 lies below -1 and never wins."""
     return np.array([np.float32(float(j) / 7.0) for j in range(-8, 8)], dtype=np.float32)
+
+
+def e2m1_value(code: int) -> float:
+    """Value of a 4-bit E2M1 code: sign bit 3, exponent bits 2..1 (bias 1),
+    mantissa bit 0; exponent field 0 is the subnormal range (m * 2^-1)."""
+    sign = -1.0 if code & 8 else 1.0
+    e = (code >> 1) & 3
+    m = code & 1
+    mag = m * 0.5 if e == 0 else (1.0 + 0.5 * m) * 2.0 ** (e - 1)
+    return sign * mag
+
+
+def fp4_codebook() -> np.ndarray:
+    """4-bit floats as an absmax code.  The paper's introduction, item (1),
+    names 4-bit floats as the other data type NF4 is compared with but does not
+    define them.  Reading: the E2M1 values (the 4-bit float of the OCP
+    microscaling formats) over their largest magnitude 6, so that +-6 carry the
+    block's absmax.  E2M1 holds 15 distinct values (+0 and -0 coincide); the
+    sixteenth entry is -8/6, the magnitude one exponent step beyond 6, which
+    lies below -1 and never wins, as -8/7 in the Int4 table."""
+    vals = sorted({e2m1_value(c) for c in range(16)})      # -0 and +0 collapse
+    assert len(vals) == 15
+    top = max(abs(v) for v in vals)
+    return np.array([np.float32(-8.0 / top)] + [np.float32(v / top) for v in vals], dtype=np.float32)
+

@@ -71,6 +71,15 @@ def test_int4_codebook_matches_oracle_bit_for_bit(lib):
     assert lib.qlora_build_int4_codebook(None) == 1
 
 
+def test_fp4_codebook_matches_oracle_bit_for_bit(lib):
+    out = (ctypes.c_float * 16)()
+    lib.qlora_build_fp4_codebook.argtypes = [ctypes.c_void_p]
+    assert lib.qlora_build_fp4_codebook(ctypes.cast(out, ctypes.c_void_p)) == 0
+    got = np.array(list(out), np.float32)
+    assert np.array_equal(got.view(np.uint32), ocb.fp4_codebook().view(np.uint32))
+    assert lib.qlora_build_fp4_codebook(None) == 1
+
+
 def test_status_strings(lib):
     lib.qlora_status_string.restype = ctypes.c_char_p
     assert lib.qlora_status_string(0) == b"QLORA_OK"

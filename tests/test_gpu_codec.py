@@ -103,6 +103,18 @@ def test_int4_codebook(q):
     assert np.all(occ.unpack(w.packed.cpu().numpy())[:64] == 8)
 
 
+def test_fp4_codebook(q):
+    """The 4-bit float (E2M1) table through the same quantizer and
+    dequantizer: ragged and LLaMA-attention-shaped tensors, bit-exact."""
+    table = q.qlora_build_fp4_codebook()
+    assert np.array_equal(np.array(table, np.float32).view(np.uint32), ocb.fp4_codebook().view(np.uint32))
+    for shape, seed in (((257, 320), 31), ((4096, 4096), 32)):
+        W = synthetic.normal(shape, 0.02, seed, torch.bfloat16)
+        w, ref = check_parity(q, W, codebook=table)
+        codes = occ.unpack(ref["packed"])
+        assert codes.min() >= 1, "index 0 (-8/6) is never the nearest value"
+
+
 def test_edge_blocks(q):
     """Zero blocks, a subnormal block, values exactly on the round-down
     midpoints (ties go to the lower code), and +-absmax."""
@@ -165,3 +177,57 @@ def test_bits_per_parameter_from_buffer_sizes(q):
     w = q.NF4Weight(4096, 4096, device="cuda")
     bits = 8 * w.nbytes / (4096 * 4096)
     assert bits == pytest.approx(occ.storage_bits_per_param(4096 * 4096), rel=1e-12)
+
+
+def _blocks_with_absmax(c1: np.ndarray, seed: int) -> torch.Tensor:
+    """fp32 weight [len(c1)/16, 1024] whose 64-blocks have exactly the given
+    absmax values: element 0 of block b is c1[b], the others lie strictly
+    inside (-c1[b], c1[b])."""
+    rng = np.random.default_rng(seed)
+    nb = len(c1)
+    blocks = (rng.uniform(-0.9, 0.9, (nb, 64)) * c1[:, None]).astype(np.float32)
+    blocks[:, 0] = c1
+    return torch.from_numpy(blocks.reshape(nb // 16, 1024))
+
+
+def _e4m3_midpoints():
+    vals = sorted({occ.e4m3_value(c) for c in range(0x7F)} | {0.0})
+    return [(a + b) / 2 for a, b in zip(vals, vals[1:])]
+
+
+def test_double_quantization_on_e4m3_ties(q):
+    """Block constants c1 = 1 +- t 2^-9 with t on every E4M3 rounding midpoint:
+    the mean is exactly 1, every group's scale exactly 2^-9 (t = 448 is in
+    each group), so (c1 - mean) / c2 = t is an exact tie that round-to-
+    nearest-even must resolve (Double Quantization, E4M3 reading)."""
+    mids = _e4m3_midpoints()
+    groups = 32
+    c1 = []
+    for g in range(groups):
+        ts = [448.0] + [mids[(127 * g + i) % len(mids)] for i in range(127)]
+        for t in ts:
+            c1 += [1.0 + t * 2.0 ** -9, 1.0 - t * 2.0 ** -9]
+    c1 = np.array(c1, np.float32)
+    assert c1.min() > 0 and len(c1) == 256 * groups
+    w, ref = check_parity(q, _blocks_with_absmax(c1, 5))
+    assert float(ref["mean"]) == 1.0 and np.all(ref["c2"] == np.float32(2.0 ** -9))
+
+
+def test_double_quantization_near_e4m3_boundaries(q):
+    """Group scale 3 2^-11 (its reciprocal is inexact) and quotients within a
+    few float32 units of E4M3 rounding boundaries: the codes must equal the
+    oracle's correctly rounded quotient everywhere."""
+    mids = _e4m3_midpoints()
+    c = 3.0 * 2.0 ** -11
+    groups = 48
+    c1 = []
+    for g in range(groups):
+        ts = [448.0]
+        for i in range(127):
+            m = mids[(5 * g + i) % len(mids)]
+            ts.append(m * (1.0 + ((i % 7) - 3) * 2.0 ** -23))
+        for t in ts:
+            c1 += [1.0 + t * c, 1.0 - t * c]
+    c1 = np.array(c1, np.float32)
+    assert c1.min() > 0
+    check_parity(q, _blocks_with_absmax(c1, 6))

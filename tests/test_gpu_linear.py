@@ -162,6 +162,14 @@ def test_int4_codebook(q, M):
     full_check(q, case, codebook=table)
 
 
+@pytest.mark.parametrize("M", [16, 200, 512])
+def test_fp4_codebook(q, M):
+    """The FP4 (E2M1) table through the decode (16 tokens), single-CTA (200)
+    and CTA-pair (512) kernels, with bf16 outputs."""
+    case = synthetic.linear_case(M, 384, 320, 16, alpha=16.0, seed=80 + M)
+    full_check(q, case, ydt=torch.bfloat16, codebook=q.qlora_build_fp4_codebook())
+
+
 def test_saved_h_equals_recomputed_h(q):
     case = synthetic.linear_case(200, 384, 512, 64, alpha=16.0, seed=5)
     run = Runner(q, case)

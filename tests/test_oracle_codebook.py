@@ -83,3 +83,24 @@ def test_int4_table_structure():
         level = Fraction(j - 8, 7)
         ulp = Fraction(float(np.spacing(np.float32(abs(v)) if v else np.float32(1e-38))))
         assert abs(Fraction(float(v)) - level) <= ulp / 2, (j, float(v))
+
+
+def test_e2m1_values_match_the_ocp_table():
+    rows = read_golden("e2m1_spec.txt")
+    assert len(rows) == 16
+    for code, val in rows:
+        got = codebook.e2m1_value(int(code, 16))
+        assert got == float(val) and np.signbit(got) == val.startswith("-"), code
+
+
+def test_fp4_table_structure():
+    q = codebook.fp4_codebook()
+    assert q.dtype == np.float32 and len(q) == 16
+    assert np.all(np.diff(q.astype(np.float64)) > 0), "strictly increasing"
+    assert np.count_nonzero(q == 0) == 1 and q[8] == 0
+    assert q[1] == -1.0 and q[15] == 1.0 and q[0] < -1.0
+    # the distinct E2M1 values over 6, each one binary32 rounding of the exact quotient
+    for v, want in zip(q[1:], [-6, -4, -3, -2, -1.5, -1, -0.5, 0, 0.5, 1, 1.5, 2, 3, 4, 6]):
+        assert v == np.float32(want / 6.0)
+    # the pad below -1 is never the nearest value of anything in [-1, 1]
+    assert (q[0] + q[1]) / 2 < -1.0
