@@ -286,6 +286,7 @@ def run_ours(args, rank, world, local_rank):
     codec = run_codec(args, q, torch, dev, peaks, peak_src) if (rank == 0 and not args.skip_codec) else None
     decode = run_decode65b(args, q, torch, dev, peaks, peak_src) if (rank == 0 and not args.skip_decode) else None
     adamw = run_adamw7b(args, q, torch, dev, peaks, peak_src) if (rank == 0 and not args.skip_optim) else None
+    blockr = run_block7b(args, q, torch, dev, peaks, peak_src) if (rank == 0 and not args.skip_block) else None
     del layers, ws, grads, flush
     stack = run_stack65b(args, q, torch, dev, peaks, peak_src) if (rank == 0 and not args.skip_stack) else None
 
@@ -314,10 +315,13 @@ def run_ours(args, rank, world, local_rank):
         line["decode65b"] = decode
     if adamw is not None:
         line["adamw7b"] = adamw
+    if blockr is not None:
+        line["block7b"] = blockr
     if stack is not None:
         line["stack65b"] = stack
     if world == 1 and not args.skip_cpu:
         line["cpu_baseline"] = cpu_baseline_linear(budget_s=args.cpu_seconds)
+        line["cpu_baseline_tiny"] = cpu_baseline_tiny()
     return line
 
 
@@ -413,6 +417,7 @@ def run_codec(args, q, torch, dev, peaks, peak_src):
     ach = qgbs if dom == "quantize" else dgbs
     peak = peaks["hbm_gbs"]
     del g
+    cpu = None if args.skip_cpu else cpu_baseline_codec(q, torch, tensors)
     return {
         "workload": "codec7b: NF4+DQ quantize->dequantize round trip, 224 LLaMA-7B tensors, "
                     f"{nweights} bf16 weights ~N(0,0.02), one CUDA graph per step",
@@ -431,6 +436,7 @@ def run_codec(args, q, torch, dev, peaks, peak_src):
                     "note": "quantize_ms / dequantize_ms: each API call bracketed by CUDA events on one stream "
                             "(quantize = workspace reset + first-level pass + double quantization); "
                             "per_kernel_ms_bracketed: every kernel bracketed separately (no overlap)"},
+        "cpu_baseline": cpu,
     }
 
 
@@ -462,6 +468,10 @@ def run_decode65b(args, q, torch, dev, peaks, peak_src):
     scale = ALPHA / R
     out = {"workload": "decode65b: forward of the 7 LLaMA-65B linears (8192x8192 x4, 22016x8192 x2, 8192x22016), "
                        "r=64, bf16 activations, tokens 1/4/16", "unit": "GB/s", "tokens": {}}
+    if not args.skip_cpu:
+        L0 = layers[0]
+        X1 = synthetic.normal((1, L0["K"]), 1.0, 70_301, torch.bfloat16, dev)
+        out["cpu_baseline"] = cpu_baseline_decode(q, torch, L0["w"], X1, L0["A"], L0["B"], 1)
     for M in (1, 4, 16):
         ws = torch.empty(max(q.qlora_linear_workspace_bytes(M, L["N"], L["K"], R) for L in layers),
                          dtype=torch.uint8, device=dev)
@@ -594,6 +604,7 @@ def run_stack65b(args, q, torch, dev, peaks, peak_src, layers_n=None, tokens=204
                      "peak_source": f"{peak_src} bf16_tflops_sustained"},
         "gpu_launches_per_step": (q.qlora_launch_count() - launches0) // steps,
         "clocks": clk.summary(),
+        "cpu_baseline": None if args.skip_cpu else cpu_baseline_stack(),
     }
 
 
@@ -666,6 +677,83 @@ def run_adamw7b(args, q, torch, dev, peaks, peak_src):
     }
 
 
+def run_block7b(args, q, torch, dev, peaks, peak_src, batch=8, seq=512):
+    """One LLaMA-7B transformer block (hidden 4096, 32 heads of 128, inter
+    11008) with QLoRA adapters (r = 64, alpha = 16) on all seven linears, at
+    4096 tokens (8 x 512): the forward pass (checkpointed: only the output is
+    kept) and the backward pass (recompute, then gradients of x and of the 14
+    adapter matrices).  FLOP are counted as the model's: every linear's
+    4MNK + 6Mr(N+K) and the attention products 12 B H S^2 D (dense count);
+    the recomputed forward is extra work the count leaves out."""
+    import synthetic
+    hidden, heads, inter = 4096, 32, 11008
+    case = synthetic.block_case(batch, seq, hidden, heads, inter, R, ALPHA, seed=95_000, device=dev)
+    weights = []
+    qws = torch.empty(q.qlora_quantize_workspace_bytes(inter, hidden), dtype=torch.uint8, device=dev)
+    for W in case["W"]:
+        w = q.NF4Weight(*W.shape, device=dev)
+        q.qlora_quantize_nf4_dq(W, w, qws)
+        weights.append(w)
+    del qws, case["W"]
+    blk = q.Block(batch, seq, hidden, heads, inter, R, ALPHA / R, weights, case["A"], case["B"],
+                  case["norm1"], case["norm2"])
+    ws = torch.empty(q.qlora_block_workspace_bytes(blk), dtype=torch.uint8, device=dev)
+    T = batch * seq
+    x, dy = case["x"], case["dy"]
+    y = torch.empty(T, hidden, dtype=torch.bfloat16, device=dev)
+    dx = torch.empty_like(y)
+    dA = [torch.empty(R, w.cols, dtype=torch.float32, device=dev) for w in weights]
+    dB = [torch.empty(w.rows, R, dtype=torch.float32, device=dev) for w in weights]
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def step():
+        q.qlora_block_fwd(blk, x, y, ws)
+        q.qlora_block_bwd(blk, x, dy, dx, dA, dB, ws)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    q.qlora_check_device_error()
+    steps = max(1, min(args.steps, 10))
+    total = 0.0
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for _ in range(steps):
+            flush.zero_()
+            torch.cuda.synchronize()
+            torch.cuda._sleep(20_000_000)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            step()
+            e1.record()
+            torch.cuda.synchronize()
+            total += e0.elapsed_time(e1)
+    q.qlora_check_device_error()
+    ms = total / steps
+    lin = sum(linear_flops(T, w.rows, w.cols, R) for w in weights)
+    att = 12 * batch * heads * seq * seq * (hidden // heads)
+    recompute = sum(2 * T * w.rows * w.cols + 2 * T * R * (w.rows + w.cols) for w in weights[:6]) + att // 3
+    model = lin + att
+    value = model / (ms * 1e-3) / 1e12
+    # per-kind device time of one step, every launch bracketed by events
+    q.qlora_timing_reset()
+    q.qlora_timing_enable(True)
+    step()
+    q.qlora_timing_enable(False)
+    kern = q.qlora_timing_read()
+    return {
+        "workload": f"block7b: one LLaMA-7B block (QLoRA on q,k,v,o,gate,up,down; RMSNorm, RoPE, causal attention, "
+                    f"SwiGLU), checkpointed forward + backward, {T} tokens ({batch}x{seq}), r=64, alpha=16",
+        "value": round(value, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 4),
+        "model_flop_per_step": model, "hardware_flop_per_step": model + recompute,
+        "hardware_tflops": round((model + recompute) / (ms * 1e-3) / 1e12, 2),
+        "roofline": {"bound": "tensor", "achieved": round(value, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(value / peaks["bf16_tflops"], 4), "traffic": None,
+                     "peak_source": f"{peak_src} bf16_tflops (burst); achieved counts model FLOP"},
+        "kernels_ms_bracketed": {k: round(v[0], 4) for k, v in kern.items() if v[1]},
+        "clocks": clk.summary(),
+    }
+
+
 # ---- CPU baselines (the oracle, as it stands) ---------------------------------------
 
 def _blas_threads():
@@ -707,6 +795,127 @@ def cpu_baseline_linear(budget_s=15.0):
             "kind": "oracle",
             "sample": f"oracle float64 fwd+bwd of one 4096x4096 linear (r=64), token batches up to {M}, "
                       f"{spent:.1f} s of host time"}
+
+
+def _omp_threads():
+    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+
+def cpu_baseline_codec(q, torch, tensors, budget_s=10.0):
+    """Oracle codec (C loops, OpenMP) on the host: quantize + dequantize of
+    one tensor of each LLaMA-7B shape in the round trip, inputs copied from
+    the device, outputs compared bit for bit with the device's."""
+    import numpy as np
+
+    from oracle import codebook as ocb
+    from oracle import codec as occ
+    Q = ocb.nf4_codebook()
+    seen, spent, nweights, exact = set(), 0.0, 0, True
+    for W, w, out in tensors:
+        shape = tuple(W.shape)
+        if shape in seen or spent > budget_s:
+            continue
+        seen.add(shape)
+        Wh = W.float().cpu().numpy()
+        t0 = time.perf_counter()
+        ref = occ.quantize(Wh, Q)
+        deq = occ.dequantize(ref["packed"], ref["e"], ref["c2"], ref["mean"], Q)
+        spent += time.perf_counter() - t0
+        nweights += Wh.size
+        exact &= bool(np.array_equal(w.packed.cpu().numpy(), ref["packed"]))
+        exact &= bool(np.array_equal(w.code2.cpu().numpy(), ref["e"]))
+        exact &= bool(np.array_equal(out.view(torch.int16).cpu().numpy().view(np.uint16).ravel(), deq))
+    return {"value": round(2 * CODEC_BYTES_PER_WEIGHT * nweights / spent / 1e9, 3), "unit": "GB/s",
+            "cores": _omp_threads(), "kind": "oracle", "bit_exact_vs_device": exact,
+            "sample": f"oracle quantize + dequantize of one tensor of each shape {sorted(seen)} "
+                      f"({nweights} weights, {spent:.1f} s of host time)"}
+
+
+def cpu_baseline_decode(q, torch, w, X, A, B, M):
+    """Oracle decode forward of one LLaMA-65B 8192x8192 linear at M tokens:
+    dequantize (C loops) then the float64 layer (numpy)."""
+    import numpy as np
+
+    from oracle import codec as occ
+    from oracle import linear as olin
+    Q = np.asarray(w.codebook, np.float32)
+    packed, e, c2 = w.packed.cpu().numpy(), w.code2.cpu().numpy(), w.c2.cpu().numpy()
+    mean = np.float32(w.mean[0].item())
+    Xh, Ah, Bh = (t.float().cpu().numpy().astype(np.float64) for t in (X, A, B))
+    t0 = time.perf_counter()
+    Wd = occ.bf16_bits_to_f32(occ.dequantize(packed, e, c2, mean, Q)).reshape(w.rows, w.cols).astype(np.float64)
+    olin.forward(Xh, Wd, Ah, Bh, ALPHA / R)
+    dt = time.perf_counter() - t0
+    nbytes = weight_bytes(w.rows, w.cols) + 2 * R * (w.rows + w.cols) + 2 * M * (w.rows + w.cols)
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"oracle dequantize + float64 forward of one 8192x8192 linear at {M} token(s), "
+                      f"{dt:.2f} s of host time"}
+
+
+def cpu_baseline_stack(budget_s=10.0):
+    """Oracle fwd+bwd of one LLaMA-65B 8192x8192 linear (r = 64) on a token
+    sample of the stack's 2048 tokens; TFLOP/s, the rate one stack layer
+    would run at."""
+    import numpy as np
+
+    import synthetic
+    from oracle import linear as olin
+    N = K = 8192
+    case = synthetic.linear_case(16, N, K, R, ALPHA, seed=8)
+    Wd = case["W"].float().numpy().astype(np.float64)   # stands for the dequantized bf16 weight
+    A, B = case["A"].float().numpy(), case["B"].float().numpy()
+    rng = np.random.default_rng(1)
+    M, spent, flops = 32, 0.0, 0.0
+    while spent < budget_s:
+        X, dY = rng.standard_normal((M, K)), rng.standard_normal((M, N))
+        t0 = time.perf_counter()
+        olin.forward(X, Wd, A, B, ALPHA / R)
+        olin.backward(X, Wd, A, B, ALPHA / R, dY)
+        dt = time.perf_counter() - t0
+        spent += dt
+        flops += linear_flops(M, N, K, R)
+        if dt < budget_s / 8 and M < 2048:
+            M *= 2
+    return {"value": round(flops / spent / 1e12, 5), "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"oracle float64 fwd+bwd of one 8192x8192 linear (r=64), token batches up to {M} of 2048, "
+                      f"{spent:.1f} s of host time"}
+
+
+def cpu_baseline_tiny():
+    """Oracle on the tiny configuration (W 256x256, 16 tokens, r = 8): codec
+    and linear fwd+bwd, timed on one core and on all cores."""
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+
+    import synthetic
+    from oracle import codebook as ocb
+    from oracle import codec as occ
+    from oracle import linear as olin
+    c = synthetic.tiny_linear(seed=0)
+    Q = ocb.nf4_codebook()
+    W = c["W"].numpy()
+    X, A, B, dY = (c[k].float().numpy().astype(np.float64) for k in ("X", "A", "B", "dY"))
+
+    def once():
+        ref = occ.quantize(W, Q)
+        Wd = occ.bf16_bits_to_f32(occ.dequantize(ref["packed"], ref["e"], ref["c2"], ref["mean"], Q))
+        Wd = Wd.reshape(W.shape).astype(np.float64)
+        olin.forward(X, Wd, A, B, c["scale"])
+        olin.backward(X, Wd, A, B, c["scale"], dY)
+
+    out = {}
+    for label, n in (("1_core", 1), ("all_cores", _blas_threads())):
+        with threadpool_limits(limits=n):
+            os.environ["OMP_NUM_THREADS"] = str(n)
+            once()
+            reps, t0 = 0, time.perf_counter()
+            while time.perf_counter() - t0 < 1.0:
+                once()
+                reps += 1
+            out[label] = {"ms_per_call": round((time.perf_counter() - t0) / reps * 1e3, 3), "cores": n}
+    os.environ.pop("OMP_NUM_THREADS", None)
+    return {"kind": "oracle", "unit": "ms per quantize + dequantize + linear fwd+bwd", **out,
+            "sample": "the whole tiny configuration, repeated for 1 s"}
 
 
 def run_reference(args, rank, world):
@@ -804,6 +1013,8 @@ def main():
     ap.add_argument("--skip-decode", action="store_true")
     ap.add_argument("--skip-stack", action="store_true")
     ap.add_argument("--skip-optim", action="store_true")
+    ap.add_argument("--skip-block", action="store_true")
+    ap.add_argument("--block-only", action="store_true", help="run only the transformer-block object (profiling runs)")
     ap.add_argument("--optim-only", action="store_true", help="run only the paged AdamW object (profiling runs)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--linears", default="llama7b",
@@ -838,6 +1049,11 @@ def main():
             import bit_nf4_quantized_16_b200 as q
             torch.cuda.set_device(local_rank)
             line = {"impl": "ours", "codec_shape": run_codec_shape(args, q, torch, torch.device("cuda", local_rank))}
+        elif args.block_only:
+            import bit_nf4_quantized_16_b200 as q
+            torch.cuda.set_device(local_rank)
+            peaks, src = load_peaks()
+            line = {"impl": "ours", "block7b": run_block7b(args, q, torch, torch.device("cuda", local_rank), peaks, src)}
         elif args.optim_only:
             import bit_nf4_quantized_16_b200 as q
             torch.cuda.set_device(local_rank)

@@ -37,10 +37,11 @@ EXPORTS = (
     "qlora_timing_enable", "qlora_timing_reset", "qlora_timing_read", "qlora_launch_count",
     "qlora_debug_inject_stall",
     "qlora_paged_alloc", "qlora_paged_free", "qlora_paged_prefetch", "qlora_adamw_step",
+    "qlora_block_workspace_bytes", "qlora_block_fwd", "qlora_block_bwd",
 )
 
 KERNEL_KINDS = ("quantize", "dq_encode", "dequantize", "fwd_fused", "bwd_fused", "lowrank", "wgrad",
-                "elementwise", "optimizer")
+                "elementwise", "optimizer", "block", "attention")
 
 
 class QLoraError(RuntimeError):
@@ -61,6 +62,14 @@ class qlora_nf4_weight(ctypes.Structure):
         ("c2", ctypes.c_void_p), ("mean", ctypes.c_void_p),
         ("codebook", ctypes.c_float * 16),
     ]
+
+
+class qlora_block(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("seq", ctypes.c_int32), ("hidden", ctypes.c_int32),
+                ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("inter", ctypes.c_int32),
+                ("r", ctypes.c_int32), ("lora_scale", ctypes.c_float), ("rms_eps", ctypes.c_float),
+                ("rope_base", ctypes.c_float), ("w", qlora_nf4_weight * 7), ("A", ctypes.c_void_p * 7),
+                ("B", ctypes.c_void_p * 7), ("norm1", ctypes.c_void_p), ("norm2", ctypes.c_void_p)]
 
 
 def _load():
@@ -92,6 +101,9 @@ def _load():
         "qlora_paged_free": (ctypes.c_int, [P]),
         "qlora_paged_prefetch": (ctypes.c_int, [P, S, ctypes.c_int, P]),
         "qlora_adamw_step": (ctypes.c_int, [P, P, P, P, P, I64, ctypes.POINTER(qlora_adamw_hparams), P]),
+        "qlora_block_workspace_bytes": (S, [ctypes.POINTER(qlora_block)]),
+        "qlora_block_fwd": (ctypes.c_int, [ctypes.POINTER(qlora_block), P, P, P, S, P]),
+        "qlora_block_bwd": (ctypes.c_int, [ctypes.POINTER(qlora_block), P, P, P, P, P, P, S, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -303,3 +315,41 @@ def qlora_adamw_step(param, param_bf16, grad, exp_avg, exp_avg_sq, lr, beta1, be
     _check(lib.qlora_adamw_step(_ptr(param), _ptr(param_bf16), _ptr(grad), _ptr(exp_avg), _ptr(exp_avg_sq),
                                 param.numel(), ctypes.byref(h), _stream(stream)),
            "qlora_adamw_step")
+
+
+# ---- transformer block ------------------------------------------------------------------
+
+BLOCK_LINEARS = ("q", "k", "v", "o", "gate", "up", "down")
+
+
+class Block:
+    """Descriptor of one QLoRA transformer block: the seven quantized weights
+    (NF4Weight, in the order of BLOCK_LINEARS), their bf16 adapters A [r][in],
+    B [out][r], and the two bf16 norm weights, all device tensors kept alive
+    by this object."""
+
+    def __init__(self, batch, seq, hidden, heads, inter, r, lora_scale, weights, A, B, norm1, norm2,
+                 rms_eps=1e-6, rope_base=10000.0):
+        self.weights, self.A, self.B, self.norm1, self.norm2 = list(weights), list(A), list(B), norm1, norm2
+        self.desc = qlora_block(batch, seq, hidden, heads, hidden // heads, inter, r, lora_scale, rms_eps,
+                                rope_base, (qlora_nf4_weight * 7)(*[w.desc for w in self.weights]),
+                                (ctypes.c_void_p * 7)(*[a.data_ptr() for a in self.A]),
+                                (ctypes.c_void_p * 7)(*[b.data_ptr() for b in self.B]),
+                                norm1.data_ptr(), norm2.data_ptr())
+
+
+def qlora_block_workspace_bytes(block: Block) -> int:
+    return lib.qlora_block_workspace_bytes(ctypes.byref(block.desc))
+
+
+def qlora_block_fwd(block: Block, x, y, workspace, stream=None):
+    _check(lib.qlora_block_fwd(ctypes.byref(block.desc), _ptr(x), _ptr(y), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), _stream(stream)), "qlora_block_fwd")
+
+
+def qlora_block_bwd(block: Block, x, dy, dx, dA, dB, workspace, stream=None):
+    pa = (ctypes.c_void_p * 7)(*[t.data_ptr() for t in dA])
+    pb = (ctypes.c_void_p * 7)(*[t.data_ptr() for t in dB])
+    _check(lib.qlora_block_bwd(ctypes.byref(block.desc), _ptr(x), _ptr(dy), _ptr(dx),
+                               ctypes.cast(pa, ctypes.c_void_p), ctypes.cast(pb, ctypes.c_void_p), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), _stream(stream)), "qlora_block_bwd")

@@ -46,8 +46,11 @@ namespace qlora {
 enum BMode : int { kBTmaK = 0, kBTmaMN = 1, kBNf4K = 2, kBNf4MN = 3 };
 // Epilogues: kEpiBf16 stores the tile as bf16; kEpiF32 stores it as fp32,
 // into plane `split` of a stack of partial products when the contraction is
-// split (out + split * split_stride).
-enum Epi : int { kEpiBf16 = 0, kEpiF32 = 1 };
+// split (out + split * split_stride).  kEpiDropBf16 / kEpiDropF32 store
+// drop_base + (kept ? drop_scale * acc : 0) (the adapter term of the input
+// gradient under LoRA dropout, added to the frozen path's fp32 product; the
+// mask holds bit c % 8 of byte (row * out_ld + c) / 8 per element).
+enum Epi : int { kEpiBf16 = 0, kEpiF32 = 1, kEpiDropBf16 = 2, kEpiDropF32 = 3 };
 
 struct GemmParams {
     CUtensorMap tm_a;    // main A operand
@@ -74,6 +77,9 @@ struct GemmParams {
     int64_t out_ld;
     int m_total, n_total;
     int64_t split_stride;  // elements between split planes (partial products)
+    const uint8_t *drop_mask;  // kEpiDrop*: kept-input bit mask, [rows][out_ld / 8]
+    const float *drop_base;    // kEpiDrop*: fp32 [rows][out_ld] added to the scaled tile
+    float drop_scale;          // kEpiDrop*: 1 / (1 - p)
     int *err;            // device error word
     uint64_t timeout_ns; // limit of every pipeline wait
     uint64_t drain_ns;   // limit of the waits for copies and MMAs already in flight after an abort
@@ -336,6 +342,41 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode, MT>::kThreads, 1)
                             v.z = pack_bf16x2(__uint_as_float(r[8 * g + 4]), __uint_as_float(r[8 * g + 5]));
                             v.w = pack_bf16x2(__uint_as_float(r[8 * g + 6]), __uint_as_float(r[8 * g + 7]));
                             *reinterpret_cast<uint4 *>(o + 8 * g) = v;
+                        }
+                    } else if (kEpi == kEpiDropBf16 || kEpi == kEpiDropF32) {
+                        // out_ld % 32 == 0 and col0 % 32 == 0: the 32 mask bits of this
+                        // chunk are one aligned 32-bit word; n_total % 32 == 0
+                        if (col0 >= p.n_total) continue;
+                        const int64_t flat = (int64_t)row * p.out_ld + col0;
+                        const uint32_t bits = *reinterpret_cast<const uint32_t *>(p.drop_mask + flat / 8);
+                        float v[32];
+#pragma unroll
+                        for (int g = 0; g < 8; g++) {
+                            const float4 b4 = *reinterpret_cast<const float4 *>(p.drop_base + flat + 4 * g);
+                            const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+                            for (int i = 0; i < 4; i++) {
+                                const int c = 4 * g + i;
+                                const float t = ((bits >> c) & 1u) ? __fmul_rn(p.drop_scale, __uint_as_float(r[c])) : 0.0f;
+                                v[c] = __fadd_rn(bb[i], t);
+                            }
+                        }
+                        if (kEpi == kEpiDropBf16) {
+                            __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.out) + flat;
+#pragma unroll
+                            for (int g = 0; g < 4; g++) {
+                                uint4 w;
+                                w.x = pack_bf16x2(v[8 * g + 0], v[8 * g + 1]);
+                                w.y = pack_bf16x2(v[8 * g + 2], v[8 * g + 3]);
+                                w.z = pack_bf16x2(v[8 * g + 4], v[8 * g + 5]);
+                                w.w = pack_bf16x2(v[8 * g + 6], v[8 * g + 7]);
+                                *reinterpret_cast<uint4 *>(o + 8 * g) = w;
+                            }
+                        } else {
+                            float *o = static_cast<float *>(p.out) + flat;
+#pragma unroll
+                            for (int g = 0; g < 8; g++)
+                                *reinterpret_cast<float4 *>(o + 4 * g) = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
                         }
                     } else {
                         float *o = static_cast<float *>(p.out) + (int64_t)sp * p.split_stride + (int64_t)row * p.out_ld + col0;

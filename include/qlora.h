@@ -338,6 +338,65 @@ typedef struct {
 QLORA_API qlora_status qlora_adamw_step(float *param, void *param_bf16, const float *grad, float *exp_avg,
                                         float *exp_avg_sq, int64_t n, const qlora_adamw_hparams *h, void *stream);
 
+/*
+ * One QLoRA transformer block ("QLoRA: Efficient Finetuning of Quantized
+ * LLMs", Introduction: LoRA adapters at every network layer, trained with
+ * gradient checkpointing).  The pages fix the seven linear shapes of the
+ * LLaMA models but not the rest of the block; it is the LLaMA decoder layer:
+ *     u1 = RMSNorm(x; norm1); q, k, v = Lq(u1), Lk(u1), Lv(u1)
+ *     q, k rotated (RoPE: pairs (i, i + D/2) of each head by p * base^(-2i/D)
+ *     at sequence position p)
+ *     a = causal softmax(q k^T / sqrt(D)) v per sequence and head
+ *     h = x + Lo(a);  u2 = RMSNorm(h; norm2)
+ *     y = h + Ldown(silu(Lgate(u2)) * Lup(u2))
+ * with RMSNorm(x; g) = x / sqrt(mean(x^2) + eps) * g.  Every L is the QLoRA
+ * linear of qlora_linear_fwd (frozen NF4 + DQ weight, adapters A, B, scale
+ * lora_scale).  Activations are bf16 [batch * seq, hidden], row = b * seq + p.
+ *   w[7], A[7], B[7]  in the order q, k, v, o, gate, up, down; w[l] as for
+ *                     qlora_linear_fwd, A[l] device bf16 [r][in], B[l] device
+ *                     bf16 [out][r].
+ *   norm1, norm2      device bf16 [hidden] (frozen).
+ * Constraints: heads * head_dim == hidden, head_dim % 8 == 0, hidden % 64 ==
+ * 0, inter % 64 == 0, seq % 8 == 0, r as for the linear layer.
+ */
+typedef struct {
+    int32_t batch, seq, hidden, heads, head_dim, inter, r;
+    float lora_scale;
+    float rms_eps;
+    float rope_base;
+    qlora_nf4_weight w[7];
+    const void *A[7];
+    const void *B[7];
+    const void *norm1;
+    const void *norm2;
+} qlora_block;
+
+/* Workspace bytes of qlora_block_fwd / qlora_block_bwd (0 for an invalid
+ * description). */
+QLORA_API size_t qlora_block_workspace_bytes(const qlora_block *blk);
+
+/*
+ * qlora_block_fwd -- y = block(x).  Keeps nothing else (gradient
+ * checkpointing: the backward pass recomputes what it needs from x).
+ *   x, y       device bf16 [batch * seq, hidden].
+ *   workspace  device, >= qlora_block_workspace_bytes(blk).
+ * Errors: INVALID_ARG, SHAPE, ALIGNMENT, WORKSPACE, CUDA, UNSUPPORTED.
+ */
+QLORA_API qlora_status qlora_block_fwd(const qlora_block *blk, const void *x, void *y, void *workspace,
+                                       size_t workspace_bytes, void *stream);
+
+/*
+ * qlora_block_bwd -- gradients of the block for dy = dL/dy: recomputes the
+ * forward pass from x, then returns dx and the adapter gradients of all seven
+ * linears (the quantized weights and the norm weights are frozen).
+ *   dy, dx     device bf16 [batch * seq, hidden].
+ *   dA[l], dB[l]  device float [r][in] and [out][r], overwritten.
+ * Errors: INVALID_ARG, SHAPE, ALIGNMENT, WORKSPACE, CUDA, UNSUPPORTED.
+ */
+QLORA_API qlora_status qlora_block_bwd(const qlora_block *blk, const void *x, const void *dy, void *dx,
+                                       float *const dA[7], float *const dB[7], void *workspace,
+                                       size_t workspace_bytes, void *stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 QLORA_API const char *qlora_status_string(qlora_status status);
 
@@ -370,7 +429,9 @@ enum {
     QLORA_KERNEL_WGRAD = 6,       /* dA and dB products                  */
     QLORA_KERNEL_ELEMENTWISE = 7, /* split-sum / hi-lo finalize kernels  */
     QLORA_KERNEL_OPTIMIZER = 8,   /* AdamW update of the adapters        */
-    QLORA_NUM_KERNELS = 9
+    QLORA_KERNEL_BLOCK = 9,       /* block norms, RoPE, SwiGLU           */
+    QLORA_KERNEL_ATTENTION = 10,  /* block attention products, softmax   */
+    QLORA_NUM_KERNELS = 11
 };
 QLORA_API qlora_status qlora_timing_enable(int enable);
 QLORA_API qlora_status qlora_timing_reset(void);

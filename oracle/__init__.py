@@ -19,6 +19,7 @@ Modules
             driven from Python).
   linear    QLoRA linear forward and backward in float64 (numpy).
   optim     AdamW update of the adapters in float64 (the paged optimizer).
+  block     one LLaMA-layout QLoRA transformer block, forward and backward, float64.
 
 Parity status: every function has a pin in tests/test_oracle_*.py except the
 individual NF4 codebook values beyond the structural invariants, and the
@@ -26,4 +27,4 @@ claim that every bin holds the same expected share of values, which the
 pages make but never back with numbers ("parity unpinned" for those two).
 """
 
-from . import codebook, exact, codec, linear, optim  # noqa: F401
+from . import codebook, exact, codec, linear, optim, block  # noqa: F401

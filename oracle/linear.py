@@ -64,6 +64,49 @@ def backward_weight_grads(X, A, B, s: float, dY):
     return s * (G.T @ X), s * (dY.T @ (X @ A.T))
 
 
+# ---- LoRA dropout on the adapter input ------------------------------------------------
+#
+# The blog's LoraConfig snippet ("Efficient Language Model Fine-Tuning with
+# QLoRA on Resource-Constrained Hardware", marciocunha.net) sets lora_dropout:
+# the adapter branch sees X_d = X * mask / (1 - p) while the frozen base sees
+# X.  With bf16 activations the dropped-out input is itself bf16: each kept
+# element is RN_bf16(RN32(x * RN32(1 / (1 - p)))), each dropped one 0.  The
+# gradient through the dropout is mask / (1 - p) (the rounding is a storage
+# step, not part of the function being differentiated):
+#   Y  = X W'^T + s (X_d A^T) B^T
+#   dX = dY W' + (s (dY B) A) * mask / (1 - p)
+#   dA = s (dY B)^T X_d,   dB = s dY^T (X_d A^T)
+
+def dropout_scale(p: float) -> np.float32:
+    return np.float32(1.0 / np.float64(np.float32(1.0) - np.float32(p))) if p > 0 else np.float32(1.0)
+
+
+def dropout_input(X, mask, p: float, bf16_round=True) -> np.ndarray:
+    """X_d: kept elements scaled by RN32(1/(1-p)) (and rounded to bf16), the
+    others 0.  mask: bool [M, K], True = kept."""
+    X = np.asarray(X, np.float32)
+    sc = dropout_scale(p)
+    v = (X * sc).astype(np.float32)
+    if bf16_round:
+        b = v.view(np.uint32).astype(np.uint64)
+        b = (b + 0x7FFF + ((b >> 16) & 1)) & 0xFFFF0000      # round to nearest even, to bf16
+        v = b.astype(np.uint32).view(np.float32)
+    return np.where(mask, v, np.float32(0.0)).astype(np.float64)
+
+
+def forward_dropout(X, Wd, A, B, s: float, Xd) -> np.ndarray:
+    X, Wd, A, B, Xd = map(_f64, (X, Wd, A, B, Xd))
+    return X @ Wd.T + s * ((Xd @ A.T) @ B.T)
+
+
+def backward_dropout(X, Wd, A, B, s: float, dY, Xd, mask, p: float):
+    """(dX, dA, dB) of forward_dropout."""
+    X, Wd, A, B, dY, Xd = map(_f64, (X, Wd, A, B, dY, Xd))
+    G = dY @ B
+    dX = dY @ Wd + s * (G @ A) * (np.asarray(mask, bool) * np.float64(dropout_scale(p)))
+    return dX, s * (G.T @ Xd), s * (dY.T @ (Xd @ A.T))
+
+
 def rel_frobenius(got, ref) -> float:
     got, ref = _f64(got), _f64(ref)
     den = np.linalg.norm(ref)

@@ -50,3 +50,25 @@ def linear_case(M: int, N: int, K: int, r: int, alpha: float, seed: int, w_dtype
         "dY": normal((M, N), 1.0, seed + 4, torch.bfloat16, device),
         "r": r, "alpha": alpha, "scale": alpha / r, "M": M, "N": N, "K": K,
     }
+
+
+def block_case(batch: int, seq: int, hidden: int, heads: int, inter: int, r: int, alpha: float, seed: int,
+               device="cpu") -> dict:
+    """One transformer block problem: the seven weights N(0, 0.02) in the
+    shapes (out, in) of q, k, v, o (hidden x hidden), gate, up (inter x
+    hidden), down (hidden x inter); adapters A N(0, 1/r), B N(0, 0.01); norm
+    weights 1 + N(0, 0.1); block input x and output gradient dy N(0, 1)."""
+    shapes = [(hidden, hidden)] * 4 + [(inter, hidden)] * 2 + [(hidden, inter)]
+    W = [normal(s, 0.02, seed + 10 * i, torch.bfloat16, device) for i, s in enumerate(shapes)]
+    A = [normal((r, s[1]), 1.0 / r, seed + 10 * i + 1, torch.bfloat16, device) for i, s in enumerate(shapes)]
+    B = [normal((s[0], r), 0.01, seed + 10 * i + 2, torch.bfloat16, device) for i, s in enumerate(shapes)]
+    T = batch * seq
+    return {
+        "W": W, "A": A, "B": B,
+        "norm1": (1.0 + normal((hidden,), 0.1, seed + 101)).to(torch.bfloat16).to(device),
+        "norm2": (1.0 + normal((hidden,), 0.1, seed + 102)).to(torch.bfloat16).to(device),
+        "x": normal((T, hidden), 1.0, seed + 103, torch.bfloat16, device),
+        "dy": normal((T, hidden), 1.0, seed + 104, torch.bfloat16, device),
+        "batch": batch, "seq": seq, "hidden": hidden, "heads": heads, "inter": inter, "r": r,
+        "alpha": alpha, "scale": alpha / r,
+    }

@@ -95,6 +95,60 @@ def test_weight_grad_helper_matches_full_backward():
             assert abs(gA[j, k] - ref) < 1e-10
 
 
+def test_dropout_gradients_against_finite_differences():
+    """With the unrounded dropped-out input, the backward pass is the exact
+    derivative of the forward pass in X, A and B."""
+    rng = np.random.default_rng(17)
+    M, K, N, r, s, p = 4, 8, 5, 3, 0.5, 0.25
+    X, W, A, B, dY = (_rand(rng, M, K), _rand(rng, N, K), _rand(rng, r, K), _rand(rng, N, r), _rand(rng, M, N))
+    mask = rng.random((M, K)) >= p
+    sc = np.float64(linear.dropout_scale(p))
+
+    def fwd(X_, A_, B_):
+        return linear.forward_dropout(X_, W, A_, B_, s, X_ * mask * sc)
+
+    def loss(X_, A_, B_):
+        return float(np.sum(dY * fwd(X_, A_, B_)))
+
+    dX, dA, dB = linear.backward_dropout(X, W, A, B, s, dY, X * mask * sc, mask, p)
+    h = 1e-6
+    for name, P, G in (("X", X, dX), ("A", A, dA), ("B", B, dB)):
+        for idx in np.ndindex(P.shape):
+            Pp, Pm = P.copy(), P.copy()
+            Pp[idx] += h
+            Pm[idx] -= h
+            ap = {"X": (Pp, A, B), "A": (X, Pp, B), "B": (X, A, Pp)}[name]
+            am = {"X": (Pm, A, B), "A": (X, Pm, B), "B": (X, A, Pm)}[name]
+            fd = (loss(*ap) - loss(*am)) / (2 * h)
+            assert abs(fd - G[idx]) < 1e-6 * max(1.0, abs(fd)), (name, idx)
+
+
+def test_dropout_special_cases():
+    rng = np.random.default_rng(18)
+    M, K, N, r, s = 3, 16, 6, 2, 2.0
+    X = np.clip(np.round(rng.standard_normal((M, K)) * 64) / 64, -3.9, 3.9)   # exact in bf16
+    W, A, B, dY = _rand(rng, N, K), _rand(rng, r, K), _rand(rng, N, r), _rand(rng, M, N)
+    # p = 0 with every input kept is the plain layer (scale 1: x_d = bf16(x) = x for bf16-exact x)
+    keep = np.ones((M, K), bool)
+    Xb = linear.dropout_input(X.astype(np.float32), keep, 0.0, bf16_round=False)
+    np.testing.assert_array_equal(Xb, X)
+    np.testing.assert_allclose(linear.forward_dropout(X, W, A, B, s, Xb), linear.forward(X, W, A, B, s), atol=1e-12)
+    for a, b in zip(linear.backward_dropout(X, W, A, B, s, dY, Xb, keep, 0.0), linear.backward(X, W, A, B, s, dY)):
+        np.testing.assert_allclose(a, b, atol=1e-12)
+    # everything dropped: the adapter branch vanishes
+    drop = np.zeros((M, K), bool)
+    Xd = linear.dropout_input(X.astype(np.float32), drop, 0.5)
+    np.testing.assert_allclose(linear.forward_dropout(X, W, A, B, s, Xd), X @ W.T, atol=1e-12)
+    dX, dA, dB = linear.backward_dropout(X, W, A, B, s, dY, Xd, drop, 0.5)
+    assert not dA.any() and not dB.any()
+    np.testing.assert_allclose(dX, dY @ W, atol=1e-12)
+    # the scale of p = 0.5 is exactly 2 and the bf16 rounding of x * 2 is exact
+    half = rng.random((M, K)) >= 0.5
+    np.testing.assert_array_equal(linear.dropout_input(X.astype(np.float32), half, 0.5), X * 2 * half)
+    # the scale of p = 0.05: RN32(1 / RN32(0.95))
+    assert linear.dropout_scale(0.05) == np.float32(1.0 / np.float64(np.float32(0.95)))
+
+
 def test_error_metrics():
     ref = np.array([[3.0, 4.0]])
     assert linear.rel_frobenius(ref, ref) == 0.0
