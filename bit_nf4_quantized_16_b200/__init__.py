@@ -20,6 +20,7 @@ QLORA_GROUP = 256
 QLORA_NOALLOC_MAX_BLOCKS = 1 << 20   # largest rows*cols/64 of qlora_quantize_nf4_dq_noalloc
 QLORA_BF16 = 0
 QLORA_FP32 = 1
+QLORA_FP16 = 2
 
 STATUS = {
     0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_SHAPE", 3: "QLORA_ERR_ALIGNMENT",
@@ -28,7 +29,8 @@ STATUS = {
 
 # every symbol the header declares
 EXPORTS = (
-    "qlora_build_nf4_codebook", "qlora_build_int4_codebook", "qlora_build_fp4_codebook",
+    "qlora_build_nf4_codebook", "qlora_build_nfk_codebook", "qlora_build_int4_codebook",
+    "qlora_build_fp4_codebook",
     "qlora_quantize_workspace_bytes",
     "qlora_quantize_nf4_dq",
     "qlora_quantize_nf4_dq_noalloc",
@@ -38,6 +40,8 @@ EXPORTS = (
     "qlora_debug_inject_stall",
     "qlora_paged_alloc", "qlora_paged_free", "qlora_paged_prefetch", "qlora_adamw_step",
     "qlora_block_workspace_bytes", "qlora_block_fwd", "qlora_block_bwd",
+    "qlora_linear_workspace_bytes_ex", "qlora_linear_fwd_ex", "qlora_linear_bwd_ex",
+    "qlora_dequantize_nf4_dq_ex",
 )
 
 KERNEL_KINDS = ("quantize", "dq_encode", "dequantize", "fwd_fused", "bwd_fused", "lowrank", "wgrad",
@@ -64,6 +68,10 @@ class qlora_nf4_weight(ctypes.Structure):
     ]
 
 
+class qlora_linear_opts(ctypes.Structure):
+    _fields_ = [("dropout_mask", ctypes.c_void_p), ("dropout_p", ctypes.c_float), ("compute_dtype", ctypes.c_int)]
+
+
 class qlora_block(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("seq", ctypes.c_int32), ("hidden", ctypes.c_int32),
                 ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("inter", ctypes.c_int32),
@@ -82,11 +90,13 @@ def _load():
     sig = {
         "qlora_build_nf4_codebook": (ctypes.c_int, [ctypes.c_double, P]),
         "qlora_build_int4_codebook": (ctypes.c_int, [P]),
+        "qlora_build_nfk_codebook": (ctypes.c_int, [ctypes.c_int, ctypes.c_double, P]),
         "qlora_build_fp4_codebook": (ctypes.c_int, [P]),
         "qlora_quantize_workspace_bytes": (S, [I64, I64]),
         "qlora_quantize_nf4_dq": (ctypes.c_int, [P, ctypes.c_int, W, P, S, P]),
         "qlora_quantize_nf4_dq_noalloc": (ctypes.c_int, [P, ctypes.c_int, W, P]),
         "qlora_dequantize_nf4_dq": (ctypes.c_int, [W, P, P]),
+        "qlora_dequantize_nf4_dq_ex": (ctypes.c_int, [W, P, ctypes.c_int, P]),
         "qlora_linear_workspace_bytes": (S, [I64, I64, I64, I32]),
         "qlora_linear_fwd": (ctypes.c_int, [W, P, I64, P, P, I32, F, P, ctypes.c_int, P, P, S, P]),
         "qlora_linear_bwd": (ctypes.c_int, [W, P, P, I64, P, P, I32, F, P, P, ctypes.c_int, P, P, P, S, P]),
@@ -102,6 +112,11 @@ def _load():
         "qlora_paged_prefetch": (ctypes.c_int, [P, S, ctypes.c_int, P]),
         "qlora_adamw_step": (ctypes.c_int, [P, P, P, P, P, I64, ctypes.POINTER(qlora_adamw_hparams), P]),
         "qlora_block_workspace_bytes": (S, [ctypes.POINTER(qlora_block)]),
+        "qlora_linear_workspace_bytes_ex": (S, [I64, I64, I64, I32, ctypes.POINTER(qlora_linear_opts)]),
+        "qlora_linear_fwd_ex": (ctypes.c_int, [W, P, I64, P, P, I32, F, P, ctypes.c_int, P, P, S, P,
+                                               ctypes.POINTER(qlora_linear_opts)]),
+        "qlora_linear_bwd_ex": (ctypes.c_int, [W, P, P, I64, P, P, I32, F, P, P, ctypes.c_int, P, P, P, S, P,
+                                               ctypes.POINTER(qlora_linear_opts)]),
         "qlora_block_fwd": (ctypes.c_int, [ctypes.POINTER(qlora_block), P, P, P, S, P]),
         "qlora_block_bwd": (ctypes.c_int, [ctypes.POINTER(qlora_block), P, P, P, P, P, P, S, P]),
     }
@@ -134,6 +149,8 @@ def _dtype_code(t):
         return QLORA_BF16
     if t.dtype == torch.float32:
         return QLORA_FP32
+    if t.dtype == torch.float16:
+        return QLORA_FP16
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
@@ -170,6 +187,12 @@ def qlora_build_nf4_codebook(delta: float = 0.0):
     return [float(v) for v in out]
 
 
+def qlora_build_nfk_codebook(k: int, delta: float = 0.0):
+    out = (ctypes.c_float * 16)()
+    _check(lib.qlora_build_nfk_codebook(k, delta, ctypes.cast(out, ctypes.c_void_p)), "qlora_build_nfk_codebook")
+    return [float(v) for v in out]
+
+
 def qlora_build_int4_codebook():
     out = (ctypes.c_float * 16)()
     _check(lib.qlora_build_int4_codebook(ctypes.cast(out, ctypes.c_void_p)), "qlora_build_int4_codebook")
@@ -200,31 +223,59 @@ def qlora_quantize_nf4_dq_noalloc(W: torch.Tensor, out: NF4Weight, stream=None):
            "qlora_quantize_nf4_dq_noalloc")
 
 
-def qlora_dequantize_nf4_dq(w: NF4Weight, out_bf16: torch.Tensor, stream=None):
-    _check(lib.qlora_dequantize_nf4_dq(ctypes.byref(w.desc), _ptr(out_bf16), _stream(stream)),
-           "qlora_dequantize_nf4_dq")
+def qlora_dequantize_nf4_dq(w: NF4Weight, out: torch.Tensor, stream=None):
+    """bf16 output (the default compute dtype), or fp16 when `out` is fp16."""
+    if out.dtype == torch.float16:
+        _check(lib.qlora_dequantize_nf4_dq_ex(ctypes.byref(w.desc), _ptr(out), QLORA_FP16, _stream(stream)),
+               "qlora_dequantize_nf4_dq_ex")
+    else:
+        _check(lib.qlora_dequantize_nf4_dq(ctypes.byref(w.desc), _ptr(out), _stream(stream)),
+               "qlora_dequantize_nf4_dq")
 
 
-def qlora_linear_workspace_bytes(M: int, N: int, K: int, r: int) -> int:
-    return lib.qlora_linear_workspace_bytes(M, N, K, r)
+def _opts(dropout, X):
+    """Options for the _ex calls, or None for the plain ones.  dropout: None, or
+    (mask, p) with mask a uint8 device tensor of M*K/8 bytes (bit k % 8 of byte
+    (m*K + k) / 8: element (m, k) kept); the compute dtype follows X (fp16
+    tensors select the fp16 compute dtype)."""
+    f16 = X is not None and X.dtype == torch.float16
+    if dropout is None and not f16:
+        return None
+    mask, p = dropout if dropout is not None else (None, 0.0)
+    return qlora_linear_opts(None if mask is None else mask.data_ptr(), p, QLORA_FP16 if f16 else QLORA_BF16)
+
+
+def qlora_linear_workspace_bytes(M: int, N: int, K: int, r: int, dropout=None) -> int:
+    if dropout is None:
+        return lib.qlora_linear_workspace_bytes(M, N, K, r)
+    o = qlora_linear_opts(1, 0.0, QLORA_BF16)   # only the presence of a mask matters for the size
+    return lib.qlora_linear_workspace_bytes_ex(M, N, K, r, ctypes.byref(o))
 
 
 def qlora_linear_fwd(w: NF4Weight, X, M: int, A, B, r: int, scale: float, Y, H_save=None,
-                     workspace=None, stream=None):
+                     workspace=None, stream=None, dropout=None):
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib.qlora_linear_fwd(ctypes.byref(w.desc), _ptr(X), M, _ptr(A), _ptr(B), r, scale, _ptr(Y),
-                                _dtype_code(Y), _ptr(H_save), _ptr(workspace), ws_bytes, _stream(stream)),
-           "qlora_linear_fwd")
+    args = (ctypes.byref(w.desc), _ptr(X), M, _ptr(A), _ptr(B), r, scale, _ptr(Y), _dtype_code(Y), _ptr(H_save),
+            _ptr(workspace), ws_bytes, _stream(stream))
+    opts = _opts(dropout, X)
+    if opts is None:
+        _check(lib.qlora_linear_fwd(*args), "qlora_linear_fwd")
+    else:
+        _check(lib.qlora_linear_fwd_ex(*args, ctypes.byref(opts)), "qlora_linear_fwd_ex")
 
 
 def qlora_linear_bwd(w: NF4Weight, X, dY, M: int, A, B, r: int, scale: float, H_saved, dX, dA, dB,
-                     workspace=None, stream=None):
+                     workspace=None, stream=None, dropout=None):
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    dx_code = QLORA_BF16 if dX is None else _dtype_code(dX)
-    _check(lib.qlora_linear_bwd(ctypes.byref(w.desc), _ptr(X), _ptr(dY), M, _ptr(A), _ptr(B), r, scale,
-                                _ptr(H_saved), _ptr(dX), dx_code, _ptr(dA), _ptr(dB), _ptr(workspace),
-                                ws_bytes, _stream(stream)),
-           "qlora_linear_bwd")
+    dx_code = (QLORA_FP16 if X is not None and X.dtype == torch.float16 else QLORA_BF16) if dX is None \
+        else _dtype_code(dX)
+    args = (ctypes.byref(w.desc), _ptr(X), _ptr(dY), M, _ptr(A), _ptr(B), r, scale, _ptr(H_saved), _ptr(dX),
+            dx_code, _ptr(dA), _ptr(dB), _ptr(workspace), ws_bytes, _stream(stream))
+    opts = _opts(dropout, X)
+    if opts is None:
+        _check(lib.qlora_linear_bwd(*args), "qlora_linear_bwd")
+    else:
+        _check(lib.qlora_linear_bwd_ex(*args, ctypes.byref(opts)), "qlora_linear_bwd_ex")
 
 
 def qlora_status_string(status: int) -> str:

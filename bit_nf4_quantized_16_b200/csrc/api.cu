@@ -160,36 +160,61 @@ static double ppnd16(double p)
 
 using namespace qlora;
 
-// NF4 construction ("QLoRA: Efficient Finetuning of Quantized LLMs", section
-// "Method", paragraph "4-bit NormalFloat Quantization"): 2^(k-1)+1 = 9
-// quantiles for the positive part and 2^(k-1) = 8 for the negative part,
-// probabilities equally spaced from 1 - delta to 1/2, union without the
-// duplicate zero, normalized by the largest magnitude into [-1, 1].
-extern "C" qlora_status qlora_build_nf4_codebook(double delta, float codebook_out[16])
+// NF-k construction ("QLoRA: Efficient Finetuning of Quantized LLMs", section
+// "Method", paragraph "4-bit NormalFloat Quantization"): 2^(k-1)+1 quantiles
+// for the positive part and 2^(k-1) for the negative part, probabilities
+// equally spaced from 1 - delta to 1/2, union without the duplicate zero,
+// normalized by the largest magnitude into [-1, 1]; v receives the 2^k
+// values ascending.
+static void nfk_values(int k, double delta, double *v)
 {
-    if (!codebook_out) return QLORA_ERR_INVALID_ARG;
-    if (delta <= 0.0) delta = 0.5 * (1.0 / 32.0 + 1.0 / 30.0);
-    if (!(delta < 0.5)) return QLORA_ERR_INVALID_ARG;
     const double hi = 1.0 - delta;
     const double top = ppnd16(hi);
-    double v[16];
+    const int npos = (1 << (k - 1)) + 1, nneg = 1 << (k - 1);
     int n = 0;
-    for (int i = 0; i < 9; i++) {        // positive part, zero included
-        double p = i < 8 ? hi + (0.5 - hi) * i / 8.0 : 0.5;
-        v[n++] = (i < 8 ? ppnd16(p) : 0.0) / top;
+    for (int i = 0; i < npos; i++) {     // positive part, zero included
+        double p = i < npos - 1 ? hi + (0.5 - hi) * i / (double)(npos - 1) : 0.5;
+        v[n++] = (i < npos - 1 ? ppnd16(p) : 0.0) / top;
     }
-    for (int i = 0; i < 7; i++) {        // negative part; its zero is the dropped duplicate
-        double p = hi + (0.5 - hi) * i / 7.0;
+    for (int i = 0; i < nneg - 1; i++) {  // negative part; its zero is the dropped duplicate
+        double p = hi + (0.5 - hi) * i / (double)(nneg - 1);
         v[n++] = -ppnd16(p) / top;
     }
-    // ascending order
-    for (int i = 1; i < 16; i++)
+    for (int i = 1; i < n; i++)           // ascending order
         for (int j = i; j > 0 && v[j - 1] > v[j]; j--) {
             double t = v[j];
             v[j] = v[j - 1];
             v[j - 1] = t;
         }
+}
+
+extern "C" qlora_status qlora_build_nf4_codebook(double delta, float codebook_out[16])
+{
+    if (!codebook_out) return QLORA_ERR_INVALID_ARG;
+    if (delta <= 0.0) delta = 0.5 * (1.0 / 32.0 + 1.0 / 30.0);
+    if (!(delta < 0.5)) return QLORA_ERR_INVALID_ARG;
+    double v[16];
+    nfk_values(4, delta, v);
     for (int i = 0; i < 16; i++) codebook_out[i] = (float)v[i];
+    return QLORA_OK;
+}
+
+// NF-k for k = 2, 3, 4 in the 16-entry table of the 4-bit codec: the 2^k
+// values, and 16 - 2^k padding values beyond +-1 (half at -1 - i/4 below,
+// half at 1 + i/4 above), never the nearest value of anything in [-1, 1].
+// Default delta: 1/2 (1/(2 * 2^k) + 1/(2 (2^k - 1))).
+extern "C" qlora_status qlora_build_nfk_codebook(int k, double delta, float codebook_out[16])
+{
+    if (!codebook_out || k < 2 || k > 4) return QLORA_ERR_INVALID_ARG;
+    const int n = 1 << k;
+    if (delta <= 0.0) delta = 0.5 * (1.0 / (2.0 * n) + 1.0 / (2.0 * (n - 1)));
+    if (!(delta < 0.5)) return QLORA_ERR_INVALID_ARG;
+    double v[16];
+    nfk_values(k, delta, v);
+    const int half = (16 - n) / 2;
+    for (int i = 0; i < half; i++) codebook_out[i] = (float)(-1.0 - (half - i) / 4.0);
+    for (int i = 0; i < n; i++) codebook_out[half + i] = (float)v[i];
+    for (int i = 0; i < half; i++) codebook_out[half + n + i] = (float)(1.0 + (i + 1) / 4.0);
     return QLORA_OK;
 }
 

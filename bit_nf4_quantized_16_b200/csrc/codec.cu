@@ -138,13 +138,17 @@ __device__ __forceinline__ uint32_t add_code(const uint32_t *lut, float n, uint3
     return acc | (part & (0xFu << (4 * I)));
 }
 
-// Magnitude maximum of two bf16 pairs, lane by lane (max.xorsign.abs: the
-// result's magnitude is max(|a|, |b|); its sign bit is meaningless and masked
-// off by the caller).
-__device__ __forceinline__ uint32_t maxabs_bf16x2(uint32_t a, uint32_t b)
+// Magnitude maximum of two bf16 (F16: fp16) pairs, lane by lane
+// (max.xorsign.abs: the result's magnitude is max(|a|, |b|); its sign bit is
+// meaningless and masked off by the caller).
+template <bool F16>
+__device__ __forceinline__ uint32_t maxabs16x2(uint32_t a, uint32_t b)
 {
     uint32_t d;
-    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    if constexpr (F16)
+        asm("max.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    else
+        asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
     return d;
 }
 
@@ -166,9 +170,13 @@ __device__ __forceinline__ uint32_t codes8(const uint32_t *lut, const float (&n)
 // of packed codes; the block absmax, the reciprocal and the block constant are
 // lane-local.  A lane's 8 (bf16) or 16 (fp32) 16-byte loads are issued
 // together; fp32 input is read twice (the second time from L1).
-template <bool kF32In>
+// kIn: 0 bf16 input, 1 fp32 input, 2 fp16 input (bf16 and fp16 stream
+// through the TMA rings).
+template <int kIn>
 __global__ void __maxnreg__(64) quantize_blocks_kernel(const __grid_constant__ QuantParams p)
 {
+    constexpr bool kF32In = kIn == 1;
+    constexpr bool kF16In = kIn == 2;
     static_assert(kQThreads >= 256, "the first 256 threads build the code table and own the buckets");
     __shared__ __align__(16) uint32_t lut[4096];
     __shared__ unsigned long long s_acc[256];
@@ -243,14 +251,15 @@ __global__ void __maxnreg__(64) quantize_blocks_kernel(const __grid_constant__ Q
             // block absmax: magnitudes of the 64 values in two lanes of bf16
             // pairs, then the larger half; magnitude bit patterns compare like
             // the values
-            uint32_t m0 = maxabs_bf16x2(v[0].x, v[0].y), m1 = maxabs_bf16x2(v[0].z, v[0].w);
+            uint32_t m0 = maxabs16x2<kF16In>(v[0].x, v[0].y), m1 = maxabs16x2<kF16In>(v[0].z, v[0].w);
 #pragma unroll
             for (int i = 1; i < 8; i++) {
-                m0 = maxabs_bf16x2(m0, maxabs_bf16x2(v[i].x, v[i].y));
-                m1 = maxabs_bf16x2(m1, maxabs_bf16x2(v[i].z, v[i].w));
+                m0 = maxabs16x2<kF16In>(m0, maxabs16x2<kF16In>(v[i].x, v[i].y));
+                m1 = maxabs16x2<kF16In>(m1, maxabs16x2<kF16In>(v[i].z, v[i].w));
             }
-            const uint32_t m = maxabs_bf16x2(m0, m1) & 0x7FFF7FFFu;
-            cv = __uint_as_float(__vmaxu2(m, m >> 16) << 16);   // larger half, as binary32
+            const uint32_t m = maxabs16x2<kF16In>(m0, m1) & 0x7FFF7FFFu;
+            const uint32_t mh = __vmaxu2(m, m >> 16) & 0xFFFFu;   // larger half
+            cv = kF16In ? __half2float(__ushort_as_half((unsigned short)mh)) : __uint_as_float(mh << 16);
             // zero block (absmax below the smallest normal): r = 0 sends every
             // element to n = +-0, whose code is the codebook's zero
             const float r = cv < 1.17549435e-38f ? 0.0f : __frcp_rn(cv);
@@ -259,8 +268,15 @@ __global__ void __maxnreg__(64) quantize_blocks_kernel(const __grid_constant__ Q
                 const uint32_t u[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
                 float n[8];
 #pragma unroll
-                for (int j = 0; j < 4; j++)
-                    nf4::mul2(__uint_as_float(u[j] << 16), __uint_as_float(u[j] & 0xFFFF0000u), r, n[2 * j], n[2 * j + 1]);
+                for (int j = 0; j < 4; j++) {
+                    if constexpr (kF16In) {
+                        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&u[j]));
+                        nf4::mul2(f.x, f.y, r, n[2 * j], n[2 * j + 1]);
+                    } else {
+                        nf4::mul2(__uint_as_float(u[j] << 16), __uint_as_float(u[j] & 0xFFFF0000u), r, n[2 * j],
+                                  n[2 * j + 1]);
+                    }
+                }
                 words[i] = codes8(lut, n);
             }
         } else {
@@ -442,6 +458,7 @@ struct DeqParams {
     float q[16];
 };
 
+template <bool F16>
 __global__ void __launch_bounds__(kThreads) dequantize_kernel(DeqParams p)
 {
     __shared__ float lut[16];
@@ -472,7 +489,7 @@ __global__ void __launch_bounds__(kThreads) dequantize_kernel(DeqParams p)
         for (int u = 0; u < kDeqUnroll; u++) {
             int64_t w = w0 + u * stride;
             if (w >= p.nwords) continue;
-            *reinterpret_cast<uint4 *>(p.out + 8 * w) = nf4::expand8(word[u], lut, c1p[u]);
+            *reinterpret_cast<uint4 *>(p.out + 8 * w) = nf4::expand8<F16>(word[u], lut, c1p[u]);
         }
     }
 }
@@ -519,18 +536,30 @@ qlora_status prepare_quantize(QuantParams &qp, const void *W, qlora_dtype w_dtyp
     if (!qp.err) return QLORA_ERR_CUDA;
     qp.timeout_ns = 2000000000ull;
     qp.stall_inject = 0;
-    if (w_dtype == QLORA_BF16) {
-        QLORA_TRY(make_map(&qp.tm_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, 64, (uint64_t)(numel / 64), 128, 64, 32,
-                           CU_TENSOR_MAP_SWIZZLE_128B));
+    if (w_dtype == QLORA_BF16 || w_dtype == QLORA_FP16) {
+        QLORA_TRY(make_map(&qp.tm_w,
+                           w_dtype == QLORA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, W,
+                           64, (uint64_t)(numel / 64), 128, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B));
         static PerDeviceOnce attr;
         QLORA_TRY(attr.run(dev.device, []() -> qlora_status {
-            QLORA_CUDA_TRY(cudaFuncSetAttribute(quantize_blocks_kernel<false>,
+            QLORA_CUDA_TRY(cudaFuncSetAttribute(quantize_blocks_kernel<0>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize, kQDynSmem));
+            QLORA_CUDA_TRY(cudaFuncSetAttribute(quantize_blocks_kernel<2>,
                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kQDynSmem));
             return QLORA_OK;
         }));
         qp.stall_inject = take_stall_injection(QLORA_KERNEL_QUANTIZE, &qp.timeout_ns) ? 1 : 0;
     }
     return QLORA_OK;
+}
+
+// The quantizer for the input type w_dtype.
+cudaError_t launch_quantize(qlora_dtype w_dtype, int grid, cudaStream_t s, const QuantParams &qp)
+{
+    if (w_dtype == QLORA_FP32) return launch_pdl(quantize_blocks_kernel<1>, dim3(grid), dim3(kQThreads), 0, s, qp);
+    if (w_dtype == QLORA_FP16)
+        return launch_pdl(quantize_blocks_kernel<2>, dim3(grid), dim3(kQThreads), kQDynSmem, s, qp);
+    return launch_pdl(quantize_blocks_kernel<0>, dim3(grid), dim3(kQThreads), kQDynSmem, s, qp);
 }
 
 int grid_for(int64_t work_items, int items_per_cta, int max_ctas)
@@ -560,7 +589,7 @@ extern "C" qlora_status qlora_quantize_nf4_dq(const void *W, qlora_dtype w_dtype
                                               void *workspace, size_t workspace_bytes, void *stream)
 {
     if (!W || !out || !workspace) return QLORA_ERR_INVALID_ARG;
-    if (w_dtype != QLORA_BF16 && w_dtype != QLORA_FP32) return QLORA_ERR_INVALID_ARG;
+    if (w_dtype != QLORA_BF16 && w_dtype != QLORA_FP32 && w_dtype != QLORA_FP16) return QLORA_ERR_INVALID_ARG;
     QLORA_TRY(check_weight(out));
     if (!aligned16(W) || !aligned16(workspace)) return QLORA_ERR_ALIGNMENT;
     if (workspace_bytes < qlora_quantize_workspace_bytes(out->rows, out->cols)) return QLORA_ERR_WORKSPACE;
@@ -590,10 +619,7 @@ extern "C" qlora_status qlora_quantize_nf4_dq(const void *W, qlora_dtype w_dtype
     int grid = grid_for(qp.nblocks, kQThreads * 2, dev.sms);
     {
         LaunchScope ls(QLORA_KERNEL_QUANTIZE, s);
-        if (w_dtype == QLORA_FP32)
-            QLORA_CUDA_TRY(launch_pdl(quantize_blocks_kernel<true>, dim3(grid), dim3(kQThreads), 0, s, qp));
-        else
-            QLORA_CUDA_TRY(launch_pdl(quantize_blocks_kernel<false>, dim3(grid), dim3(kQThreads), kQDynSmem, s, qp));
+        QLORA_CUDA_TRY(launch_quantize(w_dtype, grid, s, qp));
     }
     QLORA_TRY(launch_status());
 
@@ -612,9 +638,12 @@ extern "C" qlora_status qlora_quantize_nf4_dq(const void *W, qlora_dtype w_dtype
     return launch_status();
 }
 
-extern "C" qlora_status qlora_dequantize_nf4_dq(const qlora_nf4_weight *w, void *out_bf16, void *stream)
+extern "C" qlora_status qlora_dequantize_nf4_dq_ex(const qlora_nf4_weight *w, void *out, qlora_dtype out_dtype,
+                                                   void *stream)
 {
-    if (!w || !out_bf16) return QLORA_ERR_INVALID_ARG;
+    if (!w || !out) return QLORA_ERR_INVALID_ARG;
+    if (out_dtype != QLORA_BF16 && out_dtype != QLORA_FP16) return QLORA_ERR_INVALID_ARG;
+    void *out_bf16 = out;
     QLORA_TRY(check_weight(w));
     if (!aligned16(out_bf16)) return QLORA_ERR_ALIGNMENT;
     DeviceInfo dev;
@@ -630,10 +659,16 @@ extern "C" qlora_status qlora_dequantize_nf4_dq(const qlora_nf4_weight *w, void 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     {
         LaunchScope ls(QLORA_KERNEL_DEQUANTIZE, s);
-        QLORA_CUDA_TRY(launch_pdl(dequantize_kernel, dim3(grid_for(p.nwords, kThreads * kDeqUnroll, dev.sms * 8)),
-                                  dim3(kThreads), 0, s, p));
+        QLORA_CUDA_TRY(launch_pdl(out_dtype == QLORA_FP16 ? dequantize_kernel<true> : dequantize_kernel<false>,
+                                  dim3(grid_for(p.nwords, kThreads * kDeqUnroll, dev.sms * 8)), dim3(kThreads), 0, s,
+                                  p));
     }
     return launch_status();
+}
+
+extern "C" qlora_status qlora_dequantize_nf4_dq(const qlora_nf4_weight *w, void *out_bf16, void *stream)
+{
+    return qlora_dequantize_nf4_dq_ex(w, out_bf16, QLORA_BF16, stream);
 }
 
 // ---- quantization without allocation ------------------------------------------------
@@ -684,7 +719,7 @@ extern "C" qlora_status qlora_quantize_nf4_dq_noalloc(const void *W, qlora_dtype
                                                       const qlora_nf4_weight *out, void *stream)
 {
     if (!W || !out) return QLORA_ERR_INVALID_ARG;
-    if (w_dtype != QLORA_BF16 && w_dtype != QLORA_FP32) return QLORA_ERR_INVALID_ARG;
+    if (w_dtype != QLORA_BF16 && w_dtype != QLORA_FP32 && w_dtype != QLORA_FP16) return QLORA_ERR_INVALID_ARG;
     QLORA_TRY(check_weight(out));
     if (!aligned16(W)) return QLORA_ERR_ALIGNMENT;
     // larger than the fixed scratch (compared before multiplying)
@@ -717,10 +752,7 @@ extern "C" qlora_status qlora_quantize_nf4_dq_noalloc(const void *W, qlora_dtype
     const int grid = grid_for(qp.nblocks, kQThreads * 2, dev.sms);
     {
         LaunchScope ls(QLORA_KERNEL_QUANTIZE, s);
-        if (w_dtype == QLORA_FP32)
-            QLORA_CUDA_TRY(launch_pdl(quantize_blocks_kernel<true>, dim3(grid), dim3(kQThreads), 0, s, qp));
-        else
-            QLORA_CUDA_TRY(launch_pdl(quantize_blocks_kernel<false>, dim3(grid), dim3(kQThreads), kQDynSmem, s, qp));
+        QLORA_CUDA_TRY(launch_quantize(w_dtype, grid, s, qp));
     }
     QLORA_TRY(launch_status());
 

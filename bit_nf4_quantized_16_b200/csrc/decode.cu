@@ -25,6 +25,7 @@
 // forms H = s X A^T (fp32, optionally saved for the backward pass), adds
 // H B^T and stores Y in bf16 or fp32.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include <algorithm>
@@ -49,6 +50,7 @@ struct DecodeParams {
     const float *mean;
     float q[16];
     const __nv_bfloat16 *X;   // [M][K]
+    const __nv_bfloat16 *Xa;  // [M][K]: input of the adapter rows (X, or the dropped-out input under LoRA dropout)
     const __nv_bfloat16 *A;   // [r][K]
     int64_t N, K, kblocks;
     int M, r;
@@ -82,15 +84,23 @@ __device__ __forceinline__ uint4 ld_cached_v4(const void *p)
     return __ldg(reinterpret_cast<const uint4 *>(p));
 }
 
-// D += A B, m16n8k16, bf16 inputs, fp32 accumulators.
+// D += A B, m16n8k16, bf16 (or, F16, fp16) inputs, fp32 accumulators.
+template <bool F16>
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                                uint32_t b0, uint32_t b1)
 {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    if constexpr (F16)
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+            "{%0,%1,%2,%3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    else
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+            "{%0,%1,%2,%3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 // One 128-wide step of this lane's two rows: packed codes and block constants.
@@ -109,7 +119,7 @@ struct WStage {
 // 2c+9} is + {2, 3}: lane c's 32 consecutive k feed 8 steps, four per step.
 // mma.sync is warp-collective: every lane calls this; lanes whose k is past the
 // end pass kin = false and multiply zeros.
-template <int NT>
+template <int NT, bool F16>
 __device__ __forceinline__ void mma_step(float (&acc)[NT][2][4], const uint4 (&ea)[4], const uint4 (&eb)[4],
                                          const __nv_bfloat16 *const (&xrow)[NT], const bool (&xok)[NT], int64_t k,
                                          bool kin)
@@ -119,13 +129,14 @@ __device__ __forceinline__ void mma_step(float (&acc)[NT][2][4], const uint4 (&e
 #pragma unroll
         for (int t = 0; t < NT; t++) {
             const uint4 xb = (xok[t] && kin) ? ld_cached_v4(xrow[t] + k + 8 * w) : make_uint4(0, 0, 0, 0);
-            mma_bf16_16816(acc[t][0], ea[w].x, eb[w].x, ea[w].y, eb[w].y, xb.x, xb.y);
-            mma_bf16_16816(acc[t][0], ea[w].z, eb[w].z, ea[w].w, eb[w].w, xb.z, xb.w);
+            mma_bf16_16816<F16>(acc[t][0], ea[w].x, eb[w].x, ea[w].y, eb[w].y, xb.x, xb.y);
+            mma_bf16_16816<F16>(acc[t][0], ea[w].z, eb[w].z, ea[w].w, eb[w].w, xb.z, xb.w);
         }
     }
 }
 
-template <int NT>
+// F16: the fp16 compute dtype (fp16 X, A and expansion).
+template <int NT, bool F16>
 __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm) decode_gemv_kernel(const __grid_constant__ DecodeParams p)
 {
     __shared__ float lut[16];
@@ -157,6 +168,8 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm) decode_gemv_kernel
     if ((int)blockIdx.x >= p.row_tiles) {
         // ---- rows of A: warp task = (16-row group, piece of the contraction)
         if (sp != 0) return;
+#pragma unroll
+        for (int t = 0; t < NT; t++) xrow[t] = p.Xa + (int64_t)(xok[t] ? 8 * t + g : 0) * p.K;
         const int groups = (p.r + 15) / 16;
         const int task = ((int)blockIdx.x - p.row_tiles) * kDecWarps + warp;
         const int grp = task % groups, qtr = task / groups;
@@ -175,7 +188,7 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm) decode_gemv_kernel
                 ea[w] = (ok_g && k_ok) ? ld_cached_v4(p.A + rg * p.K + k + 8 * w) : make_uint4(0, 0, 0, 0);
                 eb[w] = (ok_g8 && k_ok) ? ld_cached_v4(p.A + rg8 * p.K + k + 8 * w) : make_uint4(0, 0, 0, 0);
             }
-            mma_step<NT>(acc, ea, eb, xrow, xok, k, k_ok);
+            mma_step<NT, F16>(acc, ea, eb, xrow, xok, k, k_ok);
         }
         float *part = p.part_h + (int64_t)qtr * p.M * p.r;
 #pragma unroll
@@ -223,15 +236,15 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm) decode_gemv_kernel
                     const float sg = (ok_g && kin) ? nf4::block_scale((uint8_t)st[i].eg, st[i].c2g, mu) : 0.0f;
                     const float sg8 = (ok_g8 && kin) ? nf4::block_scale((uint8_t)st[i].eg8, st[i].c2g8, mu) : 0.0f;
                     uint4 ea[4], eb[4];
-                    ea[0] = nf4::expand8(st[i].pg.x, lut, sg);
-                    ea[1] = nf4::expand8(st[i].pg.y, lut, sg);
-                    ea[2] = nf4::expand8(st[i].pg.z, lut, sg);
-                    ea[3] = nf4::expand8(st[i].pg.w, lut, sg);
-                    eb[0] = nf4::expand8(st[i].pg8.x, lut, sg8);
-                    eb[1] = nf4::expand8(st[i].pg8.y, lut, sg8);
-                    eb[2] = nf4::expand8(st[i].pg8.z, lut, sg8);
-                    eb[3] = nf4::expand8(st[i].pg8.w, lut, sg8);
-                    mma_step<NT>(acc, ea, eb, xrow, xok, k, kin);
+                    ea[0] = nf4::expand8<F16>(st[i].pg.x, lut, sg);
+                    ea[1] = nf4::expand8<F16>(st[i].pg.y, lut, sg);
+                    ea[2] = nf4::expand8<F16>(st[i].pg.z, lut, sg);
+                    ea[3] = nf4::expand8<F16>(st[i].pg.w, lut, sg);
+                    eb[0] = nf4::expand8<F16>(st[i].pg8.x, lut, sg8);
+                    eb[1] = nf4::expand8<F16>(st[i].pg8.y, lut, sg8);
+                    eb[2] = nf4::expand8<F16>(st[i].pg8.z, lut, sg8);
+                    eb[3] = nf4::expand8<F16>(st[i].pg8.w, lut, sg8);
+                    mma_step<NT, F16>(acc, ea, eb, xrow, xok, k, kin);
                 }
                 load(d + i + kPrefetch, st[i]);
             }
@@ -267,9 +280,11 @@ __device__ __forceinline__ void load_splits8(float (&v)[8], const float *part, i
 // not written by the GEMV; everything before the GEMV in the stream completed
 // before the GEMV let this kernel start, and the loads go through L2 only),
 // and the first token's split partials are in flight during the H reduction.
+// y_type: QLORA_BF16, QLORA_FP32 or QLORA_FP16; b_f16: B holds fp16 (the fp16
+// compute dtype) instead of bf16.
 __global__ void __launch_bounds__(256) decode_finalize_kernel(const float *part, const float *part_h, int splits,
                                                             int M, int64_t N, int r, float scale,
-                                                            const __nv_bfloat16 *B, void *Y, int y_f32,
+                                                            const __nv_bfloat16 *B, int b_f16, void *Y, int y_type,
                                                             float *H_save)
 {
     __shared__ float h[kDecodeMaxTokens * 128];
@@ -311,13 +326,24 @@ __global__ void __launch_bounds__(256) decode_finalize_kernel(const float *part,
             const uint32_t w[4] = {bv[j].x, bv[j].y, bv[j].z, bv[j].w};
 #pragma unroll
             for (int i = 0; i < 4; i++) {
-                l = __fmaf_rn(hm[8 * j + 2 * i], __uint_as_float(w[i] << 16), l);
-                l = __fmaf_rn(hm[8 * j + 2 * i + 1], __uint_as_float(w[i] & 0xFFFF0000u), l);
+                float b0, b1;
+                if (b_f16) {
+                    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[i]));
+                    b0 = f.x;
+                    b1 = f.y;
+                } else {
+                    b0 = __uint_as_float(w[i] << 16);
+                    b1 = __uint_as_float(w[i] & 0xFFFF0000u);
+                }
+                l = __fmaf_rn(hm[8 * j + 2 * i], b0, l);
+                l = __fmaf_rn(hm[8 * j + 2 * i + 1], b1, l);
             }
         }
         y = __fadd_rn(y, l);
-        if (y_f32)
+        if (y_type == QLORA_FP32)
             static_cast<float *>(Y)[(int64_t)m * N + n] = y;
+        else if (y_type == QLORA_FP16)
+            static_cast<__half *>(Y)[(int64_t)m * N + n] = __float2half_rn(y);
         else
             static_cast<__nv_bfloat16 *>(Y)[(int64_t)m * N + n] = __float2bfloat16_rn(y);
     }
@@ -355,9 +381,9 @@ size_t decode_workspace_bytes(int64_t M, int64_t N, int64_t K, int r, int sms)
     return d.part_bytes + d.part_h_bytes;
 }
 
-qlora_status run_decode_fwd(const qlora_nf4_weight *w, const void *X, int64_t M, const void *A, const void *B, int r,
-                            float scale, void *Y, qlora_dtype y_dtype, float *H_save, void *ws, size_t ws_bytes,
-                            const DeviceInfo &dev, cudaStream_t s)
+qlora_status run_decode_fwd(const qlora_nf4_weight *w, const void *X, const void *Xa, int64_t M, const void *A,
+                            const void *B, int r, float scale, void *Y, qlora_dtype y_dtype, float *H_save, void *ws,
+                            size_t ws_bytes, const DeviceInfo &dev, cudaStream_t s, bool f16)
 {
     if (M < 1 || M > kDecodeMaxTokens) return QLORA_ERR_SHAPE;
     const DecodePlan d = decode_plan(M, w->rows, w->cols, r, dev.sms);
@@ -369,6 +395,7 @@ qlora_status run_decode_fwd(const qlora_nf4_weight *w, const void *X, int64_t M,
     p.mean = w->mean;
     for (int i = 0; i < 16; i++) p.q[i] = w->codebook[i];
     p.X = static_cast<const __nv_bfloat16 *>(X);
+    p.Xa = static_cast<const __nv_bfloat16 *>(Xa);
     p.A = static_cast<const __nv_bfloat16 *>(A);
     p.N = w->rows;
     p.K = w->cols;
@@ -384,16 +411,18 @@ qlora_status run_decode_fwd(const qlora_nf4_weight *w, const void *X, int64_t M,
     {
         LaunchScope ls(QLORA_KERNEL_FWD_FUSED, s);
         if (M <= 8)
-            QLORA_CUDA_TRY(launch_pdl(decode_gemv_kernel<1>, grid, dim3(kDecThreads), 0, s, p));
+            QLORA_CUDA_TRY(launch_pdl(f16 ? decode_gemv_kernel<1, true> : decode_gemv_kernel<1, false>, grid,
+                                      dim3(kDecThreads), 0, s, p));
         else
-            QLORA_CUDA_TRY(launch_pdl(decode_gemv_kernel<2>, grid, dim3(kDecThreads), 0, s, p));
+            QLORA_CUDA_TRY(launch_pdl(f16 ? decode_gemv_kernel<2, true> : decode_gemv_kernel<2, false>, grid,
+                                      dim3(kDecThreads), 0, s, p));
     }
     {
         LaunchScope ls(QLORA_KERNEL_ELEMENTWISE, s);
         QLORA_CUDA_TRY(launch_pdl(decode_finalize_kernel, dim3(ceil_div_i(w->rows, 256)), dim3(256), 0, s,
                                   (const float *)p.part, (const float *)p.part_h, d.splits, (int)M,
-                                  (int64_t)w->rows, r, scale, static_cast<const __nv_bfloat16 *>(B), Y,
-                                  y_dtype == QLORA_FP32 ? 1 : 0, H_save));
+                                  (int64_t)w->rows, r, scale, static_cast<const __nv_bfloat16 *>(B), f16 ? 1 : 0, Y,
+                                  (int)y_dtype, H_save));
     }
     return launch_status();
 }

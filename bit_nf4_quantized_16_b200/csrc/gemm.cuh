@@ -113,7 +113,6 @@ namespace gemm_detail {
 
 using nf4::block_scale;
 using nf4::expand8;
-using nf4::pack_bf16x2;
 
 __device__ __forceinline__ void record_timeout(const GemmParams &p, int *abort_flag)
 {
@@ -123,7 +122,9 @@ __device__ __forceinline__ void record_timeout(const GemmParams &p, int *abort_f
 
 }  // namespace gemm_detail
 
-template <int BN, int kBMode, int kEpi, int MT>
+// F16: the fp16 compute dtype (fp16 operands, fp16 expansion and 16-bit
+// outputs) instead of bf16.
+template <int BN, int kBMode, int kEpi, int MT, bool F16 = false>
 __global__ void __launch_bounds__(GemmCfg<BN, kBMode, MT>::kThreads, 1)
     qgemm_kernel(const __grid_constant__ GemmParams p)
 {
@@ -259,7 +260,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode, MT>::kThreads, 1)
     } else if (warp == 1 && lane == 0) {
         // ---------------- MMA issuer ----------------
         constexpr bool kBMn = (kBMode == kBTmaMN || kBMode == kBNf4MN);
-        const uint32_t idesc = idesc_bf16_f32(128, BN, p.a_mn, kBMn ? 1 : 0);
+        const uint32_t idesc = idesc_bf16_f32(128, BN, p.a_mn, kBMn ? 1 : 0, F16);
         uint32_t it = 0, local = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < num_tiles && ok && !*vabort; t += gridDim.x, local++) {
@@ -337,10 +338,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode, MT>::kThreads, 1)
                         for (int g = 0; g < 4; g++) {
                             if (col0 + 8 * g >= p.n_total) break;
                             uint4 v;
-                            v.x = pack_bf16x2(__uint_as_float(r[8 * g + 0]), __uint_as_float(r[8 * g + 1]));
-                            v.y = pack_bf16x2(__uint_as_float(r[8 * g + 2]), __uint_as_float(r[8 * g + 3]));
-                            v.z = pack_bf16x2(__uint_as_float(r[8 * g + 4]), __uint_as_float(r[8 * g + 5]));
-                            v.w = pack_bf16x2(__uint_as_float(r[8 * g + 6]), __uint_as_float(r[8 * g + 7]));
+                            v.x = nf4::pack16x2<F16>(__uint_as_float(r[8 * g + 0]), __uint_as_float(r[8 * g + 1]));
+                            v.y = nf4::pack16x2<F16>(__uint_as_float(r[8 * g + 2]), __uint_as_float(r[8 * g + 3]));
+                            v.z = nf4::pack16x2<F16>(__uint_as_float(r[8 * g + 4]), __uint_as_float(r[8 * g + 5]));
+                            v.w = nf4::pack16x2<F16>(__uint_as_float(r[8 * g + 6]), __uint_as_float(r[8 * g + 7]));
                             *reinterpret_cast<uint4 *>(o + 8 * g) = v;
                         }
                     } else if (kEpi == kEpiDropBf16 || kEpi == kEpiDropF32) {
@@ -366,10 +367,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode, MT>::kThreads, 1)
 #pragma unroll
                             for (int g = 0; g < 4; g++) {
                                 uint4 w;
-                                w.x = pack_bf16x2(v[8 * g + 0], v[8 * g + 1]);
-                                w.y = pack_bf16x2(v[8 * g + 2], v[8 * g + 3]);
-                                w.z = pack_bf16x2(v[8 * g + 4], v[8 * g + 5]);
-                                w.w = pack_bf16x2(v[8 * g + 6], v[8 * g + 7]);
+                                w.x = nf4::pack16x2<F16>(v[8 * g + 0], v[8 * g + 1]);
+                                w.y = nf4::pack16x2<F16>(v[8 * g + 2], v[8 * g + 3]);
+                                w.z = nf4::pack16x2<F16>(v[8 * g + 4], v[8 * g + 5]);
+                                w.w = nf4::pack16x2<F16>(v[8 * g + 6], v[8 * g + 7]);
                                 *reinterpret_cast<uint4 *>(o + 8 * g) = w;
                             }
                         } else {
@@ -498,7 +499,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBMode, MT>::kThreads, 1)
                     const int dst_chunk0 = part * WPT;
 #pragma unroll
                     for (int j = 0; j < WPT; j++)
-                        *reinterpret_cast<uint4 *>(dst + (((dst_chunk0 + j) ^ (r & 7)) << 4)) = expand8(words[j], lut, c1p);
+                        *reinterpret_cast<uint4 *>(dst + (((dst_chunk0 + j) ^ (r & 7)) << 4)) = expand8<F16>(words[j], lut, c1p);
                     fence_proxy_async_smem();
                 }
                 __syncwarp();

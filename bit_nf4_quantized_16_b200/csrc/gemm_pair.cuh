@@ -61,7 +61,7 @@ struct PairCfg {
     static_assert(kSmemBytes + 64 <= 232448, "shared memory per block");
 };
 
-template <int kBMode, int kEpi, int MT>
+template <int kBMode, int kEpi, int MT, bool F16 = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<kBMode, MT>::kThreads, 1)
     qgemm_pair_kernel(const __grid_constant__ GemmParams p)
 {
@@ -193,7 +193,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<kBMode, MT>:
         }
     } else if (warp == 1 && lane == 0 && leader) {
         // ---------------- MMA issuer (leader only) ----------------
-        const uint32_t idesc = idesc_bf16_f32(256, NP, 0, kBMn ? 1 : 0);
+        const uint32_t idesc = idesc_bf16_f32(256, NP, 0, kBMn ? 1 : 0, F16);
         uint32_t it = 0, local = 0;
         bool ok = true;
         for (int t = cluster_id; t < num_tiles && ok && !*vabort; t += num_clusters, local++) {
@@ -276,10 +276,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<kBMode, MT>:
 #pragma unroll
                         for (int g = 0; g < 4; g++) {
                             uint4 v;
-                            v.x = pack_bf16x2(__uint_as_float(r[8 * g + 0]), __uint_as_float(r[8 * g + 1]));
-                            v.y = pack_bf16x2(__uint_as_float(r[8 * g + 2]), __uint_as_float(r[8 * g + 3]));
-                            v.z = pack_bf16x2(__uint_as_float(r[8 * g + 4]), __uint_as_float(r[8 * g + 5]));
-                            v.w = pack_bf16x2(__uint_as_float(r[8 * g + 6]), __uint_as_float(r[8 * g + 7]));
+                            v.x = nf4::pack16x2<F16>(__uint_as_float(r[8 * g + 0]), __uint_as_float(r[8 * g + 1]));
+                            v.y = nf4::pack16x2<F16>(__uint_as_float(r[8 * g + 2]), __uint_as_float(r[8 * g + 3]));
+                            v.z = nf4::pack16x2<F16>(__uint_as_float(r[8 * g + 4]), __uint_as_float(r[8 * g + 5]));
+                            v.w = nf4::pack16x2<F16>(__uint_as_float(r[8 * g + 6]), __uint_as_float(r[8 * g + 7]));
                             *reinterpret_cast<uint4 *>(box + lane * 64 + ((g ^ ((lane >> 1) & 3)) << 4)) = v;
                         }
                         fence_proxy_async_smem();
@@ -397,7 +397,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<kBMode, MT>:
                     const int dst_chunk0 = part * WPT;
 #pragma unroll
                     for (int j = 0; j < WPT; j++)
-                        *reinterpret_cast<uint4 *>(dst + (((dst_chunk0 + j) ^ (r & 7)) << 4)) = expand8(words[j], lut, c1p);
+                        *reinterpret_cast<uint4 *>(dst + (((dst_chunk0 + j) ^ (r & 7)) << 4)) = expand8<F16>(words[j], lut, c1p);
                     fence_proxy_async_smem();
                 }
                 __syncwarp();

@@ -31,6 +31,7 @@
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include "sm100.cuh"
@@ -90,21 +91,35 @@ struct SkinnyCfg {
 
 namespace skinny_detail {
 
-__device__ __forceinline__ uint32_t bf16_bits(float v)
+// Bits of v rounded to the 16-bit compute type, and that value back in fp32.
+template <bool F16>
+__device__ __forceinline__ uint32_t bits16(float v)
 {
-    return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v));
+    if constexpr (F16)
+        return (uint32_t)__half_as_ushort(__float2half_rn(v));
+    else
+        return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+template <bool F16>
+__device__ __forceinline__ float from16(uint32_t b)
+{
+    if constexpr (F16)
+        return __half2float(__ushort_as_half((unsigned short)b));
+    else
+        return __uint_as_float(b << 16);
 }
 
-// hi = bf16(v), lo = bf16(v - hi) of columns col..col+3 of row `row` into the
-// chunked hi/lo layout [rows][2 r_pad].
+// hi = t16(v), lo = t16(v - hi) (t16: the 16-bit compute type) of columns
+// col..col+3 of row `row` into the chunked hi/lo layout [rows][2 r_pad].
+template <bool F16>
 __device__ __forceinline__ void store_hi_lo4(__nv_bfloat16 *dst, int64_t row, int r_pad, int col, float4 v)
 {
     const float vv[4] = {v.x, v.y, v.z, v.w};
     uint32_t hi[4], lo[4];
 #pragma unroll
     for (int i = 0; i < 4; i++) {
-        hi[i] = bf16_bits(vv[i]);
-        lo[i] = bf16_bits(__fsub_rn(vv[i], __uint_as_float(hi[i] << 16)));
+        hi[i] = bits16<F16>(vv[i]);
+        lo[i] = bits16<F16>(__fsub_rn(vv[i], from16<F16>(hi[i])));
     }
     __nv_bfloat16 *d = dst + row * 2 * r_pad + 128 * (col >> 6) + (col & 63);
     *reinterpret_cast<uint2 *>(d) = make_uint2(hi[0] | (hi[1] << 16), hi[2] | (hi[3] << 16));
@@ -118,7 +133,7 @@ __device__ __forceinline__ float4 add4(float4 a, float4 b)
 
 }  // namespace skinny_detail
 
-template <int BN, int A_MN, int B_MN>
+template <int BN, int A_MN, int B_MN, bool F16 = false>
 __global__ void __launch_bounds__(256, 1) qgemm_skinny_kernel(const __grid_constant__ SkinnyParams p)
 {
     using Cfg = SkinnyCfg<BN, A_MN, B_MN>;
@@ -212,7 +227,7 @@ __global__ void __launch_bounds__(256, 1) qgemm_skinny_kernel(const __grid_const
         }
     } else if (warp == 1 && lane == 0) {
         // ---------------- MMA issuer ----------------
-        const uint32_t idesc = idesc_bf16_f32(128, BN, A_MN, B_MN);
+        const uint32_t idesc = idesc_bf16_f32(128, BN, A_MN, B_MN, F16);
         bool ok = true;
         for (int ks = 0; ks < n_k; ks++) {
             const int s = ks % S;
@@ -294,11 +309,11 @@ __global__ void __launch_bounds__(256, 1) qgemm_skinny_kernel(const __grid_const
                                        __fmul_rn(J.scale, acc.z), __fmul_rn(J.scale, acc.w));
                 if (!in) v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
                 if (J.f32_out && in) *reinterpret_cast<float4 *>(J.f32_out + grow * J.r + col) = v;
-                store_hi_lo4(J.hl_out, grow, J.r_pad, col, v);
+                store_hi_lo4<F16>(J.hl_out, grow, J.r_pad, col, v);
                 if (J.aux_in) {
                     float4 h = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
                     if (in) h = *reinterpret_cast<const float4 *>(J.aux_in + grow * J.r + col);
-                    store_hi_lo4(J.aux_out, grow, J.r_pad, col, h);
+                    store_hi_lo4<F16>(J.aux_out, grow, J.r_pad, col, h);
                 }
             } else {
                 const int j = 64 * nt + 4 * c4;

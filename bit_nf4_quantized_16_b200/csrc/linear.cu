@@ -60,12 +60,12 @@ void set_limits(GemmParams &p, int kind)
     p.stall_inject = take_stall_injection(kind, &p.timeout_ns) ? 1 : 0;
 }
 
-template <int BN, int kBMode, int kEpi, int MT = 1>
+template <int BN, int kBMode, int kEpi, int MT = 1, bool F16 = false>
 qlora_status launch_gemm(GemmParams &p, const DeviceInfo &dev, cudaStream_t s, int kind)
 {
     using Cfg = GemmCfg<BN, kBMode, MT>;
     static PerDeviceOnce attr;
-    auto kern = qgemm_kernel<BN, kBMode, kEpi, MT>;
+    auto kern = qgemm_kernel<BN, kBMode, kEpi, MT, F16>;
     QLORA_TRY(attr.run(dev.device, [&]() -> qlora_status {
         QLORA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes));
         return QLORA_OK;
@@ -85,13 +85,13 @@ qlora_status launch_gemm(GemmParams &p, const DeviceInfo &dev, cudaStream_t s, i
 // Fused dequant-GEMM on CTA pairs: p.m_tiles / p.n_tiles count pair tiles
 // (2 * 128 * MT tokens x 256 features); one cluster of two CTAs per tile,
 // persistent over tiles, at most as many clusters as can be resident at once.
-template <int kBMode, int kEpi, int MT>
+template <int kBMode, int kEpi, int MT, bool F16 = false>
 qlora_status launch_gemm_pair(GemmParams &p, const DeviceInfo &dev, cudaStream_t s, int kind)
 {
     using Cfg = PairCfg<kBMode, MT>;
     static PerDeviceOnce setup;
     static int max_clusters[kMaxDevices] = {};
-    auto kern = qgemm_pair_kernel<kBMode, kEpi, MT>;
+    auto kern = qgemm_pair_kernel<kBMode, kEpi, MT, F16>;
     QLORA_TRY(setup.run(dev.device, [&]() -> qlora_status {
         QLORA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes));
         cudaLaunchConfig_t cfg{};
@@ -124,11 +124,11 @@ int pad64(int v) { return (v + 63) / 64 * 64; }
 
 // Launches one skinny-product grid: `clusters` output tiles, `csize` CTAs per
 // cluster (the contraction split).
-template <int BN, int A_MN, int B_MN>
+template <int BN, int A_MN, int B_MN, bool F16 = false>
 qlora_status launch_skinny(SkinnyParams &p, int clusters, int csize, const DeviceInfo &dev, cudaStream_t s, int kind)
 {
     using Cfg = SkinnyCfg<BN, A_MN, B_MN>;
-    auto kern = qgemm_skinny_kernel<BN, A_MN, B_MN>;
+    auto kern = qgemm_skinny_kernel<BN, A_MN, B_MN, F16>;
     p.err = device_error_word();
     if (!p.err) return QLORA_ERR_CUDA;
     p.timeout_ns = kTimeoutNs;
@@ -156,13 +156,13 @@ qlora_status launch_skinny(SkinnyParams &p, int clusters, int csize, const Devic
 
 // Kernel attributes and the number of co-resident clusters for each cluster
 // size 1, 2, 4, 8 (once per device and instantiation).
-template <int BN, int A_MN, int B_MN>
+template <int BN, int A_MN, int B_MN, bool F16 = false>
 qlora_status skinny_setup(const DeviceInfo &dev, const int **max_clusters)
 {
     using Cfg = SkinnyCfg<BN, A_MN, B_MN>;
     static PerDeviceOnce once;
     static int maxc[kMaxDevices][4] = {};
-    auto kern = qgemm_skinny_kernel<BN, A_MN, B_MN>;
+    auto kern = qgemm_skinny_kernel<BN, A_MN, B_MN, F16>;
     QLORA_TRY(once.run(dev.device, [&]() -> qlora_status {
         QLORA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes));
         for (int i = 0; i < 4; i++) {
@@ -213,11 +213,14 @@ struct Plan {
     int64_t M, N, K;
     int r, r_pad;
     size_t off_h2, off_g2, bytes;
+    // LoRA dropout: the dropped-out input X_d (bf16 [M][K]) and the frozen
+    // path's fp32 input gradient [M][K]
+    size_t off_xd, off_dxs;
 };
 
 size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
-Plan make_plan(int64_t M, int64_t N, int64_t K, int r, int sms)
+Plan make_plan(int64_t M, int64_t N, int64_t K, int r, int sms, bool dropout = false)
 {
     Plan pl{};
     pl.M = M;
@@ -231,7 +234,79 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int r, int sms)
     pl.bytes = 2 * hl;
     // the decode forward (M <= kDecodeMaxTokens) uses the start of the workspace for its partials
     if (M <= kDecodeMaxTokens) pl.bytes = std::max(pl.bytes, align256(decode_workspace_bytes(M, N, K, r, sms)));
+    if (dropout) {
+        pl.off_xd = pl.bytes;
+        pl.off_dxs = pl.off_xd + align256((size_t)M * K * 2);
+        pl.bytes = pl.off_dxs + align256((size_t)M * K * 4);
+    }
     return pl;
+}
+
+// ---- LoRA dropout ---------------------------------------------------------------------
+//
+// The blog's LoraConfig snippet ("Efficient Language Model Fine-Tuning with
+// QLoRA on Resource-Constrained Hardware", marciocunha.net) sets lora_dropout:
+// the adapter branch sees X_d = X * mask / (1 - p), the frozen path X.  Kept
+// elements are RN_bf16(RN32(x * RN32(1 / (1 - p)))), dropped ones 0; the
+// mask holds bit k % 8 of byte (m K + k) / 8 for element (m, k), 1 = kept.
+
+bool dropout_on(const qlora_linear_opts *o) { return o && o->dropout_mask; }
+
+float dropout_scale(const qlora_linear_opts *o) { return 1.0f / (1.0f - o->dropout_p); }
+
+// X_d from X and the mask, eight elements (one mask byte) per thread (F16:
+// fp16 X and X_d).
+template <bool F16>
+__global__ void __launch_bounds__(256) dropout_input_kernel(const __nv_bfloat16 *X, const uint8_t *mask, float scale,
+                                                            __nv_bfloat16 *Xd, int64_t n8)
+{
+    sm100::pdl_wait();
+    sm100::pdl_trigger();
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
+        const uint4 xv = *reinterpret_cast<const uint4 *>(X + 8 * i);
+        const uint32_t bits = mask[i];
+        const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            float xa, xb;
+            if constexpr (F16) {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[j]));
+                xa = f.x;
+                xb = f.y;
+            } else {
+                xa = __uint_as_float(w[j] << 16);
+                xb = __uint_as_float(w[j] & 0xFFFF0000u);
+            }
+            const uint32_t packed = nf4::pack16x2<F16>(__fmul_rn(xa, scale), __fmul_rn(xb, scale));
+            const uint32_t keep = ((bits >> (2 * j)) & 1u ? 0x0000FFFFu : 0u) | ((bits >> (2 * j + 1)) & 1u ? 0xFFFF0000u : 0u);
+            o[j] = packed & keep;
+        }
+        *reinterpret_cast<uint4 *>(Xd + 8 * i) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+template <bool F16>
+qlora_status run_dropout_input(const Plan &pl, const DeviceInfo &dev, const void *X, const qlora_linear_opts *o,
+                               char *ws, cudaStream_t s)
+{
+    const int64_t n8 = pl.M * pl.K / 8;
+    const int grid = (int)std::min<int64_t>((n8 + 255) / 256, (int64_t)dev.sms * 16);
+    LaunchScope ls(QLORA_KERNEL_ELEMENTWISE, s);
+    QLORA_CUDA_TRY(launch_pdl(dropout_input_kernel<F16>, dim3(grid), dim3(256), 0, s, static_cast<const __nv_bfloat16 *>(X),
+                              o->dropout_mask, dropout_scale(o), reinterpret_cast<__nv_bfloat16 *>(ws + pl.off_xd),
+                              n8));
+    return launch_status();
+}
+
+qlora_status check_opts(const qlora_linear_opts *o)
+{
+    if (!o) return QLORA_OK;
+    if (o->compute_dtype != QLORA_BF16 && o->compute_dtype != QLORA_FP16) return QLORA_ERR_INVALID_ARG;
+    if (!o->dropout_mask) return QLORA_OK;
+    if (!(o->dropout_p >= 0.0f && o->dropout_p < 1.0f)) return QLORA_ERR_INVALID_ARG;
+    if (!aligned16(o->dropout_mask)) return QLORA_ERR_ALIGNMENT;
+    return QLORA_OK;
 }
 
 qlora_status check_linear(const qlora_nf4_weight *w, const void *X, int64_t M, const void *A, const void *B,
@@ -250,13 +325,13 @@ qlora_status check_linear(const qlora_nf4_weight *w, const void *X, int64_t M, c
 // Low-rank factor v = scale * P Q^T (P [M][Kc] bf16, Q given as the B operand)
 // into the hi/lo buffer `hl`, with an optional fp32 copy and an optional
 // hi/lo split of aux_in into aux_out.
-template <int BN, int B_MN>
+template <int BN, int B_MN, bool F16 = false>
 qlora_status run_lowrank(const Plan &pl, const DeviceInfo &dev, const void *P, int64_t Kc, const void *Q,
                          float scale, __nv_bfloat16 *hl, float *f32_out, const float *aux_in, __nv_bfloat16 *aux_out,
                          cudaStream_t s)
 {
     const int *maxc = nullptr;
-    QLORA_TRY((skinny_setup<BN, 0, B_MN>(dev, &maxc)));
+    QLORA_TRY((skinny_setup<BN, 0, B_MN, F16>(dev, &maxc)));
     SkinnyParams p{};
     SkinnyJob &J = p.job[0];
     QLORA_TRY(map_k_major(&J.tm_a, P, Kc, pl.M, 128));
@@ -278,17 +353,18 @@ qlora_status run_lowrank(const Plan &pl, const DeviceInfo &dev, const void *P, i
     p.clusters0 = J.m_tiles;
     p.wait_at_end = 0;
     const int cs = choose_csize(J.m_tiles, J.k_total, maxc);
-    return launch_skinny<BN, 0, B_MN>(p, J.m_tiles, cs, dev, s, QLORA_KERNEL_LOWRANK);
+    return launch_skinny<BN, 0, B_MN, F16>(p, J.m_tiles, cs, dev, s, QLORA_KERNEL_LOWRANK);
 }
 
 // H = s X A^T into the hi/lo buffer (and optionally fp32 H_out)
+template <bool F16>
 qlora_status run_h(const Plan &pl, const DeviceInfo &dev, const void *X, const void *A, float scale, float *H_out,
                    char *ws, cudaStream_t s)
 {
     __nv_bfloat16 *H2 = reinterpret_cast<__nv_bfloat16 *>(ws + pl.off_h2);
     if (pl.r_pad == 64)
-        return run_lowrank<64, 0>(pl, dev, X, pl.K, A, scale, H2, H_out, nullptr, nullptr, s);
-    return run_lowrank<128, 0>(pl, dev, X, pl.K, A, scale, H2, H_out, nullptr, nullptr, s);
+        return run_lowrank<64, 0, F16>(pl, dev, X, pl.K, A, scale, H2, H_out, nullptr, nullptr, s);
+    return run_lowrank<128, 0, F16>(pl, dev, X, pl.K, A, scale, H2, H_out, nullptr, nullptr, s);
 }
 
 }  // namespace
@@ -296,35 +372,48 @@ qlora_status run_h(const Plan &pl, const DeviceInfo &dev, const void *X, const v
 
 using namespace qlora;
 
-extern "C" size_t qlora_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t r)
+extern "C" size_t qlora_linear_workspace_bytes_ex(int64_t M, int64_t N, int64_t K, int32_t r,
+                                                  const qlora_linear_opts *opts)
 {
     if (M <= 0 || N <= 0 || K <= 0 || r <= 0) return 256;
     DeviceInfo dev;
     int sms = device_info(&dev) == QLORA_OK ? dev.sms : 148;
-    return make_plan(M, N, K, r, sms).bytes;
+    return make_plan(M, N, K, r, sms, dropout_on(opts)).bytes;
 }
 
-extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const void *X, int64_t M, const void *A,
-                                         const void *B, int32_t r, float scale, void *Y, qlora_dtype y_dtype,
-                                         float *H_save, void *workspace, size_t workspace_bytes, void *stream)
+extern "C" size_t qlora_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t r)
 {
-    QLORA_TRY(check_linear(w, X, M, A, B, r, workspace));
+    return qlora_linear_workspace_bytes_ex(M, N, K, r, nullptr);
+}
+
+template <bool F16>
+static qlora_status linear_fwd(const qlora_nf4_weight *w, const void *X, int64_t M, const void *A, const void *B,
+                               int32_t r, float scale, void *Y, qlora_dtype y_dtype, float *H_save, void *workspace,
+                               size_t workspace_bytes, void *stream, const qlora_linear_opts *opts)
+{
+    const bool drop = dropout_on(opts);
     if (!Y) return QLORA_ERR_INVALID_ARG;
-    if (y_dtype != QLORA_BF16 && y_dtype != QLORA_FP32) return QLORA_ERR_INVALID_ARG;
+    if (y_dtype != (F16 ? QLORA_FP16 : QLORA_BF16) && y_dtype != QLORA_FP32) return QLORA_ERR_INVALID_ARG;
     if (!aligned16(Y) || (H_save && !aligned16(H_save))) return QLORA_ERR_ALIGNMENT;
     DeviceInfo dev;
     QLORA_TRY(device_info(&dev));
     if (M == 0) return QLORA_OK;
-    const Plan pl = make_plan(M, w->rows, w->cols, r, dev.sms);
+    const Plan pl = make_plan(M, w->rows, w->cols, r, dev.sms, drop);
     if (workspace_bytes < pl.bytes) return QLORA_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     char *ws = static_cast<char *>(workspace);
+    // the adapter branch's input: X, or X_d under LoRA dropout
+    const void *Xa = X;
+    if (drop) {
+        QLORA_TRY(run_dropout_input<F16>(pl, dev, X, opts, ws, s));
+        Xa = ws + pl.off_xd;
+    }
 
     // a handful of tokens: stream the packed weight once (bound by HBM, not the tensor cores)
     if (M <= kDecodeMaxTokens)
-        return run_decode_fwd(w, X, M, A, B, r, scale, Y, y_dtype, H_save, ws, workspace_bytes, dev, s);
+        return run_decode_fwd(w, X, Xa, M, A, B, r, scale, Y, y_dtype, H_save, ws, workspace_bytes, dev, s, F16);
 
-    QLORA_TRY(run_h(pl, dev, X, A, scale, H_save, ws, s));
+    QLORA_TRY(run_h<F16>(pl, dev, Xa, A, scale, H_save, ws, s));
 
     // fused forward: 256 tokens (two 128-row accumulators) x 128 output features per tile
     constexpr int kFBN = 128, kFMT = 2;
@@ -353,26 +442,47 @@ extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const void *
     p.n_total = (int)pl.N;
     if (M > 128 * kFMT) {
         // more than one tile of tokens: CTA pairs, 512 tokens x 256 features per pair
-        if (y_dtype == QLORA_BF16)
-            QLORA_TRY(make_map(&p.tm_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, pl.N, M, pl.N * 2, 32, 32,
-                               CU_TENSOR_MAP_SWIZZLE_64B));
+        if (y_dtype != QLORA_FP32)
+            QLORA_TRY(make_map(&p.tm_out, F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y,
+                               pl.N, M, pl.N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B));
         p.m_tiles = ceil_div(M, 2 * 128 * kFMT);
         p.n_tiles = ceil_div(pl.N, 2 * kFBN);
-        if (y_dtype == QLORA_BF16) return launch_gemm_pair<kBNf4K, kEpiBf16, kFMT>(p, dev, s, QLORA_KERNEL_FWD_FUSED);
-        return launch_gemm_pair<kBNf4K, kEpiF32, kFMT>(p, dev, s, QLORA_KERNEL_FWD_FUSED);
+        if (y_dtype != QLORA_FP32) return launch_gemm_pair<kBNf4K, kEpiBf16, kFMT, F16>(p, dev, s, QLORA_KERNEL_FWD_FUSED);
+        return launch_gemm_pair<kBNf4K, kEpiF32, kFMT, F16>(p, dev, s, QLORA_KERNEL_FWD_FUSED);
     }
-    if (y_dtype == QLORA_BF16) return launch_gemm<kFBN, kBNf4K, kEpiBf16, kFMT>(p, dev, s, QLORA_KERNEL_FWD_FUSED);
-    return launch_gemm<kFBN, kBNf4K, kEpiF32, kFMT>(p, dev, s, QLORA_KERNEL_FWD_FUSED);
+    if (y_dtype != QLORA_FP32) return launch_gemm<kFBN, kBNf4K, kEpiBf16, kFMT, F16>(p, dev, s, QLORA_KERNEL_FWD_FUSED);
+    return launch_gemm<kFBN, kBNf4K, kEpiF32, kFMT, F16>(p, dev, s, QLORA_KERNEL_FWD_FUSED);
 }
 
-extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *X, const void *dY, int64_t M,
-                                         const void *A, const void *B, int32_t r, float scale,
-                                         const float *H_saved, void *dX, qlora_dtype dx_dtype, float *dA, float *dB,
-                                         void *workspace, size_t workspace_bytes, void *stream)
+extern "C" qlora_status qlora_linear_fwd_ex(const qlora_nf4_weight *w, const void *X, int64_t M, const void *A,
+                                            const void *B, int32_t r, float scale, void *Y, qlora_dtype y_dtype,
+                                            float *H_save, void *workspace, size_t workspace_bytes, void *stream,
+                                            const qlora_linear_opts *opts)
 {
     QLORA_TRY(check_linear(w, X, M, A, B, r, workspace));
+    QLORA_TRY(check_opts(opts));
+    if (opts && opts->compute_dtype == QLORA_FP16)
+        return linear_fwd<true>(w, X, M, A, B, r, scale, Y, y_dtype, H_save, workspace, workspace_bytes, stream, opts);
+    return linear_fwd<false>(w, X, M, A, B, r, scale, Y, y_dtype, H_save, workspace, workspace_bytes, stream, opts);
+}
+
+extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const void *X, int64_t M, const void *A,
+                                         const void *B, int32_t r, float scale, void *Y, qlora_dtype y_dtype,
+                                         float *H_save, void *workspace, size_t workspace_bytes, void *stream)
+{
+    return qlora_linear_fwd_ex(w, X, M, A, B, r, scale, Y, y_dtype, H_save, workspace, workspace_bytes, stream,
+                               nullptr);
+}
+
+template <bool F16>
+static qlora_status linear_bwd(const qlora_nf4_weight *w, const void *X, const void *dY, int64_t M, const void *A,
+                               const void *B, int32_t r, float scale, const float *H_saved, void *dX,
+                               qlora_dtype dx_dtype, float *dA, float *dB, void *workspace, size_t workspace_bytes,
+                               void *stream, const qlora_linear_opts *opts)
+{
+    const bool drop = dropout_on(opts);
     if (!dY || !dA || !dB) return QLORA_ERR_INVALID_ARG;
-    if (dx_dtype != QLORA_BF16 && dx_dtype != QLORA_FP32) return QLORA_ERR_INVALID_ARG;
+    if (dx_dtype != (F16 ? QLORA_FP16 : QLORA_BF16) && dx_dtype != QLORA_FP32) return QLORA_ERR_INVALID_ARG;
     if (!aligned16(dY) || !aligned16(dA) || !aligned16(dB) || (dX && !aligned16(dX)) ||
         (H_saved && !aligned16(H_saved)))
         return QLORA_ERR_ALIGNMENT;
@@ -386,21 +496,27 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *
         QLORA_CUDA_TRY(cudaMemsetAsync(dB, 0, (size_t)N * r * 4, s));
         return QLORA_OK;
     }
-    const Plan pl = make_plan(M, N, K, r, dev.sms);
+    const Plan pl = make_plan(M, N, K, r, dev.sms, drop);
     if (workspace_bytes < pl.bytes) return QLORA_ERR_WORKSPACE;
     char *ws = static_cast<char *>(workspace);
     __nv_bfloat16 *H2 = reinterpret_cast<__nv_bfloat16 *>(ws + pl.off_h2);
     __nv_bfloat16 *G2 = reinterpret_cast<__nv_bfloat16 *>(ws + pl.off_g2);
     const int hl_cols = 2 * pl.r_pad;
+    // the adapter branch's input: X, or X_d under LoRA dropout
+    const void *Xa = X;
+    if (drop) {
+        QLORA_TRY(run_dropout_input<F16>(pl, dev, X, opts, ws, s));
+        Xa = ws + pl.off_xd;
+    }
 
     // H (hi/lo) recomputed when no saved H is given
-    if (!H_saved) QLORA_TRY(run_h(pl, dev, X, A, scale, nullptr, ws, s));
+    if (!H_saved) QLORA_TRY(run_h<F16>(pl, dev, Xa, A, scale, nullptr, ws, s));
 
     // G = s dY B (contraction over N); the same kernel splits a saved H into hi/lo
     if (pl.r_pad == 64)
-        QLORA_TRY((run_lowrank<64, 1>(pl, dev, dY, N, B, scale, G2, nullptr, H_saved, H_saved ? H2 : nullptr, s)));
+        QLORA_TRY((run_lowrank<64, 1, F16>(pl, dev, dY, N, B, scale, G2, nullptr, H_saved, H_saved ? H2 : nullptr, s)));
     else
-        QLORA_TRY((run_lowrank<128, 1>(pl, dev, dY, N, B, scale, G2, nullptr, H_saved, H_saved ? H2 : nullptr, s)));
+        QLORA_TRY((run_lowrank<128, 1, F16>(pl, dev, dY, N, B, scale, G2, nullptr, H_saved, H_saved ? H2 : nullptr, s)));
 
     // dX = dY W' + bf16(G) A  (fused transposed dequant-GEMM)
     if (dX) {
@@ -429,21 +545,57 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *
         p.out_ld = K;
         p.m_total = (int)M;
         p.n_total = (int)K;
+        // under dropout the adapter term is masked elementwise: the fused GEMM
+        // forms the frozen path dY W' alone, in fp32, and a second product adds
+        // the masked adapter term (below)
+        const bool f32_out = drop || dx_dtype == QLORA_FP32;
+        if (drop) {
+            p.k_stages_lora = 0;
+            p.out = ws + pl.off_dxs;
+        }
         if (M > 128 * kBMT) {
             // CTA pairs: 512 tokens x 256 input features per pair
-            if (dx_dtype == QLORA_BF16)
-                QLORA_TRY(make_map(&p.tm_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dX, K, M, K * 2, 32, 32,
-                                   CU_TENSOR_MAP_SWIZZLE_64B));
+            if (!f32_out)
+                QLORA_TRY(make_map(&p.tm_out,
+                                   F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dX, K,
+                                   M, K * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B));
             p.m_tiles = ceil_div(M, 2 * 128 * kBMT);
             p.n_tiles = ceil_div(K, 2 * kBBN);
-            if (dx_dtype == QLORA_BF16)
-                QLORA_TRY((launch_gemm_pair<kBNf4MN, kEpiBf16, kBMT>(p, dev, s, QLORA_KERNEL_BWD_FUSED)));
+            if (!f32_out)
+                QLORA_TRY((launch_gemm_pair<kBNf4MN, kEpiBf16, kBMT, F16>(p, dev, s, QLORA_KERNEL_BWD_FUSED)));
             else
-                QLORA_TRY((launch_gemm_pair<kBNf4MN, kEpiF32, kBMT>(p, dev, s, QLORA_KERNEL_BWD_FUSED)));
-        } else if (dx_dtype == QLORA_BF16)
-            QLORA_TRY((launch_gemm<kBBN, kBNf4MN, kEpiBf16, kBMT>(p, dev, s, QLORA_KERNEL_BWD_FUSED)));
+                QLORA_TRY((launch_gemm_pair<kBNf4MN, kEpiF32, kBMT, F16>(p, dev, s, QLORA_KERNEL_BWD_FUSED)));
+        } else if (!f32_out)
+            QLORA_TRY((launch_gemm<kBBN, kBNf4MN, kEpiBf16, kBMT, F16>(p, dev, s, QLORA_KERNEL_BWD_FUSED)));
         else
-            QLORA_TRY((launch_gemm<kBBN, kBNf4MN, kEpiF32, kBMT>(p, dev, s, QLORA_KERNEL_BWD_FUSED)));
+            QLORA_TRY((launch_gemm<kBBN, kBNf4MN, kEpiF32, kBMT, F16>(p, dev, s, QLORA_KERNEL_BWD_FUSED)));
+        if (drop) {
+            // dX = frozen path + (bf16(G) A) * mask / (1 - p): the adapter product
+            // alone (LoRA steps only), its epilogue adding the masked term
+            GemmParams q{};
+            QLORA_TRY(map_bf16(&q.tm_a2, G2, hl_cols, M, hl_cols, 64, 128 * kBMT));   // hi chunks of G
+            QLORA_TRY(map_bf16(&q.tm_b2, A, K, r, K, 64, 64));                        // A[j][k]: MN-major operand
+            q.tm_a = q.tm_a2;   // main operands unused (no main steps)
+            q.tm_b = q.tm_b2;
+            q.a2_x_step = 128;
+            q.m_tiles = ceil_div(M, 128 * kBMT);
+            q.n_tiles = ceil_div(K, kBBN);
+            q.splits = 1;
+            q.k_stages_total = 0;
+            q.k_stages_split = 0;
+            q.k_stages_lora = pl.r_pad / 64;
+            q.out = dX;
+            q.out_ld = K;
+            q.m_total = (int)M;
+            q.n_total = (int)K;
+            q.drop_mask = opts->dropout_mask;
+            q.drop_base = reinterpret_cast<const float *>(ws + pl.off_dxs);
+            q.drop_scale = dropout_scale(opts);
+            if (dx_dtype != QLORA_FP32)
+                QLORA_TRY((launch_gemm<kBBN, kBTmaMN, kEpiDropBf16, kBMT, F16>(q, dev, s, QLORA_KERNEL_BWD_FUSED)));
+            else
+                QLORA_TRY((launch_gemm<kBBN, kBTmaMN, kEpiDropF32, kBMT, F16>(q, dev, s, QLORA_KERNEL_BWD_FUSED)));
+        }
     }
 
     // dA = (X^T [G_hi | G_lo])^T and dB = dY^T [H_hi | H_lo] in one launch: output rows k
@@ -451,10 +603,10 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *
     // contraction over the tokens; the reduction adds the halves
     {
         const int *maxc = nullptr;
-        QLORA_TRY((skinny_setup<128, 1, 1>(dev, &maxc)));
+        QLORA_TRY((skinny_setup<128, 1, 1, F16>(dev, &maxc)));
         SkinnyParams p{};
         SkinnyJob &Ja = p.job[0], &Jb = p.job[1];
-        QLORA_TRY(map_bf16(&Ja.tm_a, X, K, M, K, 64, 64));               // MN-major: rows k, contraction m
+        QLORA_TRY(map_bf16(&Ja.tm_a, Xa, K, M, K, 64, 64));              // MN-major: rows k, contraction m
         QLORA_TRY(map_bf16(&Ja.tm_b, G2, hl_cols, M, hl_cols, 64, 64));
         QLORA_TRY(map_bf16(&Jb.tm_a, dY, N, M, N, 64, 64));
         QLORA_TRY(map_bf16(&Jb.tm_b, H2, hl_cols, M, hl_cols, 64, 64));
@@ -477,7 +629,31 @@ extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *
         // after the dX GEMM nothing read here comes from the kernel just before
         p.wait_at_end = dX ? 1 : 0;
         const int cs = choose_csize(tiles_a + tiles_b, Ja.k_total, maxc);
-        QLORA_TRY((launch_skinny<128, 1, 1>(p, tiles_a + tiles_b, cs, dev, s, QLORA_KERNEL_WGRAD)));
+        QLORA_TRY((launch_skinny<128, 1, 1, F16>(p, tiles_a + tiles_b, cs, dev, s, QLORA_KERNEL_WGRAD)));
     }
     return launch_status();
+}
+
+extern "C" qlora_status qlora_linear_bwd_ex(const qlora_nf4_weight *w, const void *X, const void *dY, int64_t M,
+                                            const void *A, const void *B, int32_t r, float scale,
+                                            const float *H_saved, void *dX, qlora_dtype dx_dtype, float *dA,
+                                            float *dB, void *workspace, size_t workspace_bytes, void *stream,
+                                            const qlora_linear_opts *opts)
+{
+    QLORA_TRY(check_linear(w, X, M, A, B, r, workspace));
+    QLORA_TRY(check_opts(opts));
+    if (opts && opts->compute_dtype == QLORA_FP16)
+        return linear_bwd<true>(w, X, dY, M, A, B, r, scale, H_saved, dX, dx_dtype, dA, dB, workspace, workspace_bytes,
+                                stream, opts);
+    return linear_bwd<false>(w, X, dY, M, A, B, r, scale, H_saved, dX, dx_dtype, dA, dB, workspace, workspace_bytes,
+                             stream, opts);
+}
+
+extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *X, const void *dY, int64_t M,
+                                         const void *A, const void *B, int32_t r, float scale,
+                                         const float *H_saved, void *dX, qlora_dtype dx_dtype, float *dA, float *dB,
+                                         void *workspace, size_t workspace_bytes, void *stream)
+{
+    return qlora_linear_bwd_ex(w, X, dY, M, A, B, r, scale, H_saved, dX, dx_dtype, dA, dB, workspace, workspace_bytes,
+                               stream, nullptr);
 }

@@ -5,7 +5,7 @@
 // both produce the same bits.
 //
 // Per block of 64 weights: c1' = fmaf(E4M3value(code2), c2, mean); per weight:
-// w = bf16_RNE(RN32(q[code] * c1')).
+// w = bf16_RNE(RN32(q[code] * c1')) (fp16_RNE for the fp16 compute dtype).
 #pragma once
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -34,6 +34,24 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return d;
 }
 
+// Two binary32 values rounded to nearest-even binary16, lo in bits 0-15.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi)
+{
+    uint32_t d;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
+// The 16-bit compute type's pair packing: bf16 (default) or fp16.
+template <bool F16>
+__device__ __forceinline__ uint32_t pack16x2(float lo, float hi)
+{
+    if constexpr (F16)
+        return pack_f16x2(lo, hi);
+    else
+        return pack_bf16x2(lo, hi);
+}
+
 // (a, b) * (s, s), each lane an IEEE round-to-nearest-even product.
 __device__ __forceinline__ void mul2(float a, float b, float s, float &ra, float &rb)
 {
@@ -51,10 +69,12 @@ __device__ __forceinline__ float lut_at(const float *lut, uint32_t off)
     return *reinterpret_cast<const float *>(reinterpret_cast<const char *>(lut) + off);
 }
 
-// 8 consecutive codes (one 32-bit word, element 0 in bits 0-3) -> 8 bf16 in a
-// 16-byte vector (element 0 in the lowest 16 bits).  The byte offsets of the
-// even and the odd codes are formed once per word; each element then costs
-// one byte extraction and one shared-memory load.
+// 8 consecutive codes (one 32-bit word, element 0 in bits 0-3) -> 8 bf16 (or,
+// with F16, fp16: the fp16 compute dtype) in a 16-byte vector (element 0 in
+// the lowest 16 bits).  The byte offsets of the even and the odd codes are
+// formed once per word; each element then costs one byte extraction and one
+// shared-memory load.
+template <bool F16 = false>
 __device__ __forceinline__ uint4 expand8(uint32_t word, const float *lut, float c1p)
 {
     const uint32_t ev = (word << 2) & 0x3C3C3C3Cu;   // byte k: 4 * code of element 2k
@@ -73,7 +93,7 @@ __device__ __forceinline__ uint4 expand8(uint32_t word, const float *lut, float 
     for (int i = 0; i < 4; i++) {
         float lo, hi;
         mul2(q[2 * i], q[2 * i + 1], c1p, lo, hi);
-        o[i] = pack_bf16x2(lo, hi);
+        o[i] = pack16x2<F16>(lo, hi);
     }
     return make_uint4(o[0], o[1], o[2], o[3]);
 }

@@ -361,13 +361,13 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
     return d;
 }
 
-// Instruction descriptor for kind::f16 with bf16 A/B and fp32 D.
-// a_mn / b_mn: operand is MN-major (1) or K-major (0).
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn)
+// Instruction descriptor for kind::f16 with bf16 A/B (fp16 A/B when f16)
+// and fp32 D.  a_mn / b_mn: operand is MN-major (1) or K-major (0).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn, bool f16 = false)
 {
     return (1u << 4)                       // D format: f32
-           | (1u << 7)                     // A format: bf16
-           | (1u << 10)                    // B format: bf16
+           | ((f16 ? 0u : 1u) << 7)        // A format: bf16 (1) or f16 (0)
+           | ((f16 ? 0u : 1u) << 10)       // B format: bf16 (1) or f16 (0)
            | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16)
            | ((uint32_t)(N >> 3) << 17)    // N / 8
            | ((uint32_t)(M >> 4) << 24);   // M / 16

@@ -78,7 +78,7 @@ typedef enum {
     QLORA_ERR_TIMEOUT = 7      /* a kernel's bounded wait gave up (device)    */
 } qlora_status;
 
-typedef enum { QLORA_BF16 = 0, QLORA_FP32 = 1 } qlora_dtype;
+typedef enum { QLORA_BF16 = 0, QLORA_FP32 = 1, QLORA_FP16 = 2 } qlora_dtype;
 
 /*
  * A quantized weight W [rows, cols] (rows = N = out_features, cols = K =
@@ -126,6 +126,19 @@ typedef struct {
 QLORA_API qlora_status qlora_build_nf4_codebook(double delta, float codebook_out[16]);
 
 /*
+ * qlora_build_nfk_codebook -- k-bit NormalFloat (k = 2, 3, 4) from the same
+ * construction, held in the 16-entry table of the 4-bit codec: the 2^k NF-k
+ * values (ascending, -1 .. 1, one zero), then 16 - 2^k padding values beyond
+ * +-1 (half at -1 - i/4 below -1, half at 1 + i/4 above 1, i = 1, 2, ...),
+ * which are never the nearest value to a scaled element; k = 4 is NF4 itself.
+ *   delta  tail probability in (0, 0.5); <= 0 selects
+ *          1/2 (1/(2 * 2^k) + 1/(2 (2^k - 1))).
+ * Host-only, no CUDA call.  Errors: QLORA_ERR_INVALID_ARG (null pointer, k
+ * outside 2..4, delta >= 0.5).
+ */
+QLORA_API qlora_status qlora_build_nfk_codebook(int k, double delta, float codebook_out[16]);
+
+/*
  * qlora_build_int4_codebook -- a 4-bit integer table for the same codec and
  * GEMMs ("Introduction", item (1), names 4-bit integers as the baseline NF4
  * is compared with, without defining them).  Reading: the two's-complement
@@ -166,8 +179,8 @@ QLORA_API size_t qlora_quantize_workspace_bytes(int64_t rows, int64_t cols);
  * mean = binary32 nearest to the exact mean of all c1 (ties to even); per
  * group: d = RN32(c1 - mean), c2 = RN32(max|d| / 448), code2 = E4M3 with
  * round-to-nearest-even and saturation of RN32(d / c2) (all zero if c2 = 0).
- *   W          device, rows*cols elements of w_dtype (QLORA_BF16 or
- *              QLORA_FP32), row-major.
+ *   W          device, rows*cols elements of w_dtype (QLORA_BF16, QLORA_FP16
+ *              or QLORA_FP32), row-major.
  *   out        host struct: rows, cols, the four device buffers (written) and
  *              the codebook (read).  rows >= 1, cols % 64 == 0.
  *   workspace  device, at least qlora_quantize_workspace_bytes(rows, cols)
@@ -230,6 +243,14 @@ QLORA_API qlora_status qlora_quantize_nf4_dq_noalloc(const void *W, qlora_dtype 
  * Errors: INVALID_ARG, SHAPE, ALIGNMENT, CUDA, UNSUPPORTED.
  */
 QLORA_API qlora_status qlora_dequantize_nf4_dq(const qlora_nf4_weight *w, void *out_bf16, void *stream);
+
+/*
+ * qlora_dequantize_nf4_dq_ex -- the same with the output type out_dtype:
+ * QLORA_BF16 (as above) or QLORA_FP16 (w = fp16_RNE(RN32(q[code] * c1')),
+ * the fp16 compute dtype).  Errors as above, INVALID_ARG for another dtype.
+ */
+QLORA_API qlora_status qlora_dequantize_nf4_dq_ex(const qlora_nf4_weight *w, void *out, qlora_dtype out_dtype,
+                                                  void *stream);
 
 /*
  * Workspace in bytes for qlora_linear_fwd / qlora_linear_bwd at these sizes
@@ -356,7 +377,7 @@ QLORA_API qlora_status qlora_adamw_step(float *param, void *param_bf16, const fl
  *                     qlora_linear_fwd, A[l] device bf16 [r][in], B[l] device
  *                     bf16 [out][r].
  *   norm1, norm2      device bf16 [hidden] (frozen).
- * Constraints: heads * head_dim == hidden, head_dim % 8 == 0, hidden % 64 ==
+ * Constraints: heads * head_dim == hidden, head_dim % 16 == 0, hidden % 64 ==
  * 0, inter % 64 == 0, seq % 8 == 0, r as for the linear layer.
  */
 typedef struct {
@@ -396,6 +417,55 @@ QLORA_API qlora_status qlora_block_fwd(const qlora_block *blk, const void *x, vo
 QLORA_API qlora_status qlora_block_bwd(const qlora_block *blk, const void *x, const void *dy, void *dx,
                                        float *const dA[7], float *const dB[7], void *workspace,
                                        size_t workspace_bytes, void *stream);
+
+/*
+ * Options of the QLoRA linear layer (the _ex entry points below; the plain
+ * entry points are the _ex ones with opts = NULL).
+ *   dropout_mask  device or NULL.  LoRA dropout on the adapter input (the
+ *                 blog "Efficient Language Model Fine-Tuning with QLoRA on
+ *                 Resource-Constrained Hardware", LoraConfig snippet,
+ *                 lora_dropout): the adapter branch sees X_d = X * mask /
+ *                 (1 - p) while the frozen weight sees X.  Bit (k % 8) of
+ *                 byte (m * K + k) / 8 is element (m, k)'s mask bit (1 =
+ *                 kept); M * K / 8 bytes, 16-byte aligned.  Kept elements
+ *                 are bf16(RN32(x * RN32(1 / RN32(1 - p)))), dropped ones 0.
+ *                 The same mask must be passed to the forward and the
+ *                 backward call of one step.  With dropout:
+ *                     H  = s X_d A^T
+ *                     dX = dY W' + (bf16(G) A) * mask / (1 - p)
+ *                     dA = G^T X_d,  dB = dY^T H
+ *   dropout_p     probability the mask was drawn with, 0 <= p < 1.
+ *   compute_dtype QLORA_BF16 (0, the default) or QLORA_FP16: the 16-bit type
+ *                 of X, A, B, dY, of the expanded weight (w = fp16_RNE(RN32(
+ *                 q[code] * c1')) for fp16) and of 16-bit outputs; y_dtype and
+ *                 dx_dtype are then that type or QLORA_FP32 (the blog's
+ *                 BitsAndBytesConfig snippet, bnb_4bit_compute_dtype).  H and
+ *                 G are carried as hi + lo pairs of the same type.
+ */
+typedef struct {
+    const uint8_t *dropout_mask;
+    float dropout_p;
+    qlora_dtype compute_dtype;
+} qlora_linear_opts;
+
+/* Workspace bytes for the _ex entry points with these options (dropout needs
+ * 6 M K bytes more than qlora_linear_workspace_bytes). */
+QLORA_API size_t qlora_linear_workspace_bytes_ex(int64_t M, int64_t N, int64_t K, int32_t r,
+                                                 const qlora_linear_opts *opts);
+
+/* qlora_linear_fwd / qlora_linear_bwd with options (NULL: none).  Errors as
+ * for the plain calls, plus INVALID_ARG for p outside [0, 1), an unknown
+ * compute dtype or an output dtype that does not match it, and ALIGNMENT for
+ * a misaligned mask. */
+QLORA_API qlora_status qlora_linear_fwd_ex(const qlora_nf4_weight *w, const void *X, int64_t M, const void *A,
+                                           const void *B, int32_t r, float scale, void *Y, qlora_dtype y_dtype,
+                                           float *H_save, void *workspace, size_t workspace_bytes, void *stream,
+                                           const qlora_linear_opts *opts);
+QLORA_API qlora_status qlora_linear_bwd_ex(const qlora_nf4_weight *w, const void *X, const void *dY, int64_t M,
+                                           const void *A, const void *B, int32_t r, float scale,
+                                           const float *H_saved, void *dX, qlora_dtype dx_dtype, float *dA,
+                                           float *dB, void *workspace, size_t workspace_bytes, void *stream,
+                                           const qlora_linear_opts *opts);
 
 /* Human-readable name of a status code (static string, never NULL). */
 QLORA_API const char *qlora_status_string(qlora_status status);

@@ -71,6 +71,30 @@ def nfk_codebook_f64(k: int = 4, delta: float = DEFAULT_DELTA) -> np.ndarray:
     return np.array(values, dtype=np.float64)
 
 
+def nfk_default_delta(k: int) -> float:
+    """The default tail probability of the NF-k reading above for any k: the
+    centre of the outermost equal-mass bin, averaged over the 2^k- and
+    (2^k - 1)-level halves (for k = 4 this is DEFAULT_DELTA)."""
+    n = 2 ** k
+    return 0.5 * (1.0 / (2 * n) + 1.0 / (2 * (n - 1)))
+
+
+def nfk_table(k: int, delta: float = None) -> np.ndarray:
+    """NF-k (k = 2, 3, 4) as the 16 binary32 values the 4-bit codec stores:
+    the 2^k NF-k values (rounded once), with 16 - 2^k padding values beyond
+    +-1 (half below -1 at -1 - i/4, half above +1 at 1 + i/4, i = 1, 2, ...),
+    which are never the nearest value of anything in [-1, 1]; for k = 4 the
+    table is NF4 itself."""
+    if k not in (2, 3, 4):
+        raise ValueError("k must be 2, 3 or 4")
+    d = nfk_default_delta(k) if delta is None else delta
+    vals = list(nfk_codebook_f64(k, d).astype(np.float32))
+    half = (16 - 2 ** k) // 2
+    below = [np.float32(-1.0 - i / 4.0) for i in range(half, 0, -1)]
+    above = [np.float32(1.0 + i / 4.0) for i in range(1, half + 1)]
+    return np.array(below + vals + above, dtype=np.float32)
+
+
 def nf4_codebook(delta: float = DEFAULT_DELTA) -> np.ndarray:
     """NF4 as the 16 binary32 values the codec stores (rounded once)."""
     return nfk_codebook_f64(4, delta).astype(np.float32)

@@ -56,6 +56,8 @@ def _load():
         lib.oracle_dq_encode.argtypes = [P, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, P, P]
         lib.oracle_dequantize.argtypes = [P, P, P, ctypes.c_float, P, ctypes.c_int64,
                                           ctypes.c_int32, P]
+        lib.oracle_dequantize_f32.argtypes = [P, P, P, ctypes.c_float, P, ctypes.c_int64,
+                                              ctypes.c_int32, P]
         _lib = lib
     return _lib
 
@@ -150,6 +152,24 @@ def dequantize(packed, e, c2, mean, q, group: int = GROUP) -> np.ndarray:
     lib.oracle_dequantize(_ptr(packed), _ptr(e), _ptr(c2), float(mean), _ptr(q),
                           nblocks, group, _ptr(w))
     return w
+
+
+def dequantize_f16(packed, e, c2, mean, q, group: int = GROUP) -> np.ndarray:
+    """fp16 bit patterns (uint16 [numel]) of the tensor dequantized for the fp16
+    compute dtype: RN32(q[code] * c1') (C loops) rounded to nearest-even
+    binary16 (numpy's conversion)."""
+    lib = _load()
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    e = np.ascontiguousarray(e, dtype=np.uint8)
+    c2 = np.ascontiguousarray(c2, dtype=np.float32)
+    q = np.ascontiguousarray(q, dtype=np.float32)
+    nblocks = e.size
+    if packed.size != nblocks * BLOCK // 2:
+        raise ValueError("packed / e size mismatch")
+    w = np.empty(nblocks * BLOCK, np.float32)
+    lib.oracle_dequantize_f32(_ptr(packed), _ptr(e), _ptr(c2), float(mean), _ptr(q),
+                              nblocks, group, _ptr(w))
+    return w.astype(np.float16).view(np.uint16)
 
 
 def storage_bits_per_param(numel: int, group: int = GROUP) -> float:

@@ -78,7 +78,13 @@ def backward_weight_grads(X, A, B, s: float, dY):
 #   dA = s (dY B)^T X_d,   dB = s dY^T (X_d A^T)
 
 def dropout_scale(p: float) -> np.float32:
-    return np.float32(1.0 / np.float64(np.float32(1.0) - np.float32(p))) if p > 0 else np.float32(1.0)
+    """RN32(1 / RN32(1 - p)): one correctly rounded binary32 quotient (exact
+    rational arithmetic, no intermediate rounding)."""
+    from fractions import Fraction
+
+    from . import exact
+    keep = np.float32(np.float32(1.0) - np.float32(p))
+    return exact.rn32(Fraction(1) / Fraction(float(keep)))
 
 
 def dropout_input(X, mask, p: float, bf16_round=True) -> np.ndarray:

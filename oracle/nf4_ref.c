@@ -191,3 +191,23 @@ void oracle_dequantize(const uint8_t *packed, const uint8_t *e, const float *c2,
         }
     }
 }
+
+/* The products RN32(q[code] * c1') before the 16-bit rounding: the fp16
+ * compute dtype rounds these to binary16 (the caller does that). */
+void oracle_dequantize_f32(const uint8_t *packed, const uint8_t *e, const float *c2,
+                           float mu, const float q[16], int64_t nblocks, int32_t group,
+                           float *w)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t b = 0; b < nblocks; b++) {
+        float ev = (float)oracle_e4m3_value(e[b]);
+        float c1p = fmaf(ev, c2[b / group], mu);
+        for (int i = 0; i < 64; i++) {
+            int64_t idx = 64 * b + i;
+            uint8_t byte = packed[idx / 2];
+            int code = (idx & 1) ? (byte >> 4) : (byte & 15);
+            w[idx] = q[code] * c1p;
+        }
+    }
+}
+

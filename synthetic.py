@@ -40,14 +40,15 @@ def tiny_linear(seed: int = 0, device="cpu") -> dict:
 
 
 def linear_case(M: int, N: int, K: int, r: int, alpha: float, seed: int, w_dtype=torch.bfloat16,
-                device="cpu") -> dict:
-    """One QLoRA linear problem with the workload's distributions."""
+                device="cpu", act_dtype=torch.bfloat16) -> dict:
+    """One QLoRA linear problem with the workload's distributions (act_dtype:
+    the 16-bit compute dtype of X, A, B and dY)."""
     return {
         "W": normal((N, K), 0.02, seed, w_dtype, device),
-        "X": normal((M, K), 1.0, seed + 1, torch.bfloat16, device),
-        "A": normal((r, K), 1.0 / r, seed + 2, torch.bfloat16, device),
-        "B": normal((N, r), 0.01, seed + 3, torch.bfloat16, device),
-        "dY": normal((M, N), 1.0, seed + 4, torch.bfloat16, device),
+        "X": normal((M, K), 1.0, seed + 1, act_dtype, device),
+        "A": normal((r, K), 1.0 / r, seed + 2, act_dtype, device),
+        "B": normal((N, r), 0.01, seed + 3, act_dtype, device),
+        "dY": normal((M, N), 1.0, seed + 4, act_dtype, device),
         "r": r, "alpha": alpha, "scale": alpha / r, "M": M, "N": N, "K": K,
     }
 
@@ -72,3 +73,14 @@ def block_case(batch: int, seq: int, hidden: int, heads: int, inter: int, r: int
         "batch": batch, "seq": seq, "hidden": hidden, "heads": heads, "inter": inter, "r": r,
         "alpha": alpha, "scale": alpha / r,
     }
+
+
+def dropout_mask(M: int, K: int, p: float, seed: int, device="cpu"):
+    """LoRA-dropout keep mask: (bool [M, K] with P(kept) = 1 - p, and the same
+    mask packed 8 elements per byte, bit k % 8 of byte (m*K + k) / 8)."""
+    g = _gen(seed)
+    keep = torch.rand(M, K, generator=g) >= p
+    bits = keep.reshape(-1, 8).to(torch.uint8)
+    weights = torch.tensor([1, 2, 4, 8, 16, 32, 64, 128], dtype=torch.uint8)
+    packed = (bits * weights).sum(dim=1).to(torch.uint8)
+    return keep, packed.to(device)

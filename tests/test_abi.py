@@ -71,6 +71,17 @@ def test_int4_codebook_matches_oracle_bit_for_bit(lib):
     assert lib.qlora_build_int4_codebook(None) == 1
 
 
+@pytest.mark.parametrize("k", [2, 3, 4])
+def test_nfk_codebook_matches_oracle_bit_for_bit(lib, k):
+    out = (ctypes.c_float * 16)()
+    lib.qlora_build_nfk_codebook.argtypes = [ctypes.c_int, ctypes.c_double, ctypes.c_void_p]
+    assert lib.qlora_build_nfk_codebook(k, 0.0, ctypes.cast(out, ctypes.c_void_p)) == 0
+    got = np.array(list(out), np.float32)
+    assert np.array_equal(got.view(np.uint32), ocb.nfk_table(k).view(np.uint32))
+    assert lib.qlora_build_nfk_codebook(5, 0.0, ctypes.cast(out, ctypes.c_void_p)) == 1
+    assert lib.qlora_build_nfk_codebook(3, 0.5, ctypes.cast(out, ctypes.c_void_p)) == 1
+
+
 def test_fp4_codebook_matches_oracle_bit_for_bit(lib):
     out = (ctypes.c_float * 16)()
     lib.qlora_build_fp4_codebook.argtypes = [ctypes.c_void_p]

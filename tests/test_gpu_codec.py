@@ -115,6 +115,33 @@ def test_fp4_codebook(q):
         assert codes.min() >= 1, "index 0 (-8/6) is never the nearest value"
 
 
+@pytest.mark.parametrize("k", [2, 3])
+def test_nfk_codebooks(q, k):
+    """NF3 and NF2 through the 4-bit quantizer and dequantizer, bit-exact;
+    the padding codes beyond +-1 are never emitted."""
+    table = q.qlora_build_nfk_codebook(k)
+    W = synthetic.normal((300, 512), 0.02, 40 + k, torch.bfloat16)
+    w, ref = check_parity(q, W, codebook=table)
+    pad = (16 - 2 ** k) // 2
+    codes = occ.unpack(ref["packed"])
+    assert codes.min() >= pad and codes.max() < 16 - pad
+
+
+def test_fp16_input_and_fp16_dequantization(q):
+    """The fp16 compute dtype: fp16 weights quantize bit-exactly (the oracle
+    reads them as the float32 values they are), and the dequantizer's fp16
+    output is fp16_RNE(RN32(q * c1')) bit for bit."""
+    for shape, seed in (((257, 320), 51), ((4096, 4096), 52)):
+        W = synthetic.normal(shape, 0.02, seed, torch.float16)
+        w, ref = check_parity(q, W)
+        out = torch.empty(shape, dtype=torch.float16, device="cuda")
+        q.qlora_dequantize_nf4_dq(w, out)
+        torch.cuda.synchronize()
+        got = out.view(torch.int16).cpu().numpy().view(np.uint16).ravel()
+        want = occ.dequantize_f16(ref["packed"], ref["e"], ref["c2"], ref["mean"], Q)
+        assert np.array_equal(got, want)
+
+
 def test_edge_blocks(q):
     """Zero blocks, a subnormal block, values exactly on the round-down
     midpoints (ties go to the lower code), and +-absmax."""

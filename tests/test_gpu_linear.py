@@ -41,14 +41,20 @@ def half_ulp_bf16(ref):
     return 2.0 ** (e - 8)
 
 
-def assert_close(got, ref, bf16_out=False, what=""):
+def half_ulp_f16(ref):
+    a = np.abs(np.asarray(ref, np.float64))
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -14)))
+    return 2.0 ** (e - 11)
+
+
+def assert_close(got, ref, bf16_out=False, what="", f16_out=False):
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
     assert got.shape == ref.shape, what
     assert np.all(np.isfinite(got)), what
     rel = olin.rel_frobenius(got, ref)
     assert rel <= REL_FRO, f"{what}: rel Frobenius {rel:.3e}"
-    bound = MAX_ABS + (half_ulp_bf16(ref) if bf16_out else 0.0)
+    bound = MAX_ABS + (half_ulp_bf16(ref) if bf16_out else 0.0) + (half_ulp_f16(ref) if f16_out else 0.0)
     err = np.abs(got - ref)
     worst = np.unravel_index(np.argmax(err - bound), err.shape) if err.size else None
     assert np.all(err <= bound), f"{what}: max abs {err.max():.3e} at {worst}"
@@ -58,6 +64,13 @@ def oracle_weight(W, codebook=Q):
     ref = occ.quantize(W.float().numpy(), codebook)
     Wd = occ.dequantize(ref["packed"], ref["e"], ref["c2"], ref["mean"], codebook)
     return occ.bf16_bits_to_f32(Wd).reshape(W.shape).astype(np.float64)
+
+
+def oracle_weight_f16(W, codebook=Q):
+    """The weight as the fp16 compute dtype expands it."""
+    ref = occ.quantize(W.float().numpy(), codebook)
+    bits = occ.dequantize_f16(ref["packed"], ref["e"], ref["c2"], ref["mean"], codebook)
+    return bits.view(np.float16).reshape(W.shape).astype(np.float64)
 
 
 class Runner:
@@ -280,3 +293,88 @@ def test_argument_errors(q):
     with pytest.raises(q.QLoraError) as e:
         q.qlora_linear_fwd(run.w, run.X, 16, run.A, run.B, 12, 2.0, Y, None, run.ws)
     assert e.value.status == 2
+
+
+@pytest.mark.parametrize("M,N,K,r,p", [
+    (16, 384, 320, 16, 0.1),      # decode forward
+    (200, 384, 512, 64, 0.05),    # single-CTA fused GEMMs
+    (600, 264, 576, 64, 0.5),     # CTA pairs, ragged
+    (4096, 4096, 4096, 64, 0.05), # LLaMA-7B attention shape, the blog's p
+])
+def test_lora_dropout(q, M, N, K, r, p):
+    """LoRA dropout on the adapter input (the blog's LoraConfig snippet,
+    lora_dropout): Y, dX (bf16) and dA, dB against the oracle on the same
+    mask; the frozen path sees the undropped input."""
+    case = synthetic.linear_case(M, N, K, r, alpha=16.0, seed=3000 + M)
+    keep, packed = synthetic.dropout_mask(M, K, p, seed=3100 + M, device="cuda")
+    run = Runner(q, case)
+    run.ws = torch.empty(q.qlora_linear_workspace_bytes(M, N, K, r, dropout=(packed, p)), dtype=torch.uint8,
+                         device="cuda")
+    s = case["scale"]
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    H = torch.empty(M, r, dtype=torch.float32, device="cuda")
+    q.qlora_linear_fwd(run.w, run.X, M, run.A, run.B, r, s, Y, H, run.ws, dropout=(packed, p))
+    dX = torch.empty(M, K, dtype=torch.bfloat16, device="cuda")
+    dA = torch.empty(r, K, dtype=torch.float32, device="cuda")
+    dB = torch.empty(N, r, dtype=torch.float32, device="cuda")
+    q.qlora_linear_bwd(run.w, run.X, run.dY, M, run.A, run.B, r, s, H, dX, dA, dB, run.ws, dropout=(packed, p))
+    q.qlora_check_device_error()
+    Wd = oracle_weight(case["W"])
+    X, A, B, dY = (np64(case[k]) for k in ("X", "A", "B", "dY"))
+    keep = keep.numpy()
+    Xd = olin.dropout_input(case["X"].float().numpy(), keep, p)
+    rows = np.arange(M) if M <= 600 else np.sort(np.random.default_rng(7).choice(M, 48, replace=False))
+    rY = olin.forward_dropout(X[rows], Wd, A, B, s, Xd[rows])
+    assert_close(np64(Y)[rows], rY, bf16_out=True, what="Y")
+    np.testing.assert_allclose(np64(H), s * Xd @ A.T, rtol=1e-5, atol=1e-5)
+    rdX, rdA, rdB = olin.backward_dropout(X, Wd, A, B, s, dY, Xd, keep, p) if M <= 600 else (None, None, None)
+    if rdX is None:
+        G = dY @ B
+        rdX = (dY[rows] @ Wd) + s * (G[rows] @ A) * (keep[rows] * np.float64(olin.dropout_scale(p)))
+        rdA, rdB = s * (G.T @ Xd), s * (dY.T @ (Xd @ A.T))
+        assert_close(np64(dX)[rows], rdX, bf16_out=True, what="dX")
+    else:
+        assert_close(np64(dX), rdX, bf16_out=True, what="dX")
+    assert_close(np64(dA), rdA, what="dA")
+    assert_close(np64(dB), rdB, what="dB")
+
+
+
+@pytest.mark.parametrize("M", [16, 200, 600])
+@pytest.mark.parametrize("odt", [torch.float16, torch.float32])
+def test_fp16_compute_dtype(q, M, odt):
+    """The fp16 compute dtype (the blog's BitsAndBytesConfig snippet,
+    bnb_4bit_compute_dtype=torch.float16): fp16 X, A, B, dY, the weight
+    expanded to fp16, fp16 or fp32 outputs; through the decode (16 tokens),
+    single-CTA (200) and CTA-pair (600) kernels."""
+    case = synthetic.linear_case(M, 384, 512, 64, alpha=16.0, seed=4000 + M, act_dtype=torch.float16)
+    run = Runner(q, case)
+    Wd = oracle_weight_f16(case["W"])
+    X, A, B, dY = (np64(case[k]) for k in ("X", "A", "B", "dY"))
+    s = case["scale"]
+    f16 = odt == torch.float16
+    Y, H = run.fwd(odt, save_h=True)
+    assert_close(np64(Y), olin.forward(X, Wd, A, B, s), f16_out=f16, what="Y")
+    dX, dA, dB = run.bwd(odt, H=H)
+    rdX, rdA, rdB = olin.backward(X, Wd, A, B, s, dY)
+    assert_close(np64(dX), rdX, f16_out=f16, what="dX")
+    assert_close(np64(dA), rdA, what="dA")
+    assert_close(np64(dB), rdB, what="dB")
+
+
+def test_fp16_compute_dtype_llama7b_gate(q):
+    """fp16 compute dtype at the LLaMA-7B gate shape (11008 x 4096), 4096 tokens:
+    Y and dX on sampled rows, dA and dB in full."""
+    case = synthetic.linear_case(4096, 11008, 4096, 64, alpha=16.0, seed=4100, act_dtype=torch.float16)
+    run = Runner(q, case)
+    Wd = oracle_weight_f16(case["W"])
+    X, A, B, dY = (np64(case[k]) for k in ("X", "A", "B", "dY"))
+    s = case["scale"]
+    rows = np.sort(np.random.default_rng(11).choice(4096, 48, replace=False))
+    Y, H = run.fwd(torch.float16, save_h=True)
+    assert_close(np64(Y)[rows], olin.forward_rows(X, Wd, A, B, s, rows), f16_out=True, what="Y")
+    dX, dA, dB = run.bwd(torch.float16, H=H)
+    assert_close(np64(dX)[rows], olin.backward_dx_rows(Wd, A, B, s, dY, rows), f16_out=True, what="dX")
+    rdA, rdB = olin.backward_weight_grads(X, A, B, s, dY)
+    assert_close(np64(dA), rdA, what="dA")
+    assert_close(np64(dB), rdB, what="dB")

@@ -104,3 +104,29 @@ def test_fp4_table_structure():
         assert v == np.float32(want / 6.0)
     # the pad below -1 is never the nearest value of anything in [-1, 1]
     assert (q[0] + q[1]) / 2 < -1.0
+
+
+
+@pytest.mark.parametrize("k", [2, 3, 4])
+def test_nfk_tables(k):
+    """NF-k in the 16-entry table: 2^k NormalFloat values with the page's
+    structure (2^(k-1) negative, one zero, 2^(k-1) positive, +-1 at the ends),
+    equally spaced probabilities behind them (undone with scipy's Phi), and
+    never-nearest pads beyond +-1."""
+    t = codebook.nfk_table(k)
+    assert len(t) == 16 and np.all(np.diff(t.astype(np.float64)) > 0)
+    n = 2 ** k
+    pad = (16 - n) // 2
+    v = t[pad:pad + n].astype(np.float64)
+    assert v[0] == -1.0 and v[-1] == 1.0 and np.count_nonzero(v == 0) == 1
+    assert np.count_nonzero(v < 0) == n // 2 - 1 and np.count_nonzero(v > 0) == n // 2
+    if pad:
+        assert (t[pad - 1] + t[pad]) / 2 < -1.0 and (t[pad + n - 1] + t[pad + n]) / 2 > 1.0
+    d = codebook.nfk_default_delta(k)
+    top = special.ndtri(1.0 - d)
+    for side in (v[v > 0], -v[v < 0]):
+        # the zero (probability 1/2) and the side's values, undone with Phi
+        steps = np.diff(np.sort(np.concatenate([[0.5], special.ndtr(side * top)])))
+        np.testing.assert_allclose(steps, steps[0], rtol=1e-6)
+    if k == 4:
+        assert np.array_equal(t.view(np.uint32), codebook.nf4_codebook().view(np.uint32))

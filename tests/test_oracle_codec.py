@@ -240,3 +240,25 @@ def test_storage_bits_per_parameter_match_the_page():
     saving = without_dq - bits
     assert saving == pytest.approx(FIG["dq_saving_bits"], abs=0.005)
     assert 65e9 * saving / 8 / 1e9 == pytest.approx(FIG["dq_saving_65b_gb"], abs=0.1)
+
+
+
+def test_fp16_dequantization_shares_the_products_of_the_bf16_one():
+    """The fp16 compute dtype rounds the same binary32 products RN32(q * c1')
+    to binary16: rounding those products to bf16 instead must give exactly the
+    bf16 dequantizer's bits, and every fp16 value must be the nearest binary16
+    of its product (checked against torch's conversion)."""
+    import torch
+    rng = np.random.default_rng(9)
+    W = (rng.standard_normal((64, 256)) * 0.02).astype(np.float32)
+    q = codebook.nf4_codebook()
+    ref = codec.quantize(W, q)
+    h = codec.dequantize_f16(ref["packed"], ref["e"], ref["c2"], ref["mean"], q)
+    lib = codec._load()
+    prods = np.empty(W.size, np.float32)
+    lib.oracle_dequantize_f32(codec._ptr(ref["packed"]), codec._ptr(ref["e"]), codec._ptr(ref["c2"]),
+                              float(ref["mean"]), codec._ptr(q), ref["e"].size, 256, codec._ptr(prods))
+    assert np.array_equal(codec.bf16_rne(prods),
+                          codec.dequantize(ref["packed"], ref["e"], ref["c2"], ref["mean"], q))
+    want = torch.from_numpy(prods).to(torch.float16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(h, want)

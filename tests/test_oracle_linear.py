@@ -145,8 +145,10 @@ def test_dropout_special_cases():
     # the scale of p = 0.5 is exactly 2 and the bf16 rounding of x * 2 is exact
     half = rng.random((M, K)) >= 0.5
     np.testing.assert_array_equal(linear.dropout_input(X.astype(np.float32), half, 0.5), X * 2 * half)
-    # the scale of p = 0.05: RN32(1 / RN32(0.95))
-    assert linear.dropout_scale(0.05) == np.float32(1.0 / np.float64(np.float32(0.95)))
+    # the scale of p = 0.05: RN32(1 / RN32(0.95)), checked against the correctly
+    # rounded float32 division of numpy
+    assert linear.dropout_scale(0.05) == np.float32(1.0) / np.float32(0.95)
+    assert linear.dropout_scale(0.1) == np.float32(1.0) / np.float32(0.9)
 
 
 def test_error_metrics():
