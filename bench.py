@@ -1016,6 +1016,7 @@ def main():
     ap.add_argument("--skip-block", action="store_true")
     ap.add_argument("--block-only", action="store_true", help="run only the transformer-block object (profiling runs)")
     ap.add_argument("--optim-only", action="store_true", help="run only the paged AdamW object (profiling runs)")
+    ap.add_argument("--decode-only", action="store_true", help="run only the decode-shaped forward (profiling runs)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--linears", default="llama7b",
                     help="llama7b (the seven linears of one layer) or NxK for one linear (profiling runs)")
@@ -1054,6 +1055,12 @@ def main():
             torch.cuda.set_device(local_rank)
             peaks, src = load_peaks()
             line = {"impl": "ours", "block7b": run_block7b(args, q, torch, torch.device("cuda", local_rank), peaks, src)}
+        elif args.decode_only:
+            import bit_nf4_quantized_16_b200 as q
+            torch.cuda.set_device(local_rank)
+            peaks, src = load_peaks()
+            line = {"impl": "ours",
+                    "decode65b": run_decode65b(args, q, torch, torch.device("cuda", local_rank), peaks, src)}
         elif args.optim_only:
             import bit_nf4_quantized_16_b200 as q
             torch.cuda.set_device(local_rank)

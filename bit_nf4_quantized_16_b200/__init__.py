@@ -13,7 +13,9 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libqlora_b200.so")
+# QLORA_B200_BUILD=debug selects the bounds-checked build (libqlora_b200_debug.so)
+LIB_PATH = os.path.join(_HERE, "libqlora_b200_debug.so" if os.environ.get("QLORA_B200_BUILD") == "debug"
+                        else "libqlora_b200.so")
 
 QLORA_BLOCK = 64
 QLORA_GROUP = 256
@@ -37,7 +39,7 @@ EXPORTS = (
     "qlora_dequantize_nf4_dq", "qlora_linear_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd",
     "qlora_status_string", "qlora_check_device_error",
     "qlora_timing_enable", "qlora_timing_reset", "qlora_timing_read", "qlora_launch_count",
-    "qlora_debug_inject_stall",
+    "qlora_debug_inject_stall", "qlora_debug_bounds", "qlora_debug_bounds_selftest",
     "qlora_paged_alloc", "qlora_paged_free", "qlora_paged_prefetch", "qlora_adamw_step",
     "qlora_block_workspace_bytes", "qlora_block_fwd", "qlora_block_bwd",
     "qlora_linear_workspace_bytes_ex", "qlora_linear_fwd_ex", "qlora_linear_bwd_ex",
@@ -107,6 +109,8 @@ def _load():
         "qlora_timing_read": (ctypes.c_int, [P, P]),
         "qlora_launch_count": (ctypes.c_int64, []),
         "qlora_debug_inject_stall": (ctypes.c_int, [ctypes.c_int, ctypes.c_uint64]),
+        "qlora_debug_bounds": (ctypes.c_int, [ctypes.c_char_p, S]),
+        "qlora_debug_bounds_selftest": (ctypes.c_int, []),
         "qlora_paged_alloc": (ctypes.c_int, [S, ctypes.POINTER(ctypes.c_void_p)]),
         "qlora_paged_free": (ctypes.c_int, [P]),
         "qlora_paged_prefetch": (ctypes.c_int, [P, S, ctypes.c_int, P]),
@@ -312,6 +316,20 @@ def qlora_debug_inject_stall(kind: str, timeout_ns: int = 1_000_000):
     kernel family `kind` ("quantize", "fwd_fused" or "bwd_fused"; None disarms)."""
     code = -1 if kind is None else KERNEL_KINDS.index(kind)
     _check(lib.qlora_debug_inject_stall(code, timeout_ns), "qlora_debug_inject_stall")
+
+
+def qlora_debug_bounds_selftest():
+    """Bounds-checked build only: records one failed check without touching memory."""
+    _check(lib.qlora_debug_bounds_selftest(), "qlora_debug_bounds_selftest")
+
+
+def qlora_debug_bounds():
+    """The bounds-checked build's record: (line, source file) of the first
+    failed index check since the last call, (0, "") if none; (-1, "") in the
+    ordinary build."""
+    buf = ctypes.create_string_buffer(128)
+    line = lib.qlora_debug_bounds(buf, 128)
+    return line, buf.value.decode()
 
 
 # ---- paged optimizer -----------------------------------------------------------------

@@ -4,7 +4,11 @@ Every translation unit under csrc/ is compiled for sm_100a only
 (-gencode arch=compute_100a,code=sm_100a) and linked with the static CUDA
 runtime; the library loads without PyTorch.
 
-Usage: python bit_nf4_quantized_16_b200/build.py [--force] [-v]
+With --debug the same sources are compiled with QLORA_DEBUG into
+libqlora_b200_debug.so: the bounds-checked build, whose kernels record a
+failed index check instead of faulting (qlora_debug_bounds in qlora.h).
+
+Usage: python bit_nf4_quantized_16_b200/build.py [--force] [-v] [--debug]
 (run by path: importing the package itself needs the built library)
 """
 
@@ -18,6 +22,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libqlora_b200.so")
+LIB_DEBUG = os.path.join(HERE, "libqlora_b200_debug.so")
 OBJ_DIR = os.path.join(ROOT, "_build")
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
@@ -35,37 +40,41 @@ def _deps():
         os.path.join(ROOT, "include", "qlora.h"), __file__]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(debug: bool = False) -> bool:
+    lib = LIB_DEBUG if debug else LIB
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    os.makedirs(OBJ_DIR, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    lib = LIB_DEBUG if debug else LIB
+    if not force and up_to_date(debug):
+        return lib
+    obj_dir = os.path.join(OBJ_DIR, "debug") if debug else OBJ_DIR
+    os.makedirs(obj_dir, exist_ok=True)
     objs = []
     for src in _sources():
-        obj = os.path.join(OBJ_DIR, os.path.basename(src) + ".o")
-        cmd = [NVCC] + ARCH + FLAGS + ["-c", src, "-o", obj]
+        obj = os.path.join(obj_dir, os.path.basename(src) + ".o")
+        cmd = [NVCC] + ARCH + FLAGS + (["-DQLORA_DEBUG"] if debug else []) + ["-c", src, "-o", obj]
         if verbose:
             cmd += ["-Xptxas", "-v"]
             print(" ".join(cmd), flush=True)
         subprocess.check_call(cmd)
         objs.append(obj)
-    cmd = [NVCC] + ARCH + ["-shared", "-o", LIB] + objs + ["-cudart", "static"]
+    cmd = [NVCC] + ARCH + ["-shared", "-o", lib] + objs + ["-cudart", "static"]
     subprocess.check_call(cmd)
-    return LIB
+    return lib
 
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("-v", "--verbose", action="store_true")
+    ap.add_argument("--debug", action="store_true", help="the bounds-checked build (QLORA_DEBUG)")
     a = ap.parse_args(argv)
-    print(build(force=a.force, verbose=a.verbose))
+    print(build(force=a.force, verbose=a.verbose, debug=a.debug))
 
 
 if __name__ == "__main__":

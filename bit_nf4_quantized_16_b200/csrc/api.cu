@@ -10,6 +10,7 @@
 #include <string.h>
 
 #include "common.cuh"
+#include "debug.cuh"
 
 namespace qlora {
 
@@ -305,6 +306,77 @@ extern "C" qlora_status qlora_debug_inject_stall(int kind, uint64_t timeout_ns)
     g_stall_kind = kind;
     g_stall_ns = timeout_ns;
     return QLORA_OK;
+}
+
+// ---- bounds-checked build ------------------------------------------------------------
+
+namespace qlora {
+namespace {
+struct BoundsRegistry {
+    std::mutex mu;
+    std::vector<std::pair<BoundsReader, const char *>> readers;
+};
+BoundsRegistry &bounds_registry()
+{
+    static BoundsRegistry r;
+    return r;
+}
+}  // namespace
+
+void register_bounds_reader(BoundsReader reader, const char *unit)
+{
+    BoundsRegistry &r = bounds_registry();
+    std::lock_guard<std::mutex> lock(r.mu);
+    r.readers.emplace_back(reader, unit);
+}
+}  // namespace qlora
+
+#ifdef QLORA_DEBUG
+namespace qlora {
+namespace {
+// Evaluates one check whose index is past its extent; touches no memory.
+__global__ void bounds_selftest_kernel(int64_t i, int64_t n, int *sink)
+{
+    if (!QLORA_IN(i, n) && sink) *sink = 1;
+}
+}  // namespace
+}  // namespace qlora
+#endif
+
+extern "C" qlora_status qlora_debug_bounds_selftest(void)
+{
+#ifdef QLORA_DEBUG
+    qlora::bounds_selftest_kernel<<<1, 1>>>(4, 4, nullptr);
+    return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+#else
+    return QLORA_ERR_UNSUPPORTED;
+#endif
+}
+
+extern "C" int qlora_debug_bounds(char *unit, size_t unit_len)
+{
+#ifdef QLORA_DEBUG
+    if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+    qlora::BoundsRegistry &r = qlora::bounds_registry();
+    std::lock_guard<std::mutex> lock(r.mu);
+    int first = 0;
+    for (auto &e : r.readers) {
+        const int line = e.first();
+        if (line != 0 && first == 0) {
+            first = line;
+            if (unit && unit_len) {
+                const char *base = strrchr(e.second, '/');
+                base = base ? base + 1 : e.second;
+                strncpy(unit, base, unit_len - 1);
+                unit[unit_len - 1] = 0;
+            }
+        }
+    }
+    return first;
+#else
+    if (unit && unit_len) unit[0] = 0;
+    return -1;
+#endif
 }
 
 // ---- kernel timing ------------------------------------------------------------------

@@ -34,7 +34,7 @@ size_t al(size_t v) { return (v + 255) / 256 * 256; }
 
 struct BlockLayout {
     int64_t T, d, I, Z, S;
-    size_t u1, q, k, v, a, ao, h, u2, gt, up, m, rstd1, rstd2, hs[kL], sc, P;
+    size_t u1, q, k, v, a, ao, h, u2, gt, up, m, rstd1, rstd2, hs[kL], sc, P, rope;
     size_t dm, dgt, dup, dxg, dxu, dh, da, dq, dk, dv, dxq, dxk, dxv, lin, lin_bytes, bytes;
 };
 
@@ -72,6 +72,7 @@ BlockLayout layout(const qlora_block *b)
     for (int l = 0; l < kL; l++) L.hs[l] = take((size_t)L.T * b->r * 4);
     L.sc = take((size_t)L.Z * L.S * L.S * 4);
     L.P = take((size_t)L.Z * L.S * L.S * 2);
+    L.rope = take((size_t)L.S * (b->head_dim / 2) * 8);
     L.dm = take(ti);
     L.dgt = take(ti);
     L.dup = take(ti);
@@ -101,7 +102,7 @@ qlora_status check_block(const qlora_block *b)
     if (!b) return QLORA_ERR_INVALID_ARG;
     if (b->batch < 1 || b->seq < 1 || b->heads < 1 || b->head_dim < 8 || b->hidden < 8 || b->inter < 8)
         return QLORA_ERR_SHAPE;
-    if (b->head_dim % 8 || b->hidden % 64 || b->inter % 64 || b->seq % 8) return QLORA_ERR_SHAPE;
+    if (b->head_dim % 16 || b->hidden % 64 || b->inter % 64 || b->seq % 8) return QLORA_ERR_SHAPE;
     if ((int64_t)b->heads * b->head_dim != b->hidden) return QLORA_ERR_SHAPE;
     const int64_t want[kL][2] = {{b->hidden, b->hidden}, {b->hidden, b->hidden}, {b->hidden, b->hidden},
                                  {b->hidden, b->hidden}, {b->inter, b->hidden}, {b->inter, b->hidden},
@@ -153,6 +154,11 @@ qlora_status bmm(const Ctx &c, blk::BmmArgs a, int kind)
     return QLORA_OK;
 }
 
+// elements of a [T][hidden] activation and of the [Z][S][S] score buffers
+// (the extents the bounds-checked build checks attention operands against)
+int64_t act_elems(const Ctx &c) { return c.L.T * c.L.d; }
+int64_t score_elems(const Ctx &c) { return c.L.Z * c.L.S * c.L.S; }
+
 // batch strides of a [T][hidden] activation viewed as (sequence, head) tiles
 void act_view(const Ctx &c, int64_t &ld, int64_t &s0, int64_t &s1)
 {
@@ -188,13 +194,17 @@ qlora_status forward(const Ctx &c, const bf16 *x, bf16 *y, bool save)
     QLORA_TRY(lin_fwd(c, Lk, c.at(L.u1), c.at(L.k), hs[Lk]));
     QLORA_TRY(lin_fwd(c, Lv, c.at(L.u1), c.at(L.v), hs[Lv]));
     const float log2b = log2f(b->rope_base);
-    const int64_t pairs = L.T * b->heads * (b->head_dim / 2);
+    const int64_t groups = L.T * b->heads * (b->head_dim / 16);
+    const float2 *cs = c.at<float2>(L.rope);
     {
         LaunchScope ls(QLORA_KERNEL_BLOCK, c.s);
-        QLORA_CUDA_TRY(launch_pdl(blk::rope_kernel, dim3(grid_for(pairs, c.sms)), dim3(256), 0, c.s, c.at(L.q), L.T,
-                                  b->seq, b->heads, b->head_dim, log2b, 1.0f));
-        QLORA_CUDA_TRY(launch_pdl(blk::rope_kernel, dim3(grid_for(pairs, c.sms)), dim3(256), 0, c.s, c.at(L.k), L.T,
-                                  b->seq, b->heads, b->head_dim, log2b, 1.0f));
+        const int entries = (int)(L.S * (b->head_dim / 2));
+        QLORA_CUDA_TRY(launch_pdl(blk::rope_table_kernel, dim3((entries + 255) / 256), dim3(256), 0, c.s,
+                                  c.at<float2>(L.rope), (int)L.S, b->head_dim, log2b));
+        QLORA_CUDA_TRY(launch_pdl(blk::rope_kernel, dim3(grid_for(groups, c.sms)), dim3(256), 0, c.s, c.at(L.q), cs,
+                                  L.T, b->seq, b->heads, b->head_dim, 1.0f));
+        QLORA_CUDA_TRY(launch_pdl(blk::rope_kernel, dim3(grid_for(groups, c.sms)), dim3(256), 0, c.s, c.at(L.k), cs,
+                                  L.T, b->seq, b->heads, b->head_dim, 1.0f));
     }
     int64_t ald, as0, as1, sld, ss0, ss1;
     act_view(c, ald, as0, as1);
@@ -203,8 +213,11 @@ qlora_status forward(const Ctx &c, const bf16 *x, bf16 *y, bool save)
         // scores = q k^T / sqrt(D), causal
         blk::BmmArgs a{};
         a.A = c.at(L.q);
+        a.a_n = act_elems(c);
         a.B = c.at(L.k);
+        a.b_n = act_elems(c);
         a.C = c.at<float>(L.sc);
+        a.c_n = score_elems(c);
         a.M = (int)L.S; a.N = (int)L.S; a.K = b->head_dim;
         a.lda = ald; a.sa0 = as0; a.sa1 = as1;
         a.ldb = ald; a.sb0 = as0; a.sb1 = as1;
@@ -224,8 +237,11 @@ qlora_status forward(const Ctx &c, const bf16 *x, bf16 *y, bool save)
         // a = P v (P is zero above the diagonal)
         blk::BmmArgs a{};
         a.A = c.at(L.P);
+        a.a_n = score_elems(c);
         a.B = c.at(L.v);
+        a.b_n = act_elems(c);
         a.C = c.at(L.a);
+        a.c_n = act_elems(c);
         a.M = (int)L.S; a.N = b->head_dim; a.K = (int)L.S;
         a.lda = sld; a.sa0 = ss0; a.sa1 = ss1;
         a.ldb = ald; a.sb0 = as0; a.sb1 = as1;
@@ -247,7 +263,7 @@ qlora_status forward(const Ctx &c, const bf16 *x, bf16 *y, bool save)
     QLORA_TRY(lin_fwd(c, Lup, c.at(L.u2), c.at(L.up), hs[Lup]));
     {
         LaunchScope ls(QLORA_KERNEL_BLOCK, c.s);
-        QLORA_CUDA_TRY(launch_pdl(blk::swiglu_fwd_kernel, dim3(grid_for(L.T * L.I, c.sms)), dim3(256), 0, c.s,
+        QLORA_CUDA_TRY(launch_pdl(blk::swiglu_fwd_kernel, dim3(grid_for(L.T * L.I / 8, c.sms)), dim3(256), 0, c.s,
                                   (const bf16 *)c.at(L.gt), (const bf16 *)c.at(L.up), c.at(L.m), L.T * L.I));
     }
     if (save) return launch_status();
@@ -311,7 +327,7 @@ extern "C" qlora_status qlora_block_bwd(const qlora_block *b, const void *x, con
     QLORA_TRY(lin_bwd(c, Ldown, c.at(L.m), dyb, nullptr, c.at(L.dm), dA[Ldown], dB[Ldown]));
     {
         LaunchScope ls(QLORA_KERNEL_BLOCK, c.s);
-        QLORA_CUDA_TRY(launch_pdl(blk::swiglu_bwd_kernel, dim3(grid_for(L.T * L.I, c.sms)), dim3(256), 0, c.s,
+        QLORA_CUDA_TRY(launch_pdl(blk::swiglu_bwd_kernel, dim3(grid_for(L.T * L.I / 8, c.sms)), dim3(256), 0, c.s,
                                   (const bf16 *)c.at(L.dm), (const bf16 *)c.at(L.gt), (const bf16 *)c.at(L.up),
                                   c.at(L.dgt), c.at(L.dup), L.T * L.I));
     }
@@ -334,8 +350,11 @@ extern "C" qlora_status qlora_block_bwd(const qlora_block *b, const void *x, con
         // dv = P^T da (row i of P^T, key i, is non-zero only for queries i and later)
         blk::BmmArgs a{};
         a.A = c.at(L.P);
+        a.a_n = score_elems(c);
         a.B = c.at(L.da);
+        a.b_n = act_elems(c);
         a.C = c.at(L.dv);
+        a.c_n = act_elems(c);
         a.M = (int)L.S; a.N = b->head_dim; a.K = (int)L.S;
         a.lda = sld; a.sa0 = ss0; a.sa1 = ss1;
         a.ldb = ald; a.sb0 = as0; a.sb1 = as1;
@@ -349,8 +368,11 @@ extern "C" qlora_status qlora_block_bwd(const qlora_block *b, const void *x, con
         // dP = da v^T (the scores buffer)
         blk::BmmArgs a{};
         a.A = c.at(L.da);
+        a.a_n = act_elems(c);
         a.B = c.at(L.v);
+        a.b_n = act_elems(c);
         a.C = c.at<float>(L.sc);
+        a.c_n = score_elems(c);
         a.M = (int)L.S; a.N = (int)L.S; a.K = b->head_dim;
         a.lda = ald; a.sa0 = as0; a.sa1 = as1;
         a.ldb = ald; a.sb0 = as0; a.sb1 = as1;
@@ -371,8 +393,11 @@ extern "C" qlora_status qlora_block_bwd(const qlora_block *b, const void *x, con
         // dq = dS k
         blk::BmmArgs a{};
         a.A = c.at(L.P);
+        a.a_n = score_elems(c);
         a.B = c.at(L.k);
+        a.b_n = act_elems(c);
         a.C = c.at(L.dq);
+        a.c_n = act_elems(c);
         a.M = (int)L.S; a.N = b->head_dim; a.K = (int)L.S;
         a.lda = sld; a.sa0 = ss0; a.sa1 = ss1;
         a.ldb = ald; a.sb0 = as0; a.sb1 = as1;
@@ -383,18 +408,20 @@ extern "C" qlora_status qlora_block_bwd(const qlora_block *b, const void *x, con
         QLORA_TRY((bmm<false, false, false>(c, a, QLORA_KERNEL_ATTENTION)));
         // dk = dS^T q
         a.B = c.at(L.q);
+        a.b_n = act_elems(c);
         a.C = c.at(L.dk);
+        a.c_n = act_elems(c);
         a.tri = 2;
         QLORA_TRY((bmm<true, false, false>(c, a, QLORA_KERNEL_ATTENTION)));
     }
-    const float log2b = log2f(b->rope_base);
-    const int64_t pairs = L.T * b->heads * (b->head_dim / 2);
+    const int64_t groups = L.T * b->heads * (b->head_dim / 16);
+    const float2 *cs = c.at<float2>(L.rope);   // written by the recomputed forward pass
     {
         LaunchScope ls(QLORA_KERNEL_BLOCK, c.s);
-        QLORA_CUDA_TRY(launch_pdl(blk::rope_kernel, dim3(grid_for(pairs, c.sms)), dim3(256), 0, c.s, c.at(L.dq), L.T,
-                                  b->seq, b->heads, b->head_dim, log2b, -1.0f));
-        QLORA_CUDA_TRY(launch_pdl(blk::rope_kernel, dim3(grid_for(pairs, c.sms)), dim3(256), 0, c.s, c.at(L.dk), L.T,
-                                  b->seq, b->heads, b->head_dim, log2b, -1.0f));
+        QLORA_CUDA_TRY(launch_pdl(blk::rope_kernel, dim3(grid_for(groups, c.sms)), dim3(256), 0, c.s, c.at(L.dq), cs,
+                                  L.T, b->seq, b->heads, b->head_dim, -1.0f));
+        QLORA_CUDA_TRY(launch_pdl(blk::rope_kernel, dim3(grid_for(groups, c.sms)), dim3(256), 0, c.s, c.at(L.dk), cs,
+                                  L.T, b->seq, b->heads, b->head_dim, -1.0f));
     }
 
     // 4. q, k, v, first norm (+ residual)

@@ -7,6 +7,7 @@
 #include <stdint.h>
 
 #include "sm100.cuh"
+#include "debug.cuh"
 
 namespace qlora {
 namespace blk {
@@ -28,6 +29,7 @@ __global__ void __launch_bounds__(256) rmsnorm_fwd_kernel(const __nv_bfloat16 *x
     __shared__ float red[8];
     float ss = 0.0f;
     for (int c = threadIdx.x * 8; c < d; c += 256 * 8) {
+        if (!QLORA_IN(c + 7, d)) break;
         uint4 xv = *reinterpret_cast<const uint4 *>(xr + c);
         if (res) {
             const uint4 rv = *reinterpret_cast<const uint4 *>(res + row * d + c);
@@ -62,6 +64,7 @@ __global__ void __launch_bounds__(256) rmsnorm_fwd_kernel(const __nv_bfloat16 *x
     if (threadIdx.x == 0 && rstd_out) rstd_out[row] = rstd;
     const __nv_bfloat16 *xs = res ? x_out + row * d : xr;
     for (int c = threadIdx.x * 8; c < d; c += 256 * 8) {
+        if (!QLORA_IN(c + 7, d)) break;
         const uint4 xv = *reinterpret_cast<const uint4 *>(xs + c);
         const uint4 gv = *reinterpret_cast<const uint4 *>(g + c);
         const __nv_bfloat162 *a = reinterpret_cast<const __nv_bfloat162 *>(&xv);
@@ -118,6 +121,7 @@ __global__ void __launch_bounds__(256) rmsnorm_bwd_kernel(const __nv_bfloat16 *x
     };
     float dot = 0.0f;
     for (int c = threadIdx.x * 8; c < d; c += 256 * 8) {
+        if (!QLORA_IN(c + 7, d)) break;
         float du[8], xv[8], gv[8];
         du_at(c, du);
         load8(x + row * d + c, xv);
@@ -134,6 +138,7 @@ __global__ void __launch_bounds__(256) rmsnorm_bwd_kernel(const __nv_bfloat16 *x
     for (int w = 0; w < 8; w++) tot += red[w];
     const float mean = tot / (float)d;
     for (int c = threadIdx.x * 8; c < d; c += 256 * 8) {
+        if (!QLORA_IN(c + 7, d)) break;
         float du[8], xv[8], gv[8], rv[8];
         du_at(c, du);
         load8(x + row * d + c, xv);
@@ -155,60 +160,122 @@ __global__ void __launch_bounds__(256) rmsnorm_bwd_kernel(const __nv_bfloat16 *x
 }
 
 // ---- rotary position embedding --------------------------------------------------
-// t [rows][heads * hd], row = b * seq + p: the pairs (i, i + hd/2) of each
-// head rotate by the angle p * base^(-2i/hd) (sign < 0: the inverse rotation,
-// which is the backward pass).  One thread per pair.
-__global__ void __launch_bounds__(256) rope_kernel(__nv_bfloat16 *t, int64_t rows, int seq, int heads, int hd,
-                                                   float log2_base, float sign)
+// Angle table: cs[p][i] = (cos, sin) of p * base^(-2i/hd) for positions p <
+// seq and pairs i < hd/2, computed once per block call.
+__global__ void __launch_bounds__(256) rope_table_kernel(float2 *cs, int seq, int hd, float log2_base)
 {
     sm100::pdl_wait();
     sm100::pdl_trigger();
     const int half = hd / 2;
-    const int64_t n = rows * heads * half;
+    const int id = blockIdx.x * blockDim.x + threadIdx.x;
+    if (id >= seq * half || !QLORA_IN(id, seq * half)) return;
+    const int p = id / half, i = id % half;
+    const float inv = exp2f(-2.0f * (float)i / (float)hd * log2_base);
+    float s, c;
+    sincosf((float)p * inv, &s, &c);
+    cs[id] = make_float2(c, s);
+}
+
+// t [rows][heads * hd], row = b * seq + p: the pairs (i, i + hd/2) of each
+// head rotate by the table's angle for (p, i) (sign < 0: the inverse rotation,
+// which is the backward pass).  One thread per 8 consecutive pairs (16-byte
+// accesses); hd % 16 == 0.
+__global__ void __launch_bounds__(256) rope_kernel(__nv_bfloat16 *t, const float2 *cs, int64_t rows, int seq,
+                                                   int heads, int hd, float sign)
+{
+    sm100::pdl_wait();
+    sm100::pdl_trigger();
+    const int half = hd / 2, groups = half / 8;
+    const int64_t n = rows * heads * groups;
     for (int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; id < n; id += (int64_t)gridDim.x * blockDim.x) {
-        const int i = (int)(id % half);
-        const int64_t rh = id / half;
+        const int i0 = (int)(id % groups) * 8;
+        const int64_t rh = id / groups;
         const int h = (int)(rh % heads);
         const int64_t row = rh / heads;
         const int p = (int)(row % seq);
-        const float inv = exp2f(-2.0f * (float)i / (float)hd * log2_base);
-        float s, c;
-        sincosf((float)p * inv, &s, &c);
-        s *= sign;
         __nv_bfloat16 *base = t + row * (int64_t)heads * hd + (int64_t)h * hd;
-        const float a = bf(base[i]), b = bf(base[i + half]);
-        base[i] = __float2bfloat16_rn(a * c - b * s);
-        base[i + half] = __float2bfloat16_rn(a * s + b * c);
+        if (!QLORA_IN(row * (int64_t)heads * hd + (int64_t)h * hd + i0 + half + 7, rows * heads * hd) ||
+            !QLORA_IN((int64_t)p * half + i0 + 7, (int64_t)seq * half))
+            continue;
+        uint4 av = *reinterpret_cast<const uint4 *>(base + i0);
+        uint4 bv = *reinterpret_cast<const uint4 *>(base + i0 + half);
+        __nv_bfloat162 *a2 = reinterpret_cast<__nv_bfloat162 *>(&av);
+        __nv_bfloat162 *b2 = reinterpret_cast<__nv_bfloat162 *>(&bv);
+        const float2 *tab = cs + (int64_t)p * half + i0;
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const float2 fa = __bfloat1622float2(a2[j]), fb = __bfloat1622float2(b2[j]);
+            const float2 c0 = tab[2 * j], c1 = tab[2 * j + 1];
+            const float s0 = sign * c0.y, s1 = sign * c1.y;
+            a2[j] = __floats2bfloat162_rn(fa.x * c0.x - fb.x * s0, fa.y * c1.x - fb.y * s1);
+            b2[j] = __floats2bfloat162_rn(fa.x * s0 + fb.x * c0.x, fa.y * s1 + fb.y * c1.x);
+        }
+        *reinterpret_cast<uint4 *>(base + i0) = av;
+        *reinterpret_cast<uint4 *>(base + i0 + half) = bv;
     }
 }
 
 // ---- SwiGLU -----------------------------------------------------------------------
 __device__ __forceinline__ float sigmoidf_(float z) { return 1.0f / (1.0f + __expf(-z)); }
 
-// m = bf16(silu(gate) * up)
+__device__ __forceinline__ void unpack8(uint4 v, float (&f)[8])
+{
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const float2 x = __bfloat1622float2(h[i]);
+        f[2 * i] = x.x;
+        f[2 * i + 1] = x.y;
+    }
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&f)[8])
+{
+    uint4 v;
+    __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; i++) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+    return v;
+}
+
+// m = bf16(silu(gate) * up), 8 elements per thread (n % 8 == 0)
 __global__ void __launch_bounds__(256) swiglu_fwd_kernel(const __nv_bfloat16 *gate, const __nv_bfloat16 *up,
                                                          __nv_bfloat16 *m, int64_t n)
 {
     sm100::pdl_wait();
     sm100::pdl_trigger();
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-        const float gt = bf(gate[i]);
-        m[i] = __float2bfloat16_rn(gt * sigmoidf_(gt) * bf(up[i]));
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; 8 * i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        float g[8], u[8], o[8];
+        if (!QLORA_IN(8 * i + 7, n)) break;
+        unpack8(*reinterpret_cast<const uint4 *>(gate + 8 * i), g);
+        unpack8(*reinterpret_cast<const uint4 *>(up + 8 * i), u);
+#pragma unroll
+        for (int j = 0; j < 8; j++) o[j] = g[j] * sigmoidf_(g[j]) * u[j];
+        *reinterpret_cast<uint4 *>(m + 8 * i) = pack8(o);
     }
 }
 
-// dgate = dm * up * silu'(gate), dup = dm * silu(gate)
+// dgate = dm * up * silu'(gate), dup = dm * silu(gate), 8 elements per thread
 __global__ void __launch_bounds__(256) swiglu_bwd_kernel(const __nv_bfloat16 *dm, const __nv_bfloat16 *gate,
                                                          const __nv_bfloat16 *up, __nv_bfloat16 *dgate,
                                                          __nv_bfloat16 *dup, int64_t n)
 {
     sm100::pdl_wait();
     sm100::pdl_trigger();
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-        const float gt = bf(gate[i]), u = bf(up[i]), d = bf(dm[i]);
-        const float sg = sigmoidf_(gt);
-        dgate[i] = __float2bfloat16_rn(d * u * (sg + gt * sg * (1.0f - sg)));
-        dup[i] = __float2bfloat16_rn(d * gt * sg);
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; 8 * i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        float d[8], g[8], u[8], og[8], ou[8];
+        if (!QLORA_IN(8 * i + 7, n)) break;
+        unpack8(*reinterpret_cast<const uint4 *>(dm + 8 * i), d);
+        unpack8(*reinterpret_cast<const uint4 *>(gate + 8 * i), g);
+        unpack8(*reinterpret_cast<const uint4 *>(up + 8 * i), u);
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+            const float sg = sigmoidf_(g[j]);
+            og[j] = d[j] * u[j] * (sg + g[j] * sg * (1.0f - sg));
+            ou[j] = d[j] * g[j] * sg;
+        }
+        *reinterpret_cast<uint4 *>(dgate + 8 * i) = pack8(og);
+        *reinterpret_cast<uint4 *>(dup + 8 * i) = pack8(ou);
     }
 }
 
@@ -233,6 +300,7 @@ struct BmmArgs {
     float alpha;
     int tri;
     int causal;
+    int64_t a_n, b_n, c_n;   // elements of the buffers behind A, B and C (bounds-checked build)
 };
 
 constexpr int kBM = 128, kBN = 128, kBK = 32;
@@ -292,7 +360,8 @@ __global__ void __launch_bounds__(256) bmm_kernel(const BmmArgs p)
         float *C = static_cast<float *>(p.C) + z0 * p.sc0 + z1 * p.sc1;
         for (int e = tid; e < kBM * kBN; e += 256) {
             const int i = i0 + e / kBN, j = j0 + e % kBN;
-            if (i < p.M && j < p.N) C[(int64_t)i * p.ldc + j] = -INFINITY;
+            if (i < p.M && j < p.N && QLORA_IN(z0 * p.sc0 + z1 * p.sc1 + (int64_t)i * p.ldc + j, p.c_n))
+                C[(int64_t)i * p.ldc + j] = -INFINITY;
         }
         return;
     }
@@ -309,12 +378,14 @@ __global__ void __launch_bounds__(256) bmm_kernel(const BmmArgs p)
             if (!AT) {
                 const int r = ch >> 2, c = (ch & 3) * 8;            // [128 rows][32 k]
                 const int gi = i0 + r, gk = k0 + c;
-                const bool ok = gi < p.M && gk < kend;
+                const bool ok = gi < p.M && gk < kend &&
+                                QLORA_IN(z0 * p.sa0 + z1 * p.sa1 + (int64_t)gi * p.lda + gk + 7, p.a_n);
                 cp_async16(&sA[st][r * kPadK + c], A + (ok ? (int64_t)gi * p.lda + gk : 0), ok);
             } else {
                 const int r = ch >> 4, c = (ch & 15) * 8;           // [32 k][128 rows]
                 const int gk = k0 + r, gi = i0 + c;
-                const bool ok = gk < kend && gi < p.M;
+                const bool ok = gk < kend && gi < p.M &&
+                                QLORA_IN(z0 * p.sa0 + z1 * p.sa1 + (int64_t)gk * p.lda + gi + 7, p.a_n);
                 cp_async16(&sA[st][r * kPadMN + c], A + (ok ? (int64_t)gk * p.lda + gi : 0), ok);
             }
         }
@@ -324,12 +395,14 @@ __global__ void __launch_bounds__(256) bmm_kernel(const BmmArgs p)
             if (BT) {
                 const int r = ch >> 2, c = (ch & 3) * 8;            // [128 cols][32 k]
                 const int gj = j0 + r, gk = k0 + c;
-                const bool ok = gj < p.N && gk < kend;
+                const bool ok = gj < p.N && gk < kend &&
+                                QLORA_IN(z0 * p.sb0 + z1 * p.sb1 + (int64_t)gj * p.ldb + gk + 7, p.b_n);
                 cp_async16(&sB[st][r * kPadK + c], B + (ok ? (int64_t)gj * p.ldb + gk : 0), ok);
             } else {
                 const int r = ch >> 4, c = (ch & 15) * 8;           // [32 k][128 cols]
                 const int gk = k0 + r, gj = j0 + c;
-                const bool ok = gk < kend && gj < p.N;
+                const bool ok = gk < kend && gj < p.N &&
+                                QLORA_IN(z0 * p.sb0 + z1 * p.sb1 + (int64_t)gk * p.ldb + gj + 7, p.b_n);
                 cp_async16(&sB[st][r * kPadMN + c], B + (ok ? (int64_t)gk * p.ldb + gj : 0), ok);
             }
         }
@@ -407,6 +480,7 @@ __global__ void __launch_bounds__(256) bmm_kernel(const BmmArgs p)
                 const int i = i0 + wm * 64 + mi * 16 + g + 8 * half;
                 const int j = j0 + wn * 32 + nj * 8 + 2 * c;
                 if (i >= p.M || j >= p.N) continue;
+                if (!QLORA_IN(z0 * p.sc0 + z1 * p.sc1 + (int64_t)i * p.ldc + j + 1, p.c_n)) continue;
                 float v0 = p.alpha * acc[mi][nj][2 * half], v1 = p.alpha * acc[mi][nj][2 * half + 1];
                 if (OUT_F32) {
                     if (p.causal) {

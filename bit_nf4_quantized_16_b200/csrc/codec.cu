@@ -24,6 +24,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "debug.cuh"
 #include "exact_mean.cuh"
 #include "nf4_expand.cuh"
 #include "sm100.cuh"
@@ -284,7 +285,7 @@ __global__ void __maxnreg__(64) quantize_blocks_kernel(const __grid_constant__ Q
             float m = 0.0f;
 #pragma unroll
             for (int i = 0; i < 16; i++) {
-                const uint4 v = act ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+                const uint4 v = act && QLORA_IN(b, p.nblocks) ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
                 m = fmaxf(fmaxf(m, fmaxf(fabsf(__uint_as_float(v.x)), fabsf(__uint_as_float(v.y)))),
                           fmaxf(fabsf(__uint_as_float(v.z)), fabsf(__uint_as_float(v.w))));
             }
@@ -302,7 +303,7 @@ __global__ void __maxnreg__(64) quantize_blocks_kernel(const __grid_constant__ Q
                 words[i] = codes8(lut, n);
             }
         }
-        if (act) {
+        if (act && QLORA_IN(b, p.nblocks)) {
             st_v8(reinterpret_cast<uint4 *>(p.packed) + 2 * b, make_uint4(words[0], words[1], words[2], words[3]),
                   make_uint4(words[4], words[5], words[6], words[7]));   // 64 codes = 32 B
             p.c1[b] = cv;
@@ -429,12 +430,12 @@ __global__ void __launch_bounds__(kThreads) dq_encode_kernel(DqParams p)
 #pragma unroll
         for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
         const float s = __fdiv_rn(amax, 448.0f);
-        if (lane == 0) p.c2[g] = s;
+        if (lane == 0 && QLORA_IN(g, p.ngroups)) p.c2[g] = s;
         const float rs = s >= 0x1p-100f ? __frcp_rn(s) : 0.0f;
         uint8_t e[8];
 #pragma unroll
         for (int i = 0; i < 8; i++) e[i] = s == 0.0f ? (uint8_t)0 : e4m3_of_quotient(d[i], s, rs);
-        if (b0 + 8 <= p.nblocks) {
+        if (b0 + 8 <= p.nblocks && QLORA_IN(b0 + 7, p.nblocks)) {
             uint2 v;
             v.x = e[0] | (e[1] << 8) | (e[2] << 16) | ((uint32_t)e[3] << 24);
             v.y = e[4] | (e[5] << 8) | (e[6] << 16) | ((uint32_t)e[7] << 24);
@@ -482,13 +483,14 @@ __global__ void __launch_bounds__(kThreads) dequantize_kernel(DeqParams p)
             if (w < p.nwords) {
                 word[u] = ld_stream_u32(p.packed + 4 * w);
                 int64_t b = w >> 3;
-                c1p[u] = nf4::block_scale(p.code2[b], p.c2[b / QLORA_GROUP], mu);
+                if (QLORA_IN(b, (p.nwords + 7) / 8) && QLORA_IN(b / QLORA_GROUP, (p.nwords / 8 + QLORA_GROUP - 1) / QLORA_GROUP))
+                    c1p[u] = nf4::block_scale(p.code2[b], p.c2[b / QLORA_GROUP], mu);
             }
         }
 #pragma unroll
         for (int u = 0; u < kDeqUnroll; u++) {
             int64_t w = w0 + u * stride;
-            if (w >= p.nwords) continue;
+            if (w >= p.nwords || !QLORA_IN(w, p.nwords)) continue;
             *reinterpret_cast<uint4 *>(p.out + 8 * w) = nf4::expand8<F16>(word[u], lut, c1p[u]);
         }
     }

@@ -31,6 +31,7 @@
 #include <algorithm>
 
 #include "common.cuh"
+#include "debug.cuh"
 #include "decode.cuh"
 #include "nf4_expand.cuh"
 #include "sm100.cuh"
@@ -122,13 +123,15 @@ struct WStage {
 template <int NT, bool F16>
 __device__ __forceinline__ void mma_step(float (&acc)[NT][2][4], const uint4 (&ea)[4], const uint4 (&eb)[4],
                                          const __nv_bfloat16 *const (&xrow)[NT], const bool (&xok)[NT], int64_t k,
-                                         bool kin)
+                                         bool kin, [[maybe_unused]] const __nv_bfloat16 *xbase,
+                                         [[maybe_unused]] int64_t xlen)
 {
 #pragma unroll
     for (int w = 0; w < 4; w++) {
 #pragma unroll
         for (int t = 0; t < NT; t++) {
-            const uint4 xb = (xok[t] && kin) ? ld_cached_v4(xrow[t] + k + 8 * w) : make_uint4(0, 0, 0, 0);
+            const uint4 xb = (xok[t] && kin && QLORA_IN((xrow[t] - xbase) + k + 8 * w + 7, xlen))
+                                 ? ld_cached_v4(xrow[t] + k + 8 * w) : make_uint4(0, 0, 0, 0);
             mma_bf16_16816<F16>(acc[t][0], ea[w].x, eb[w].x, ea[w].y, eb[w].y, xb.x, xb.y);
             mma_bf16_16816<F16>(acc[t][0], ea[w].z, eb[w].z, ea[w].w, eb[w].w, xb.z, xb.w);
         }
@@ -185,10 +188,12 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm) decode_gemv_kernel
             uint4 ea[4], eb[4];
 #pragma unroll
             for (int w = 0; w < 4; w++) {
-                ea[w] = (ok_g && k_ok) ? ld_cached_v4(p.A + rg * p.K + k + 8 * w) : make_uint4(0, 0, 0, 0);
-                eb[w] = (ok_g8 && k_ok) ? ld_cached_v4(p.A + rg8 * p.K + k + 8 * w) : make_uint4(0, 0, 0, 0);
+                ea[w] = (ok_g && k_ok && QLORA_IN(rg * p.K + k + 8 * w + 7, (int64_t)p.r * p.K))
+                            ? ld_cached_v4(p.A + rg * p.K + k + 8 * w) : make_uint4(0, 0, 0, 0);
+                eb[w] = (ok_g8 && k_ok && QLORA_IN(rg8 * p.K + k + 8 * w + 7, (int64_t)p.r * p.K))
+                            ? ld_cached_v4(p.A + rg8 * p.K + k + 8 * w) : make_uint4(0, 0, 0, 0);
             }
-            mma_step<NT, F16>(acc, ea, eb, xrow, xok, k, k_ok);
+            mma_step<NT, F16>(acc, ea, eb, xrow, xok, k, k_ok, p.Xa, (int64_t)p.M * p.K);
         }
         float *part = p.part_h + (int64_t)qtr * p.M * p.r;
 #pragma unroll
@@ -197,7 +202,8 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm) decode_gemv_kernel
             for (int i = 0; i < 4; i++) {
                 const int tok = 8 * t + 2 * c + (i & 1);
                 const int64_t row = (i < 2) ? rg : rg8;
-                if (tok < p.M && row < p.r) part[(int64_t)tok * p.r + row] = __fadd_rn(acc[t][0][i], acc[t][1][i]);
+                if (tok < p.M && row < p.r && QLORA_IN(((int64_t)qtr * p.M + tok) * p.r + row, (int64_t)kAPieces * p.M * p.r))
+                    part[(int64_t)tok * p.r + row] = __fadd_rn(acc[t][0][i], acc[t][1][i]);
             }
         }
         return;
@@ -215,13 +221,19 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm) decode_gemv_kernel
         const int64_t k = (int64_t)d * 128 + 32 * c;
         const bool in = d < d1 && k < p.K;
         const uint4 z = make_uint4(0, 0, 0, 0);
-        st.pg = (in && ok_g) ? ld_stream_v4(p.packed + rg * half_k + k / 2) : z;
-        st.pg8 = (in && ok_g8) ? ld_stream_v4(p.packed + rg8 * half_k + k / 2) : z;
+        [[maybe_unused]] const int64_t nblk = p.N * p.kblocks;
+        // (checked only where the access happens)
+        const bool ld_g = in && ok_g && QLORA_IN(rg * half_k + k / 2 + 15, p.N * half_k) &&
+                          QLORA_IN(rg * p.kblocks + k / 64, nblk) && QLORA_IN((rg * p.kblocks + k / 64) >> 8, (nblk + 255) / 256);
+        const bool ld_g8 = in && ok_g8 && QLORA_IN(rg8 * half_k + k / 2 + 15, p.N * half_k) &&
+                           QLORA_IN(rg8 * p.kblocks + k / 64, nblk) && QLORA_IN((rg8 * p.kblocks + k / 64) >> 8, (nblk + 255) / 256);
+        st.pg = ld_g ? ld_stream_v4(p.packed + rg * half_k + k / 2) : z;
+        st.pg8 = ld_g8 ? ld_stream_v4(p.packed + rg8 * half_k + k / 2) : z;
         const int64_t b = rg * p.kblocks + k / 64, b8 = rg8 * p.kblocks + k / 64;
-        st.eg = (in && ok_g) ? (uint32_t)__ldg(p.code2 + b) : 0u;
-        st.c2g = (in && ok_g) ? __ldg(p.c2 + (b >> 8)) : 0.0f;
-        st.eg8 = (in && ok_g8) ? (uint32_t)__ldg(p.code2 + b8) : 0u;
-        st.c2g8 = (in && ok_g8) ? __ldg(p.c2 + (b8 >> 8)) : 0.0f;
+        st.eg = ld_g ? (uint32_t)__ldg(p.code2 + b) : 0u;
+        st.c2g = ld_g ? __ldg(p.c2 + (b >> 8)) : 0.0f;
+        st.eg8 = ld_g8 ? (uint32_t)__ldg(p.code2 + b8) : 0u;
+        st.c2g8 = ld_g8 ? __ldg(p.c2 + (b8 >> 8)) : 0.0f;
     };
     WStage st[kPrefetch];
 #pragma unroll
@@ -244,7 +256,7 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm) decode_gemv_kernel
                     eb[1] = nf4::expand8<F16>(st[i].pg8.y, lut, sg8);
                     eb[2] = nf4::expand8<F16>(st[i].pg8.z, lut, sg8);
                     eb[3] = nf4::expand8<F16>(st[i].pg8.w, lut, sg8);
-                    mma_step<NT, F16>(acc, ea, eb, xrow, xok, k, kin);
+                    mma_step<NT, F16>(acc, ea, eb, xrow, xok, k, kin, p.X, (int64_t)p.M * p.K);
                 }
                 load(d + i + kPrefetch, st[i]);
             }
@@ -259,7 +271,8 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm) decode_gemv_kernel
         for (int i = 0; i < 4; i++) {
             const int tok = 8 * t + 2 * c + (i & 1);
             const int64_t row = (i < 2) ? rg : rg8;
-            if (tok < p.M && row < p.N) part[(int64_t)tok * p.N + row] = __fadd_rn(acc[t][0][i], acc[t][1][i]);
+            if (tok < p.M && row < p.N && QLORA_IN(((int64_t)sp * p.M + tok) * p.N + row, (int64_t)gridDim.y * p.M * p.N))
+                part[(int64_t)tok * p.N + row] = __fadd_rn(acc[t][0][i], acc[t][1][i]);
         }
     }
 }
@@ -300,6 +313,7 @@ __global__ void __launch_bounds__(256) decode_finalize_kernel(const float *part,
     float v[8];
     load_splits8(v, part, 0, has_row ? splits : 0, 0, M, N, n);
     for (int i = threadIdx.x; i < M * r; i += blockDim.x) {
+        if (!QLORA_IN(i, kDecodeMaxTokens * 128)) break;
         float hv = 0.0f;
 #pragma unroll
         for (int s = 0; s < kAPieces; s++) hv = __fadd_rn(hv, part_h[(int64_t)s * M * r + i]);

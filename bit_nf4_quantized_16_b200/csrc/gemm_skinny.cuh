@@ -35,6 +35,7 @@
 #include <stdint.h>
 
 #include "sm100.cuh"
+#include "debug.cuh"
 
 namespace qlora {
 
@@ -301,13 +302,14 @@ __global__ void __launch_bounds__(256, 1) qgemm_skinny_kernel(const __grid_const
                 acc = add4(acc, lo);
             }
             const int64_t grow = (int64_t)mt * 128 + lr;
-            if (grow >= J.m_total) continue;
+            if (grow >= J.m_total || !QLORA_IN(grow, J.m_total)) continue;
             if (!wgrad) {
                 const int col = 4 * c4;
                 const bool in = col < J.r;   // r % 8 == 0: four columns are all in or all out
                 float4 v = make_float4(__fmul_rn(J.scale, acc.x), __fmul_rn(J.scale, acc.y),
                                        __fmul_rn(J.scale, acc.z), __fmul_rn(J.scale, acc.w));
                 if (!in) v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                if (!QLORA_IN(col + 3, J.r_pad)) continue;
                 if (J.f32_out && in) *reinterpret_cast<float4 *>(J.f32_out + grow * J.r + col) = v;
                 store_hi_lo4<F16>(J.hl_out, grow, J.r_pad, col, v);
                 if (J.aux_in) {
@@ -318,6 +320,10 @@ __global__ void __launch_bounds__(256, 1) qgemm_skinny_kernel(const __grid_const
             } else {
                 const int j = 64 * nt + 4 * c4;
                 if (j >= J.r) continue;
+                if (!QLORA_IN((int64_t)(j + 3) * (J.fin == kFinWgradT ? J.out_ld : 1) +
+                                  grow * (J.fin == kFinWgradT ? 1 : J.out_ld),
+                              (int64_t)(J.fin == kFinWgradT ? J.r : J.m_total) * J.out_ld))
+                    continue;
                 if (J.fin == kFinWgradT) {
                     J.f32_out[(int64_t)(j + 0) * J.out_ld + grow] = acc.x;
                     J.f32_out[(int64_t)(j + 1) * J.out_ld + grow] = acc.y;

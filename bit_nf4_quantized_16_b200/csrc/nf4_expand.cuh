@@ -73,8 +73,10 @@ __device__ __forceinline__ float lut_at(const float *lut, uint32_t off)
 // with F16, fp16: the fp16 compute dtype) in a 16-byte vector (element 0 in
 // the lowest 16 bits).  The byte offsets of the even and the odd codes are
 // formed once per word; each element then costs one byte extraction and one
-// shared-memory load.
-template <bool F16 = false>
+// shared-memory load.  kPairMul: the products as paired f32x2 multiplies (half
+// the multiply instructions) or as scalar ones (no register pairing); both
+// are IEEE round-to-nearest products, so the bits are the same.
+template <bool F16 = false, bool kPairMul = true>
 __device__ __forceinline__ uint4 expand8(uint32_t word, const float *lut, float c1p)
 {
     const uint32_t ev = (word << 2) & 0x3C3C3C3Cu;   // byte k: 4 * code of element 2k
@@ -92,7 +94,12 @@ __device__ __forceinline__ uint4 expand8(uint32_t word, const float *lut, float 
 #pragma unroll
     for (int i = 0; i < 4; i++) {
         float lo, hi;
-        mul2(q[2 * i], q[2 * i + 1], c1p, lo, hi);
+        if constexpr (kPairMul) {
+            mul2(q[2 * i], q[2 * i + 1], c1p, lo, hi);
+        } else {
+            lo = __fmul_rn(q[2 * i], c1p);
+            hi = __fmul_rn(q[2 * i + 1], c1p);
+        }
         o[i] = pack16x2<F16>(lo, hi);
     }
     return make_uint4(o[0], o[1], o[2], o[3]);

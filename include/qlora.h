@@ -509,6 +509,26 @@ QLORA_API qlora_status qlora_timing_read(double ms[QLORA_NUM_KERNELS], int64_t l
 QLORA_API int64_t qlora_launch_count(void);
 
 /*
+ * qlora_debug_bounds -- the bounds-checked build (library compiled with
+ * QLORA_DEBUG, libqlora_b200_debug.so).  Its kernels check every computed
+ * index of a raw pointer access against the extent of the buffer the
+ * arguments describe; a failed check records its source line and skips the
+ * access instead of faulting.  Synchronizes the current device, then returns
+ * the first recorded line (0 if no check failed since the last call) and
+ * clears it; `unit` (nullable, `unit_len` bytes) receives the source file's
+ * name.  Returns -1 in the ordinary build, which has no checks.
+ */
+QLORA_API int qlora_debug_bounds(char *unit, size_t unit_len);
+
+/*
+ * qlora_debug_bounds_selftest -- launches (on the current device, default
+ * stream) one thread that evaluates a single bounds check whose index equals
+ * its extent and touches no memory, so that qlora_debug_bounds() then reports
+ * that check's line in api.cu.  QLORA_ERR_UNSUPPORTED in the ordinary build.
+ */
+QLORA_API qlora_status qlora_debug_bounds_selftest(void);
+
+/*
  * qlora_debug_inject_stall -- failure-detection test hook (the pages describe
  * no such facility; it exists so that tests can drive the bounded-wait path
  * without faulting the GPU).  Arms a one-shot fault in the next launch of

@@ -19,3 +19,13 @@ def read_golden(name):
             if line:
                 rows.append(line.split())
     return rows
+
+
+def pytest_runtest_teardown(item, nextitem):
+    """Under the bounds-checked build (QLORA_B200_BUILD=debug), every GPU test
+    must leave no failed index check behind."""
+    if os.environ.get("QLORA_B200_BUILD") != "debug" or item.get_closest_marker("gpu") is None:
+        return
+    import bit_nf4_quantized_16_b200 as q
+    line, unit = q.qlora_debug_bounds()
+    assert line == 0, f"bounds check failed at {unit}:{line} during {item.nodeid}"

@@ -42,6 +42,29 @@ def test_every_declared_symbol_is_exported(lib):
         assert hasattr(lib, n), n
 
 
+def test_bounds_checked_build_exports_every_symbol():
+    """The QLORA_DEBUG build (libqlora_b200_debug.so) is the same ABI."""
+    path = os.path.join(ROOT, "bit_nf4_quantized_16_b200", "libqlora_b200_debug.so")
+    if not os.path.exists(path):
+        import importlib.util
+        spec = importlib.util.spec_from_file_location("qbuild", os.path.join(ROOT, "bit_nf4_quantized_16_b200", "build.py"))
+        mod = importlib.util.module_from_spec(spec)
+        spec.loader.exec_module(mod)
+        mod.build(debug=True)
+    dlib = ctypes.CDLL(path)
+    for n in declared_symbols():
+        assert hasattr(dlib, n), n
+
+
+def test_ordinary_build_has_no_bounds_checks(lib):
+    """qlora_debug_bounds answers -1 and the self-test is unsupported (no CUDA call)."""
+    lib.qlora_debug_bounds.restype = ctypes.c_int
+    lib.qlora_debug_bounds.argtypes = [ctypes.c_char_p, ctypes.c_size_t]
+    buf = ctypes.create_string_buffer(16)
+    assert lib.qlora_debug_bounds(buf, 16) == -1 and buf.value == b""
+    assert lib.qlora_debug_bounds_selftest() == 6   # QLORA_ERR_UNSUPPORTED
+
+
 def test_binding_lists_the_same_symbols():
     src = open(os.path.join(ROOT, "bit_nf4_quantized_16_b200", "__init__.py")).read()
     exports = re.search(r"EXPORTS = \((.*?)\)", src, re.S).group(1)
