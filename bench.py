@@ -283,6 +283,8 @@ def run_ours(args, rank, world, local_rank):
     breakdown = {k: {"ms_per_step": round(v[0] / args.steps, 4), "launches_per_step": v[1] // args.steps}
                  for k, v in kern.items() if v[1]}
 
+    variants = run_variants7b(args, q, torch, dev, layers, timed_steps, step_flops, TOKENS, scale, peaks, peak_src) \
+        if (rank == 0 and not args.skip_variants and args.linears == "llama7b") else None
     codec = run_codec(args, q, torch, dev, peaks, peak_src) if (rank == 0 and not args.skip_codec) else None
     decode = run_decode65b(args, q, torch, dev, peaks, peak_src) if (rank == 0 and not args.skip_decode) else None
     adamw = run_adamw7b(args, q, torch, dev, peaks, peak_src) if (rank == 0 and not args.skip_optim) else None
@@ -309,6 +311,8 @@ def run_ours(args, rank, world, local_rank):
         "kernels": breakdown,
         "clocks": clocks,
     }
+    if variants is not None:
+        line["variants7b"] = variants
     if codec is not None:
         line["codec"] = codec
     if decode is not None:
@@ -323,6 +327,65 @@ def run_ours(args, rank, world, local_rank):
         line["cpu_baseline"] = cpu_baseline_linear(budget_s=args.cpu_seconds)
         line["cpu_baseline_tiny"] = cpu_baseline_tiny()
     return line
+
+
+def run_variants7b(args, q, torch, dev, layers, timed_steps, step_flops, tokens, scale, peaks, peak_src):
+    """The headline's LLaMA-7B layer step (7 linears fwd+bwd, 4096 tokens) under
+    the variant knobs, timed the same way: the fp16 compute dtype (fp16
+    activations, adapters and outputs, fp16 expansion of the 4-bit weight) and
+    LoRA dropout (p = 0.05, keep mask drawn once, bf16)."""
+    import synthetic
+    out = {"workload": "linear7b step (7 LLaMA-7B QLoRA linears fwd+bwd, 4096 tokens, r=64) with the variant knobs",
+           "unit": "TFLOP/s"}
+    steps = max(args.steps // 2, 3)
+    # fp16 compute dtype: same quantized weights, fp16 tensors
+    f16 = []
+    for L in layers:
+        f16.append({k: L[k].to(torch.float16) for k in ("X", "A", "B", "dY")})
+        f16[-1].update(Y=torch.empty_like(L["Y"], dtype=torch.float16), dX=torch.empty_like(L["dX"], dtype=torch.float16))
+    ws = torch.empty(max(q.qlora_linear_workspace_bytes(tokens, L["N"], L["K"], R) for L in layers),
+                     dtype=torch.uint8, device=dev)
+
+    def step_f16():
+        for L, F in zip(layers, f16):
+            q.qlora_linear_fwd(L["w"], F["X"], tokens, F["A"], F["B"], R, scale, F["Y"], L["H"], ws)
+        for L, F in zip(reversed(layers), reversed(f16)):
+            q.qlora_linear_bwd(L["w"], F["X"], F["dY"], tokens, F["A"], F["B"], R, scale, L["H"], F["dX"],
+                               L["dA"], L["dB"], ws)
+
+    for _ in range(3):
+        step_f16()
+    torch.cuda.synchronize()
+    q.qlora_check_device_error()
+    ms = timed_steps(steps, step_f16)
+    out["fp16_compute"] = {"value": round(step_flops * steps / (ms * 1e-3) / 1e12, 2),
+                           "ms_per_step": round(ms / steps, 4), "frac_of_bf16_peak": None}
+    out["fp16_compute"]["frac_of_bf16_peak"] = round(out["fp16_compute"]["value"] / peaks["bf16_tflops"], 4)
+    del f16
+    # LoRA dropout: one mask per linear (M*K/8 bytes)
+    masks = [synthetic.dropout_mask(tokens, L["K"], 0.05, 90_000 + i, dev)[1] for i, L in enumerate(layers)]
+    wsd = torch.empty(max(q.qlora_linear_workspace_bytes(tokens, L["N"], L["K"], R, dropout=(masks[0], 0.05))
+                          for L in layers), dtype=torch.uint8, device=dev)
+
+    def step_drop():
+        for L, m in zip(layers, masks):
+            q.qlora_linear_fwd(L["w"], L["X"], tokens, L["A"], L["B"], R, scale, L["Y"], L["H"], wsd,
+                               dropout=(m, 0.05))
+        for L, m in zip(reversed(layers), reversed(masks)):
+            q.qlora_linear_bwd(L["w"], L["X"], L["dY"], tokens, L["A"], L["B"], R, scale, L["H"], L["dX"],
+                               L["dA"], L["dB"], wsd, dropout=(m, 0.05))
+
+    for _ in range(3):
+        step_drop()
+    torch.cuda.synchronize()
+    q.qlora_check_device_error()
+    ms = timed_steps(steps, step_drop)
+    out["lora_dropout_0.05"] = {"value": round(step_flops * steps / (ms * 1e-3) / 1e12, 2),
+                                "ms_per_step": round(ms / steps, 4),
+                                "note": "FLOP counted as without dropout (the dropped-input pass and the separate "
+                                        "adapter dX product are extra work)"}
+    out["peak_source"] = f"{peak_src} bf16_tflops (burst); fp16 dense peak taken equal to bf16"
+    return out
 
 
 def run_codec(args, q, torch, dev, peaks, peak_src):
@@ -1014,6 +1077,7 @@ def main():
     ap.add_argument("--skip-stack", action="store_true")
     ap.add_argument("--skip-optim", action="store_true")
     ap.add_argument("--skip-block", action="store_true")
+    ap.add_argument("--skip-variants", action="store_true")
     ap.add_argument("--block-only", action="store_true", help="run only the transformer-block object (profiling runs)")
     ap.add_argument("--optim-only", action="store_true", help="run only the paged AdamW object (profiling runs)")
     ap.add_argument("--decode-only", action="store_true", help="run only the decode-shaped forward (profiling runs)")

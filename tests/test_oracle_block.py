@@ -94,3 +94,12 @@ def test_attention_closed_forms():
     a, _ = block.attention(q, k, v, 1, 3, H, D)
     want = np.cumsum(v, axis=0) / np.arange(1, 4)[:, None]
     np.testing.assert_allclose(a, want, rtol=1e-13)
+
+
+def test_silu_closed_forms():
+    """silu(z) = z * sigmoid(z): sigmoid(ln 3) = 3/4 exactly, silu(0) = 0, and
+    silu(z) - silu(-z) = z for every z (sigmoid(z) + sigmoid(-z) = 1)."""
+    ln3 = np.log(3.0)
+    np.testing.assert_allclose(block.silu(np.array([ln3, -ln3, 0.0])), [0.75 * ln3, -0.25 * ln3, 0.0], rtol=1e-15)
+    z = np.linspace(-20, 20, 81)
+    np.testing.assert_allclose(block.silu(z) - block.silu(-z), z, rtol=1e-14, atol=1e-14)
