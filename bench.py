@@ -178,6 +178,7 @@ def run_ours(args, rank, world, local_rank):
             "dX": torch.empty(TOKENS, K, dtype=torch.bfloat16, device=dev),
             "dA": grads[off: off + R * K].view(R, K),
             "dB": grads[off + R * K: off + R * K + N * R].view(N, R),
+            "grad": grads[off: off + R * K + N * R],
         }
         off += R * K + N * R
         layers.append(L)
@@ -188,14 +189,16 @@ def run_ours(args, rank, world, local_rank):
     step_flops = sum(linear_flops(TOKENS, L["N"], L["K"], R) for L in layers)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)   # > 126 MB L2
 
+    reducer = dp.OverlappedGradSum()
+
     def step():
         for L in layers:
             q.qlora_linear_fwd(L["w"], L["X"], TOKENS, L["A"], L["B"], R, scale, L["Y"], L["H"], ws)
         for L in reversed(layers):
             q.qlora_linear_bwd(L["w"], L["X"], L["dY"], TOKENS, L["A"], L["B"], R, scale, L["H"], L["dX"],
                                L["dA"], L["dB"], ws)
-        if world > 1:
-            dp.allreduce_adapter_grads(grads)
+            reducer.ready(L["grad"])   # this linear's dA, dB: summed while the backward goes on
+        reducer.wait()
 
     def timed_steps(k, fn):
         """Device time of k steps, each after an L2 flush, CUDA events on the
@@ -256,8 +259,8 @@ def run_ours(args, rank, world, local_rank):
             L["dY"].copy_(pin[L["name"]]["dY"], non_blocking=True)
             q.qlora_linear_bwd(L["w"], L["X"], L["dY"], TOKENS, L["A"], L["B"], R, scale, L["H"], L["dX"],
                                L["dA"], L["dB"], ws)
-        if world > 1:
-            dp.allreduce_adapter_grads(grads)
+            reducer.ready(L["grad"])
+        reducer.wait()
         host_grads.copy_(grads, non_blocking=True)
 
     e2e_step()
@@ -575,8 +578,30 @@ def run_decode65b(args, q, torch, dev, peaks, peak_src):
                          for L in layers)
         gbs = nbytes / (ms * 1e-3) / 1e9
         ach = gemv_bytes / (gemv_ms * 1e-3) / 1e9
+        # end to end: every linear's X from pinned host memory, Y back to pinned host memory
+        pin_x = [L["X"].cpu().pin_memory() for L in layers]
+        pin_y = [torch.empty(L["Y"].shape, dtype=L["Y"].dtype).pin_memory() for L in layers]
+
+        def e2e_step():
+            for L, hx, hy in zip(layers, pin_x, pin_y):
+                L["X"].copy_(hx, non_blocking=True)
+                q.qlora_linear_fwd(L["w"], L["X"], M, L["A"], L["B"], R, scale, L["Y"], None, ws)
+                hy.copy_(L["Y"], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        torch.cuda._sleep(20_000_000)
+        e0.record()
+        for _ in range(reps):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / reps
         out["tokens"][str(M)] = {
             "value": round(gbs, 1), "us_per_layer": round(ms * 1e3, 2), "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
+            "e2e": {"value": round(nbytes / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s", "us_per_layer": round(e2e_ms * 1e3, 2),
+                    "h2d_bytes_per_step": sum(2 * M * L["K"] for L in layers),
+                    "d2h_bytes_per_step": sum(2 * M * L["N"] for L in layers)},
             "roofline": {"kernel": "decode_gemv", "bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": None,
                          "peak_source": f"{peak_src} hbm_gbs"},
@@ -837,7 +862,7 @@ def cpu_baseline_linear(budget_s=15.0):
     from oracle import linear as olin
     N = K = 4096
     case = synthetic.linear_case(64, N, K, R, ALPHA, seed=7)
-    Wd = case["W"].float().numpy().astype(np.float64)   # stands for the dequantized bf16 weight
+    Wd = case["W"].float().numpy().astype(np.float64)   # raw N(0, 0.02) weight: the same arithmetic as a dequantized one
     A = case["A"].float().numpy()
     B = case["B"].float().numpy()
     rng = np.random.default_rng(0)
@@ -856,8 +881,8 @@ def cpu_baseline_linear(budget_s=15.0):
             M *= 2
     return {"value": round(flops / spent / 1e12, 5), "unit": "TFLOP/s", "cores": _blas_threads(),
             "kind": "oracle",
-            "sample": f"oracle float64 fwd+bwd of one 4096x4096 linear (r=64), token batches up to {M}, "
-                      f"{spent:.1f} s of host time"}
+            "sample": f"oracle float64 fwd+bwd of one 4096x4096 linear (r=64; the raw N(0,0.02) weight stands "
+                      f"for the dequantized one), token batches up to {M}, {spent:.1f} s of host time"}
 
 
 def _omp_threads():
@@ -925,7 +950,7 @@ def cpu_baseline_stack(budget_s=10.0):
     from oracle import linear as olin
     N = K = 8192
     case = synthetic.linear_case(16, N, K, R, ALPHA, seed=8)
-    Wd = case["W"].float().numpy().astype(np.float64)   # stands for the dequantized bf16 weight
+    Wd = case["W"].float().numpy().astype(np.float64)   # raw N(0, 0.02) weight: the same arithmetic as a dequantized one
     A, B = case["A"].float().numpy(), case["B"].float().numpy()
     rng = np.random.default_rng(1)
     M, spent, flops = 32, 0.0, 0.0

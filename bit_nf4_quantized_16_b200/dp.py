@@ -28,6 +28,34 @@ def allreduce_adapter_grads(flat_grads: torch.Tensor, group=None):
     return flat_grads
 
 
+class OverlappedGradSum:
+    """Sums adapter gradients over the ranks while the backward pass goes on.
+
+    The backward pass runs the linears in reverse order; as soon as one
+    linear's dA and dB are written, `ready(buf)` starts an asynchronous
+    all-reduce of that buffer (a contiguous view of the flattened gradients),
+    so the exchange of the last linears' gradients overlaps the backward of
+    the earlier ones.  `wait()` blocks the current stream (not the host) on
+    every reduction started since the last wait.  Each rank must call
+    `ready` on the same buffers in the same order, which holds when every
+    rank runs the same layer sequence.  With one rank both calls do nothing.
+    """
+
+    def __init__(self, group=None):
+        self.group = group
+        self.pending = []
+        self.active = dist.is_initialized() and dist.get_world_size(group) > 1
+
+    def ready(self, buf: torch.Tensor):
+        if self.active:
+            self.pending.append(dist.all_reduce(buf, op=dist.ReduceOp.SUM, group=self.group, async_op=True))
+
+    def wait(self):
+        for work in self.pending:
+            work.wait()
+        self.pending = []
+
+
 def max_over_ranks(value: float, device=None, group=None) -> float:
     """The largest of the ranks' values (a step time measured on each rank)."""
     if not (dist.is_initialized() and dist.get_world_size(group) > 1):

@@ -101,3 +101,62 @@ def test_two_gloo_ranks_sum_to_the_full_batch_gradient():
         assert t == 2.5          # max over ranks of 1.5 + rank
         shards.append(shard)
     assert shards == [(0, 19), (19, 37)]
+
+
+def _worker_overlapped(rank, world, port, out):
+    """Three linears' backward in reverse order; each linear's dA, dB are
+    handed to the overlapped reducer as soon as they exist (views of one
+    flattened buffer), and the reducer is waited on once at the end."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import sys
+        sys.path.insert(0, os.path.join(HERE, ".."))
+        from oracle import linear as olin
+        dp = _load_dp()
+        cases = [_case(seed=10 + i, N=48 + 8 * i, K=64 + 16 * i) for i in range(3)]
+        sizes = [c["A"].size + c["B"].size for c in cases]
+        flat = torch.zeros(sum(sizes), dtype=torch.float64)
+        offs = np.cumsum([0] + sizes)
+        red = dp.OverlappedGradSum()
+        for i in reversed(range(3)):
+            c = cases[i]
+            a, b = dp.shard_tokens(c["X"].shape[0], rank, world)
+            _, dA, dB = olin.backward(c["X"][a:b], c["W"], c["A"], c["B"], c["s"], c["dY"][a:b])
+            view = flat[offs[i]: offs[i + 1]]
+            view.copy_(torch.from_numpy(np.concatenate([dA.ravel(), dB.ravel()])))
+            red.ready(view)
+        red.wait()
+        out[rank] = (flat.numpy().copy(), len(red.pending))
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def test_overlapped_reduction_sums_every_linear():
+    from oracle import linear as olin
+    world = 2
+    port = _free_port()
+    manager = mp.get_context("spawn").Manager()
+    out = manager.dict()
+    mp.start_processes(_worker_overlapped, args=(world, port, out), nprocs=world, start_method="spawn", join=True)
+    want = []
+    for i in range(3):
+        c = _case(seed=10 + i, N=48 + 8 * i, K=64 + 16 * i)
+        _, dA, dB = olin.backward(c["X"], c["W"], c["A"], c["B"], c["s"], c["dY"])
+        want.append(np.concatenate([dA.ravel(), dB.ravel()]))
+    want = np.concatenate(want)
+    for rank in range(world):
+        got, pending = out[rank]
+        np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+        assert pending == 0
+
+
+def test_overlapped_reduction_is_a_no_op_on_one_rank():
+    dp = _load_dp()
+    red = dp.OverlappedGradSum()
+    buf = torch.arange(6, dtype=torch.float32)
+    red.ready(buf)
+    red.wait()
+    assert torch.equal(buf, torch.arange(6, dtype=torch.float32)) and red.pending == []
