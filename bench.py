@@ -483,6 +483,38 @@ def run_codec(args, q, torch, dev, peaks, peak_src):
     ach = qgbs if dom == "quantize" else dgbs
     peak = peaks["hbm_gbs"]
     del g
+    # end to end on one layer's 7 tensors: each weight copied in from pinned host
+    # memory, quantized, dequantized, and the bf16 result copied back, over the
+    # same four streams
+    layer = tensors[:len(synthetic.LLAMA7B_LINEARS)]
+    pin_in = [W.cpu().pin_memory() for W, _, _ in layer]
+    pin_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _, _, out in layer]
+    lw = sum(W.numel() for W, _, _ in layer)
+
+    def e2e_step():
+        main = torch.cuda.current_stream()
+        for st in side:
+            st.wait_stream(main)
+        for i, ((W, w, out), hi, ho) in enumerate(zip(layer, pin_in, pin_out)):
+            with torch.cuda.stream(side[i % n_streams]):
+                W.copy_(hi, non_blocking=True)
+                q.qlora_quantize_nf4_dq(W, w, qws[i % n_streams])
+                q.qlora_dequantize_nf4_dq(w, out)
+                ho.copy_(out, non_blocking=True)
+        for st in side:
+            main.wait_stream(st)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+    e2e = {"value": round(2 * CODEC_BYTES_PER_WEIGHT * lw / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+           "ms_per_layer": round(e2e_ms, 4), "h2d_bytes_per_step": 2 * lw, "d2h_bytes_per_step": 2 * lw,
+           "workload": "one layer's 7 tensors: pinned host bf16 in, quantize, dequantize, pinned host bf16 out"}
     cpu = None if args.skip_cpu else cpu_baseline_codec(q, torch, tensors)
     return {
         "workload": "codec7b: NF4+DQ quantize->dequantize round trip, 224 LLaMA-7B tensors, "
@@ -502,6 +534,7 @@ def run_codec(args, q, torch, dev, peaks, peak_src):
                     "note": "quantize_ms / dequantize_ms: each API call bracketed by CUDA events on one stream "
                             "(quantize = workspace reset + first-level pass + double quantization); "
                             "per_kernel_ms_bracketed: every kernel bracketed separately (no overlap)"},
+        "e2e": e2e,
         "cpu_baseline": cpu,
     }
 
@@ -676,10 +709,37 @@ def run_stack65b(args, q, torch, dev, peaks, peak_src, layers_n=None, tokens=204
             step()
         e1.record()
         torch.cuda.synchronize()
+    launches = q.qlora_launch_count() - launches0
     q.qlora_check_device_error()
     ms = e0.elapsed_time(e1) / steps
     flops = sum(linear_flops(tokens, L["N"], L["K"], R) for L in lin)
     value = flops / (ms * 1e-3) / 1e12
+    # end to end: the stack's input activation and output gradient come from
+    # pinned host memory each step, and the gradients of the first linear (the
+    # last ones the backward writes) go back to pinned host memory
+    x0, dy0 = act[("X", lin[0]["K"])], act[("dY", lin[-1]["N"])]
+    hx, hdy = x0.cpu().pin_memory(), dy0.cpu().pin_memory()
+    hda = torch.empty(lin[0]["dA"].shape, dtype=torch.float32).pin_memory()
+    hdb = torch.empty(lin[0]["dB"].shape, dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        x0.copy_(hx, non_blocking=True)
+        dy0.copy_(hdy, non_blocking=True)
+        step()
+        hda.copy_(lin[0]["dA"], non_blocking=True)
+        hdb.copy_(lin[0]["dB"], non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / steps
+    e2e = {"value": round(flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 3),
+           "h2d_bytes_per_step": 2 * (x0.numel() + dy0.numel()),
+           "d2h_bytes_per_step": 4 * (lin[0]["dA"].numel() + lin[0]["dB"].numel())}
     return {
         "workload": f"stack65b: {n_layers} LLaMA-65B layers x 7 QLoRA linears fwd+bwd, {tokens} tokens, r=64, "
                     "alpha=16, no attention",
@@ -690,8 +750,9 @@ def run_stack65b(args, q, torch, dev, peaks, peak_src, layers_n=None, tokens=204
                      "unit": "TFLOP/s", "frac": round(value / peaks["bf16_tflops_sustained"], 4),
                      "frac_of_burst_peak": round(value / peaks["bf16_tflops"], 4), "traffic": None,
                      "peak_source": f"{peak_src} bf16_tflops_sustained"},
-        "gpu_launches_per_step": (q.qlora_launch_count() - launches0) // steps,
+        "gpu_launches_per_step": launches // steps,
         "clocks": clk.summary(),
+        "e2e": e2e,
         "cpu_baseline": None if args.skip_cpu else cpu_baseline_stack(),
     }
 
