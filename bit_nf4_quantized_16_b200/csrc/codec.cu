@@ -88,36 +88,48 @@ constexpr uint32_t kQDynSmem = (kQThreads / 32) * kQStages * kQStageBytes + 1024
 // rounded down to binary32, so "n > midpoint_j" holds exactly when n is nearer
 // to value j+1 than to value j (a tie stays with the lower index), and the
 // code is the number of midpoints below n.
-// Keys: an order-preserving integer key of n has the same top 12 bits as a
-// 2^20-wide interval of keys; each such interval holds at most one midpoint
-// (the host checks this), so with
-//   E(j) = (midpoints below interval j) << 20, plus 2^20-1 - low20(key_m) if
+// Keys: an order-preserving integer key of n has the same top 11 bits as a
+// 2^21-wide interval of keys; each interval that scaled elements reach
+// (|n| <= 1, plus rounding) holds at most one midpoint (the host checks this),
+// so with
+//   E(j) = (midpoints below interval j) << 21, plus 2^21-1 - low21(key_m) if
 //          midpoint m lies inside interval j,
-// the code is (E(j) + low20(key)) >> 20 (the carry decides the one midpoint).
-// The kernel uses k = bits(n) with its low 20 bits flipped when n < 0: the
-// top 12 bits of k are the raw sign/exponent/3-bit index i of n, and the low
-// 20 bits of k equal those of the order-preserving key.  Entry i of the
-// table holds E(j(i)) - (i << 20), so that t = table[i] + k holds the code in
-// bits 20..23 and zeros above.
+// the code is (E(j) + low21(key)) >> 21 (the carry decides the one midpoint).
+// The kernel uses k = bits(n) with its low 21 bits flipped when n < 0, and
+// also bit 25 (index bit 4): the top 11 bits of k are the raw sign, exponent
+// and 2-bit mantissa prefix of n, with bit 4 flipped for negative n so that
+// the most used negative and positive intervals of a warp's lookups fall in
+// different shared-memory banks; the low 21 bits of k equal those of the
+// order-preserving key.  Entry i of the table holds E(j(i)) - (i << 21), so
+// that t = table[i] + k holds the code in bits 21..24 and zeros above.
 // The steps are split between the integer and the multiply-add pipes (all of
 // them on the multiply-add pipe, through multiply-high, saturated it and
 // measured 20% slower; all of them on the integer pipe saturated that one).
-// Every CTA builds the table once: thread t fills the entries of ordered
-// intervals j = 16t..16t+15, walking the sorted midpoint keys once.
+// Every CTA builds the table once: thread t < 256 fills the entries of
+// ordered intervals j = 8t..8t+7, walking the sorted midpoint keys once.
+constexpr int kLutShift = 21;
+constexpr uint32_t kLutEntries = 1u << (32 - kLutShift);       // 2048
+constexpr uint32_t kLutLow = (1u << kLutShift) - 1;
+constexpr uint32_t kLutNegSwizzle = 16u;                        // index bits flipped for n < 0
+constexpr uint32_t kLutSignMask = kLutLow | (kLutNegSwizzle << kLutShift);
+
 __device__ __forceinline__ void build_code_lut(uint32_t *lut, const uint32_t *mkey_smem)
 {
-    const uint32_t first = threadIdx.x * 16u;
+    constexpr uint32_t kPer = kLutEntries / 256;
+    const uint32_t first = threadIdx.x * kPer;
     uint32_t j = 0;
-    while (j < 15 && mkey_smem[j] < (first << 20)) j++;
+    while (j < 15 && mkey_smem[j] < (first << kLutShift)) j++;
 #pragma unroll
-    for (int t = 0; t < 16; t++) {
+    for (uint32_t t = 0; t < kPer; t++) {
         const uint32_t idx = first + t;    // interval of the order-preserving key
-        while (j < 15 && mkey_smem[j] < (idx << 20)) j++;
+        while (j < 15 && mkey_smem[j] < (idx << kLutShift)) j++;
         uint32_t inc = 0;
-        if (j < 15 && (mkey_smem[j] >> 20) == idx) inc = 0xFFFFFu - (mkey_smem[j] & 0xFFFFFu);
-        // raw index: positive numbers have key = bits | 2^31, negative ones ~bits
-        const uint32_t raw = idx >= 2048u ? idx - 2048u : 4095u - idx;
-        lut[raw] = (j << 20) + inc - (raw << 20);
+        if (j < 15 && (mkey_smem[j] >> kLutShift) == idx) inc = kLutLow - (mkey_smem[j] & kLutLow);
+        // raw index: positive numbers have key = bits | 2^31, negative ones ~bits;
+        // negative ones also have index bit 4 flipped (the bank swizzle)
+        const uint32_t half = kLutEntries / 2;
+        const uint32_t raw = idx >= half ? idx - half : ((kLutEntries - 1) - idx) ^ kLutNegSwizzle;
+        lut[raw] = (j << kLutShift) + inc - (raw << kLutShift);
     }
 }
 
@@ -130,12 +142,11 @@ __device__ __forceinline__ uint32_t add_code(const uint32_t *lut, float n, uint3
 {
     const uint32_t b = __float_as_uint(n);
     const uint32_t s = (uint32_t)__mulhi((int)b, 2);        // 0 or all ones: the sign mask
-    const uint32_t k = b ^ (s & 0xFFFFFu);                  // low 20 bits flipped for n < 0
-    const uint32_t t = lut[k >> 20] + k;                    // code in bits 20..23, zero above
+    const uint32_t k = b ^ (s & kLutSignMask);              // low 21 bits and bit 25 flipped for n < 0
+    const uint32_t t = lut[k >> kLutShift] + k;             // code in bits 21..24, zero above
     uint32_t part;
-    if constexpr (4 * I < 20) part = __umulhi(t, 1u << (12 + 4 * I));  // t >> (20 - 4I)
-    else if constexpr (4 * I == 20) part = t;
-    else part = t * (1u << (4 * I - 20));                              // t << (4I - 20)
+    if constexpr (4 * I < kLutShift) part = __umulhi(t, 1u << (32 - kLutShift + 4 * I));   // t >> (21 - 4I)
+    else part = t * (1u << (4 * I - kLutShift));                                          // t << (4I - 21)
     return acc | (part & (0xFu << (4 * I)));
 }
 
@@ -179,7 +190,7 @@ __global__ void __maxnreg__(64) quantize_blocks_kernel(const __grid_constant__ Q
     constexpr bool kF32In = kIn == 1;
     constexpr bool kF16In = kIn == 2;
     static_assert(kQThreads >= 256, "the first 256 threads build the code table and own the buckets");
-    __shared__ __align__(16) uint32_t lut[4096];
+    __shared__ __align__(16) uint32_t lut[kLutEntries];
     __shared__ unsigned long long s_acc[256];
     __shared__ uint32_t s_mkey[16];
     __shared__ bool s_last;
@@ -524,7 +535,12 @@ qlora_status midpoint_keys(const float q[16], uint32_t out[15])
         float m = round_down_f32(sum / 2.0);
         if (m == 0.0f) m = 0.0f;  // +0, never -0
         out[j] = host_sortable_key(m);
-        if (j > 0 && (out[j] >> 20) == (out[j - 1] >> 20)) return QLORA_ERR_UNSUPPORTED;
+        // two midpoints in one key interval: only an interval that scaled
+        // elements reach (|n| <= 1, plus rounding) must hold at most one
+        const uint32_t iv = out[j] >> kLutShift;
+        if (j > 0 && iv == (out[j - 1] >> kLutShift) && iv >= (host_sortable_key(-1.0001f) >> kLutShift) &&
+            iv <= (host_sortable_key(1.0001f) >> kLutShift))
+            return QLORA_ERR_UNSUPPORTED;
     }
     return QLORA_OK;
 }

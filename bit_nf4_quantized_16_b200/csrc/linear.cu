@@ -31,6 +31,7 @@
 #include <utility>
 
 #include "common.cuh"
+#include "debug.cuh"
 #include "decode.cuh"
 #include "gemm.cuh"
 #include "gemm_pair.cuh"
@@ -213,12 +214,28 @@ struct Plan {
     int64_t M, N, K;
     int r, r_pad;
     size_t off_h2, off_g2, bytes;
+    // 17..256 tokens (single-CTA engine): contraction splits of the fused
+    // forward and input gradient when their output tiles would leave SMs idle,
+    // and the fp32 partial planes they write
+    int split_fwd, split_dx;
+    size_t off_split;
     // LoRA dropout: the dropped-out input X_d (bf16 [M][K]) and the frozen
     // path's fp32 input gradient [M][K]
     size_t off_xd, off_dxs;
 };
 
 size_t align256(size_t v) { return (v + 255) / 256 * 256; }
+
+// Contraction splits for a single-CTA fused GEMM with `tiles` output tiles and
+// `k_steps` 64-deep steps: enough CTAs to cover the SMs, at most 8 splits and
+// at least 8 steps per split.
+int choose_splits(int tiles, int k_steps, int sms)
+{
+    int sp = tiles > 0 ? sms / tiles : 1;
+    sp = std::max(1, std::min(sp, 8));
+    while (sp > 1 && k_steps / sp < 8) sp--;
+    return sp;
+}
 
 Plan make_plan(int64_t M, int64_t N, int64_t K, int r, int sms, bool dropout = false)
 {
@@ -239,7 +256,59 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int r, int sms, bool dropout = f
         pl.off_dxs = pl.off_xd + align256((size_t)M * K * 2);
         pl.bytes = pl.off_dxs + align256((size_t)M * K * 4);
     }
+    pl.split_fwd = pl.split_dx = 1;
+    if (M > kDecodeMaxTokens && M <= 256) {
+        pl.split_fwd = choose_splits(ceil_div(N, 128), (int)(K / 64), sms);
+        pl.split_dx = dropout ? 1 : choose_splits(ceil_div(K, 128), ceil_div(N, 64), sms);
+        const size_t planes = std::max((size_t)pl.split_fwd * M * N, (size_t)pl.split_dx * M * K);
+        if (pl.split_fwd > 1 || pl.split_dx > 1) {
+            pl.off_split = pl.bytes;
+            pl.bytes = pl.off_split + align256(planes * 4);
+        }
+    }
     return pl;
+}
+
+// ---- split contraction of the single-CTA fused GEMMs ------------------------------------
+
+// out[m][c] = sum over s = 0 .. splits-1 (in that order) of planes[s][m][c],
+// stored as bf16 / fp16 / fp32; four columns per thread (cols % 4 == 0).
+__global__ void __launch_bounds__(256) split_sum_kernel(const float *planes, int splits, int64_t rows, int64_t cols,
+                                                        void *out, int out_type)
+{
+    sm100::pdl_wait();
+    sm100::pdl_trigger();
+    const int64_t n4 = rows * cols / 4, plane = rows * cols;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+        float4 a = __ldcg(reinterpret_cast<const float4 *>(planes) + i);
+        for (int sp = 1; sp < splits; sp++) {
+            if (!QLORA_IN(sp * plane + 4 * i + 3, splits * plane)) break;
+            const float4 b = __ldcg(reinterpret_cast<const float4 *>(planes + sp * plane) + i);
+            a = make_float4(__fadd_rn(a.x, b.x), __fadd_rn(a.y, b.y), __fadd_rn(a.z, b.z), __fadd_rn(a.w, b.w));
+        }
+        if (out_type == QLORA_FP32) {
+            reinterpret_cast<float4 *>(out)[i] = a;
+        } else if (out_type == QLORA_FP16) {
+            const __half2 lo = __floats2half2_rn(a.x, a.y), hi = __floats2half2_rn(a.z, a.w);
+            reinterpret_cast<uint2 *>(out)[i] =
+                make_uint2(*reinterpret_cast<const uint32_t *>(&lo), *reinterpret_cast<const uint32_t *>(&hi));
+        } else {
+            const __nv_bfloat162 lo = __floats2bfloat162_rn(a.x, a.y), hi = __floats2bfloat162_rn(a.z, a.w);
+            reinterpret_cast<uint2 *>(out)[i] =
+                make_uint2(*reinterpret_cast<const uint32_t *>(&lo), *reinterpret_cast<const uint32_t *>(&hi));
+        }
+    }
+}
+
+qlora_status run_split_sum(const float *planes, int splits, int64_t rows, int64_t cols, void *out, qlora_dtype out_type,
+                           const DeviceInfo &dev, cudaStream_t s, int kind)
+{
+    const int64_t n4 = rows * cols / 4;
+    const int grid = (int)std::min<int64_t>((n4 + 255) / 256, 4 * dev.sms);
+    LaunchScope ls(kind, s);
+    QLORA_CUDA_TRY(launch_pdl(split_sum_kernel, dim3(grid), dim3(256), 0, s, planes, splits, rows, cols, out,
+                              (int)out_type));
+    return launch_status();
 }
 
 // ---- LoRA dropout ---------------------------------------------------------------------
@@ -450,6 +519,16 @@ static qlora_status linear_fwd(const qlora_nf4_weight *w, const void *X, int64_t
         if (y_dtype != QLORA_FP32) return launch_gemm_pair<kBNf4K, kEpiBf16, kFMT, F16>(p, dev, s, QLORA_KERNEL_FWD_FUSED);
         return launch_gemm_pair<kBNf4K, kEpiF32, kFMT, F16>(p, dev, s, QLORA_KERNEL_FWD_FUSED);
     }
+    if (pl.split_fwd > 1) {
+        // few output tiles: split the contraction, then sum the planes in order
+        float *planes = reinterpret_cast<float *>(ws + pl.off_split);
+        p.splits = pl.split_fwd;
+        p.k_stages_split = ceil_div(p.k_stages_total, p.splits);
+        p.out = planes;
+        p.split_stride = M * pl.N;
+        QLORA_TRY((launch_gemm<kFBN, kBNf4K, kEpiF32, kFMT, F16>(p, dev, s, QLORA_KERNEL_FWD_FUSED)));
+        return run_split_sum(planes, p.splits, M, pl.N, Y, y_dtype, dev, s, QLORA_KERNEL_ELEMENTWISE);
+    }
     if (y_dtype != QLORA_FP32) return launch_gemm<kFBN, kBNf4K, kEpiBf16, kFMT, F16>(p, dev, s, QLORA_KERNEL_FWD_FUSED);
     return launch_gemm<kFBN, kBNf4K, kEpiF32, kFMT, F16>(p, dev, s, QLORA_KERNEL_FWD_FUSED);
 }
@@ -565,6 +644,15 @@ static qlora_status linear_bwd(const qlora_nf4_weight *w, const void *X, const v
                 QLORA_TRY((launch_gemm_pair<kBNf4MN, kEpiBf16, kBMT, F16>(p, dev, s, QLORA_KERNEL_BWD_FUSED)));
             else
                 QLORA_TRY((launch_gemm_pair<kBNf4MN, kEpiF32, kBMT, F16>(p, dev, s, QLORA_KERNEL_BWD_FUSED)));
+        } else if (pl.split_dx > 1) {
+            // few output tiles: split the contraction, then sum the planes in order
+            float *planes = reinterpret_cast<float *>(ws + pl.off_split);
+            p.splits = pl.split_dx;
+            p.k_stages_split = ceil_div(p.k_stages_total, p.splits);
+            p.out = planes;
+            p.split_stride = M * K;
+            QLORA_TRY((launch_gemm<kBBN, kBNf4MN, kEpiF32, kBMT, F16>(p, dev, s, QLORA_KERNEL_BWD_FUSED)));
+            QLORA_TRY(run_split_sum(planes, p.splits, M, K, dX, dx_dtype, dev, s, QLORA_KERNEL_ELEMENTWISE));
         } else if (!f32_out)
             QLORA_TRY((launch_gemm<kBBN, kBNf4MN, kEpiBf16, kBMT, F16>(p, dev, s, QLORA_KERNEL_BWD_FUSED)));
         else

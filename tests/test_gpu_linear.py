@@ -165,6 +165,15 @@ def test_single_cta_fused_bf16_outputs(q, M):
     full_check(q, synthetic.linear_case(M, 384, 512, 64, alpha=16.0, seed=300 + M), ydt=torch.bfloat16)
 
 
+@pytest.mark.parametrize("M,N,K", [(17, 1024, 4096), (200, 1024, 4096), (256, 4096, 4096), (100, 512, 8192)])
+@pytest.mark.parametrize("ydt", [torch.float32, torch.bfloat16])
+def test_single_cta_split_contraction(q, M, N, K, ydt):
+    """17..256 tokens with few output tiles: the single-CTA fused forward and
+    input gradient split the contraction over idle SMs (fp32 planes summed in
+    order by a second kernel)."""
+    full_check(q, synthetic.linear_case(M, N, K, 64, alpha=16.0, seed=500 + M + N), ydt=ydt)
+
+
 @pytest.mark.parametrize("M", [16, 200, 512])
 def test_int4_codebook(q, M):
     """The Int4 table through the same kernels: the decode forward (16
