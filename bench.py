@@ -251,12 +251,28 @@ def run_ours(args, rank, world, local_rank):
     h2d = sum(L["X"].numel() * 2 + L["dY"].numel() * 2 for L in layers)
     d2h = grads.numel() * 4
 
+    copy_s = torch.cuda.Stream()
+
     def e2e_step():
-        for L in layers:
-            L["X"].copy_(pin[L["name"]]["X"], non_blocking=True)
+        # host-to-device copies on a side stream, in the order the kernels
+        # need them, so that they overlap the compute of the linears before
+        main = torch.cuda.current_stream()
+        copy_s.wait_stream(main)   # the previous step no longer reads these buffers
+        ev_x, ev_dy = [], []
+        with torch.cuda.stream(copy_s):
+            for L in layers:
+                L["X"].copy_(pin[L["name"]]["X"], non_blocking=True)
+                ev_x.append(torch.cuda.Event())
+                ev_x[-1].record(copy_s)
+            for L in reversed(layers):
+                L["dY"].copy_(pin[L["name"]]["dY"], non_blocking=True)
+                ev_dy.append(torch.cuda.Event())
+                ev_dy[-1].record(copy_s)
+        for L, e in zip(layers, ev_x):
+            main.wait_event(e)
             q.qlora_linear_fwd(L["w"], L["X"], TOKENS, L["A"], L["B"], R, scale, L["Y"], L["H"], ws)
-        for L in reversed(layers):
-            L["dY"].copy_(pin[L["name"]]["dY"], non_blocking=True)
+        for L, e in zip(reversed(layers), ev_dy):
+            main.wait_event(e)
             q.qlora_linear_bwd(L["w"], L["X"], L["dY"], TOKENS, L["A"], L["B"], R, scale, L["H"], L["dX"],
                                L["dA"], L["dB"], ws)
             reducer.ready(L["grad"])
@@ -406,7 +422,7 @@ def run_codec(args, q, torch, dev, peaks, peak_src):
     # the tensors are independent: they are spread over a few streams (one
     # quantize workspace each) so that one tensor's launch and tail overlap
     # another's streaming
-    n_streams = 4
+    n_streams = args.codec_streams
     qws_bytes = max(q.qlora_quantize_workspace_bytes(N, K) for N, K in shapes)
     qws = [torch.empty(qws_bytes, dtype=torch.uint8, device=dev) for _ in range(n_streams)]
     side = [torch.cuda.Stream() for _ in range(n_streams)]
@@ -1175,6 +1191,7 @@ def main():
     ap.add_argument("--codec-tensors", type=int, default=0,
                     help="limit the codec round trip to the first N LLaMA-7B tensors (profiling runs)")
     ap.add_argument("--codec-only", action="store_true", help="run only the codec round trip (profiling runs)")
+    ap.add_argument("--codec-streams", type=int, default=4, help="streams the independent codec tensors spread over")
     ap.add_argument("--codec-shape", default=None,
                     help="NxK: time quantize and dequantize of one tensor of this shape only (profiling runs)")
     args = ap.parse_args()
