@@ -88,34 +88,35 @@ constexpr uint32_t kQDynSmem = (kQThreads / 32) * kQStages * kQStageBytes + 1024
 // rounded down to binary32, so "n > midpoint_j" holds exactly when n is nearer
 // to value j+1 than to value j (a tie stays with the lower index), and the
 // code is the number of midpoints below n.
-// Keys: an order-preserving integer key of n has the same top 11 bits as a
-// 2^21-wide interval of keys; each interval that scaled elements reach
-// (|n| <= 1, plus rounding) holds at most one midpoint (the host checks this),
-// so with
-//   E(j) = (midpoints below interval j) << 21, plus 2^21-1 - low21(key_m) if
-//          midpoint m lies inside interval j,
-// the code is (E(j) + low21(key)) >> 21 (the carry decides the one midpoint).
-// The kernel uses k = bits(n) with its low 21 bits flipped when n < 0, and
-// also bit 25 (index bit 4): the top 11 bits of k are the raw sign, exponent
-// and 2-bit mantissa prefix of n, with bit 4 flipped for negative n so that
-// the most used negative and positive intervals of a warp's lookups fall in
-// different shared-memory banks; the low 21 bits of k equal those of the
-// order-preserving key.  Entry i of the table holds E(j(i)) - (i << 21), so
-// that t = table[i] + k holds the code in bits 21..24 and zeros above.
-// The steps are split between the integer and the multiply-add pipes (all of
-// them on the multiply-add pipe, through multiply-high, saturated it and
-// measured 20% slower; all of them on the integer pipe saturated that one).
-// Every CTA builds the table once: thread t < 256 fills the entries of
-// ordered intervals j = 8t..8t+7, walking the sorted midpoint keys once.
+// Keys: the order-preserving integer key of n (bits | 2^31 for n >= +0, ~bits
+// for n <= -0) splits into an 11-bit interval index and a 21-bit offset; each
+// interval that scaled elements reach (|n| <= 1, plus rounding) holds at most
+// one midpoint (the host checks this).  The table is indexed by the top 11 RAW
+// bits of n (sign, exponent, two mantissa bits), which name one interval; its
+// entry plus the raw bits of n gives, through the carry out of the low 21
+// bits, the code in bits 28..31 (bits 21..27 of the entry are ones so that the
+// carry reaches bit 28):
+//  - n >= +0: offset = low21(bits) grows with n; with j midpoints below the
+//    interval and midpoint m inside it, the entry adds 2^21-1 - low21(key_m),
+//    so the carry is [n > m] and the nibble j + [n > m];
+//  - n <= -0: low21(bits) grows as n falls, so the entry yields 15 - code
+//    (the nibble rises with |n| as the code falls): its top is 15 - j, or
+//    14 - j and 1 + low21(key_m) added when m lies inside; the packed word's
+//    nibbles of negative elements are complemented afterwards, from the input
+//    sign bits (eight at a time with byte permutes).
+// Entry i holds its value minus i << 21, so the sum's top bits depend only on
+// the entry.  Per element: a shift (the index), a shared load, an add and a
+// funnel shift that moves the nibble into the packed word.
+// Every CTA builds the table once: thread t < 256 fills the entries of the
+// key-ordered intervals 8t..8t+7, walking the sorted midpoint keys once.
 constexpr int kLutShift = 21;
 constexpr uint32_t kLutEntries = 1u << (32 - kLutShift);       // 2048
 constexpr uint32_t kLutLow = (1u << kLutShift) - 1;
-constexpr uint32_t kLutNegSwizzle = 16u;                        // index bits flipped for n < 0
-constexpr uint32_t kLutSignMask = kLutLow | (kLutNegSwizzle << kLutShift);
 
 __device__ __forceinline__ void build_code_lut(uint32_t *lut, const uint32_t *mkey_smem)
 {
     constexpr uint32_t kPer = kLutEntries / 256;
+    constexpr uint32_t kHalf = kLutEntries / 2;
     const uint32_t first = threadIdx.x * kPer;
     uint32_t j = 0;
     while (j < 15 && mkey_smem[j] < (first << kLutShift)) j++;
@@ -123,31 +124,68 @@ __device__ __forceinline__ void build_code_lut(uint32_t *lut, const uint32_t *mk
     for (uint32_t t = 0; t < kPer; t++) {
         const uint32_t idx = first + t;    // interval of the order-preserving key
         while (j < 15 && mkey_smem[j] < (idx << kLutShift)) j++;
-        uint32_t inc = 0;
-        if (j < 15 && (mkey_smem[j] >> kLutShift) == idx) inc = kLutLow - (mkey_smem[j] & kLutLow);
-        // raw index: positive numbers have key = bits | 2^31, negative ones ~bits;
-        // negative ones also have index bit 4 flipped (the bank swizzle)
-        const uint32_t half = kLutEntries / 2;
-        const uint32_t raw = idx >= half ? idx - half : ((kLutEntries - 1) - idx) ^ kLutNegSwizzle;
-        lut[raw] = (j << kLutShift) + inc - (raw << kLutShift);
+        const bool inside = j < 15 && (mkey_smem[j] >> kLutShift) == idx;
+        const uint32_t low_m = inside ? mkey_smem[j] & kLutLow : 0u;
+        uint32_t raw, top, inc;
+        if (idx >= kHalf) {                // n >= +0: key = bits | 2^31
+            raw = idx - kHalf;
+            top = j;
+            inc = inside ? kLutLow - low_m : 0u;
+        } else {                           // n <= -0: key = ~bits
+            raw = (kLutEntries - 1) - idx;
+            top = inside ? 14 - j : 15 - j;
+            inc = inside ? low_m + 1 : 0u;
+        }
+        lut[raw] = (((top << 7) | 0x7Fu) << kLutShift) + inc - (raw << kLutShift);
     }
 }
 
-// Code of n inserted at nibble position 4*I of acc (whose nibble I is zero).
-// The sign mask and the move of the code to its nibble are multiplications
-// (multiply-add pipe), the table index, the add and the logic ops integer-pipe
-// instructions: the two pipes carry about equal shares.
-template <int I>
-__device__ __forceinline__ uint32_t add_code(const uint32_t *lut, float n, uint32_t acc)
+// Table entry plus the raw bits of n: the code of n (15 - code for n <= -0)
+// in bits 28..31.
+__device__ __forceinline__ uint32_t code_top(const uint32_t *lut, float n)
 {
     const uint32_t b = __float_as_uint(n);
-    const uint32_t s = (uint32_t)__mulhi((int)b, 2);        // 0 or all ones: the sign mask
-    const uint32_t k = b ^ (s & kLutSignMask);              // low 21 bits and bit 25 flipped for n < 0
-    const uint32_t t = lut[k >> kLutShift] + k;             // code in bits 21..24, zero above
-    uint32_t part;
-    if constexpr (4 * I < kLutShift) part = __umulhi(t, 1u << (32 - kLutShift + 4 * I));   // t >> (21 - 4I)
-    else part = t * (1u << (4 * I - kLutShift));                                          // t << (4I - 21)
-    return acc | (part & (0xFu << (4 * I)));
+    return lut[b >> kLutShift] + b;
+}
+
+// 8 nibbles of 8 consecutive values (already multiplied by r), element 0 in
+// bits 0-3, those of negative elements still complemented: each funnel shift
+// moves the word up one nibble and brings in the next lower element's nibble.
+__device__ __forceinline__ uint32_t codes8(const uint32_t *lut, const float (&n)[8])
+{
+    uint32_t word = code_top(lut, n[7]) >> 28;
+#pragma unroll
+    for (int e = 6; e >= 0; e--) word = __funnelshift_l(code_top(lut, n[e]), word, 4);
+    return word;
+}
+
+// Byte permute whose selector nibbles with bit 3 set replicate the sign bit
+// of the chosen byte (0x00 or 0xFF).
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
+{
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// Nibble mask of the negative elements among 8 elements given as 16-bit
+// pairs u0..u3 (element 2j in the low half of uj): 0xF at nibble e where
+// element e has its sign bit set.
+__device__ __forceinline__ uint32_t neg_nibbles16(uint32_t u0, uint32_t u1, uint32_t u2, uint32_t u3)
+{
+    const uint32_t x = prmt(u0, u1, 0xFDB9);   // byte k: sign of element k (0..3)
+    const uint32_t y = prmt(u2, u3, 0xFDB9);   // elements 4..7
+    const uint32_t even = prmt(x, y, 0x6420);  // elements 0, 2, 4, 6
+    const uint32_t odd = prmt(x, y, 0x7531);   // elements 1, 3, 5, 7
+    return (even & 0x0F0F0F0Fu) | (odd & 0xF0F0F0F0u);
+}
+
+// The same for 8 binary32 elements (sign in byte 3 of each word).
+__device__ __forceinline__ uint32_t neg_nibbles32(const uint4 &v0, const uint4 &v1)
+{
+    const uint32_t even = prmt(prmt(v0.x, v0.z, 0xFFFB), prmt(v1.x, v1.z, 0xFFFB), 0x5410);
+    const uint32_t odd = prmt(prmt(v0.y, v0.w, 0xFFFB), prmt(v1.y, v1.w, 0xFFFB), 0x5410);
+    return (even & 0x0F0F0F0Fu) | (odd & 0xF0F0F0F0u);
 }
 
 // Magnitude maximum of two bf16 (F16: fp16) pairs, lane by lane
@@ -162,19 +200,6 @@ __device__ __forceinline__ uint32_t maxabs16x2(uint32_t a, uint32_t b)
     else
         asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
     return d;
-}
-
-// 8 codes of 8 consecutive values (already multiplied by r), element 0 in bits 0-3.
-__device__ __forceinline__ uint32_t codes8(const uint32_t *lut, const float (&n)[8])
-{
-    uint32_t word = add_code<0>(lut, n[0], 0u);
-    word = add_code<1>(lut, n[1], word);
-    word = add_code<2>(lut, n[2], word);
-    word = add_code<3>(lut, n[3], word);
-    word = add_code<4>(lut, n[4], word);
-    word = add_code<5>(lut, n[5], word);
-    word = add_code<6>(lut, n[6], word);
-    return add_code<7>(lut, n[7], word);
 }
 
 // One lane per block of 64 weights, 32 consecutive blocks per warp and step:
@@ -208,19 +233,13 @@ __global__ void __maxnreg__(64) quantize_blocks_kernel(const __grid_constant__ Q
     uint8_t *ring = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(q_dyn) + 1023) & ~uintptr_t(1023)) +
                     warp * kQStages * kQStageBytes;
     __shared__ uint64_t s_bar[kQThreads / 32][kQStages];
-    // launched with programmatic serialization: the input may come from the
-    // kernel before this one; the double-quantization kernel after it may
-    // become resident now and wait for this grid's completion
-    sm100::pdl_wait();
-    sm100::pdl_trigger();
+    // Set-up that reads no memory another kernel writes (barriers, the code
+    // table from the parameters) runs before the dependency wait: launched with
+    // programmatic serialization, it overlaps the tail of the kernel before
+    // (for a quantize call, the kernel that reset its reduction slots).
     if (!kF32In && lane == 0) {
         for (int st = 0; st < kQStages; st++) sm100::mbar_init(&s_bar[warp][st], 1);
         sm100::fence_barrier_init();
-        const bool skip = p.stall_inject && blockIdx.x == 0 && warp == 0;
-        if (first < p.nblocks && !skip) {
-            sm100::mbar_arrive_expect_tx(&s_bar[warp][0], kQStageBytes);
-            sm100::tma_load_2d(ring, &p.tm_w, &s_bar[warp][0], 0, (int32_t)first);
-        }
     }
     if (threadIdx.x == 0) {
 #pragma unroll
@@ -229,6 +248,18 @@ __global__ void __maxnreg__(64) quantize_blocks_kernel(const __grid_constant__ Q
     if (threadIdx.x < 256) s_acc[threadIdx.x] = 0;
     __syncthreads();
     if (threadIdx.x < 256) build_code_lut(lut, s_mkey);
+    // the input, the reduction slots and the outputs from here on; the
+    // double-quantization kernel after this one may become resident now and
+    // wait for this grid's completion
+    sm100::pdl_wait();
+    sm100::pdl_trigger();
+    if (!kF32In && lane == 0) {
+        const bool skip = p.stall_inject && blockIdx.x == 0 && warp == 0;
+        if (first < p.nblocks && !skip) {
+            sm100::mbar_arrive_expect_tx(&s_bar[warp][0], kQStageBytes);
+            sm100::tma_load_2d(ring, &p.tm_w, &s_bar[warp][0], 0, (int32_t)first);
+        }
+    }
     __syncthreads();
     uint32_t it = 0;
     for (int64_t b0 = first; b0 < p.nblocks; b0 += nwarps * 32, it++) {
@@ -289,7 +320,7 @@ __global__ void __maxnreg__(64) quantize_blocks_kernel(const __grid_constant__ Q
                                   n[2 * j + 1]);
                     }
                 }
-                words[i] = codes8(lut, n);
+                words[i] = codes8(lut, n) ^ neg_nibbles16(u[0], u[1], u[2], u[3]);
             }
         } else {
             const uint4 *src = static_cast<const uint4 *>(p.W) + 16 * b;  // 64 fp32 = 16 x 16 B
@@ -311,7 +342,7 @@ __global__ void __maxnreg__(64) quantize_blocks_kernel(const __grid_constant__ Q
                 nf4::mul2(__uint_as_float(v0.z), __uint_as_float(v0.w), r, n[2], n[3]);
                 nf4::mul2(__uint_as_float(v1.x), __uint_as_float(v1.y), r, n[4], n[5]);
                 nf4::mul2(__uint_as_float(v1.z), __uint_as_float(v1.w), r, n[6], n[7]);
-                words[i] = codes8(lut, n);
+                words[i] = codes8(lut, n) ^ neg_nibbles32(v0, v1);
             }
         }
         if (act && QLORA_IN(b, p.nblocks)) {
@@ -571,6 +602,17 @@ qlora_status prepare_quantize(QuantParams &qp, const void *W, qlora_dtype w_dtyp
     return QLORA_OK;
 }
 
+// Resets the quantizer's reduction slots (bucket sums and the CTA ticket) at
+// the start of a call; a kernel rather than a memset so that the quantizer's
+// set-up can overlap it under programmatic dependent launch.
+__global__ void __launch_bounds__(64) reset_slots_kernel(unsigned long long *acc, unsigned int *ticket)
+{
+    sm100::pdl_wait();   // the previous call on this workspace may still read the slots
+    sm100::pdl_trigger();
+    for (int i = threadIdx.x; i < 256; i += 64) acc[i] = 0ull;
+    if (threadIdx.x == 0) *ticket = 0u;
+}
+
 // The quantizer for the input type w_dtype.
 cudaError_t launch_quantize(qlora_dtype w_dtype, int grid, cudaStream_t s, const QuantParams &qp)
 {
@@ -591,6 +633,19 @@ int grid_for(int64_t work_items, int items_per_cta, int max_ctas)
 
 // Workspace layout for the quantizer: [acc 256 u64][ticket u32 + pad to 16][c1 floats]
 static constexpr size_t kAccBytes = 256 * sizeof(unsigned long long) + 16;
+
+// The reduction slots and the arrival ticket start at zero on every call.
+static qlora_status reset_slots(void *ws, cudaStream_t s)
+{
+    {
+        LaunchScope ls(QLORA_KERNEL_ELEMENTWISE, s);
+        QLORA_CUDA_TRY(launch_pdl(reset_slots_kernel, dim3(1), dim3(64), 0, s,
+                                  static_cast<unsigned long long *>(ws),
+                                  reinterpret_cast<unsigned int *>(static_cast<char *>(ws) +
+                                                                   256 * sizeof(unsigned long long))));
+    }
+    return launch_status();
+}
 
 }  // namespace qlora
 
@@ -621,7 +676,7 @@ extern "C" qlora_status qlora_quantize_nf4_dq(const void *W, qlora_dtype w_dtype
     const int64_t numel = out->rows * out->cols;
     const int64_t nblocks = numel / QLORA_BLOCK;
     char *ws = static_cast<char *>(workspace);
-    QLORA_CUDA_TRY(cudaMemsetAsync(ws, 0, kAccBytes, s));
+    QLORA_TRY(reset_slots(ws, s));
 
     QuantParams qp;
     qp.W = W;
@@ -753,8 +808,7 @@ extern "C" qlora_status qlora_quantize_nf4_dq_noalloc(const void *W, qlora_dtype
     QLORA_TRY(static_scratch(dev.device, &ws));
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // the reduction slots and the arrival ticket start at zero on every call
-    QLORA_CUDA_TRY(cudaMemsetAsync(ws, 0, kAccBytes, s));
+    QLORA_TRY(reset_slots(ws, s));
 
     QuantParams qp;
     qp.W = W;

@@ -497,7 +497,7 @@ enum {
     QLORA_KERNEL_BWD_FUSED = 4,   /* fused dequant-GEMM, input gradient  */
     QLORA_KERNEL_LOWRANK = 5,     /* H = X A^T and G = dY B products     */
     QLORA_KERNEL_WGRAD = 6,       /* dA and dB products                  */
-    QLORA_KERNEL_ELEMENTWISE = 7, /* split-sum / hi-lo finalize kernels  */
+    QLORA_KERNEL_ELEMENTWISE = 7, /* split-sum, finalize, slot resets    */
     QLORA_KERNEL_OPTIMIZER = 8,   /* AdamW update of the adapters        */
     QLORA_KERNEL_BLOCK = 9,       /* block norms, RoPE, SwiGLU           */
     QLORA_KERNEL_ATTENTION = 10,  /* block attention products, softmax   */

@@ -258,3 +258,26 @@ def test_double_quantization_near_e4m3_boundaries(q):
     c1 = np.array(c1, np.float32)
     assert c1.min() > 0
     check_parity(q, _blocks_with_absmax(c1, 6))
+
+
+def test_back_to_back_calls_share_one_workspace(q):
+    """Several quantize calls queued on one stream with one workspace and no
+    host synchronization between them: each call resets the shared reduction
+    slots and arrival ticket only after the call before it has finished with
+    them, so every weight matches the oracle."""
+    shapes = [(4096, 4096), (64, 4096), (11008, 4096), (3, 192), (4096, 11008)]
+    Ws = [synthetic.normal(s, 0.02, seed=90 + i, dtype=torch.bfloat16) for i, s in enumerate(shapes)]
+    nbytes = max(q.qlora_quantize_workspace_bytes(r, c) for r, c in shapes)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    Wd = [W.cuda() for W in Ws]
+    outs = [q.NF4Weight(r, c, device="cuda") for r, c in shapes]
+    torch.cuda.synchronize()
+    for W, w in zip(Wd, outs):
+        q.qlora_quantize_nf4_dq(W, w, ws)
+    torch.cuda.synchronize()
+    for W, w in zip(Ws, outs):
+        ref = occ.quantize(W.float().numpy(), Q)
+        assert np.array_equal(w.packed.cpu().numpy(), ref["packed"]), "packed codes"
+        assert np.array_equal(w.code2.cpu().numpy(), ref["e"]), "E4M3 codes"
+        assert np.array_equal(w.c2.cpu().numpy().view(np.uint32), ref["c2"].view(np.uint32)), "group scales"
+        assert w.mean[0].item() == float(ref["mean"]), "mean"
