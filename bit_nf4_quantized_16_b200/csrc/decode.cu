@@ -12,8 +12,12 @@
 // decode_gemv_kernel: each warp owns 16 rows of W (or of A) and a range of the
 // contraction.  Every lane streams the packed codes of its two rows with
 // 16-byte loads (32 codes = 32 consecutive k per row), expands them with the
-// dequantizer's own arithmetic (nf4::expand8, bit-identical bf16) straight
-// into the A fragments of mma.sync m16n8k16, and multiplies them with X.  The
+// dequantizer's arithmetic (w = bf16(RN32(q[code] * c1')), bit-identical)
+// straight into the A fragments of mma.sync m16n8k16, and multiplies them with
+// X.  One byte of packed codes is one A register (two neighbouring k), so the
+// expansion looks up both codebook values of a byte at once in a 256-entry
+// pair table in shared memory.  The block constants c1' of a warp's 16 rows
+// are decoded once per 12 steps into shared memory.  The
 // contraction index is permuted the same way on both operands (a fragment's
 // k slots map to the lane's 32 consecutive k), so no shared-memory transpose
 // is needed; the tensor cores only replace the 2 M FMAs per weight that CUDA
@@ -70,6 +74,39 @@ constexpr int kAPieces = 8;
 // accumulators and X fragments take the registers)
 template <int NT>
 constexpr int prefetch_depth() { return NT == 1 ? 4 : 3; }
+// 128-wide steps whose block constants a warp decodes at once (a multiple of
+// both prefetch depths): 24 blocks of each of its 16 rows.
+constexpr int kScaleSteps = 12;
+constexpr int kScaleBlocks = 2 * kScaleSteps;
+constexpr int kScaleStride = kScaleBlocks + 1;   // odd row stride: a warp's reads hit distinct banks
+
+// Pair table: entry e (one byte of packed codes, the lower k in its low
+// nibble) holds (q[e & 15], q[e >> 4]).  Each entry is a 256-byte row of 32
+// copies, one 8-byte slot per lane, so the 32 lookups of a warp never share a
+// bank whatever their entries.  Then the block constants: per warp 16 rows x
+// kScaleStride floats.
+constexpr uint32_t kPairTableBytes = 256 * 32 * 8;   // 64 KB
+constexpr uint32_t kDecSmem = kPairTableBytes + kDecWarps * 16 * kScaleStride * 4;
+
+// Two dequantized weights (one byte of codes, the lower k in the low half):
+// the shared-memory offset [lane slot, entry] is one byte permute of the code
+// word and lane8 (= 8 * lane).  Same products and rounding as nf4::expand8.
+template <bool F16, int kByte>
+__device__ __forceinline__ uint32_t expand_pair(uint32_t word, uint32_t lane8, const char *tab, float c1p)
+{
+    const uint32_t off = __byte_perm(word, lane8, 0x5504u | (kByte << 4));   // lane8 + 256 * byte
+    const float2 qv = *reinterpret_cast<const float2 *>(tab + off);
+    float lo, hi;
+    nf4::mul2(qv.x, qv.y, c1p, lo, hi);
+    return nf4::pack16x2<F16>(lo, hi);
+}
+
+template <bool F16>
+__device__ __forceinline__ uint4 expand8_pairs(uint32_t word, uint32_t lane8, const char *tab, float c1p)
+{
+    return make_uint4(expand_pair<F16, 0>(word, lane8, tab, c1p), expand_pair<F16, 1>(word, lane8, tab, c1p),
+                      expand_pair<F16, 2>(word, lane8, tab, c1p), expand_pair<F16, 3>(word, lane8, tab, c1p));
+}
 
 __device__ __forceinline__ uint4 ld_stream_v4(const void *p)
 {
@@ -104,13 +141,11 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
             : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// One 128-wide step of this lane's two rows: packed codes and block constants.
-// Loads only: nothing computed from a loaded value until the step is used,
-// so issuing the next step's loads never waits for them.
+// One 128-wide step of this lane's two rows: packed codes.  Loads only:
+// nothing computed from a loaded value until the step is used, so issuing the
+// next step's loads never waits for them.
 struct WStage {
     uint4 pg, pg8;
-    uint32_t eg, eg8;   // E4M3 block codes of rows g and g+8
-    float c2g, c2g8;
 };
 
 // Fragment layout (lane = 4 g + c): A regs {a0a1, a2a3, a4a5, a6a7} hold rows
@@ -133,7 +168,7 @@ __device__ __forceinline__ void mma_step(float (&acc)[NT][2][4], const uint4 (&e
             const uint4 xb = (xok[t] && kin && QLORA_IN((xrow[t] - xbase) + k + 8 * w + 7, xlen))
                                  ? ld_cached_v4(xrow[t] + k + 8 * w) : make_uint4(0, 0, 0, 0);
             mma_bf16_16816<F16>(acc[t][0], ea[w].x, eb[w].x, ea[w].y, eb[w].y, xb.x, xb.y);
-            mma_bf16_16816<F16>(acc[t][0], ea[w].z, eb[w].z, ea[w].w, eb[w].w, xb.z, xb.w);
+            mma_bf16_16816<F16>(acc[t][1], ea[w].z, eb[w].z, ea[w].w, eb[w].w, xb.z, xb.w);
         }
     }
 }
@@ -142,11 +177,23 @@ __device__ __forceinline__ void mma_step(float (&acc)[NT][2][4], const uint4 (&e
 template <int NT, bool F16>
 __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm) decode_gemv_kernel(const __grid_constant__ DecodeParams p)
 {
-    __shared__ float lut[16];
+    extern __shared__ __align__(16) char dec_smem[];
+    __shared__ float s_q[16];
+    const bool w_rows = (int)blockIdx.x < p.row_tiles;
+    if (w_rows) {
+        // the pair table depends on the parameters only: built before the
+        // dependency wait, overlapping the previous kernel's tail
+        if (threadIdx.x < 16) s_q[threadIdx.x] = p.q[threadIdx.x];
+        __syncthreads();
+        float2 *tab = reinterpret_cast<float2 *>(dec_smem);
+        for (int i = threadIdx.x; i < 256 * 32; i += kDecThreads) {
+            const int e = i >> 5;   // a warp writes one entry's 32 slots
+            tab[i] = make_float2(s_q[e & 15], s_q[e >> 4]);
+        }
+        __syncthreads();
+    }
     sm100::pdl_wait();
     sm100::pdl_trigger();
-    if (threadIdx.x < 16) lut[threadIdx.x] = p.q[threadIdx.x];
-    __syncthreads();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, c = lane & 3;
@@ -168,7 +215,7 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm) decode_gemv_kernel
         xrow[t] = p.X + (int64_t)(xok[t] ? tok : 0) * p.K;
     }
 
-    if ((int)blockIdx.x >= p.row_tiles) {
+    if (!w_rows) {
         // ---- rows of A: warp task = (16-row group, piece of the contraction)
         if (sp != 0) return;
 #pragma unroll
@@ -211,51 +258,69 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm) decode_gemv_kernel
 
     // ---- rows of W: packed codes streamed kPrefetch steps ahead
     constexpr int kPrefetch = prefetch_depth<NT>();
+    static_assert(kScaleSteps % kPrefetch == 0, "block constants are refilled at a prefetch boundary");
     const int64_t row0 = (int64_t)blockIdx.x * kDecRows + 16 * warp;
     if (row0 >= p.N) return;
     const int64_t rg = row0 + g, rg8 = row0 + g + 8;
     const bool ok_g = rg < p.N, ok_g8 = rg8 < p.N;
     const float mu = *p.mean;
     const int64_t half_k = p.K / 2;
+    const char *tab = dec_smem;
+    const uint32_t lane8 = 8u * (uint32_t)lane;
+    float *sc = reinterpret_cast<float *>(dec_smem + kPairTableBytes) + warp * 16 * kScaleStride;
     auto load = [&](int d, WStage &st) {
         const int64_t k = (int64_t)d * 128 + 32 * c;
         const bool in = d < d1 && k < p.K;
         const uint4 z = make_uint4(0, 0, 0, 0);
-        [[maybe_unused]] const int64_t nblk = p.N * p.kblocks;
         // (checked only where the access happens)
-        const bool ld_g = in && ok_g && QLORA_IN(rg * half_k + k / 2 + 15, p.N * half_k) &&
-                          QLORA_IN(rg * p.kblocks + k / 64, nblk) && QLORA_IN((rg * p.kblocks + k / 64) >> 8, (nblk + 255) / 256);
-        const bool ld_g8 = in && ok_g8 && QLORA_IN(rg8 * half_k + k / 2 + 15, p.N * half_k) &&
-                           QLORA_IN(rg8 * p.kblocks + k / 64, nblk) && QLORA_IN((rg8 * p.kblocks + k / 64) >> 8, (nblk + 255) / 256);
+        const bool ld_g = in && ok_g && QLORA_IN(rg * half_k + k / 2 + 15, p.N * half_k);
+        const bool ld_g8 = in && ok_g8 && QLORA_IN(rg8 * half_k + k / 2 + 15, p.N * half_k);
         st.pg = ld_g ? ld_stream_v4(p.packed + rg * half_k + k / 2) : z;
         st.pg8 = ld_g8 ? ld_stream_v4(p.packed + rg8 * half_k + k / 2) : z;
-        const int64_t b = rg * p.kblocks + k / 64, b8 = rg8 * p.kblocks + k / 64;
-        st.eg = ld_g ? (uint32_t)__ldg(p.code2 + b) : 0u;
-        st.c2g = ld_g ? __ldg(p.c2 + (b >> 8)) : 0.0f;
-        st.eg8 = ld_g8 ? (uint32_t)__ldg(p.code2 + b8) : 0u;
-        st.c2g8 = ld_g8 ? __ldg(p.c2 + (b8 >> 8)) : 0.0f;
+    };
+    // c1' of the warp's 16 rows for the blocks of steps d .. d+kScaleSteps-1,
+    // one row at a time: lane j < 24 takes block 2d + j, so each load
+    // instruction reads one contiguous run of a row's block codes (and mostly
+    // one group scale); blocks past the row's end (the upper half of a final
+    // 64-wide step) get 0
+    auto fill_scales = [&](int d) {
+        const int64_t blk = 2 * (int64_t)d + lane;
+        [[maybe_unused]] const int64_t nblk = p.N * p.kblocks;
+        __syncwarp();   // every lane has read the previous range
+        if (lane < kScaleBlocks) {
+#pragma unroll
+            for (int r = 0; r < 16; r++) {
+                const int64_t row = row0 + r;
+                const int64_t b = row * p.kblocks + blk;
+                const bool ok = row < p.N && blk < p.kblocks && QLORA_IN(b, nblk) && QLORA_IN(b >> 8, (nblk + 255) / 256);
+                sc[r * kScaleStride + lane] = ok ? nf4::block_scale(__ldg(p.code2 + b), __ldg(p.c2 + (b >> 8)), mu) : 0.0f;
+            }
+        }
+        __syncwarp();
     };
     WStage st[kPrefetch];
 #pragma unroll
     for (int i = 0; i < kPrefetch; i++) load(d0 + i, st[i]);
     for (int d = d0; d < d1; d += kPrefetch) {
+        if ((d - d0) % kScaleSteps == 0) fill_scales(d);
+        const float *sc_d = sc + 2 * ((d - d0) % kScaleSteps) + (c >> 1);
 #pragma unroll
         for (int i = 0; i < kPrefetch; i++) {
             if (d + i < d1) {
                 const int64_t k = (int64_t)(d + i) * 128 + 32 * c;
                 const bool kin = k < p.K;   // false only for the upper half of a final 64-wide step
                 {
-                    const float sg = (ok_g && kin) ? nf4::block_scale((uint8_t)st[i].eg, st[i].c2g, mu) : 0.0f;
-                    const float sg8 = (ok_g8 && kin) ? nf4::block_scale((uint8_t)st[i].eg8, st[i].c2g8, mu) : 0.0f;
+                    const float sg = sc_d[g * kScaleStride + 2 * i];
+                    const float sg8 = sc_d[(g + 8) * kScaleStride + 2 * i];
                     uint4 ea[4], eb[4];
-                    ea[0] = nf4::expand8<F16>(st[i].pg.x, lut, sg);
-                    ea[1] = nf4::expand8<F16>(st[i].pg.y, lut, sg);
-                    ea[2] = nf4::expand8<F16>(st[i].pg.z, lut, sg);
-                    ea[3] = nf4::expand8<F16>(st[i].pg.w, lut, sg);
-                    eb[0] = nf4::expand8<F16>(st[i].pg8.x, lut, sg8);
-                    eb[1] = nf4::expand8<F16>(st[i].pg8.y, lut, sg8);
-                    eb[2] = nf4::expand8<F16>(st[i].pg8.z, lut, sg8);
-                    eb[3] = nf4::expand8<F16>(st[i].pg8.w, lut, sg8);
+                    ea[0] = expand8_pairs<F16>(st[i].pg.x, lane8, tab, sg);
+                    ea[1] = expand8_pairs<F16>(st[i].pg.y, lane8, tab, sg);
+                    ea[2] = expand8_pairs<F16>(st[i].pg.z, lane8, tab, sg);
+                    ea[3] = expand8_pairs<F16>(st[i].pg.w, lane8, tab, sg);
+                    eb[0] = expand8_pairs<F16>(st[i].pg8.x, lane8, tab, sg8);
+                    eb[1] = expand8_pairs<F16>(st[i].pg8.y, lane8, tab, sg8);
+                    eb[2] = expand8_pairs<F16>(st[i].pg8.z, lane8, tab, sg8);
+                    eb[3] = expand8_pairs<F16>(st[i].pg8.w, lane8, tab, sg8);
                     mma_step<NT, F16>(acc, ea, eb, xrow, xok, k, kin, p.X, (int64_t)p.M * p.K);
                 }
                 load(d + i + kPrefetch, st[i]);
@@ -376,9 +441,9 @@ DecodePlan decode_plan(int64_t M, int64_t N, int64_t K, int r, int sms)
     d.row_tiles = ceil_div_i(N, kDecRows);
     d.a_ctas = ceil_div_i((int64_t)((r + 15) / 16) * kAPieces, kDecWarps);
     d.n_dblk = ceil_div_i(K, 128);
-    // about three CTAs per SM in all (1.5 waves at two resident per SM: measured
-    // faster than a single wave), at least two 128-wide steps per split
-    int want = ceil_div_i((int64_t)3 * sms, d.row_tiles + d.a_ctas);
+    // about four CTAs per SM in all (two waves at two resident per SM: measured
+    // faster than one or one and a half), at least two 128-wide steps per split
+    int want = ceil_div_i((int64_t)4 * sms, d.row_tiles + d.a_ctas);
     want = std::max(1, std::min(want, std::max(1, d.n_dblk / 2)));
     d.per = ceil_div_i(d.n_dblk, want);
     d.splits = ceil_div_i(d.n_dblk, d.per);
@@ -422,14 +487,22 @@ qlora_status run_decode_fwd(const qlora_nf4_weight *w, const void *X, const void
     p.part = static_cast<float *>(ws);
     p.part_h = reinterpret_cast<float *>(static_cast<char *>(ws) + d.part_bytes);
     const dim3 grid(d.row_tiles + d.a_ctas, d.splits);
+    static PerDeviceOnce attr;
+    QLORA_TRY(attr.run(dev.device, []() -> qlora_status {
+        QLORA_CUDA_TRY(cudaFuncSetAttribute(decode_gemv_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem));
+        QLORA_CUDA_TRY(cudaFuncSetAttribute(decode_gemv_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem));
+        QLORA_CUDA_TRY(cudaFuncSetAttribute(decode_gemv_kernel<2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem));
+        QLORA_CUDA_TRY(cudaFuncSetAttribute(decode_gemv_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem));
+        return QLORA_OK;
+    }));
     {
         LaunchScope ls(QLORA_KERNEL_FWD_FUSED, s);
         if (M <= 8)
             QLORA_CUDA_TRY(launch_pdl(f16 ? decode_gemv_kernel<1, true> : decode_gemv_kernel<1, false>, grid,
-                                      dim3(kDecThreads), 0, s, p));
+                                      dim3(kDecThreads), kDecSmem, s, p));
         else
             QLORA_CUDA_TRY(launch_pdl(f16 ? decode_gemv_kernel<2, true> : decode_gemv_kernel<2, false>, grid,
-                                      dim3(kDecThreads), 0, s, p));
+                                      dim3(kDecThreads), kDecSmem, s, p));
     }
     {
         LaunchScope ls(QLORA_KERNEL_ELEMENTWISE, s);
