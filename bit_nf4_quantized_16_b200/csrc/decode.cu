@@ -86,7 +86,22 @@ constexpr int kScaleStride = kScaleBlocks + 1;   // odd row stride: a warp's rea
 // bank whatever their entries.  Then the block constants: per warp 16 rows x
 // kScaleStride floats.
 constexpr uint32_t kPairTableBytes = 256 * 32 * 8;   // 64 KB
-constexpr uint32_t kDecSmem = kPairTableBytes + kDecWarps * 16 * kScaleStride * 4;
+constexpr uint32_t kScaleBytes = kDecWarps * 16 * kScaleStride * 4;
+// X of the CTA's current kPrefetch steps, double-buffered: (8 NT) token rows
+// of 128 kPrefetch bf16 (24 KB for two token tiles)
+template <int NT>
+constexpr uint32_t x_stage_bytes() { return 2u * (8 * NT) * (128 * prefetch_depth<NT>()) * 2; }
+template <int NT>
+constexpr uint32_t dec_smem_bytes() { return kPairTableBytes + kScaleBytes + (NT == 2 ? x_stage_bytes<2>() : 0u); }
+
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem)),
+                 "l"(gmem)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 // Two dequantized weights (one byte of codes, the lower k in the low half):
 // the shared-memory offset [lane slot, entry] is one byte permute of the code
@@ -167,6 +182,28 @@ __device__ __forceinline__ void mma_step(float (&acc)[NT][2][4], const uint4 (&e
         for (int t = 0; t < NT; t++) {
             const uint4 xb = (xok[t] && kin && QLORA_IN((xrow[t] - xbase) + k + 8 * w + 7, xlen))
                                  ? ld_cached_v4(xrow[t] + k + 8 * w) : make_uint4(0, 0, 0, 0);
+            mma_bf16_16816<F16>(acc[t][0], ea[w].x, eb[w].x, ea[w].y, eb[w].y, xb.x, xb.y);
+            mma_bf16_16816<F16>(acc[t][1], ea[w].z, eb[w].z, ea[w].w, eb[w].w, xb.z, xb.w);
+        }
+    }
+}
+
+// mma_step with X from the staged chunk: xs_row[t] is token 8t+g's row of the
+// chunk; 16-byte unit u of a row sits at u ^ (bit 3 of u) ^ (2 * (token & 1)),
+// so the 8 lanes of each quarter-warp (two tokens, four k slices 64 bytes
+// apart) read 8 distinct bank groups.  jb = 16 * (step in chunk) + 4 c, sw the
+// lane's swizzle bits.
+template <int NT, bool F16>
+__device__ __forceinline__ void mma_step_xs(float (&acc)[NT][2][4], const uint4 (&ea)[4], const uint4 (&eb)[4],
+                                            const char *const (&xs_row)[NT], const bool (&xok)[NT], int jb, int sw,
+                                            bool kin)
+{
+#pragma unroll
+    for (int w = 0; w < 4; w++) {
+#pragma unroll
+        for (int t = 0; t < NT; t++) {
+            const uint4 xb = (xok[t] && kin) ? *reinterpret_cast<const uint4 *>(xs_row[t] + ((jb + (w ^ sw)) << 4))
+                                             : make_uint4(0, 0, 0, 0);
             mma_bf16_16816<F16>(acc[t][0], ea[w].x, eb[w].x, ea[w].y, eb[w].y, xb.x, xb.y);
             mma_bf16_16816<F16>(acc[t][1], ea[w].z, eb[w].z, ea[w].w, eb[w].w, xb.z, xb.w);
         }
@@ -259,8 +296,14 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm) decode_gemv_kernel
     // ---- rows of W: packed codes streamed kPrefetch steps ahead
     constexpr int kPrefetch = prefetch_depth<NT>();
     static_assert(kScaleSteps % kPrefetch == 0, "block constants are refilled at a prefetch boundary");
+    // X staged in shared memory once per CTA (two token tiles: measured faster
+    // than every warp loading it through L1) or loaded by each warp (one tile)
+    constexpr bool kStageX = NT == 2;
     const int64_t row0 = (int64_t)blockIdx.x * kDecRows + 16 * warp;
-    if (row0 >= p.N) return;
+    // with staged X a warp past the last row still takes part in the CTA's
+    // chunk barriers
+    const bool wrow = row0 < p.N;
+    if (!kStageX && !wrow) return;
     const int64_t rg = row0 + g, rg8 = row0 + g + 8;
     const bool ok_g = rg < p.N, ok_g8 = rg8 < p.N;
     const float mu = *p.mean;
@@ -298,10 +341,38 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm) decode_gemv_kernel
         }
         __syncwarp();
     };
+    // X of steps d .. d+kPrefetch-1 into buffer buf, by all threads of the CTA
+    constexpr int kXUnits = 16 * kPrefetch;               // 16-byte units per token row
+    constexpr uint32_t kXRowBytes = 16 * kXUnits;
+    constexpr uint32_t kXBufBytes = 8 * NT * kXRowBytes;
+    char *xs = dec_smem + kPairTableBytes + kScaleBytes;
+    auto stage_x = [&](int d, int buf) {
+        char *dst = xs + buf * kXBufBytes;
+        const int64_t kb = (int64_t)d * 128;
+        const int64_t kend = min((int64_t)d1 * 128, p.K);
+        for (int idx = threadIdx.x; idx < 8 * NT * kXUnits; idx += kDecThreads) {
+            const int row = idx / kXUnits, u = idx % kXUnits;
+            const int64_t k = kb + 8 * u;
+            if (row < p.M && k < kend && QLORA_IN(row * p.K + k + 7, (int64_t)p.M * p.K))
+                cp_async16(dst + row * kXRowBytes + ((u ^ ((u >> 3) & 1) ^ ((row & 1) << 1)) << 4), p.X + row * p.K + k);
+        }
+        cp_async_commit();
+    };
+    const int sw = (c >> 1) ^ ((g & 1) << 1);
     WStage st[kPrefetch];
 #pragma unroll
     for (int i = 0; i < kPrefetch; i++) load(d0 + i, st[i]);
-    for (int d = d0; d < d1; d += kPrefetch) {
+    if constexpr (kStageX) stage_x(d0, 0);
+    for (int d = d0, ci = 0; d < d1; d += kPrefetch, ci++) {
+        if constexpr (kStageX) {
+            cp_async_wait_all();
+            __syncthreads();   // this chunk's X is visible; every warp is done with the previous chunk
+            if (d + kPrefetch < d1) stage_x(d + kPrefetch, (ci + 1) & 1);
+            if (!wrow) continue;
+        }
+        const char *xs_row[NT];
+#pragma unroll
+        for (int t = 0; t < NT; t++) xs_row[t] = xs + (ci & 1) * kXBufBytes + (8 * t + g) * kXRowBytes;
         if ((d - d0) % kScaleSteps == 0) fill_scales(d);
         const float *sc_d = sc + 2 * ((d - d0) % kScaleSteps) + (c >> 1);
 #pragma unroll
@@ -321,7 +392,10 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm) decode_gemv_kernel
                     eb[1] = expand8_pairs<F16>(st[i].pg8.y, lane8, tab, sg8);
                     eb[2] = expand8_pairs<F16>(st[i].pg8.z, lane8, tab, sg8);
                     eb[3] = expand8_pairs<F16>(st[i].pg8.w, lane8, tab, sg8);
-                    mma_step<NT, F16>(acc, ea, eb, xrow, xok, k, kin, p.X, (int64_t)p.M * p.K);
+                    if constexpr (kStageX)
+                        mma_step_xs<NT, F16>(acc, ea, eb, xs_row, xok, 16 * i + 4 * c, sw, kin);
+                    else
+                        mma_step<NT, F16>(acc, ea, eb, xrow, xok, k, kin, p.X, (int64_t)p.M * p.K);
                 }
                 load(d + i + kPrefetch, st[i]);
             }
@@ -489,20 +563,24 @@ qlora_status run_decode_fwd(const qlora_nf4_weight *w, const void *X, const void
     const dim3 grid(d.row_tiles + d.a_ctas, d.splits);
     static PerDeviceOnce attr;
     QLORA_TRY(attr.run(dev.device, []() -> qlora_status {
-        QLORA_CUDA_TRY(cudaFuncSetAttribute(decode_gemv_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem));
-        QLORA_CUDA_TRY(cudaFuncSetAttribute(decode_gemv_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem));
-        QLORA_CUDA_TRY(cudaFuncSetAttribute(decode_gemv_kernel<2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem));
-        QLORA_CUDA_TRY(cudaFuncSetAttribute(decode_gemv_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem));
+        QLORA_CUDA_TRY(cudaFuncSetAttribute(decode_gemv_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            dec_smem_bytes<1>()));
+        QLORA_CUDA_TRY(cudaFuncSetAttribute(decode_gemv_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            dec_smem_bytes<1>()));
+        QLORA_CUDA_TRY(cudaFuncSetAttribute(decode_gemv_kernel<2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            dec_smem_bytes<2>()));
+        QLORA_CUDA_TRY(cudaFuncSetAttribute(decode_gemv_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            dec_smem_bytes<2>()));
         return QLORA_OK;
     }));
     {
         LaunchScope ls(QLORA_KERNEL_FWD_FUSED, s);
         if (M <= 8)
             QLORA_CUDA_TRY(launch_pdl(f16 ? decode_gemv_kernel<1, true> : decode_gemv_kernel<1, false>, grid,
-                                      dim3(kDecThreads), kDecSmem, s, p));
+                                      dim3(kDecThreads), dec_smem_bytes<1>(), s, p));
         else
             QLORA_CUDA_TRY(launch_pdl(f16 ? decode_gemv_kernel<2, true> : decode_gemv_kernel<2, false>, grid,
-                                      dim3(kDecThreads), kDecSmem, s, p));
+                                      dim3(kDecThreads), dec_smem_bytes<2>(), s, p));
     }
     {
         LaunchScope ls(QLORA_KERNEL_ELEMENTWISE, s);
