@@ -51,13 +51,13 @@ _CSRC = os.path.join("bit_nf4_quantized_16_b200", "csrc")
 MEASURED_TRAFFIC = {
     "linear": {
         "sources": ['gemm_pair.cuh', 'gemm.cuh', 'sm100.cuh', 'nf4_expand.cuh', 'linear.cu'],
-        "sha256": "1ccbc42721627aefd77b9259ee66f420d0666f4766604e66f399f42f88f59587",
-        "bytes": {"fwd_fused": 97.24e6, "bwd_fused": 110.51e6},
+        "sha256": "91e995f9aadab535a367885e1c0c562d3d12f730b08e80da02a71502fcaeb880",
+        "bytes": {"fwd_fused": 99.60e6, "bwd_fused": 112.17e6},
     },
     "codec": {
         "sources": ['codec.cu', 'nf4_expand.cuh', 'exact_mean.cuh'],
-        "sha256": "933d060941c097dd3bf7b0596d4d03881978f300097f0ecddebe2db101e420cb",
-        "bytes": {"quantize": 58.71e6, "dequantize": 27.13e6},
+        "sha256": "9a7b14c79aad62eb21d1fa0581aa376d3ad0e7f64654f9402d7a4711c77a9406",
+        "bytes": {"quantize": 58.64e6, "dequantize": 27.07e6},
     },
 }
 
