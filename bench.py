@@ -191,14 +191,70 @@ def run_ours(args, rank, world, local_rank):
 
     reducer = dp.OverlappedGradSum()
 
+    # The seven linears are independent, so each linear's small adapter
+    # products (H in the forward, G in the backward) run on a low-priority
+    # side stream through the split-off adapter calls, beside the previous
+    # linear's fused GEMM: they become runnable when that GEMM does (an event
+    # recorded just before it), the GEMM's CTAs take the SMs first, and the
+    # adapter kernels fill the SMs its partial last round of tiles leaves
+    # idle.  Each linear then has its own workspace.
+    mode = {"split": not args.no_adapter_split}
+    gemm_s = torch.cuda.Stream(priority=-1)
+    side_s = torch.cuda.Stream(priority=0)
+    for L in layers:
+        L["ws"] = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if mode["split"] else ws
+        L["ev"] = [torch.cuda.Event() for _ in range(4)]   # fwd adapter done, fwd GEMM next, same for bwd
+
     def step():
-        for L in layers:
-            q.qlora_linear_fwd(L["w"], L["X"], TOKENS, L["A"], L["B"], R, scale, L["Y"], L["H"], ws)
-        for L in reversed(layers):
-            q.qlora_linear_bwd(L["w"], L["X"], L["dY"], TOKENS, L["A"], L["B"], R, scale, L["H"], L["dX"],
-                               L["dA"], L["dB"], ws)
-            reducer.ready(L["grad"])   # this linear's dA, dB: summed while the backward goes on
-        reducer.wait()
+        if not mode["split"]:
+            for L in layers:
+                q.qlora_linear_fwd(L["w"], L["X"], TOKENS, L["A"], L["B"], R, scale, L["Y"], L["H"], ws)
+            for L in reversed(layers):
+                q.qlora_linear_bwd(L["w"], L["X"], L["dY"], TOKENS, L["A"], L["B"], R, scale, L["H"], L["dX"],
+                                   L["dA"], L["dB"], ws)
+                reducer.ready(L["grad"])   # this linear's dA, dB: summed while the backward goes on
+            reducer.wait()
+            return
+        cur = torch.cuda.current_stream()
+        gemm_s.wait_stream(cur)
+        side_s.wait_stream(cur)
+        for phase, order in (("fwd", layers), ("bwd", list(reversed(layers)))):
+            done, go = (0, 1) if phase == "fwd" else (2, 3)
+
+            def adapter(L):
+                with torch.cuda.stream(side_s):
+                    if phase == "fwd":
+                        q.qlora_linear_adapter_fwd(L["w"], L["X"], TOKENS, L["A"], L["B"], R, scale, L["H"],
+                                                   L["ws"], stream=side_s)
+                    else:
+                        q.qlora_linear_adapter_bwd(L["w"], L["X"], L["dY"], TOKENS, L["A"], L["B"], R, scale,
+                                                   L["H"], L["ws"], stream=side_s)
+                    L["ev"][done].record(side_s)
+
+            # host order matters: every event is recorded before a stream waits on it
+            adapter(order[0])
+            for i, L in enumerate(order):
+                with torch.cuda.stream(gemm_s):
+                    gemm_s.wait_event(L["ev"][done])
+                    L["ev"][go].record(gemm_s)
+                    if phase == "fwd":
+                        q.qlora_linear_fwd(L["w"], L["X"], TOKENS, L["A"], L["B"], R, scale, L["Y"], L["H"],
+                                           L["ws"], stream=gemm_s, adapter_ready=True)
+                    else:
+                        q.qlora_linear_bwd(L["w"], L["X"], L["dY"], TOKENS, L["A"], L["B"], R, scale, L["H"],
+                                           L["dX"], L["dA"], L["dB"], L["ws"], stream=gemm_s, adapter_ready=True)
+                        reducer.ready(L["grad"])   # this linear's dA, dB: summed while the backward goes on
+                if i + 1 < len(order):
+                    # the next linear's adapter products become runnable with this GEMM
+                    side_s.wait_event(L["ev"][go])
+                    adapter(order[i + 1])
+            if phase == "fwd":
+                # the backward's adapter call rewrites the workspace the forward GEMM read
+                side_s.wait_stream(gemm_s)
+        with torch.cuda.stream(gemm_s):
+            reducer.wait()
+        cur.wait_stream(gemm_s)
+        cur.wait_stream(side_s)
 
     def timed_steps(k, fn):
         """Device time of k steps, each after an L2 flush, CUDA events on the
@@ -232,11 +288,15 @@ def run_ours(args, rank, world, local_rank):
     launches = q.qlora_launch_count() - launches0
     q.qlora_check_device_error()
     # ---- per-kernel device times: the same steps again with CUDA events around
-    # every launch (on the launching stream)
+    # every launch (on the launching stream), undivided calls on one stream so
+    # that each launch's time is its own and not shared with a concurrent one
+    split_headline = mode["split"]
+    mode["split"] = False
     q.qlora_timing_reset()
     q.qlora_timing_enable(True)
     ms_events = timed_steps(args.steps, step)
     q.qlora_timing_enable(False)
+    mode["split"] = split_headline
     kern = q.qlora_timing_read()
     q.qlora_check_device_error()
     clocks = clk.summary()
@@ -298,7 +358,9 @@ def run_ours(args, rank, world, local_rank):
     roofline = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
                 "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": measured_traffic("linear", dom),
                 "peak_source": f"{peak_src} bf16_tflops (burst)",
-                "launches": dom_n, "avg_launch_ms": round(dom_ms / max(dom_n, 1), 4)}
+                "launches": dom_n, "avg_launch_ms": round(dom_ms / max(dom_n, 1), 4),
+                "timing": "CUDA events around every launch on its stream, in a second pass of the same steps "
+                          "with undivided linear calls on one stream (no concurrent kernel)"}
     breakdown = {k: {"ms_per_step": round(v[0] / args.steps, 4), "launches_per_step": v[1] // args.steps}
                  for k, v in kern.items() if v[1]}
 
@@ -322,7 +384,9 @@ def run_ours(args, rank, world, local_rank):
                                 "r=64, alpha=16, bf16 activations") if args.linears == "llama7b" else
                                f"single QLoRA linear {args.linears} fwd+bwd, {TOKENS} tokens, r=64, alpha=16",
                    "tokens_per_gpu": TOKENS, "rank": R, "alpha": ALPHA, "l2": "flushed (256 MB write) before each step",
-                   "parallelism": f"dp{world}", "flop_per_step_per_gpu": step_flops},
+                   "parallelism": f"dp{world}", "flop_per_step_per_gpu": step_flops,
+                   "adapter_products": ("split off to a low-priority side stream, beside the previous linear's "
+                                        "fused GEMM" if split_headline else "inside each linear call, one stream")},
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
@@ -1176,6 +1240,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--skip-codec", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--no-adapter-split", action="store_true",
+                    help="linear7b step: undivided linear calls on one stream (no side stream for H and G)")
     ap.add_argument("--skip-decode", action="store_true")
     ap.add_argument("--skip-stack", action="store_true")
     ap.add_argument("--skip-optim", action="store_true")

@@ -43,6 +43,7 @@ EXPORTS = (
     "qlora_paged_alloc", "qlora_paged_free", "qlora_paged_prefetch", "qlora_adamw_step",
     "qlora_block_workspace_bytes", "qlora_block_fwd", "qlora_block_bwd",
     "qlora_linear_workspace_bytes_ex", "qlora_linear_fwd_ex", "qlora_linear_bwd_ex",
+    "qlora_linear_adapter_fwd", "qlora_linear_adapter_bwd",
     "qlora_dequantize_nf4_dq_ex",
 )
 
@@ -71,7 +72,8 @@ class qlora_nf4_weight(ctypes.Structure):
 
 
 class qlora_linear_opts(ctypes.Structure):
-    _fields_ = [("dropout_mask", ctypes.c_void_p), ("dropout_p", ctypes.c_float), ("compute_dtype", ctypes.c_int)]
+    _fields_ = [("dropout_mask", ctypes.c_void_p), ("dropout_p", ctypes.c_float), ("compute_dtype", ctypes.c_int),
+                ("adapter_ready", ctypes.c_int32)]
 
 
 class qlora_block(ctypes.Structure):
@@ -121,6 +123,10 @@ def _load():
                                                ctypes.POINTER(qlora_linear_opts)]),
         "qlora_linear_bwd_ex": (ctypes.c_int, [W, P, P, I64, P, P, I32, F, P, P, ctypes.c_int, P, P, P, S, P,
                                                ctypes.POINTER(qlora_linear_opts)]),
+        "qlora_linear_adapter_fwd": (ctypes.c_int, [W, P, I64, P, P, I32, F, P, P, S, P,
+                                                    ctypes.POINTER(qlora_linear_opts)]),
+        "qlora_linear_adapter_bwd": (ctypes.c_int, [W, P, P, I64, P, P, I32, F, P, P, S, P,
+                                                    ctypes.POINTER(qlora_linear_opts)]),
         "qlora_block_fwd": (ctypes.c_int, [ctypes.POINTER(qlora_block), P, P, P, S, P]),
         "qlora_block_bwd": (ctypes.c_int, [ctypes.POINTER(qlora_block), P, P, P, P, P, P, S, P]),
     }
@@ -237,31 +243,33 @@ def qlora_dequantize_nf4_dq(w: NF4Weight, out: torch.Tensor, stream=None):
                "qlora_dequantize_nf4_dq")
 
 
-def _opts(dropout, X):
+def _opts(dropout, X, adapter_ready=False, always=False):
     """Options for the _ex calls, or None for the plain ones.  dropout: None, or
     (mask, p) with mask a uint8 device tensor of M*K/8 bytes (bit k % 8 of byte
     (m*K + k) / 8: element (m, k) kept); the compute dtype follows X (fp16
-    tensors select the fp16 compute dtype)."""
+    tensors select the fp16 compute dtype); adapter_ready: the adapter's
+    products were written into the workspace by the matching adapter call."""
     f16 = X is not None and X.dtype == torch.float16
-    if dropout is None and not f16:
+    if dropout is None and not f16 and not adapter_ready and not always:
         return None
     mask, p = dropout if dropout is not None else (None, 0.0)
-    return qlora_linear_opts(None if mask is None else mask.data_ptr(), p, QLORA_FP16 if f16 else QLORA_BF16)
+    return qlora_linear_opts(None if mask is None else mask.data_ptr(), p, QLORA_FP16 if f16 else QLORA_BF16,
+                             1 if adapter_ready else 0)
 
 
 def qlora_linear_workspace_bytes(M: int, N: int, K: int, r: int, dropout=None) -> int:
     if dropout is None:
         return lib.qlora_linear_workspace_bytes(M, N, K, r)
-    o = qlora_linear_opts(1, 0.0, QLORA_BF16)   # only the presence of a mask matters for the size
+    o = qlora_linear_opts(1, 0.0, QLORA_BF16, 0)   # only the presence of a mask matters for the size
     return lib.qlora_linear_workspace_bytes_ex(M, N, K, r, ctypes.byref(o))
 
 
 def qlora_linear_fwd(w: NF4Weight, X, M: int, A, B, r: int, scale: float, Y, H_save=None,
-                     workspace=None, stream=None, dropout=None):
+                     workspace=None, stream=None, dropout=None, adapter_ready=False):
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     args = (ctypes.byref(w.desc), _ptr(X), M, _ptr(A), _ptr(B), r, scale, _ptr(Y), _dtype_code(Y), _ptr(H_save),
             _ptr(workspace), ws_bytes, _stream(stream))
-    opts = _opts(dropout, X)
+    opts = _opts(dropout, X, adapter_ready)
     if opts is None:
         _check(lib.qlora_linear_fwd(*args), "qlora_linear_fwd")
     else:
@@ -269,17 +277,40 @@ def qlora_linear_fwd(w: NF4Weight, X, M: int, A, B, r: int, scale: float, Y, H_s
 
 
 def qlora_linear_bwd(w: NF4Weight, X, dY, M: int, A, B, r: int, scale: float, H_saved, dX, dA, dB,
-                     workspace=None, stream=None, dropout=None):
+                     workspace=None, stream=None, dropout=None, adapter_ready=False):
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     dx_code = (QLORA_FP16 if X is not None and X.dtype == torch.float16 else QLORA_BF16) if dX is None \
         else _dtype_code(dX)
     args = (ctypes.byref(w.desc), _ptr(X), _ptr(dY), M, _ptr(A), _ptr(B), r, scale, _ptr(H_saved), _ptr(dX),
             dx_code, _ptr(dA), _ptr(dB), _ptr(workspace), ws_bytes, _stream(stream))
-    opts = _opts(dropout, X)
+    opts = _opts(dropout, X, adapter_ready)
     if opts is None:
         _check(lib.qlora_linear_bwd(*args), "qlora_linear_bwd")
     else:
         _check(lib.qlora_linear_bwd_ex(*args, ctypes.byref(opts)), "qlora_linear_bwd_ex")
+
+
+def qlora_linear_adapter_fwd(w: NF4Weight, X, M: int, A, B, r: int, scale: float, H_save=None,
+                             workspace=None, stream=None, dropout=None):
+    """The forward's adapter products alone (H into the workspace and H_save);
+    follow with qlora_linear_fwd(..., adapter_ready=True) on the same workspace."""
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    opts = _opts(dropout, X, always=True)
+    _check(lib.qlora_linear_adapter_fwd(ctypes.byref(w.desc), _ptr(X), M, _ptr(A), _ptr(B), r, scale, _ptr(H_save),
+                                        _ptr(workspace), ws_bytes, _stream(stream), ctypes.byref(opts)),
+           "qlora_linear_adapter_fwd")
+
+
+def qlora_linear_adapter_bwd(w: NF4Weight, X, dY, M: int, A, B, r: int, scale: float, H_saved,
+                             workspace=None, stream=None, dropout=None):
+    """The backward's adapter products alone (G, and H's hi/lo halves, into the
+    workspace); follow with qlora_linear_bwd(..., adapter_ready=True)."""
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    opts = _opts(dropout, X, always=True)
+    _check(lib.qlora_linear_adapter_bwd(ctypes.byref(w.desc), _ptr(X), _ptr(dY), M, _ptr(A), _ptr(B), r, scale,
+                                        _ptr(H_saved), _ptr(workspace), ws_bytes, _stream(stream),
+                                        ctypes.byref(opts)),
+           "qlora_linear_adapter_bwd")
 
 
 def qlora_status_string(status: int) -> str:

@@ -321,6 +321,11 @@ qlora_status run_split_sum(const float *planes, int splits, int64_t rows, int64_
 
 bool dropout_on(const qlora_linear_opts *o) { return o && o->dropout_mask; }
 
+// Which part of a linear call runs: all of it, only the adapter's low-rank
+// products (the split-off first step), or all but them (adapter_ready).
+enum Phase { kPhaseAll, kPhaseAdapter, kPhaseMain };
+Phase phase_of(const qlora_linear_opts *o) { return o && o->adapter_ready ? kPhaseMain : kPhaseAll; }
+
 float dropout_scale(const qlora_linear_opts *o) { return 1.0f / (1.0f - o->dropout_p); }
 
 // X_d from X and the mask, eight elements (one mask byte) per thread (F16:
@@ -372,6 +377,7 @@ qlora_status check_opts(const qlora_linear_opts *o)
 {
     if (!o) return QLORA_OK;
     if (o->compute_dtype != QLORA_BF16 && o->compute_dtype != QLORA_FP16) return QLORA_ERR_INVALID_ARG;
+    if (o->adapter_ready != 0 && o->adapter_ready != 1) return QLORA_ERR_INVALID_ARG;
     if (!o->dropout_mask) return QLORA_OK;
     if (!(o->dropout_p >= 0.0f && o->dropout_p < 1.0f)) return QLORA_ERR_INVALID_ARG;
     if (!aligned16(o->dropout_mask)) return QLORA_ERR_ALIGNMENT;
@@ -458,12 +464,15 @@ extern "C" size_t qlora_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, 
 template <bool F16>
 static qlora_status linear_fwd(const qlora_nf4_weight *w, const void *X, int64_t M, const void *A, const void *B,
                                int32_t r, float scale, void *Y, qlora_dtype y_dtype, float *H_save, void *workspace,
-                               size_t workspace_bytes, void *stream, const qlora_linear_opts *opts)
+                               size_t workspace_bytes, void *stream, const qlora_linear_opts *opts, Phase phase)
 {
     const bool drop = dropout_on(opts);
-    if (!Y) return QLORA_ERR_INVALID_ARG;
-    if (y_dtype != (F16 ? QLORA_FP16 : QLORA_BF16) && y_dtype != QLORA_FP32) return QLORA_ERR_INVALID_ARG;
-    if (!aligned16(Y) || (H_save && !aligned16(H_save))) return QLORA_ERR_ALIGNMENT;
+    if (phase != kPhaseAdapter) {
+        if (!Y) return QLORA_ERR_INVALID_ARG;
+        if (y_dtype != (F16 ? QLORA_FP16 : QLORA_BF16) && y_dtype != QLORA_FP32) return QLORA_ERR_INVALID_ARG;
+        if (!aligned16(Y)) return QLORA_ERR_ALIGNMENT;
+    }
+    if (H_save && !aligned16(H_save)) return QLORA_ERR_ALIGNMENT;
     DeviceInfo dev;
     QLORA_TRY(device_info(&dev));
     if (M == 0) return QLORA_OK;
@@ -474,15 +483,19 @@ static qlora_status linear_fwd(const qlora_nf4_weight *w, const void *X, int64_t
     // the adapter branch's input: X, or X_d under LoRA dropout
     const void *Xa = X;
     if (drop) {
-        QLORA_TRY(run_dropout_input<F16>(pl, dev, X, opts, ws, s));
+        if (phase != kPhaseMain) QLORA_TRY(run_dropout_input<F16>(pl, dev, X, opts, ws, s));
         Xa = ws + pl.off_xd;
     }
 
-    // a handful of tokens: stream the packed weight once (bound by HBM, not the tensor cores)
-    if (M <= kDecodeMaxTokens)
+    // a handful of tokens: stream the packed weight once (bound by HBM, not
+    // the tensor cores); H is formed inside that path
+    if (M <= kDecodeMaxTokens) {
+        if (phase == kPhaseAdapter) return launch_status();
         return run_decode_fwd(w, X, Xa, M, A, B, r, scale, Y, y_dtype, H_save, ws, workspace_bytes, dev, s, F16);
+    }
 
-    QLORA_TRY(run_h<F16>(pl, dev, Xa, A, scale, H_save, ws, s));
+    if (phase != kPhaseMain) QLORA_TRY(run_h<F16>(pl, dev, Xa, A, scale, H_save, ws, s));
+    if (phase == kPhaseAdapter) return launch_status();
 
     // fused forward: 256 tokens (two 128-row accumulators) x 128 output features per tile
     constexpr int kFBN = 128, kFMT = 2;
@@ -541,8 +554,25 @@ extern "C" qlora_status qlora_linear_fwd_ex(const qlora_nf4_weight *w, const voi
     QLORA_TRY(check_linear(w, X, M, A, B, r, workspace));
     QLORA_TRY(check_opts(opts));
     if (opts && opts->compute_dtype == QLORA_FP16)
-        return linear_fwd<true>(w, X, M, A, B, r, scale, Y, y_dtype, H_save, workspace, workspace_bytes, stream, opts);
-    return linear_fwd<false>(w, X, M, A, B, r, scale, Y, y_dtype, H_save, workspace, workspace_bytes, stream, opts);
+        return linear_fwd<true>(w, X, M, A, B, r, scale, Y, y_dtype, H_save, workspace, workspace_bytes, stream, opts,
+                                phase_of(opts));
+    return linear_fwd<false>(w, X, M, A, B, r, scale, Y, y_dtype, H_save, workspace, workspace_bytes, stream, opts,
+                             phase_of(opts));
+}
+
+extern "C" qlora_status qlora_linear_adapter_fwd(const qlora_nf4_weight *w, const void *X, int64_t M, const void *A,
+                                                 const void *B, int32_t r, float scale, float *H_save,
+                                                 void *workspace, size_t workspace_bytes, void *stream,
+                                                 const qlora_linear_opts *opts)
+{
+    QLORA_TRY(check_linear(w, X, M, A, B, r, workspace));
+    QLORA_TRY(check_opts(opts));
+    const qlora_dtype none = QLORA_FP32;
+    if (opts && opts->compute_dtype == QLORA_FP16)
+        return linear_fwd<true>(w, X, M, A, B, r, scale, nullptr, none, H_save, workspace, workspace_bytes, stream,
+                                opts, kPhaseAdapter);
+    return linear_fwd<false>(w, X, M, A, B, r, scale, nullptr, none, H_save, workspace, workspace_bytes, stream, opts,
+                             kPhaseAdapter);
 }
 
 extern "C" qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const void *X, int64_t M, const void *A,
@@ -557,19 +587,22 @@ template <bool F16>
 static qlora_status linear_bwd(const qlora_nf4_weight *w, const void *X, const void *dY, int64_t M, const void *A,
                                const void *B, int32_t r, float scale, const float *H_saved, void *dX,
                                qlora_dtype dx_dtype, float *dA, float *dB, void *workspace, size_t workspace_bytes,
-                               void *stream, const qlora_linear_opts *opts)
+                               void *stream, const qlora_linear_opts *opts, Phase phase)
 {
     const bool drop = dropout_on(opts);
-    if (!dY || !dA || !dB) return QLORA_ERR_INVALID_ARG;
-    if (dx_dtype != (F16 ? QLORA_FP16 : QLORA_BF16) && dx_dtype != QLORA_FP32) return QLORA_ERR_INVALID_ARG;
-    if (!aligned16(dY) || !aligned16(dA) || !aligned16(dB) || (dX && !aligned16(dX)) ||
-        (H_saved && !aligned16(H_saved)))
-        return QLORA_ERR_ALIGNMENT;
+    if (!dY) return QLORA_ERR_INVALID_ARG;
+    if (phase != kPhaseAdapter) {
+        if (!dA || !dB) return QLORA_ERR_INVALID_ARG;
+        if (dx_dtype != (F16 ? QLORA_FP16 : QLORA_BF16) && dx_dtype != QLORA_FP32) return QLORA_ERR_INVALID_ARG;
+        if (!aligned16(dA) || !aligned16(dB) || (dX && !aligned16(dX))) return QLORA_ERR_ALIGNMENT;
+    }
+    if (!aligned16(dY) || (H_saved && !aligned16(H_saved))) return QLORA_ERR_ALIGNMENT;
     DeviceInfo dev;
     QLORA_TRY(device_info(&dev));
     const int64_t N = w->rows, K = w->cols;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (M == 0) {
+        if (phase == kPhaseAdapter) return QLORA_OK;
         // no tokens: the adapter gradients are zero
         QLORA_CUDA_TRY(cudaMemsetAsync(dA, 0, (size_t)r * K * 4, s));
         QLORA_CUDA_TRY(cudaMemsetAsync(dB, 0, (size_t)N * r * 4, s));
@@ -584,18 +617,22 @@ static qlora_status linear_bwd(const qlora_nf4_weight *w, const void *X, const v
     // the adapter branch's input: X, or X_d under LoRA dropout
     const void *Xa = X;
     if (drop) {
-        QLORA_TRY(run_dropout_input<F16>(pl, dev, X, opts, ws, s));
+        if (phase != kPhaseMain) QLORA_TRY(run_dropout_input<F16>(pl, dev, X, opts, ws, s));
         Xa = ws + pl.off_xd;
     }
 
-    // H (hi/lo) recomputed when no saved H is given
-    if (!H_saved) QLORA_TRY(run_h<F16>(pl, dev, Xa, A, scale, nullptr, ws, s));
-
-    // G = s dY B (contraction over N); the same kernel splits a saved H into hi/lo
-    if (pl.r_pad == 64)
-        QLORA_TRY((run_lowrank<64, 1, F16>(pl, dev, dY, N, B, scale, G2, nullptr, H_saved, H_saved ? H2 : nullptr, s)));
-    else
-        QLORA_TRY((run_lowrank<128, 1, F16>(pl, dev, dY, N, B, scale, G2, nullptr, H_saved, H_saved ? H2 : nullptr, s)));
+    if (phase != kPhaseMain) {
+        // H (hi/lo) recomputed when no saved H is given
+        if (!H_saved) QLORA_TRY(run_h<F16>(pl, dev, Xa, A, scale, nullptr, ws, s));
+        // G = s dY B (contraction over N); the same kernel splits a saved H into hi/lo
+        if (pl.r_pad == 64)
+            QLORA_TRY((run_lowrank<64, 1, F16>(pl, dev, dY, N, B, scale, G2, nullptr, H_saved, H_saved ? H2 : nullptr,
+                                               s)));
+        else
+            QLORA_TRY((run_lowrank<128, 1, F16>(pl, dev, dY, N, B, scale, G2, nullptr, H_saved, H_saved ? H2 : nullptr,
+                                                s)));
+        if (phase == kPhaseAdapter) return launch_status();
+    }
 
     // dX = dY W' + bf16(G) A  (fused transposed dequant-GEMM)
     if (dX) {
@@ -732,9 +769,24 @@ extern "C" qlora_status qlora_linear_bwd_ex(const qlora_nf4_weight *w, const voi
     QLORA_TRY(check_opts(opts));
     if (opts && opts->compute_dtype == QLORA_FP16)
         return linear_bwd<true>(w, X, dY, M, A, B, r, scale, H_saved, dX, dx_dtype, dA, dB, workspace, workspace_bytes,
-                                stream, opts);
+                                stream, opts, phase_of(opts));
     return linear_bwd<false>(w, X, dY, M, A, B, r, scale, H_saved, dX, dx_dtype, dA, dB, workspace, workspace_bytes,
-                             stream, opts);
+                             stream, opts, phase_of(opts));
+}
+
+extern "C" qlora_status qlora_linear_adapter_bwd(const qlora_nf4_weight *w, const void *X, const void *dY, int64_t M,
+                                                 const void *A, const void *B, int32_t r, float scale,
+                                                 const float *H_saved, void *workspace, size_t workspace_bytes,
+                                                 void *stream, const qlora_linear_opts *opts)
+{
+    QLORA_TRY(check_linear(w, X, M, A, B, r, workspace));
+    QLORA_TRY(check_opts(opts));
+    const qlora_dtype none = QLORA_FP32;
+    if (opts && opts->compute_dtype == QLORA_FP16)
+        return linear_bwd<true>(w, X, dY, M, A, B, r, scale, H_saved, nullptr, none, nullptr, nullptr, workspace,
+                                workspace_bytes, stream, opts, kPhaseAdapter);
+    return linear_bwd<false>(w, X, dY, M, A, B, r, scale, H_saved, nullptr, none, nullptr, nullptr, workspace,
+                             workspace_bytes, stream, opts, kPhaseAdapter);
 }
 
 extern "C" qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const void *X, const void *dY, int64_t M,

@@ -441,11 +441,16 @@ QLORA_API qlora_status qlora_block_bwd(const qlora_block *blk, const void *x, co
  *                 dx_dtype are then that type or QLORA_FP32 (the blog's
  *                 BitsAndBytesConfig snippet, bnb_4bit_compute_dtype).  H and
  *                 G are carried as hi + lo pairs of the same type.
+ *   adapter_ready 0 (default) or 1: the adapter's low-rank products of this
+ *                 call are already in the workspace, written by
+ *                 qlora_linear_adapter_fwd / qlora_linear_adapter_bwd with the
+ *                 same arguments and options; the call runs the rest only.
  */
 typedef struct {
     const uint8_t *dropout_mask;
     float dropout_p;
     qlora_dtype compute_dtype;
+    int32_t adapter_ready;
 } qlora_linear_opts;
 
 /* Workspace bytes for the _ex entry points with these options (dropout needs
@@ -466,6 +471,33 @@ QLORA_API qlora_status qlora_linear_bwd_ex(const qlora_nf4_weight *w, const void
                                            const float *H_saved, void *dX, qlora_dtype dx_dtype, float *dA,
                                            float *dB, void *workspace, size_t workspace_bytes, void *stream,
                                            const qlora_linear_opts *opts);
+
+/*
+ * The first step of a linear call on its own: the adapter's low-rank products
+ * (and, under LoRA dropout, the dropped-out input), written into the
+ * workspace.  A later qlora_linear_fwd_ex / qlora_linear_bwd_ex on the same
+ * workspace, with the same arguments and opts->adapter_ready = 1, runs the
+ * rest and produces the same bits as the undivided call.  Splitting lets a
+ * caller run these small, bandwidth-bound products of independent linears on
+ * a second stream, beside another linear's fused GEMM (the two halves must
+ * then be ordered by an event; nothing else may use the workspace between
+ * them).
+ *   qlora_linear_adapter_fwd: H = s X A^T (X_d under dropout), into the
+ *       workspace and into H_save if given.  At 16 tokens or fewer H is formed
+ *       inside the decode forward instead; this call then only prepares X_d
+ *       (if dropout is on), and the forward writes H_save.
+ *   qlora_linear_adapter_bwd: H recomputed if H_saved is NULL (else split
+ *       into its hi + lo halves) and G = s dY B.
+ * Arguments as for qlora_linear_fwd_ex / qlora_linear_bwd_ex (Y, dX, dA, dB
+ * omitted).  Errors as there.
+ */
+QLORA_API qlora_status qlora_linear_adapter_fwd(const qlora_nf4_weight *w, const void *X, int64_t M, const void *A,
+                                                const void *B, int32_t r, float scale, float *H_save, void *workspace,
+                                                size_t workspace_bytes, void *stream, const qlora_linear_opts *opts);
+QLORA_API qlora_status qlora_linear_adapter_bwd(const qlora_nf4_weight *w, const void *X, const void *dY, int64_t M,
+                                                const void *A, const void *B, int32_t r, float scale,
+                                                const float *H_saved, void *workspace, size_t workspace_bytes,
+                                                void *stream, const qlora_linear_opts *opts);
 
 /* Human-readable name of a status code (static string, never NULL). */
 QLORA_API const char *qlora_status_string(qlora_status status);

@@ -387,3 +387,57 @@ def test_fp16_compute_dtype_llama7b_gate(q):
     rdA, rdB = olin.backward_weight_grads(X, A, B, s, dY)
     assert_close(np64(dA), rdA, what="dA")
     assert_close(np64(dB), rdB, what="dB")
+
+
+def _whole_or_split(q, run, ydt, dropout, split, side=None):
+    """Forward then backward, either as single calls or with the adapter
+    products split off (optionally on a side stream, ordered by events)."""
+    M, N, K, r, s = run.M, run.w.rows, run.w.cols, run.c["r"], run.c["scale"]
+    ws = torch.zeros(q.qlora_linear_workspace_bytes(M, N, K, r, dropout=dropout), dtype=torch.uint8, device="cuda")
+    Y = torch.empty(M, N, dtype=ydt, device="cuda")
+    H = torch.empty(M, r, dtype=torch.float32, device="cuda")
+    dX = torch.empty(M, K, dtype=ydt, device="cuda")
+    dA = torch.empty(r, K, dtype=torch.float32, device="cuda")
+    dB = torch.empty(N, r, dtype=torch.float32, device="cuda")
+    main = torch.cuda.current_stream()
+    args_f = (run.w, run.X, M, run.A, run.B, r, s)
+    args_b = (run.w, run.X, run.dY, M, run.A, run.B, r, s, H)
+    if not split:
+        q.qlora_linear_fwd(*args_f, Y, H, ws, dropout=dropout)
+        q.qlora_linear_bwd(*args_b, dX, dA, dB, ws, dropout=dropout)
+    else:
+        for phase in ("fwd", "bwd"):
+            st = side if side is not None else main
+            st.wait_stream(main)
+            with torch.cuda.stream(st):
+                if phase == "fwd":
+                    q.qlora_linear_adapter_fwd(*args_f, H, ws, stream=st, dropout=dropout)
+                else:
+                    q.qlora_linear_adapter_bwd(*args_b, ws, stream=st, dropout=dropout)
+            main.wait_stream(st)
+            if phase == "fwd":
+                q.qlora_linear_fwd(*args_f, Y, H, ws, dropout=dropout, adapter_ready=True)
+            else:
+                q.qlora_linear_bwd(*args_b, dX, dA, dB, ws, dropout=dropout, adapter_ready=True)
+    q.qlora_check_device_error()
+    return Y, H, dX, dA, dB
+
+
+@pytest.mark.parametrize("M,p", [(512, None), (600, 0.1), (200, None), (16, None), (16, 0.1), (4096, None)])
+@pytest.mark.parametrize("ydt", [torch.bfloat16, torch.float32])
+def test_adapter_split_equals_whole_call(q, M, p, ydt):
+    """The adapter products run on their own first (qlora_linear_adapter_fwd /
+    _bwd, on a side stream for the CTA-pair sizes), then the rest of each
+    call with adapter_ready: the same bits as the undivided calls, for the
+    CTA-pair, single-CTA and decode paths, with and without LoRA dropout."""
+    N, K, r = (4096, 4096, 64) if M == 4096 else (384, 512, 64)
+    run = Runner(q, synthetic.linear_case(M, N, K, r, alpha=16.0, seed=4000 + M))
+    dropout = None
+    if p is not None:
+        _, packed = synthetic.dropout_mask(M, K, p, seed=4100 + M, device="cuda")
+        dropout = (packed, p)
+    side = torch.cuda.Stream() if M > 256 else None
+    whole = _whole_or_split(q, run, ydt, dropout, split=False)
+    split = _whole_or_split(q, run, ydt, dropout, split=True, side=side)
+    for name, a, b in zip(("Y", "H", "dX", "dA", "dB"), whole, split):
+        assert torch.equal(a, b), name
