@@ -239,6 +239,50 @@ def test_validation_of_the_linear_layer(lib):
     assert b(r=200) == 2
 
 
+class Opts(ctypes.Structure):
+    _fields_ = [("dropout_mask", ctypes.c_void_p), ("dropout_p", ctypes.c_float), ("compute_dtype", ctypes.c_int),
+                ("adapter_ready", ctypes.c_int32)]
+
+
+def test_validation_of_the_split_adapter_step(lib):
+    """qlora_linear_adapter_fwd / _bwd and the adapter_ready option reject bad
+    arguments before any CUDA call; the adapter calls need no output buffers."""
+    q = ocb.nf4_codebook()
+    fake = 0x10000
+    P, I64, I32, F, S, I = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t,
+                            ctypes.c_int)
+    W, O = ctypes.POINTER(Weight), ctypes.POINTER(Opts)
+    afwd = lib.qlora_linear_adapter_fwd
+    afwd.argtypes = [W, P, I64, P, P, I32, F, P, P, S, P, O]
+    abwd = lib.qlora_linear_adapter_bwd
+    abwd.argtypes = [W, P, P, I64, P, P, I32, F, P, P, S, P, O]
+    fwd_ex = lib.qlora_linear_fwd_ex
+    fwd_ex.argtypes = [W, P, I64, P, P, I32, F, P, I, P, P, S, P, O]
+    w = Weight(256, 256, fake, fake, fake, fake, (ctypes.c_float * 16)(*q))
+    good = Opts(None, 0.0, 0, 0)
+
+    def af(X=fake, M=64, A=fake, r=16, H=None, ws=fake, opts=good):
+        return afwd(ctypes.byref(w), X, M, A, fake, r, 1.0, H, ws, 1 << 30, None,
+                    None if opts is None else ctypes.byref(opts))
+
+    def ab(dY=fake, M=64, r=16, H=None, opts=good):
+        return abwd(ctypes.byref(w), fake, dY, M, fake, fake, r, 1.0, H, fake, 1 << 30, None,
+                    None if opts is None else ctypes.byref(opts))
+
+    assert af(X=None) == 1 and af(A=None) == 1 and af(ws=None) == 1 and af(M=-1) == 1
+    assert af(r=12) == 2
+    assert af(X=fake + 2) == 3 and af(H=fake + 4) == 3
+    assert af(opts=Opts(None, 0.0, 0, 2)) == 1                 # adapter_ready is 0 or 1
+    assert af(opts=Opts(None, 0.0, 9, 0)) == 1                 # unknown compute dtype
+    assert af(opts=Opts(fake + 4, 0.1, 0, 0)) == 3             # misaligned dropout mask
+    assert af(opts=Opts(fake, 1.0, 0, 0)) == 1                 # p outside [0, 1)
+    assert ab(dY=None) == 1 and ab(dY=fake + 2) == 3 and ab(H=fake + 4) == 3 and ab(r=136) == 2
+    assert ab(opts=Opts(None, 0.0, 0, 3)) == 1
+    bad = Opts(None, 0.0, 0, 2)
+    assert fwd_ex(ctypes.byref(w), fake, 64, fake, fake, 16, 1.0, fake, 1, None, fake, 1 << 30, None,
+                  ctypes.byref(bad)) == 1
+
+
 def test_stall_hook_validation(lib):
     """The failure-detection test hook only arms the kernel families that have
     pipeline waits, with a limit in range; it makes no CUDA call."""
