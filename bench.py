@@ -192,12 +192,12 @@ def run_ours(args, rank, world, local_rank):
     reducer = dp.OverlappedGradSum()
 
     # The seven linears are independent, so each linear's small adapter
-    # products (H in the forward, G in the backward) run on a low-priority
-    # side stream through the split-off adapter calls, beside the previous
-    # linear's fused GEMM: they become runnable when that GEMM does (an event
-    # recorded just before it), the GEMM's CTAs take the SMs first, and the
-    # adapter kernels fill the SMs its partial last round of tiles leaves
-    # idle.  Each linear then has its own workspace.
+    # products (H in the forward; G, then dA and dB, in the backward) run on a
+    # low-priority side stream through the split-off adapter calls, beside
+    # the previous linear's fused GEMM: they become runnable when that GEMM
+    # does (an event recorded just before it), the GEMM's CTAs take the SMs
+    # first, and the small kernels fill the SMs its partial last round of
+    # tiles leaves idle.  Each linear then has its own workspace.
     mode = {"split": not args.no_adapter_split}
     gemm_s = torch.cuda.Stream(priority=-1)
     side_s = torch.cuda.Stream(priority=0)
@@ -241,13 +241,18 @@ def run_ours(args, rank, world, local_rank):
                         q.qlora_linear_fwd(L["w"], L["X"], TOKENS, L["A"], L["B"], R, scale, L["Y"], L["H"],
                                            L["ws"], stream=gemm_s, adapter_ready=True)
                     else:
+                        # the input gradient alone: dA and dB need G, not dX, and follow on the side stream
                         q.qlora_linear_bwd(L["w"], L["X"], L["dY"], TOKENS, L["A"], L["B"], R, scale, L["H"],
-                                           L["dX"], L["dA"], L["dB"], L["ws"], stream=gemm_s, adapter_ready=True)
-                        reducer.ready(L["grad"])   # this linear's dA, dB: summed while the backward goes on
+                                           L["dX"], None, None, L["ws"], stream=gemm_s, adapter_ready=True)
                 if i + 1 < len(order):
                     # the next linear's adapter products become runnable with this GEMM
                     side_s.wait_event(L["ev"][go])
                     adapter(order[i + 1])
+                if phase == "bwd":
+                    with torch.cuda.stream(side_s):
+                        q.qlora_linear_bwd(L["w"], L["X"], L["dY"], TOKENS, L["A"], L["B"], R, scale, L["H"],
+                                           None, L["dA"], L["dB"], L["ws"], stream=side_s, adapter_ready=True)
+                        reducer.ready(L["grad"])   # this linear's dA, dB: summed while the backward goes on
             if phase == "fwd":
                 # the backward's adapter call rewrites the workspace the forward GEMM read
                 side_s.wait_stream(gemm_s)

@@ -591,10 +591,14 @@ static qlora_status linear_bwd(const qlora_nf4_weight *w, const void *X, const v
 {
     const bool drop = dropout_on(opts);
     if (!dY) return QLORA_ERR_INVALID_ARG;
+    // the weight gradients are formed unless both dA and dB are NULL, which
+    // only the rest of a split call allows (it then forms dX alone)
+    const bool wgrad = dA || dB;
     if (phase != kPhaseAdapter) {
-        if (!dA || !dB) return QLORA_ERR_INVALID_ARG;
+        if (wgrad && (!dA || !dB)) return QLORA_ERR_INVALID_ARG;
+        if (!wgrad && (phase != kPhaseMain || !dX)) return QLORA_ERR_INVALID_ARG;
         if (dx_dtype != (F16 ? QLORA_FP16 : QLORA_BF16) && dx_dtype != QLORA_FP32) return QLORA_ERR_INVALID_ARG;
-        if (!aligned16(dA) || !aligned16(dB) || (dX && !aligned16(dX))) return QLORA_ERR_ALIGNMENT;
+        if ((wgrad && (!aligned16(dA) || !aligned16(dB))) || (dX && !aligned16(dX))) return QLORA_ERR_ALIGNMENT;
     }
     if (!aligned16(dY) || (H_saved && !aligned16(H_saved))) return QLORA_ERR_ALIGNMENT;
     DeviceInfo dev;
@@ -602,7 +606,7 @@ static qlora_status linear_bwd(const qlora_nf4_weight *w, const void *X, const v
     const int64_t N = w->rows, K = w->cols;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (M == 0) {
-        if (phase == kPhaseAdapter) return QLORA_OK;
+        if (phase == kPhaseAdapter || !wgrad) return QLORA_OK;
         // no tokens: the adapter gradients are zero
         QLORA_CUDA_TRY(cudaMemsetAsync(dA, 0, (size_t)r * K * 4, s));
         QLORA_CUDA_TRY(cudaMemsetAsync(dB, 0, (size_t)N * r * 4, s));
@@ -726,7 +730,7 @@ static qlora_status linear_bwd(const qlora_nf4_weight *w, const void *X, const v
     // dA = (X^T [G_hi | G_lo])^T and dB = dY^T [H_hi | H_lo] in one launch: output rows k
     // (resp. n), 128-column tiles = the hi and lo halves of one 64-column chunk,
     // contraction over the tokens; the reduction adds the halves
-    {
+    if (wgrad) {
         const int *maxc = nullptr;
         QLORA_TRY((skinny_setup<128, 1, 1, F16>(dev, &maxc)));
         SkinnyParams p{};

@@ -490,6 +490,10 @@ QLORA_API qlora_status qlora_linear_bwd_ex(const qlora_nf4_weight *w, const void
  *       into its hi + lo halves) and G = s dY B.
  * Arguments as for qlora_linear_fwd_ex / qlora_linear_bwd_ex (Y, dX, dA, dB
  * omitted).  Errors as there.
+ * The rest of a split backward (adapter_ready = 1) may also be divided: with
+ * dA = dB = NULL it forms dX alone, with dX = NULL dA and dB alone (the weight
+ * gradients need G, not dX, so they may run on another stream than dX).  The
+ * undivided backward requires dA and dB (INVALID_ARG otherwise).
  */
 QLORA_API qlora_status qlora_linear_adapter_fwd(const qlora_nf4_weight *w, const void *X, int64_t M, const void *A,
                                                 const void *B, int32_t r, float scale, float *H_save, void *workspace,

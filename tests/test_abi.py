@@ -278,6 +278,18 @@ def test_validation_of_the_split_adapter_step(lib):
     assert af(opts=Opts(fake, 1.0, 0, 0)) == 1                 # p outside [0, 1)
     assert ab(dY=None) == 1 and ab(dY=fake + 2) == 3 and ab(H=fake + 4) == 3 and ab(r=136) == 2
     assert ab(opts=Opts(None, 0.0, 0, 3)) == 1
+    bwd_ex = lib.qlora_linear_bwd_ex
+    bwd_ex.argtypes = [W, P, P, I64, P, P, I32, F, P, P, I, P, P, P, S, P, O]
+    ready = Opts(None, 0.0, 0, 1)
+
+    def b(dX=fake, dA=fake, dB=fake, opts=ready):
+        return bwd_ex(ctypes.byref(w), fake, fake, 64, fake, fake, 16, 1.0, None, dX, 1, dA, dB, fake, 1 << 30, None,
+                      ctypes.byref(opts))
+
+    assert b(dA=None) == 1 and b(dB=None) == 1                   # dA and dB come together
+    assert b(dX=None, dA=None, dB=None) == 1                     # nothing to form
+    assert b(dA=None, dB=None, opts=good) == 1                   # the undivided backward needs dA, dB
+    assert b(dA=None, dB=None, dX=fake + 4) == 3
     bad = Opts(None, 0.0, 0, 2)
     assert fwd_ex(ctypes.byref(w), fake, 64, fake, fake, 16, 1.0, fake, 1, None, fake, 1 << 30, None,
                   ctypes.byref(bad)) == 1

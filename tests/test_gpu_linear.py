@@ -389,9 +389,11 @@ def test_fp16_compute_dtype_llama7b_gate(q):
     assert_close(np64(dB), rdB, what="dB")
 
 
-def _whole_or_split(q, run, ydt, dropout, split, side=None):
+def _whole_or_split(q, run, ydt, dropout, split, side=None, divide_bwd=False):
     """Forward then backward, either as single calls or with the adapter
-    products split off (optionally on a side stream, ordered by events)."""
+    products split off (optionally on a side stream, ordered by events);
+    divide_bwd: the rest of the backward as two calls, dA and dB on the side
+    stream and dX on the main one."""
     M, N, K, r, s = run.M, run.w.rows, run.w.cols, run.c["r"], run.c["scale"]
     ws = torch.zeros(q.qlora_linear_workspace_bytes(M, N, K, r, dropout=dropout), dtype=torch.uint8, device="cuda")
     Y = torch.empty(M, N, dtype=ydt, device="cuda")
@@ -417,6 +419,11 @@ def _whole_or_split(q, run, ydt, dropout, split, side=None):
             main.wait_stream(st)
             if phase == "fwd":
                 q.qlora_linear_fwd(*args_f, Y, H, ws, dropout=dropout, adapter_ready=True)
+            elif divide_bwd:
+                q.qlora_linear_bwd(*args_b, dX, None, None, ws, dropout=dropout, adapter_ready=True)
+                with torch.cuda.stream(st):
+                    q.qlora_linear_bwd(*args_b, None, dA, dB, ws, stream=st, dropout=dropout, adapter_ready=True)
+                main.wait_stream(st)
             else:
                 q.qlora_linear_bwd(*args_b, dX, dA, dB, ws, dropout=dropout, adapter_ready=True)
     q.qlora_check_device_error()
@@ -441,3 +448,6 @@ def test_adapter_split_equals_whole_call(q, M, p, ydt):
     split = _whole_or_split(q, run, ydt, dropout, split=True, side=side)
     for name, a, b in zip(("Y", "H", "dX", "dA", "dB"), whole, split):
         assert torch.equal(a, b), name
+    divided = _whole_or_split(q, run, ydt, dropout, split=True, side=side or torch.cuda.Stream(), divide_bwd=True)
+    for name, a, b in zip(("Y", "H", "dX", "dA", "dB"), whole, divided):
+        assert torch.equal(a, b), "divided backward: " + name
